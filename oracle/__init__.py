@@ -1,0 +1,125 @@
+"""CPU oracle for the weight-only quantized Linear -- TEST INFRASTRUCTURE ONLY.
+
+A plain fp64 C statement of RTN quantization and of the quantized Linear (see
+``wlq_oracle.c`` for the arithmetic and the pages each step follows).  It is
+independent of the CUDA library: the two share no code, and the oracle never
+calls the library or the library the oracle.  Only ``tests/``,
+``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg may import it.
+
+Parity: every function here is pinned by tests that do not re-use it
+(brute-force enumeration, closed-form bounds, invariants, special cases that
+reduce to library routines).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "wlq_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+OK, ERR_ARG, ERR_NONFINITE = 0, 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (OpenMP, strict IEEE: no contraction)."""
+    if force or not os.path.exists(_LIB_PATH) or (
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    ):
+        tmp = _LIB_PATH + ".tmp.%d" % os.getpid()
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+               "-shared", "-fPIC", _SRC, "-o", tmp, "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def bind(path: str):
+    """Load an oracle shared object and declare its entry points."""
+    lib = ctypes.CDLL(path)
+    i64, i32, vp = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
+    lib.oracle_quantize.argtypes = [vp, i64, i64, i32, i32, vp, vp]
+    lib.oracle_dequantize.argtypes = [vp, vp, i64, i64, i32, vp]
+    lib.oracle_linear.argtypes = [vp, i64, i64, vp, vp, i64, i32, vp, vp, vp, i32, vp]
+    for f in (lib.oracle_quantize, lib.oracle_dequantize, lib.oracle_linear):
+        f.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = bind(build())
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def _check(rc):
+    if rc == ERR_NONFINITE:
+        raise OracleError("non-finite weight")
+    if rc != OK:
+        raise OracleError("invalid argument (rc=%d)" % rc)
+
+
+def groups_of(K: int, group: int) -> int:
+    return 1 if group == 0 else K // group
+
+
+def quantize(W: np.ndarray, bits: int, group: int):
+    """RTN symmetric quantization: returns (codes int8 [N,K], scales fp32 [N,G])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    codes = np.empty((N, K), np.int8)
+    scales = np.empty((N, groups_of(K, group)), np.float32)
+    _check(_load().oracle_quantize(_p(W), N, K, bits, group, _p(codes), _p(scales)))
+    return codes, scales
+
+
+def dequantize(codes: np.ndarray, scales: np.ndarray, group: int) -> np.ndarray:
+    """deq[n,k] = q[n,k] * s[n, k/g], exact in fp64."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    N, K = codes.shape
+    out = np.empty((N, K), np.float64)
+    _check(_load().oracle_dequantize(_p(codes), _p(scales), N, K, group, _p(out)))
+    return out
+
+
+def linear(x_bits: np.ndarray, codes: np.ndarray, scales: np.ndarray, group: int,
+           bias_bits=None, L1_bits=None, L2_bits=None) -> np.ndarray:
+    """y = x deq(codes, scales)^T [+ (x L1) L2] [+ b] in fp64.
+
+    x_bits, bias_bits, L1_bits, L2_bits are bf16 bit patterns (uint16):
+    x [M,K], bias [N], L1 [K,r], L2 [r,N].
+    """
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    M, K = x_bits.shape
+    N = codes.shape[0]
+    assert codes.shape[1] == K
+    r = 0
+    if L1_bits is not None:
+        L1_bits = np.ascontiguousarray(L1_bits, dtype=np.uint16)
+        L2_bits = np.ascontiguousarray(L2_bits, dtype=np.uint16)
+        r = L1_bits.shape[1]
+        assert L1_bits.shape == (K, r) and L2_bits.shape == (r, N)
+    if bias_bits is not None:
+        bias_bits = np.ascontiguousarray(bias_bits, dtype=np.uint16)
+        assert bias_bits.shape == (N,)
+    y = np.empty((M, N), np.float64)
+    _check(_load().oracle_linear(_p(x_bits), M, K, _p(codes), _p(scales), N, group,
+                                 _p(bias_bits), _p(L1_bits), _p(L2_bits), r, _p(y)))
+    return y

@@ -1,0 +1,61 @@
+"""The oracle's pins are sensitive: a copy of the oracle with one planted
+mistake (compiled on the CPU into a temporary directory, never committed)
+must fail at least one pin.  Each mutation is a plausible slip: a wrong tie
+rule, a wrong qmax, a signed max in place of the absmax, a dropped term, a
+transposed index, a wrong group index.
+"""
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+import tests.test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "wlq_oracle.c")
+
+MUTATIONS = {
+    "ties_round_up": ("return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;", "return f + 1.0;"),
+    "qmax_off_by_one": ("const double qmax = (double)((1 << (bits - 1)) - 1);",
+                        "const double qmax = (double)(1 << (bits - 1));"),
+    "bias_dropped": ("if (bias) acc += bf16_value(bias[n]);", "(void)bias;"),
+    "low_rank_transposed": ("acc += T[j] * bf16_value(L2[(int64_t)j * N + n]);",
+                            "acc += T[j] * bf16_value(L2[n * (int64_t)r + j]);"),
+    "group_index": ("(double)scales[n * G + k / g];\n                acc",
+                    "(double)scales[n * G + k % G];\n                acc"),
+    "signed_max": ("double v = fabs((double)w[k]);", "double v = (double)w[k];"),
+}
+
+PIN_TESTS = [
+    lambda: pins.test_quantize_matches_brute_force(8),
+    lambda: pins.test_quantize_matches_brute_force(4),
+    lambda: pins.test_exact_ties_round_to_even(),
+    lambda: pins.test_grouping_matches_brute_force(4, 16),
+    lambda: pins.test_rtn_error_bound(4, 64),
+    lambda: pins.test_linear_exact_rationals_tiny(),
+    lambda: pins.test_linear_matches_numpy_matmul(4, 16),
+    lambda: pins.test_linear_matches_numpy_matmul(8, 0),
+    lambda: pins.test_linear_low_rank_only_and_plain_only(),
+]
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name, monkeypatch):
+    old, new = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, name
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "mut.c")
+        so = os.path.join(d, "libmut.so")
+        open(c, "w").write(src.replace(old, new))
+        subprocess.check_call(["gcc", "-O1", "-std=c11", "-fopenmp", "-ffp-contract=off",
+                               "-shared", "-fPIC", c, "-o", so, "-lm"])
+        monkeypatch.setattr(oracle, "_lib", oracle.bind(so))
+        failures = 0
+        for t in PIN_TESTS:
+            try:
+                t()
+            except (AssertionError, oracle.OracleError):
+                failures += 1
+        assert failures > 0, "mutation %s slipped past every pin" % name
