@@ -1,0 +1,152 @@
+/*
+ * wlq.h -- weight-only quantized Linear for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (web pages, cited by title and section):
+ *  - "Joy-face_change_optimized" model card (README), section "what this
+ *    branch does", files table: a weight-only Linear whose weights are int8
+ *    with one scale per output channel, or int4 grouped along the input
+ *    dimension, plus a loader for the exported codes; tools row: RTN int8,
+ *    RTN int4 with group size 64, and attention-int8 / MLP-int4 with group
+ *    size 16.
+ *  - "Nunchaku Lite: loading and running 4-bit SVDQuant" (news article),
+ *    section "why it matters": the hard part of the weights is carried by a
+ *    16-bit low-rank correction; section "how it works": the W4A16 kernels
+ *    keep activations in 16 bits.
+ *
+ * Conventions shared by every call:
+ *  - W is [N, K] row-major (N outputs, K inputs); x is [M, K] and y is [M, N],
+ *    both row-major.  qmax = 2^(bits-1) - 1.
+ *  - Every pointer is a DEVICE pointer owned by the caller, on the current
+ *    CUDA device, unless stated otherwise.  The library allocates no device
+ *    memory and keeps no state other than one error word per device.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Compute calls are asynchronous on it: argument errors are
+ *    returned before anything is enqueued; faults detected on the device
+ *    (non-finite weights, a bounded wait that ran out) are recorded in the
+ *    device error word and returned by wlq_get_status().
+ *  - Supported recipes (bits, group): (8, 0) = int8 per output channel;
+ *    (4, 64) and (4, 16) = int4 grouped along K.  wlq_quantize also accepts
+ *    (8, g) and (4, 0) for g in {16, 32, 64, 128}.
+ *  - Requirements: K % 8 == 0, K % group == 0, pointers 16-byte aligned.
+ *  - Only sm_100 devices are supported (WLQ_ERR_UNSUPPORTED otherwise).
+ */
+#ifndef WLQ_H_
+#define WLQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    WLQ_OK = 0,
+    WLQ_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad dtype     */
+    WLQ_ERR_SHAPE = 2,       /* K % 8, K % group, r out of range           */
+    WLQ_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned           */
+    WLQ_ERR_UNSUPPORTED = 4, /* recipe or device architecture not handled  */
+    WLQ_ERR_NONFINITE = 5,   /* a weight was NaN or +-Inf (device-detected) */
+    WLQ_ERR_WORKSPACE = 6,   /* workspace missing or smaller than required */
+    WLQ_ERR_TIMEOUT = 7,     /* a bounded device wait ran out              */
+    WLQ_ERR_CUDA = 8         /* a CUDA runtime / driver call failed        */
+} wlq_status;
+
+typedef enum { WLQ_OUT_BF16 = 0, WLQ_OUT_F32 = 1 } wlq_out_dtype;
+
+/*
+ * RTN symmetric quantization ("Joy-face_change_optimized", files table and
+ * tools row).  For each group (a whole row when group == 0, else `group`
+ * contiguous inputs of a row, starting at k = 0):
+ *   a = max |W|,  s = fp32(a / qmax)  (IEEE division, round to nearest even),
+ *   q = clamp(round_half_even(W / s), -qmax, qmax) computed exactly,
+ *   s == 0 (all-zero group) gives q = 0.
+ * W      : fp32 [N, K]
+ * codes  : int8 [N, K] (values in [-qmax, qmax])
+ * scales : fp32 [N, K / g] with g = K when group == 0
+ * A non-finite weight sets WLQ_ERR_NONFINITE in the device error word (its
+ * code is written as 0); the call itself still returns WLQ_OK.
+ * N == 0 is a no-op.
+ */
+wlq_status wlq_quantize(const float* W, int64_t N, int64_t K, int bits, int group,
+                        int8_t* codes, float* scales, void* stream);
+
+/*
+ * Bytes of the packed operand produced by wlq_pack (0 for an unsupported
+ * recipe or a bad shape).  Host-only, no device access.
+ * Layout: ceil(N/128) * ceil(K/64) tiles of 128 outputs x 64 inputs, each
+ * holding the codes (int8: 8192 B; int4: 4096 B) followed, for int4, by the
+ * tile's group scales in fp16 (gs64: 256 B; gs16: 1024 B), then one fp32
+ * factor per padded output row (int8: the channel scale; int4: the power of
+ * two that undoes the row's fp16 scale normalisation).
+ */
+size_t wlq_packed_bytes(int64_t N, int64_t K, int bits, int group);
+
+/*
+ * Lay codes and scales out for the GEMM (the pages' "loader" step).  Codes
+ * are stored offset-binary (q + 2^(bits-1)); int4 group scales are stored as
+ * fp16(s * 2^e_n) with one power of two e_n per output row, chosen so the
+ * row's largest scale lands in [2^8, 2^9).  Rows and inputs beyond N and K
+ * are zero-filled.
+ * codes: int8 [N, K]; scales: fp32 [N, K / g]; packed: wlq_packed_bytes().
+ */
+wlq_status wlq_pack(const int8_t* codes, const float* scales, int64_t N, int64_t K,
+                    int bits, int group, void* packed, void* stream);
+
+/* Inverse of the code part of wlq_pack: packed -> codes int8 [N, K]. */
+wlq_status wlq_unpack(const void* packed, int64_t N, int64_t K, int bits, int group,
+                      int8_t* codes, void* stream);
+
+/*
+ * Workspace bytes wlq_linear needs for this shape (host-only).  The
+ * workspace must be zero-filled once after it is allocated; every successful
+ * wlq_linear call leaves its counters zeroed again.  A workspace must not be
+ * shared by calls that may run concurrently.
+ */
+size_t wlq_linear_workspace(int64_t M, int64_t N, int64_t K, int bits, int group, int r);
+
+/*
+ * Weight-only quantized Linear ("Joy-face_change_optimized", files table;
+ * "Nunchaku Lite", why it matters / how it works):
+ *   y[m,n] = sum_k x[m,k] q[n,k] s[n, k/g]  +  sum_j (x L1)[m,j] L2[j,n]  +  b[n]
+ * accumulated in fp32 on the tensor cores.
+ * x      : bf16 [M, K]
+ * packed : output of wlq_pack for (N, K, bits, group)
+ * bias   : bf16 [N] or NULL
+ * L1, L2 : bf16 [K, r] and [r, N], or NULL with r == 0; r in {0, 16, 32, 64}
+ * y      : [M, N] in y_dtype (WLQ_OUT_BF16 or WLQ_OUT_F32)
+ * workspace / ws_bytes : at least wlq_linear_workspace(M, N, K, bits, group, r)
+ *                        bytes (may be NULL when that is 0)
+ * M == 0 or N == 0 is a no-op.  Results are bitwise reproducible run to run.
+ */
+wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, int64_t K,
+                      int bits, int group, const void* bias, const void* L1, const void* L2,
+                      int r, void* y, int y_dtype, void* workspace, size_t ws_bytes,
+                      void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear this device's error word:
+ * WLQ_OK, WLQ_ERR_NONFINITE or WLQ_ERR_TIMEOUT (or WLQ_ERR_CUDA).
+ */
+wlq_status wlq_get_status(void* stream);
+
+/*
+ * Exercise the bounded device wait on its own: one CTA waits, through the
+ * same helper the GEMM uses, on a barrier that nothing ever arrives at, for
+ * at most `timeout_ns` nanoseconds (capped at 10 s), then records
+ * WLQ_ERR_TIMEOUT in the device error word and exits.  No other work is
+ * touched; the device stays usable.  For failure-path tests.
+ */
+wlq_status wlq_probe_wait_timeout(uint64_t timeout_ns, void* stream);
+
+/* Human-readable text of the last error returned on this host thread. */
+const char* wlq_last_error(void);
+
+/* Library version, e.g. "0.1.0". */
+const char* wlq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WLQ_H_ */

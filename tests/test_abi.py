@@ -1,0 +1,124 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point include/wlq.h declares, and its host-only logic (sizes, argument
+checks that run before any device access) behaves as documented."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests.test_golden_shapes import load_golden
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wlq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from weight_only_quantized_rtn_b200 import _build
+    path = _build.build()
+    L = ctypes.CDLL(path)
+    L.wlq_packed_bytes.restype = ctypes.c_size_t
+    L.wlq_packed_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int]
+    L.wlq_linear_workspace.restype = ctypes.c_size_t
+    L.wlq_linear_workspace.argtypes = [ctypes.c_int64] * 3 + [ctypes.c_int] * 3
+    L.wlq_version.restype = ctypes.c_char_p
+    L.wlq_last_error.restype = ctypes.c_char_p
+    return L
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(wlq_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version(lib):
+    assert lib.wlq_version().decode().count(".") == 2
+
+
+def test_packed_bytes(lib):
+    # int8: 8192 B per 128x64 tile + 4 B per padded row
+    assert lib.wlq_packed_bytes(4096, 4096, 8, 0) == 32 * 64 * 8192 + 4096 * 4
+    assert lib.wlq_packed_bytes(4096, 4096, 4, 64) == 32 * 64 * (4096 + 256) + 4096 * 4
+    assert lib.wlq_packed_bytes(4096, 4096, 4, 16) == 32 * 64 * (4096 + 1024) + 4096 * 4
+    # ragged: N and K are padded to the tile
+    assert lib.wlq_packed_bytes(130, 72, 8, 0) == 2 * 2 * 8192 + 256 * 4
+    # unsupported recipes / shapes
+    assert lib.wlq_packed_bytes(64, 64, 4, 0) == 0
+    assert lib.wlq_packed_bytes(64, 60, 8, 0) == 0
+    assert lib.wlq_packed_bytes(64, 72, 4, 64) == 0
+
+
+def test_packed_bytes_match_the_pages_weight_totals(lib):
+    """'Joy-face_change_optimized', quantization results table: 15.2 GiB
+    (int8 per channel), 8.1 GiB (int4 gs64), 11.4 GiB (attention int8 + MLP
+    int4 gs16).  The block Linears (80 = 40 blocks x 2 streams, 99% of the
+    parameters) packed in this library's layout must come in just under each
+    total, the rest being the remaining 1% of the model; fp32 group scales
+    would overshoot the int4 figures, which is why group scales are packed as
+    16-bit values."""
+    g = load_golden()
+    n_blocks = int(g["blocks"] * g["streams"])
+    GiB = 2.0 ** 30
+    attn = [(4096, 4096)] * 4
+    mlp = [(16384, 4096), (4096, 16384)]
+
+    def total(recipe_attn, recipe_mlp):
+        b = sum(lib.wlq_packed_bytes(N, K, *recipe_attn) for N, K in attn)
+        b += sum(lib.wlq_packed_bytes(N, K, *recipe_mlp) for N, K in mlp)
+        return n_blocks * b / GiB
+
+    cases = [
+        (total((8, 0), (8, 0)), g["bytes_int8_per_channel_GiB"]),
+        (total((4, 64), (4, 64)), g["bytes_int4_gs64_GiB"]),
+        (total((8, 0), (4, 16)), g["bytes_attn_int8_mlp_int4_gs16_GiB"]),
+    ]
+    for ours, page in cases:
+        assert page - 0.3 < ours < page, (ours, page)
+    # with 4-byte group scales the int4 totals would exceed what the page prints
+    fp32_scales_gs64 = n_blocks * sum(N * K // 2 + N * K // 64 * 4 for N, K in attn + mlp) / GiB
+    assert fp32_scales_gs64 > g["bytes_int4_gs64_GiB"]
+
+
+def test_workspace_sizes(lib):
+    assert lib.wlq_linear_workspace(0, 4096, 4096, 8, 0, 0) == 0
+    # int8 at large M needs no workspace
+    assert lib.wlq_linear_workspace(4096, 4096, 4096, 8, 0, 0) == 0
+    # small M splits K: partial sums + counters
+    assert lib.wlq_linear_workspace(16, 4096, 4096, 8, 0, 0) > 0
+    # int4 stages an fp16 copy of x (+ row scales)
+    assert lib.wlq_linear_workspace(4096, 4096, 4096, 4, 64, 0) >= 4096 * 4096 * 2 + 4096 * 4
+    # low rank adds T (hi/lo) and the transposed L2
+    assert (lib.wlq_linear_workspace(4096, 4096, 4096, 4, 64, 32)
+            > lib.wlq_linear_workspace(4096, 4096, 4096, 4, 64, 0))
+    assert lib.wlq_linear_workspace(16, 64, 64, 4, 64, 8) == 0  # bad rank
+
+
+def test_argument_errors_before_any_device_access(lib):
+    vp = ctypes.c_void_p
+    lib.wlq_quantize.argtypes = [vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int, vp, vp, vp]
+    lib.wlq_linear.argtypes = [vp, ctypes.c_int64, vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                               vp, vp, vp, ctypes.c_int, vp, ctypes.c_int, vp, ctypes.c_size_t, vp]
+    assert lib.wlq_quantize(None, 4, 64, 5, 0, None, None, None) == 4          # bits
+    assert lib.wlq_quantize(None, 4, 64, 4, 48, None, None, None) == 4         # group
+    assert lib.wlq_quantize(None, 4, 60, 8, 0, None, None, None) == 2          # K % 8
+    assert lib.wlq_quantize(None, 4, 64, 8, 0, None, None, None) == 1          # null
+    assert lib.wlq_quantize(None, 0, 64, 8, 0, None, None, None) == 0          # N == 0: no-op
+    assert lib.wlq_quantize(vp(16), 4, 64, 8, 0, vp(17), vp(16), None) == 3    # alignment
+    assert b"16-byte" in lib.wlq_last_error()
+    # M == 0 is a no-op
+    assert lib.wlq_linear(None, 0, None, 64, 64, 8, 0, None, None, None, 0, None, 0, None, 0, None) == 0
+    assert lib.wlq_linear(None, 4, None, 64, 64, 4, 0, None, None, None, 0, None, 0, None, 0, None) == 4
+    assert lib.wlq_linear(None, 4, None, 64, 64, 8, 0, None, None, None, 8, None, 0, None, 0, None) == 2
+    assert lib.wlq_linear(None, 4, None, 64, 64, 8, 0, None, None, None, 16, None, 0, None, 0, None) == 1
+    assert lib.wlq_linear(None, 4, None, 64, 64, 8, 0, None, None, None, 0, None, 7, None, 0, None) == 1
+    # misaligned x is rejected before any device access
+    assert lib.wlq_linear(vp(18), 4, vp(32), 64, 64, 8, 0, None, None, None, 0, vp(64), 0, None, 0, None) == 3

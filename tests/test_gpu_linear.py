@@ -1,0 +1,166 @@
+"""GPU weight-only quantized Linear against the oracle.
+
+Bar ("Joy-face_change_optimized" files table: weight-only Linear; "Nunchaku
+Lite" 16-bit low-rank correction): with identical codes,
+max|y - y_ref| <= 1e-2 * rms(y_ref) in the fp32-output mode; the bf16-output
+mode equals bf16(fp32-output y) bit for bit; results are bitwise
+reproducible.  Small cases span several 128 x BN tiles with ragged tails in
+N, K and M; the five workloads run at full size in the launch configuration
+the benchmark uses and are checked on sampled rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import wlq_inputs as wi
+from tests.gpu_helpers import TOL, dev_bf16, dev_f32, linear_case, rel_err, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+RECIPES = [(8, 0), (4, 64), (4, 16)]
+
+
+def wlq():
+    import weight_only_quantized_rtn_b200 as m
+    return m
+
+
+def small_case(seed, M, N, K, bits, group, bias=True, r=0, outliers=0.02):
+    x = wi.activations(seed, 1, M, K)
+    W = wi.weight(seed, 2, N, K, outlier_frac=outliers)
+    b = wi.bias(seed, 3, N) if bias else None
+    L1 = L2 = None
+    if r:
+        L1 = wi.normal_bf16(wi.rng(seed, 4), (K, r), 0.05)
+        L2 = wi.normal_bf16(wi.rng(seed, 5), (r, N), 0.05)
+    return x, W, b, L1, L2
+
+
+@pytest.mark.parametrize("bits,group", RECIPES)
+@pytest.mark.parametrize("M", [1, 16, 17, 40, 64, 100, 128, 200, 300, 520])
+def test_parity_small_ragged(bits, group, M):
+    N, K = 300, 448  # 3 n-tiles (last one ragged), 7 K blocks
+    x, W, b, _, _ = small_case(100 + M, M, N, K, bits, group)
+    err, _, _ = linear_case(x, W, bits, group, b)
+    assert err <= TOL, err
+
+
+@pytest.mark.parametrize("bits,group", RECIPES)
+@pytest.mark.parametrize("N,K", [(1, 64), (129, 64), (64, 1088), (513, 2112)])
+def test_parity_shapes(bits, group, N, K):
+    M = 37
+    x, W, b, _, _ = small_case(7 * N + K, M, N, K, bits, group, bias=(N % 2 == 1))
+    err, _, _ = linear_case(x, W, bits, group, b)
+    assert err <= TOL, err
+
+
+def test_parity_k_not_multiple_of_64():
+    # int8 per channel only needs K % 8 == 0: the last K block is partial
+    for K in (8, 72, 200):
+        x, W, b, _, _ = small_case(K, 50, 140, K, 8, 0)
+        err, _, _ = linear_case(x, W, 8, 0, b)
+        assert err <= TOL, (K, err)
+
+
+@pytest.mark.parametrize("bits,group", RECIPES)
+@pytest.mark.parametrize("r", [16, 32, 64])
+@pytest.mark.parametrize("M", [16, 130])
+def test_parity_low_rank(bits, group, r, M):
+    x, W, b, L1, L2 = small_case(300 + r + M, M, 260, 512, bits, group, r=r)
+    err, _, _ = linear_case(x, W, bits, group, b, L1, L2)
+    assert err <= TOL, err
+
+
+@pytest.mark.parametrize("bits,group", RECIPES)
+def test_bf16_output_is_rounded_fp32_output(bits, group):
+    m = wlq()
+    for M in (16, 300):
+        x, W, b, _, _ = small_case(5, M, 384, 512, bits, group)
+        codes, scales = m.quantize(dev_f32(W), bits, group)
+        packed = m.pack(codes, scales, bits, group)
+        xd, bd = dev_bf16(x), dev_bf16(b)
+        y32 = m.linear(xd, packed, 384, 512, bits, group, bd, out_dtype=torch.float32)
+        y16 = m.linear(xd, packed, 384, 512, bits, group, bd, out_dtype=torch.bfloat16)
+        assert torch.equal(y16, y32.to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("bits,group", RECIPES)
+def test_bitwise_reproducible(bits, group):
+    m = wlq()
+    for M in (16, 48, 1000):  # split-K and persistent paths
+        x, W, b, L1, L2 = small_case(6, M, 1024, 1024, bits, group, r=32)
+        codes, scales = m.quantize(dev_f32(W), bits, group)
+        packed = m.pack(codes, scales, bits, group)
+        args = (dev_bf16(x), packed, 1024, 1024, bits, group, dev_bf16(b), dev_bf16(L1), dev_bf16(L2))
+        ys = [m.linear(*args, out_dtype=torch.float32) for _ in range(3)]
+        assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
+
+
+def test_empty_and_errors():
+    m = wlq()
+    W = wi.weight(8, 1, 64, 128)
+    codes, scales = m.quantize(dev_f32(W), 8, 0)
+    packed = m.pack(codes, scales, 8, 0)
+    x = torch.zeros((0, 128), dtype=torch.bfloat16, device="cuda")
+    assert m.linear(x, packed, 64, 128, 8, 0).shape == (0, 64)
+    x = dev_bf16(wi.activations(8, 2, 16, 128))
+    y = torch.empty((16, 64), dtype=torch.float32, device="cuda")
+    need = m.workspace_bytes(16, 64, 128, 8, 0)
+    if need:
+        small = torch.zeros(need - 16, dtype=torch.uint8, device="cuda")
+        with pytest.raises(m.WlqError) as e:
+            m.linear_into(y, x, packed, 64, 128, 8, 0, workspace=small)
+        assert e.value.status == m.ERR_WORKSPACE
+    with pytest.raises(m.WlqError) as e:
+        m.linear_into(y, x, packed, 64, 128, 4, 64)
+    assert e.value.status in (m.ERR_WORKSPACE, m.ERR_UNSUPPORTED, m.ERR_SHAPE)
+    m.check_status()
+
+
+# ------------------------------------------------------------ full workloads
+def _check_full(x, W, bits, group, b, L1=None, L2=None):
+    M = x.shape[0]
+    rows = sample_rows(M, 12, seed=M)
+    err, _, _ = linear_case(x, W, bits, group, b, L1, L2, rows=rows)
+    assert err <= TOL, err
+    return err
+
+
+def test_full_tiny_w8():
+    d = wi.tiny_w8()
+    err, _, _ = linear_case(d["x"], d["W"], 8, 0, d["b"])
+    assert err <= TOL, err
+
+
+@pytest.mark.parametrize("M", [16, 256, 4096])
+def test_full_attention_w8(M):
+    d = wi.attn_w8(M)
+    _check_full(d["x"], d["W"], 8, 0, d["b"])
+
+
+@pytest.mark.parametrize("which", ["up", "down"])
+@pytest.mark.parametrize("M", [16, 1560, 6240])
+def test_full_mlp_w4_gs64(which, M):
+    d = wi.mlp_w4(M, which)
+    _check_full(d["x"], d["W"], 4, 64, d["b"])
+
+
+_MIXED = {}
+
+
+@pytest.mark.parametrize("name", [n for n, *_ in wi.MIXED_LAYERS])
+def test_full_mixed_block(name):
+    if not _MIXED:
+        _MIXED.update(wi.mixed_block(4096))
+    blk = _MIXED
+    layer = blk["layers"][name]
+    K = layer["W"].shape[1]
+    x = blk["x"] if K == wi.HIDDEN else wi.activations(3, 99, 4096, K)
+    _check_full(x, layer["W"], layer["bits"], layer["group"], layer["b"])
+
+
+@pytest.mark.parametrize("M", [256, 4096])
+def test_full_svdq_low_rank(M):
+    d = wi.svdq_w4_lr(M)
+    _check_full(d["x"], d["W"], 4, 64, d["b"], d["L1"], d["L2"])

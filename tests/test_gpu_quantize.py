@@ -1,0 +1,96 @@
+"""GPU quantization and packing against the oracle: codes and fp32 scales
+bit-exact on the weights of all five workloads and on edge cases; pack/unpack
+round trip; device-side error reporting."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import wlq_inputs as wi
+from tests.gpu_helpers import assert_codes_equal, dev_f32, quantize_both
+
+pytestmark = pytest.mark.gpu
+
+
+def wlq():
+    import weight_only_quantized_rtn_b200 as m
+    return m
+
+
+def _workload_weights():
+    yield "tiny", wi.tiny_w8()["W"], 8, 0
+    yield "attn", wi.attn_w8(1)["W"], 8, 0
+    yield "mlp_up", wi.mlp_w4(1, "up")["W"], 4, 64
+    yield "mlp_down", wi.mlp_w4(1, "down")["W"], 4, 64
+    blk = wi.mixed_block(1)
+    for name, layer in blk["layers"].items():
+        yield "mixed_" + name, layer["W"], layer["bits"], layer["group"]
+    yield "svdq_residual", wi.svdq_w4_lr(1)["W"], 4, 64
+
+
+@pytest.mark.parametrize("case", list(range(11)))
+def test_quantize_bit_exact_on_workload_weights(case):
+    name, W, bits, group = list(_workload_weights())[case]
+    cg, sg, co, so = quantize_both(W, bits, group)
+    assert_codes_equal(cg, sg, co, so)
+
+
+@pytest.mark.parametrize("bits,group", [(8, 0), (4, 64), (4, 16), (8, 64), (4, 0), (8, 16), (4, 32), (4, 128)])
+def test_quantize_edge_cases(bits, group):
+    g = np.random.default_rng(99)
+    K = 384
+    W = (g.standard_normal((37, K)) * 0.02).astype(np.float32)
+    W[0] = 0.0                                            # all-zero row
+    W[1] = g.integers(-9, 10, K).astype(np.float32) * 0.5  # many exact halves (ties)
+    W[1, ::16] = 7.0 if bits == 4 else 127.0               # absmax sets s = 1
+    W[2] *= 1e-38                                         # tiny / subnormal range
+    W[3] *= 1e36                                          # huge
+    W[4, 5] = -50.0                                       # a single outlier, negative
+    W[5, :] = 3.0                                         # constant row
+    cg, sg, co, so = quantize_both(W, bits, group)
+    assert_codes_equal(cg, sg, co, so)
+
+
+def test_quantize_ragged_and_single_row():
+    for N, K in [(1, 8), (3, 24), (129, 1000), (257, 4104)]:
+        W = wi.weight(21, N, N, K)
+        for bits, group in [(8, 0), (4, 0)]:
+            cg, sg, co, so = quantize_both(W, bits, group)
+            assert_codes_equal(cg, sg, co, so)
+
+
+def test_nonfinite_weight_is_reported():
+    m = wlq()
+    W = wi.weight(22, 1, 64, 128)
+    W[7, 3] = np.nan
+    m.quantize(dev_f32(W), 8, 0)
+    assert m.get_status() == m.ERR_NONFINITE
+    assert m.get_status() == m.OK  # the word is cleared once read
+    W[7, 3] = np.inf
+    m.quantize(dev_f32(W), 4, 16)
+    assert m.get_status() == m.ERR_NONFINITE
+    W[7, 3] = 0.0
+    m.quantize(dev_f32(W), 4, 16)
+    assert m.get_status() == m.OK
+
+
+@pytest.mark.parametrize("bits,group", [(8, 0), (4, 64), (4, 16)])
+@pytest.mark.parametrize("N,K", [(128, 64), (300, 320), (1, 64), (257, 4160)])
+def test_pack_unpack_roundtrip(bits, group, N, K):
+    m = wlq()
+    W = wi.weight(23, N + K, N, K, outlier_frac=0.02)
+    codes, scales = m.quantize(dev_f32(W), bits, group)
+    packed = m.pack(codes, scales, bits, group)
+    assert packed.numel() == m.packed_bytes(N, K, bits, group)
+    back = m.unpack(packed, N, K, bits, group)
+    assert torch.equal(back, codes)
+
+
+def test_wait_probe_times_out_and_device_stays_usable():
+    m = wlq()
+    m.probe_wait_timeout(2_000_000)  # 2 ms on a barrier nothing arrives at
+    assert m.get_status() == m.ERR_TIMEOUT
+    assert m.get_status() == m.OK
+    W = wi.weight(24, 1, 16, 64)
+    cg, sg, co, so = quantize_both(W, 8, 0)
+    assert_codes_equal(cg, sg, co, so)

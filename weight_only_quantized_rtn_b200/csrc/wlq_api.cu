@@ -1,0 +1,443 @@
+// wlq_api.cu -- the C ABI (include/wlq.h): argument checks, launch plans,
+// TMA descriptors and kernel launches.  Single translation unit: every kernel
+// header is included here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/wlq.h"
+#include "gemm.cuh"
+#include "pack.cuh"
+#include "prep.cuh"
+#include "ptx.cuh"
+#include "quantize.cuh"
+
+namespace {
+
+thread_local char g_msg[512] = "no error";
+
+wlq_status fail(wlq_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+wlq_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(WLQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int fmt_of(int bits, int group) {
+    if (bits == 8 && group == 0) return wlq::FMT_W8;
+    if (bits == 4 && group == 64) return wlq::FMT_W4G64;
+    if (bits == 4 && group == 16) return wlq::FMT_W4G16;
+    return -1;
+}
+
+// ----------------------------------------------------------------- device
+struct DeviceInfo {
+    int checked = 0;  // 0 unknown, 1 supported, -1 not
+    int sms = 0;
+    bool smem_set[3] = {false, false, false};
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+wlq_status current_device(int* dev_out, DeviceInfo** info_out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(WLQ_ERR_UNSUPPORTED, "device index %d", dev);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (d.checked == 0) {
+        int major = 0, minor = 0, sms = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute");
+        d.checked = (major == 10 && minor == 0) ? 1 : -1;
+        d.sms = sms;
+    }
+    if (d.checked < 0) return fail(WLQ_ERR_UNSUPPORTED, "this library is built for sm_100 (B200) only");
+    *dev_out = dev;
+    *info_out = &d;
+    return WLQ_OK;
+}
+
+// ------------------------------------------------------------- TMA encode
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D tensor of 16-bit elements [rows, cols] (cols contiguous), tiles of
+// box_rows x 64 with a 128-byte swizzle; out-of-range elements read as zero.
+wlq_status make_map_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                       uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(WLQ_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(WLQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return WLQ_OK;
+}
+
+// ------------------------------------------------------------------ plan
+constexpr uint64_t kDefaultTimeoutNs = 2ull * 1000 * 1000 * 1000;
+constexpr size_t kSmemLimit = 232448;  // 227 KB opt-in per block on sm_100
+
+struct Plan {
+    int fmt = -1;
+    int M = 0, N = 0, K = 0, r = 0;
+    int NT = 0, KT = 0, MT = 0, S = 1, kbps = 0, BN = 0, total_tiles = 0, grid = 0;
+    int stages = 0, lr_kb = 0, acc_bufs = 1;
+    uint32_t tmem_cols = 0, lr_col0 = 0, wtile = 0, wstage = 0, xstage = 0;
+    size_t smem = 0;
+    size_t off_x16 = 0, off_xs = 0, off_thl = 0, off_l2t = 0, off_part = 0, off_cnt = 0, ws = 0;
+};
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms) {
+    p.fmt = fmt;
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.r = r;
+    p.NT = static_cast<int>(cdiv(N, 128));
+    p.KT = static_cast<int>(cdiv(K, 64));
+    p.lr_kb = r ? static_cast<int>(cdiv(2 * r, 64)) : 0;
+    // token tile: the MMA N dimension
+    if (M <= 16) p.BN = 16;
+    else if (M <= 32) p.BN = 32;
+    else if (M <= 64) p.BN = 64;
+    else if (M <= 128 || r) p.BN = 128;
+    else p.BN = 256;
+    p.MT = static_cast<int>(cdiv(M, p.BN));
+    const int tiles_nm = p.NT * p.MT;
+    // split K so that small problems still cover the SMs
+    int S = 1;
+    if (tiles_nm < sms) S = std::max(1, sms / tiles_nm);
+    S = std::min(S, std::max(1, p.KT / 2));
+    S = std::min(S, 16);
+    p.kbps = static_cast<int>(cdiv(p.KT, S));
+    p.S = static_cast<int>(cdiv(p.KT, p.kbps));
+    p.total_tiles = tiles_nm * p.S;
+    p.grid = std::min(p.total_tiles, sms);
+    // TMEM: A ring + accumulator(s), double-buffered when they fit
+    const uint32_t acc_cols = static_cast<uint32_t>(p.BN) * (r ? 2u : 1u);
+    p.acc_bufs = (wlq::ACC_COL0 + 2 * acc_cols <= 512) ? 2 : 1;
+    if (wlq::ACC_COL0 + acc_cols > 512) return false;
+    const uint32_t need = wlq::ACC_COL0 + p.acc_bufs * acc_cols;
+    p.tmem_cols = 32;
+    while (p.tmem_cols < need) p.tmem_cols <<= 1;
+    p.lr_col0 = wlq::ACC_COL0 + p.acc_bufs * static_cast<uint32_t>(p.BN);
+    // shared memory ring
+    p.wtile = wlq::tile_bytes(fmt);
+    p.wstage = (p.wtile + 1023u) & ~1023u;
+    p.xstage = static_cast<uint32_t>(p.BN) * 128u;
+    const size_t lr_bytes = r ? (wlq::LR_TILE_A_BYTES + p.xstage) : 0;
+    const size_t fixed = 1024 /* alignment */ + 512 /* barriers */ + lr_bytes;
+    const size_t per_stage = p.xstage + p.wstage;
+    p.stages = static_cast<int>(std::min<size_t>(16, (kSmemLimit - fixed) / per_stage));
+    if (p.stages < 2) return false;
+    p.smem = fixed + p.stages * per_stage;
+    // workspace
+    size_t off = 0;
+    if (fmt != wlq::FMT_W8) {
+        p.off_x16 = off; off = align256(off + static_cast<size_t>(M) * K * 2);
+        p.off_xs = off;  off = align256(off + static_cast<size_t>(M) * 4);
+    }
+    if (r) {
+        p.off_thl = off; off = align256(off + static_cast<size_t>(M) * p.lr_kb * 64 * 2);
+        p.off_l2t = off; off = align256(off + static_cast<size_t>(p.NT) * 128 * p.lr_kb * 64 * 2);
+    }
+    if (p.S > 1) {
+        p.off_part = off; off = align256(off + static_cast<size_t>(p.S) * p.MT * p.NT * p.BN * 128 * 4);
+        p.off_cnt = off;  off = align256(off + static_cast<size_t>(p.MT) * p.NT * 4);
+    }
+    p.ws = off;
+    return true;
+}
+
+wlq_status check_shape(int64_t N, int64_t K, int bits, int group) {
+    if (N < 0 || K <= 0) return fail(WLQ_ERR_INVALID_ARG, "N must be >= 0 and K > 0");
+    if (N > (int64_t(1) << 30) || K > (int64_t(1) << 30)) return fail(WLQ_ERR_SHAPE, "N or K too large");
+    if (K % 8) return fail(WLQ_ERR_SHAPE, "K %% 8 != 0 (K = %lld)", static_cast<long long>(K));
+    if (group && K % group) return fail(WLQ_ERR_SHAPE, "K %% group != 0");
+    (void)bits;
+    return WLQ_OK;
+}
+
+template <int FMT>
+wlq_status launch_gemm(const Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, const CUtensorMap& tl,
+                       const wlq::GemmArgs& a, DeviceInfo* d, cudaStream_t st) {
+    if (!d->smem_set[FMT]) {
+        cudaError_t e = cudaFuncSetAttribute(wlq::gemm_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kSmemLimit));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        d->smem_set[FMT] = true;
+    }
+    wlq::gemm_kernel<FMT><<<p.grid, wlq::GEMM_THREADS, p.smem, st>>>(tx, tt, tl, a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+    return WLQ_OK;
+}
+
+int grid_for(int64_t work, int per_block, int sms) {
+    const int64_t b = cdiv(std::max<int64_t>(work, 1), per_block);
+    return static_cast<int>(std::min<int64_t>(b, int64_t(sms) * 32));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* wlq_version(void) { return "0.1.0"; }
+
+const char* wlq_last_error(void) { return g_msg; }
+
+wlq_status wlq_quantize(const float* W, int64_t N, int64_t K, int bits, int group, int8_t* codes,
+                        float* scales, void* stream) {
+    if (bits != 8 && bits != 4) return fail(WLQ_ERR_UNSUPPORTED, "bits must be 8 or 4");
+    if (!(group == 0 || group == 16 || group == 32 || group == 64 || group == 128))
+        return fail(WLQ_ERR_UNSUPPORTED, "group must be 0, 16, 32, 64 or 128");
+    wlq_status st = check_shape(N, K, bits, group);
+    if (st != WLQ_OK) return st;
+    if (N == 0) return WLQ_OK;
+    if (!W || !codes || !scales) return fail(WLQ_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(W) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+        return fail(WLQ_ERR_ALIGN, "W and codes must be 16-byte aligned, scales 4-byte aligned");
+    int dev;
+    DeviceInfo* d;
+    if ((st = current_device(&dev, &d)) != WLQ_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int qmax = (1 << (bits - 1)) - 1;
+    if (group == 0) {
+        const int grid = static_cast<int>(std::min<int64_t>(N, int64_t(d->sms) * 8));
+        wlq::quantize_rows_kernel<256><<<grid, 256, 0, s>>>(W, N, K, qmax, codes, scales);
+    } else {
+        const int64_t total4 = N * K / 4;
+        wlq::quantize_groups_kernel<<<grid_for(total4, 256, d->sms), 256, 0, s>>>(W, total4, group / 4, qmax,
+                                                                                   codes, scales);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+    return WLQ_OK;
+}
+
+size_t wlq_packed_bytes(int64_t N, int64_t K, int bits, int group) {
+    const int fmt = fmt_of(bits, group);
+    if (fmt < 0 || N < 0 || K <= 0 || K % 8 || (group && K % group)) return 0;
+    const int64_t NT = cdiv(N, 128), KT = cdiv(K, 64);
+    return static_cast<size_t>(NT * KT) * wlq::tile_bytes(fmt) + static_cast<size_t>(NT) * 128 * 4;
+}
+
+wlq_status wlq_pack(const int8_t* codes, const float* scales, int64_t N, int64_t K, int bits, int group,
+                    void* packed, void* stream) {
+    const int fmt = fmt_of(bits, group);
+    if (fmt < 0) return fail(WLQ_ERR_UNSUPPORTED, "pack supports (8,0), (4,64) and (4,16)");
+    wlq_status st = check_shape(N, K, bits, group);
+    if (st != WLQ_OK) return st;
+    if (N == 0) return WLQ_OK;
+    if (!codes || !scales || !packed) return fail(WLQ_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(packed)) return fail(WLQ_ERR_ALIGN, "packed must be 16-byte aligned");
+    int dev;
+    DeviceInfo* d;
+    if ((st = current_device(&dev, &d)) != WLQ_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t NT = cdiv(N, 128), KT = cdiv(K, 64);
+    const int64_t G = group ? K / group : 1;
+    uint8_t* base = static_cast<uint8_t*>(packed);
+    float* rowf = reinterpret_cast<float*>(base + NT * KT * wlq::tile_bytes(fmt));
+    wlq::pack_rowfactor_kernel<<<grid_for(NT * 128 * 32, 256, d->sms), 256, 0, s>>>(scales, N, G, fmt, NT * 128, rowf);
+    wlq::pack_tiles_kernel<<<static_cast<unsigned>(NT * KT), 128, 0, s>>>(codes, scales, N, K, G, fmt,
+                                                                          static_cast<int>(KT), rowf, base);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "pack launch");
+    return WLQ_OK;
+}
+
+wlq_status wlq_unpack(const void* packed, int64_t N, int64_t K, int bits, int group, int8_t* codes,
+                      void* stream) {
+    const int fmt = fmt_of(bits, group);
+    if (fmt < 0) return fail(WLQ_ERR_UNSUPPORTED, "unpack supports (8,0), (4,64) and (4,16)");
+    wlq_status st = check_shape(N, K, bits, group);
+    if (st != WLQ_OK) return st;
+    if (N == 0) return WLQ_OK;
+    if (!codes || !packed) return fail(WLQ_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(packed)) return fail(WLQ_ERR_ALIGN, "packed must be 16-byte aligned");
+    int dev;
+    DeviceInfo* d;
+    if ((st = current_device(&dev, &d)) != WLQ_OK) return st;
+    const int64_t NT = cdiv(N, 128), KT = cdiv(K, 64);
+    wlq::unpack_tiles_kernel<<<static_cast<unsigned>(NT * KT), 128, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint8_t*>(packed), N, K, fmt, static_cast<int>(KT), codes);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "unpack launch");
+    return WLQ_OK;
+}
+
+size_t wlq_linear_workspace(int64_t M, int64_t N, int64_t K, int bits, int group, int r) {
+    const int fmt = fmt_of(bits, group);
+    if (fmt < 0 || M < 0 || N < 0 || K <= 0 || !(r == 0 || r == 16 || r == 32 || r == 64)) return 0;
+    if (M == 0 || N == 0) return 0;
+    int sms = 148;
+    int dev;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) sms = v;
+    } else {
+        cudaGetLastError();
+    }
+    Plan p;
+    if (!make_plan(p, M, N, K, fmt, r, sms)) return 0;
+    return p.ws;
+}
+
+wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, int64_t K, int bits, int group,
+                      const void* bias, const void* L1, const void* L2, int r, void* y, int y_dtype,
+                      void* workspace, size_t ws_bytes, void* stream) {
+    const int fmt = fmt_of(bits, group);
+    if (fmt < 0) return fail(WLQ_ERR_UNSUPPORTED, "linear supports (8,0), (4,64) and (4,16)");
+    wlq_status st = check_shape(N, K, bits, group);
+    if (st != WLQ_OK) return st;
+    if (M < 0) return fail(WLQ_ERR_INVALID_ARG, "M < 0");
+    if (M > (int64_t(1) << 30)) return fail(WLQ_ERR_SHAPE, "M too large");
+    if (!(r == 0 || r == 16 || r == 32 || r == 64)) return fail(WLQ_ERR_SHAPE, "r must be 0, 16, 32 or 64");
+    if (r && (!L1 || !L2)) return fail(WLQ_ERR_INVALID_ARG, "r > 0 needs L1 and L2");
+    if (y_dtype != WLQ_OUT_BF16 && y_dtype != WLQ_OUT_F32) return fail(WLQ_ERR_INVALID_ARG, "bad y_dtype");
+    if (M == 0 || N == 0) return WLQ_OK;
+    if (!x || !packed || !y) return fail(WLQ_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(x) || !aligned16(packed)) return fail(WLQ_ERR_ALIGN, "x and packed must be 16-byte aligned");
+    if ((bias && (reinterpret_cast<uintptr_t>(bias) & 1u)) || (L1 && (reinterpret_cast<uintptr_t>(L1) & 1u)) ||
+        (L2 && (reinterpret_cast<uintptr_t>(L2) & 1u)) || (reinterpret_cast<uintptr_t>(y) & 3u))
+        return fail(WLQ_ERR_ALIGN, "bias/L1/L2 must be 2-byte aligned, y 4-byte aligned");
+    int dev;
+    DeviceInfo* d;
+    if ((st = current_device(&dev, &d)) != WLQ_OK) return st;
+    Plan p;
+    if (!make_plan(p, M, N, K, fmt, r, d->sms)) return fail(WLQ_ERR_UNSUPPORTED, "no launch plan for this shape");
+    if (p.ws > 0 && (!workspace || ws_bytes < p.ws))
+        return fail(WLQ_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", p.ws, ws_bytes);
+    if (workspace && !aligned16(workspace)) return fail(WLQ_ERR_ALIGN, "workspace must be 16-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const int64_t NT = p.NT, KT = p.KT;
+
+    // --- operand preparation
+    const void* xin = x;
+    float* xs = nullptr;
+    if (fmt != wlq::FMT_W8) {
+        __half* x16 = reinterpret_cast<__half*>(ws + p.off_x16);
+        xs = reinterpret_cast<float*>(ws + p.off_xs);
+        wlq::prep_x16_kernel<<<grid_for(M * 32, 256, d->sms), 256, 0, s>>>(static_cast<const uint16_t*>(x), p.M,
+                                                                          p.K, x16, xs);
+        xin = x16;
+    }
+    uint16_t* thl = nullptr;
+    uint16_t* l2t = nullptr;
+    const int W = p.lr_kb * 64;
+    if (r) {
+        thl = reinterpret_cast<uint16_t*>(ws + p.off_thl);
+        l2t = reinterpret_cast<uint16_t*>(ws + p.off_l2t);
+        wlq::prep_lr_t_kernel<<<static_cast<unsigned>(cdiv(M, wlq::LR_ROWS)), 128, 0, s>>>(
+            static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(L1), p.M, p.K, r, W, thl);
+        wlq::prep_lr_l2t_kernel<<<grid_for(NT * 128 * W, 256, d->sms), 256, 0, s>>>(
+            static_cast<const uint16_t*>(L2), p.N, static_cast<int>(NT * 128), r, W, l2t);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "prep launch");
+
+    // --- descriptors
+    CUtensorMap tx, tt, tl;
+    std::memset(&tt, 0, sizeof tt);
+    std::memset(&tl, 0, sizeof tl);
+    if ((st = make_map_2d(&tx, xin, M, K, p.BN)) != WLQ_OK) return st;
+    if (r) {
+        if ((st = make_map_2d(&tt, thl, M, W, p.BN)) != WLQ_OK) return st;
+        if ((st = make_map_2d(&tl, l2t, NT * 128, W, 128)) != WLQ_OK) return st;
+    }
+    wlq::GemmArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.packed = static_cast<const uint8_t*>(packed);
+    a.rowf = reinterpret_cast<const float*>(a.packed + NT * KT * wlq::tile_bytes(fmt));
+    a.xs = xs;
+    a.bias = static_cast<const uint16_t*>(bias);
+    a.y = y;
+    a.partials = p.S > 1 ? reinterpret_cast<float*>(ws + p.off_part) : nullptr;
+    a.counters = p.S > 1 ? reinterpret_cast<unsigned*>(ws + p.off_cnt) : nullptr;
+    a.M = p.M; a.N = p.N; a.K = p.K;
+    a.NT = p.NT; a.KT = p.KT; a.MT = p.MT; a.S = p.S; a.kbps = p.kbps; a.BN = p.BN;
+    a.stages = p.stages; a.lr = r ? 1 : 0; a.lr_kb = p.lr_kb; a.acc_bufs = p.acc_bufs;
+    a.y_f32 = (y_dtype == WLQ_OUT_F32) ? 1 : 0;
+    a.total_tiles = p.total_tiles;
+    a.tmem_cols = p.tmem_cols; a.lr_col0 = p.lr_col0;
+    a.wtile_bytes = p.wtile; a.wstage_bytes = p.wstage; a.xstage_bytes = p.xstage;
+    a.timeout_ns = kDefaultTimeoutNs;
+    switch (fmt) {
+        case wlq::FMT_W8: return launch_gemm<wlq::FMT_W8>(p, tx, tt, tl, a, d, s);
+        case wlq::FMT_W4G64: return launch_gemm<wlq::FMT_W4G64>(p, tx, tt, tl, a, d, s);
+        default: return launch_gemm<wlq::FMT_W4G16>(p, tx, tt, tl, a, d, s);
+    }
+}
+
+wlq_status wlq_get_status(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned word = 0;
+    if ((e = cudaMemcpyFromSymbol(&word, wlq::g_error_word, sizeof word)) != cudaSuccess)
+        return cuda_fail(e, "read error word");
+    if (word) {
+        const unsigned zero = 0;
+        if ((e = cudaMemcpyToSymbol(wlq::g_error_word, &zero, sizeof zero)) != cudaSuccess)
+            return cuda_fail(e, "clear error word");
+    }
+    if (word & wlq::ERRBIT_TIMEOUT) return fail(WLQ_ERR_TIMEOUT, "a bounded device wait ran out");
+    if (word & wlq::ERRBIT_NONFINITE) return fail(WLQ_ERR_NONFINITE, "non-finite weight");
+    return WLQ_OK;
+}
+
+wlq_status wlq_probe_wait_timeout(uint64_t timeout_ns, void* stream) {
+    int dev;
+    DeviceInfo* d;
+    wlq_status st = current_device(&dev, &d);
+    if (st != WLQ_OK) return st;
+    const uint64_t cap = 10ull * 1000 * 1000 * 1000;
+    wlq::wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(std::min(timeout_ns, cap));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "probe launch");
+    return WLQ_OK;
+}
+
+}  // extern "C"
