@@ -1,0 +1,364 @@
+"""Benchmark: the weight-only quantized Linear of a DiT attention projection.
+
+Workload (seeded, synthetic): W [4096, 4096] ~ N(0, 0.02) fp32 with 1% of the
+input columns x20, RTN int8 per output channel; x bf16 [M, 4096] ~ N(0, 1)
+for M in {16, 256, 4096}; bias [4096] ~ N(0, 0.01).  One step is one pass of
+the whole path: quantize W, pack it, then the Linear at M = 16, 256 and 4096
+(inputs already in HBM; L2 flushed between steps).  value = total Linear
+FLOPs (2 M N K) of all ranks / the max over ranks of the device time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun every rank runs an independent replica (weak scaling); there
+is no collective on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import wlq_inputs as wi  # noqa: E402
+
+N_OUT, K_IN, BITS, GROUP = 4096, 4096, 8, 0
+MS = (16, 256, 4096)
+METRIC = "quantized-linear TFLOP/s and HBM GB/s vs B200 roofline, M=16..4096"
+WORKLOAD = ("DiT attention projection W8A16: W[4096,4096] fp32 N(0,0.02), 1% input columns x20, "
+            "RTN int8 per output channel; x bf16 [M,4096] N(0,1), M in {16,256,4096}; bias N(0,0.01); "
+            "step = quantize + pack + Linear at the three M")
+PROFILE = os.path.join(ROOT, "profiles", "gemm_w8_attn_m4096.txt")
+
+
+def linear_flops():
+    return sum(2.0 * M * N_OUT * K_IN for M in MS)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "weight_only_quantized_rtn_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the M=4096 GEMM from the committed ncu summary,
+    or None when the kernel sources changed since that capture."""
+    if not os.path.exists(PROFILE):
+        return None
+    vals = {}
+    for line in open(PROFILE):
+        if ":" in line and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        time.sleep(0.25)
+        self.p.terminate()
+        try:
+            self.p.wait(5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        rows = []
+        for line in open(self.f.name):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        loaded = [v for v in sm if v > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def cpu_baseline(n_rows_per_m=(16, 64, 944)):
+    """The oracle as it stands on this host's cores: quantize the whole W, then
+    the Linear for a bounded sample of rows of each M batch."""
+    import oracle
+    d = wi.attn_w8(1)
+    W = d["W"]
+    t0 = time.perf_counter()
+    codes, scales = oracle.quantize(W, BITS, GROUP)
+    flops = 0.0
+    for M, nr in zip(MS, n_rows_per_m):
+        x = wi.attn_w8(M)["x"][:nr]
+        oracle.linear(x, codes, scales, GROUP, d["b"])
+        flops += 2.0 * x.shape[0] * N_OUT * K_IN
+    dt = time.perf_counter() - t0
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": int(os.environ.get("OMP_NUM_THREADS", cores)),
+            "kind": "oracle", "seconds": round(dt, 3),
+            "sample": "quantize all of W + Linear on %s rows of the M=%s batches (fp64 C, OpenMP)"
+                      % ("/".join(map(str, n_rows_per_m)), "/".join(map(str, MS)))}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    d = wi.attn_w8(1)
+    xs = {M: wi.attn_w8(M)["x"][:16] for M in MS}
+    times, flops = [], 0.0
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        codes, scales = oracle.quantize(d["W"], BITS, GROUP)
+        f = 0.0
+        for M in MS:
+            oracle.linear(xs[M], codes, scales, GROUP, d["b"])
+            f += 2.0 * xs[M].shape[0] * N_OUT * K_IN
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+            flops = f
+    ms = 1e3 * sum(times) / len(times)
+    value = flops / (ms * 1e-3) / 1e12
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    sample = "per step: quantize all of W + Linear on 16 rows of each M batch (fp64 C oracle, OpenMP)"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": list(MS), "N": N_OUT, "K": K_IN, "sampled_rows_per_M": 16},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_gpu(args):
+    import torch
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    import weight_only_quantized_rtn_b200 as wlq
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    # ---- inputs, resident in HBM before the timed region
+    base = wi.attn_w8(1)
+    W = torch.from_numpy(base["W"]).to(dev)
+    b = torch.from_numpy(base["b"].view(np.int16)).to(dev).view(torch.bfloat16)
+    xs = {M: torch.from_numpy(wi.attn_w8(M)["x"].view(np.int16)).to(dev).view(torch.bfloat16) for M in MS}
+    codes = torch.empty((N_OUT, K_IN), dtype=torch.int8, device=dev)
+    scales = torch.empty((N_OUT, 1), dtype=torch.float32, device=dev)
+    packed = torch.empty(wlq.packed_bytes(N_OUT, K_IN, BITS, GROUP), dtype=torch.uint8, device=dev)
+    ys = {M: torch.empty((M, N_OUT), dtype=torch.bfloat16, device=dev) for M in MS}
+    wss = {M: wlq.new_workspace(M, N_OUT, K_IN, BITS, GROUP, 0, device=dev) for M in MS}
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    lib, ptr, st = wlq.lib, wlq._ptr, wlq._stream(stream)
+
+    def step(ev=None):
+        wlq._check(lib.wlq_quantize(ptr(W), N_OUT, K_IN, BITS, GROUP, ptr(codes), ptr(scales), st))
+        wlq._check(lib.wlq_pack(ptr(codes), ptr(scales), N_OUT, K_IN, BITS, GROUP, ptr(packed), st))
+        for M in MS:
+            if ev is not None:
+                ev[M][0].record(stream)
+            wlq.linear_into(ys[M], xs[M], packed, N_OUT, K_IN, BITS, GROUP, bias=b, workspace=wss[M],
+                            stream=stream)
+            if ev is not None:
+                ev[M][1].record(stream)
+
+    launches_per_step = 1 + 2 + len(MS)  # quantize, pack (row factors + tiles), one GEMM per M
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    wlq.check_status()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    inner = [{M: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for M in MS}
+             for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()  # evict L2 between steps (outside the timed events)
+        torch.cuda.nvtx.range_push("timed_step")
+        starts[i].record(stream)
+        step(inner[i])
+        ends[i].record(stream)
+        torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    wlq.check_status()
+
+    ms_step = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
+    per_m_ms = {M: sum(ev[M][0].elapsed_time(ev[M][1]) for ev in inner) / args.steps for M in MS}
+    if dist:
+        t = torch.tensor([ms_step] + [per_m_ms[M] for M in MS], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t[0])
+        per_m_ms = {M: float(t[1 + i]) for i, M in enumerate(MS)}
+
+    # ---- per-M kernels in isolation (L2 flushed before every launch)
+    iso = {}
+    for M in MS:
+        evs = []
+        for _ in range(max(5, args.steps)):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            wlq.linear_into(ys[M], xs[M], packed, N_OUT, K_IN, BITS, GROUP, bias=b, workspace=wss[M],
+                            stream=stream)
+            e1.record(stream)
+            evs.append((e0, e1))
+        torch.cuda.synchronize()
+        iso[M] = statistics.median(a.elapsed_time(c) for a, c in evs)
+
+    # ---- end to end through the public API with pinned host buffers
+    W_h = torch.from_numpy(base["W"]).pin_memory()
+    x_h = {M: xs[M].cpu().pin_memory() for M in MS}
+    y_h = {M: torch.empty((M, N_OUT), dtype=torch.bfloat16).pin_memory() for M in MS}
+    h2d = W_h.numel() * 4 + sum(x_h[M].numel() * 2 for M in MS)
+    d2h = sum(y_h[M].numel() * 2 for M in MS)
+    e2e_steps = max(3, min(args.steps, 20))
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    torch.cuda.synchronize()
+    for i in range(e2e_steps):
+        flush.zero_()
+        e_s[i].record(stream)
+        W.copy_(W_h, non_blocking=True)
+        for M in MS:
+            xs[M].copy_(x_h[M], non_blocking=True)
+        step()
+        for M in MS:
+            y_h[M].copy_(ys[M], non_blocking=True)
+        e_e[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(c) for a, c in zip(e_s, e_e)) / e2e_steps
+    if dist:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    wlq.check_status()
+
+    hbm_peak, tc_peak, tc_sust, peak_src = measured_peaks()
+    flops = linear_flops()
+    value = world * flops / (ms_step * 1e-3) / 1e12
+    per_m = {}
+    for M in MS:
+        f = 2.0 * M * N_OUT * K_IN
+        byts = wlq.packed_bytes(N_OUT, K_IN, BITS, GROUP) + M * K_IN * 2 + M * N_OUT * 2 + N_OUT * 2
+        t_iso = iso[M] * 1e-3
+        per_m[str(M)] = {
+            "in_step_us": round(per_m_ms[M] * 1e3, 2), "isolated_us": round(iso[M] * 1e3, 2),
+            "tflops": round(f / t_iso / 1e12, 1), "hbm_gbs": round(byts / t_iso / 1e9, 1),
+            "tensor_frac": round(f / t_iso / 1e12 / tc_peak, 4), "hbm_frac": round(byts / t_iso / 1e9 / hbm_peak, 4),
+            "algorithmic_bytes": int(byts)}
+    # roofline of the dominant kernel (the M=4096 GEMM), timed live in the step
+    t_dom = per_m_ms[4096] * 1e-3
+    achieved = 2.0 * 4096 * N_OUT * K_IN / t_dom / 1e12
+    roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tc_peak, "unit": "TFLOP/s",
+            "frac": round(achieved / tc_peak, 4), "traffic": profiled_traffic(),
+            "peak_source": peak_src + " bf16_tflops (burst); sustained %s" % tc_sust,
+            "kernel": "gemm_kernel<FMT_W8> at M=4096 (one launch per step)"}
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": list(MS), "N": N_OUT, "K": K_IN, "bits": BITS,
+                       "group": "per-channel", "out": "bf16", "parallelism": "replicas x%d" % world,
+                       "l2": "flushed between steps (256 MiB write outside the timed events)"},
+            "per_m": per_m, "roofline": roof, "clocks": clocks,
+            "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                    "ms_per_step": round(e2e_ms, 4)},
+            "gpu_launches": launches_per_step * args.steps}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
