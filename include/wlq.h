@@ -125,6 +125,33 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
                       void* stream);
 
 /*
+ * wlq_linear without a workspace argument, for callers that cannot allocate
+ * device memory: for example code running inside a host framework that owns
+ * a fixed device-memory pool and does not let libraries call cudaMalloc, or a
+ * latency-critical loop where cudaMalloc / cudaFree would synchronise the
+ * device.  (The pages have no counterpart to this entry point; it is a
+ * deployment convenience.)
+ *
+ * The scratch it needs lives in one built-in device array of 32 MiB, which
+ * every GPU that loads the library holds until the process exits.  Shapes
+ * whose scratch (wlq_linear_workspace) exceeds 32 MiB are rejected with
+ * WLQ_ERR_WORKSPACE; int4 weights need about 2*M*K bytes, so e.g. K = 4096
+ * allows up to roughly 4000 tokens.  This call allocates nothing: no
+ * cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ * Its first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call shares the one array and leaves its
+ * contents behind; the parts that must start at zero are cleared on the
+ * stream at the start of each call.  Calls that may overlap on the GPU (other
+ * streams, other host threads) race on the array and must be serialised by
+ * the caller.  Arguments and results are otherwise those of wlq_linear.
+ */
+wlq_status wlq_linear_noalloc(const void* x, int64_t M, const void* packed, int64_t N, int64_t K,
+                              int bits, int group, const void* bias, const void* L1, const void* L2,
+                              int r, void* y, int y_dtype, void* stream);
+
+/*
  * Synchronise `stream`, then read and clear this device's error word:
  * WLQ_OK, WLQ_ERR_NONFINITE or WLQ_ERR_TIMEOUT (or WLQ_ERR_CUDA).
  */

@@ -25,7 +25,8 @@ STATUS_NAMES = {
     ERR_TIMEOUT: "WLQ_ERR_TIMEOUT", ERR_CUDA: "WLQ_ERR_CUDA",
 }
 EXPORTS = ("wlq_quantize", "wlq_packed_bytes", "wlq_pack", "wlq_unpack", "wlq_linear_workspace",
-           "wlq_linear", "wlq_get_status", "wlq_probe_wait_timeout", "wlq_last_error", "wlq_version")
+           "wlq_linear", "wlq_linear_noalloc", "wlq_get_status", "wlq_probe_wait_timeout", "wlq_last_error",
+           "wlq_version")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("libwlq.so is not built; run `python -m weight_only_quantized_rtn_b200._build`")
@@ -40,11 +41,13 @@ lib.wlq_unpack.argtypes = [_vp, _i64, _i64, _i32, _i32, _vp, _vp]
 lib.wlq_linear_workspace.argtypes = [_i64, _i64, _i64, _i32, _i32, _i32]
 lib.wlq_linear_workspace.restype = _sz
 lib.wlq_linear.argtypes = [_vp, _i64, _vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _sz, _vp]
+lib.wlq_linear_noalloc.argtypes = [_vp, _i64, _vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _vp]
 lib.wlq_get_status.argtypes = [_vp]
 lib.wlq_probe_wait_timeout.argtypes = [_u64, _vp]
 lib.wlq_last_error.restype = ctypes.c_char_p
 lib.wlq_version.restype = ctypes.c_char_p
-for _f in ("wlq_quantize", "wlq_pack", "wlq_unpack", "wlq_linear", "wlq_get_status", "wlq_probe_wait_timeout"):
+for _f in ("wlq_quantize", "wlq_pack", "wlq_unpack", "wlq_linear", "wlq_linear_noalloc", "wlq_get_status",
+           "wlq_probe_wait_timeout"):
     getattr(lib, _f).restype = ctypes.c_int
 
 
@@ -132,6 +135,16 @@ def linear(x, packed, N, K, bits, group, bias=None, L1=None, L2=None, out_dtype=
     if workspace is None:
         workspace = new_workspace(M, N, K, bits, group, r, device=x.device)
     return linear_into(y, x, packed, N, K, bits, group, bias, L1, L2, workspace, stream)
+
+
+def linear_noalloc_into(y, x, packed, N, K, bits, group, bias=None, L1=None, L2=None, stream=None):
+    """wlq_linear_noalloc: like linear_into, with the library's built-in scratch."""
+    M = x.shape[0]
+    r = 0 if L1 is None else L1.shape[1]
+    out = OUT_F32 if y.dtype == torch.float32 else OUT_BF16
+    _check(lib.wlq_linear_noalloc(_ptr(x), M, _ptr(packed), N, K, bits, group, _ptr(bias), _ptr(L1), _ptr(L2), r,
+                                  _ptr(y), out, _stream(stream)))
+    return y
 
 
 def get_status(stream=None) -> int:

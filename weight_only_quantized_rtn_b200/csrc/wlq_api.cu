@@ -412,6 +412,68 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
     }
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of wlq_linear.  Its scratch lives in this file-scope
+// device array (held by every GPU that loads the library, until exit).  In
+// host code the array's name only stands in for it; the device address is
+// fetched once per device with cudaGetSymbolAddress, with that device current.
+namespace {
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;  // 32 MiB
+}  // namespace
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+namespace {
+void* g_static_scratch_ptr[kMaxDevices] = {};
+std::mutex g_static_mu;
+
+wlq_status static_scratch(int dev, void** out) {
+    std::lock_guard<std::mutex> lk(g_static_mu);
+    if (!g_static_scratch_ptr[dev]) {
+        void* ptr = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+        g_static_scratch_ptr[dev] = ptr;
+    }
+    *out = g_static_scratch_ptr[dev];
+    return WLQ_OK;
+}
+}  // namespace
+
+extern "C" {
+
+wlq_status wlq_linear_noalloc(const void* x, int64_t M, const void* packed, int64_t N, int64_t K, int bits,
+                              int group, const void* bias, const void* L1, const void* L2, int r, void* y,
+                              int y_dtype, void* stream) {
+    // Shapes the ordinary entry point rejects, and empty problems, go straight
+    // through it (it reports the error or does nothing); nothing here allocates.
+    const int fmt = fmt_of(bits, group);
+    if (fmt < 0 || M <= 0 || N <= 0 || check_shape(N, K, bits, group) != WLQ_OK)
+        return wlq_linear(x, M, packed, N, K, bits, group, bias, L1, L2, r, y, y_dtype, nullptr, 0, stream);
+    int dev;
+    DeviceInfo* d;
+    wlq_status st = current_device(&dev, &d);
+    if (st != WLQ_OK) return st;
+    Plan p;
+    if (!make_plan(p, M, N, K, fmt, r, d->sms)) return fail(WLQ_ERR_UNSUPPORTED, "no launch plan for this shape");
+    if (p.ws > kStaticScratchBytes)
+        return fail(WLQ_ERR_WORKSPACE,
+                    "this shape needs %zu bytes of scratch but the built-in scratch holds %zu; "
+                    "call wlq_linear with a caller-owned workspace instead",
+                    p.ws, kStaticScratchBytes);
+    void* scratch = nullptr;
+    if ((st = static_scratch(dev, &scratch)) != WLQ_OK) return st;
+    if (p.S > 1) {
+        // the split counters must start at zero; the last call may have left anything
+        cudaError_t e = cudaMemsetAsync(static_cast<uint8_t*>(scratch) + p.off_cnt, 0,
+                                        static_cast<size_t>(p.MT) * p.NT * 4, static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "clear split counters");
+    }
+    return wlq_linear(x, M, packed, N, K, bits, group, bias, L1, L2, r, y, y_dtype, scratch, kStaticScratchBytes,
+                      stream);
+}
+
 wlq_status wlq_get_status(void* stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
