@@ -98,10 +98,10 @@ wlq_status wlq_unpack(const void* packed, int64_t N, int64_t K, int bits, int gr
                       int8_t* codes, void* stream);
 
 /*
- * Workspace bytes wlq_linear needs for this shape (host-only).  The
- * workspace must be zero-filled once after it is allocated; every successful
- * wlq_linear call leaves its counters zeroed again.  A workspace must not be
- * shared by calls that may run concurrently.
+ * Workspace bytes wlq_linear needs for this shape (host-only; 0 when it
+ * needs none: int8 weights without the low-rank branch).  The contents need
+ * no initialisation.  A workspace must not be shared by calls that may run
+ * concurrently.
  */
 size_t wlq_linear_workspace(int64_t M, int64_t N, int64_t K, int bits, int group, int r);
 
@@ -142,8 +142,8 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
  * Its first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
  * before any stream capture.  Every call shares the one array and leaves its
- * contents behind; the parts that must start at zero are cleared on the
- * stream at the start of each call.  Calls that may overlap on the GPU (other
+ * contents behind; nothing in it has to start at zero, because each call
+ * writes every byte it later reads.  Calls that may overlap on the GPU (other
  * streams, other host threads) race on the array and must be serialised by
  * the caller.  Arguments and results are otherwise those of wlq_linear.
  */

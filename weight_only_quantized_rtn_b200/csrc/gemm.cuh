@@ -19,18 +19,24 @@
 //   low rank          : a second TMEM accumulator gets [Th|Tl] [L2^T|L2^T]^T
 //                       (one MMA K-step per 64 of 2r, bf16, both from smem)
 //
+// Work split: an output tile is 128 channels x BN tokens.  With few tiles the
+// K range is split over the S CTAs of a thread-block cluster (S in 1,2,4,8);
+// each CTA leaves its fp32 partial in its own shared memory and every CTA then
+// sums a 1/S share of the tile's tokens over all S partials, read through
+// distributed shared memory in split order, so results are bitwise
+// reproducible and no partial sum goes through global memory.
+//
 // Warp roles (448 threads, one CTA per SM, persistent over tiles):
 //   warps 0-7   dequant: warp w handles rows 32(w%4)..+31 and k-half w/4 of
 //               every 64-wide K block; reads codes+scales from smem, converts
 //               in registers, tcgen05.st into a 4-deep ring of A stages.
 //   warps 8-11  epilogue: tcgen05.ld the accumulator (lane = n), scale, add
-//               the low-rank accumulator and the bias, store y (or an fp32
-//               split-K partial; the last split to finish sums the partials in
-//               split order, so results are bitwise reproducible).
+//               the low-rank accumulator and the bias, store y (or the split
+//               partial, then the cluster reduction).
 //   warp 12     producer: TMA for x tiles, one bulk copy per packed weight tile.
 //   warp 13     MMA issuer (one thread) + TMEM owner.
-// All waits are bounded (see ptx.cuh); on a timeout the kernel drains what it
-// issued, frees TMEM and returns with the error bit set.
+// All waits are bounded; on a timeout the kernel drains what it issued,
+// frees TMEM and returns with the error bit set.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -51,6 +57,7 @@ constexpr uint32_t A_STAGE_COLS = 32;  // 128 lanes x 64 16-bit values
 constexpr uint32_t ACC_COL0 = A_STAGES * A_STAGE_COLS;
 constexpr uint32_t LR_TILE_A_BYTES = 128 * 128;  // 128 rows x 64 bf16
 constexpr uint64_t DRAIN_TIMEOUT_NS = 200ull * 1000 * 1000;
+constexpr int MAX_SPLITS = 8;
 
 struct GemmArgs {
     const uint8_t* packed;
@@ -58,14 +65,12 @@ struct GemmArgs {
     const float* xs;        // int4 only
     const uint16_t* bias;   // bf16 bits or null
     void* y;
-    float* partials;        // split-K only
-    unsigned* counters;     // split-K only
     int M, N, K;
     int NT, KT, MT, S, kbps, BN;
     int stages, lr, lr_kb, acc_bufs, y_f32;
-    int total_tiles;
+    int tiles_nm;
     uint32_t tmem_cols, lr_col0;
-    uint32_t wtile_bytes, wstage_bytes, xstage_bytes;
+    uint32_t wtile_bytes, wstage_bytes, xstage_bytes, red_bytes;
     uint64_t timeout_ns;
 };
 
@@ -73,13 +78,13 @@ struct TileCoord {
     int nt, mt, sp, kb0, kb1;
 };
 
-__device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t) {
+// Output tile g of this cluster, K split `rank`.
+__device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int g, int rank) {
     TileCoord c;
-    c.nt = t % a.NT;
-    const int rest = t / a.NT;
-    c.mt = rest % a.MT;
-    c.sp = rest / a.MT;
-    c.kb0 = c.sp * a.kbps;
+    c.nt = g % a.NT;
+    c.mt = g / a.NT;
+    c.sp = rank;
+    c.kb0 = rank * a.kbps;
     c.kb1 = min(a.KT, c.kb0 + a.kbps);
     return c;
 }
@@ -89,6 +94,7 @@ struct Smem {
     uint8_t* w;      // stages x wstage_bytes
     uint8_t* lrA;    // 16 KB
     uint8_t* lrB;    // xstage_bytes
+    float* red;      // split partial [BN][128] fp32 (S > 1)
     uint64_t* full;
     uint64_t* empty;
     uint64_t* afull;
@@ -98,12 +104,25 @@ struct Smem {
     uint64_t* lrfull;
     uint64_t* lrempty;
     uint64_t* drain;
-    uint64_t* splitw;
-    uint64_t* splitd;
+    uint64_t* redw;   // local: every epilogue warp wrote its part of red
+    uint64_t* readw;  // local: every epilogue warp finished reading the cluster's partials
+    uint64_t* ready;  // cluster: every CTA's partial is in its smem (S arrivals)
+    uint64_t* freed;  // cluster: every CTA finished reading this CTA's partial (S arrivals)
     uint32_t* tmem_slot;
-    volatile int* split_last;
     volatile int* abort_flag;
 };
+
+struct Sched {
+    int cid, ncl, rank;
+};
+
+__device__ __forceinline__ Sched sched() {
+    Sched s;
+    s.cid = static_cast<int>(cluster_id_x());
+    s.ncl = static_cast<int>(cluster_count_x());
+    s.rank = static_cast<int>(cluster_ctarank());
+    return s;
+}
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, const GemmArgs& a,
                                               volatile int* abort_flag) {
@@ -124,13 +143,14 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, co
 // Warp-uniform variant for warps whose lanes all consume the guarded data:
 // every lane polls the barrier, and the decision to give up is taken by lane
 // 0 and broadcast, so lanes never diverge on an abort (no __syncwarp may then
-// wait for a lane that left).
+// wait for a lane that left).  `cluster_scope` acquires at cluster scope, for
+// barriers other CTAs of the cluster arrive on.
 __device__ __forceinline__ bool warp_wait_or_abort(uint64_t* bar, uint32_t parity, const GemmArgs& a,
-                                                   volatile int* abort_flag) {
+                                                   volatile int* abort_flag, bool cluster_scope = false) {
     const int lane = threadIdx.x & 31;
     uint64_t t0 = 0;
     for (uint32_t spin = 0;; ++spin) {
-        const bool done = mbar_try_wait(bar, parity);
+        const bool done = cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
         if (__all_sync(0xffffffffu, done)) return true;
         int give_up = 0;
         if (lane == 0 && (spin & 63) == 63) {
@@ -152,16 +172,21 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t b) {
 }
 
 // ------------------------------------------------------------- conversions
-// int8 offset-binary byte -> exact fp32 via the 2^23 magic number, then two
-// values packed into one bf16x2 (exact: |q| <= 127 needs 7 bits).
+// int8 offset-binary byte u = q + 128 -> fp32 2^23 + u by byte permutation,
+// minus (2^23 + 128) gives q exactly; |q| <= 127 has at most 7 significant
+// bits, so the low 16 bits of that fp32 are zero and its upper half IS
+// bf16(q).  Two values are packed by one more permutation: no conversion
+// instruction is involved.
 __device__ __forceinline__ uint32_t bytes_to_bf16x2(uint32_t w, uint32_t sel_lo, uint32_t sel_hi) {
-    uint32_t a, b;
+    uint32_t a, b, out;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(a) : "r"(w), "r"(0x4B000000u), "r"(sel_lo));
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(b) : "r"(w), "r"(0x4B000000u), "r"(sel_hi));
-    const float f0 = __uint_as_float(a) - 8388736.0f;  // 2^23 + 128
-    const float f1 = __uint_as_float(b) - 8388736.0f;
-    uint32_t out;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(f1), "f"(f0));
+    const uint64_t ab = (static_cast<uint64_t>(b) << 32) | a;
+    const uint64_t magic = (static_cast<uint64_t>(0x4B000080u) << 32) | 0x4B000080u;  // 2^23 + 128
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(ab), "l"(magic));
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(out) : "r"(static_cast<uint32_t>(d)), "r"(static_cast<uint32_t>(d >> 32)),
+        "r"(0x7632u));
     return out;
 }
 
@@ -200,11 +225,11 @@ __device__ __forceinline__ void nibbles_to_f16x2(uint32_t w, __half2 sig, uint32
 
 // ------------------------------------------------------------------- roles
 __device__ void producer_role(const GemmArgs& a, const CUtensorMap* tm_x, const CUtensorMap* tm_t,
-                              const CUtensorMap* tm_l2, const Smem& s) {
+                              const CUtensorMap* tm_l2, const Smem& s, const Sched& sc) {
     int it = 0, lrit = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < a.total_tiles && ok; t += gridDim.x) {
-        const TileCoord c = tile_coord(a, t);
+    for (int g = sc.cid; g < a.tiles_nm && ok; g += sc.ncl) {
+        const TileCoord c = tile_coord(a, g, sc.rank);
         for (int kb = c.kb0; kb < c.kb1; ++kb) {
             const int st = it % a.stages;
             const uint32_t ph = (it / a.stages) & 1;
@@ -235,14 +260,15 @@ __device__ void producer_role(const GemmArgs& a, const CUtensorMap* tm_x, const 
 }
 
 template <int FMT>
-__device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, int warp, int lane) {
+__device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc, int warp,
+                             int lane) {
     const int q = warp & 3;   // TMEM lane quarter this warp may access
     const int h = warp >> 2;  // which 32 of the 64 inputs of a K block
     const int row = q * 32 + lane;
     const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
     int it = 0;
-    for (int t = blockIdx.x; t < a.total_tiles; t += gridDim.x) {
-        const TileCoord c = tile_coord(a, t);
+    for (int g = sc.cid; g < a.tiles_nm; g += sc.ncl) {
+        const TileCoord c = tile_coord(a, g, sc.rank);
         for (int kb = c.kb0; kb < c.kb1; ++kb, ++it) {
             const int st = it % a.stages;
             if (!warp_wait_or_abort(&s.full[st], (it / a.stages) & 1, a, s.abort_flag)) return;
@@ -289,13 +315,13 @@ __device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, in
 }
 
 template <int FMT>
-__device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s) {
+__device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc) {
     const uint32_t idesc = idesc_f16(FMT == FMT_W8 ? 1u : 0u, 128, a.BN);
     const uint32_t idesc_lr = idesc_f16(1u, 128, a.BN);
     int it = 0, lrit = 0, tc = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < a.total_tiles && ok; t += gridDim.x, ++tc) {
-        const TileCoord c = tile_coord(a, t);
+    for (int g = sc.cid; g < a.tiles_nm && ok; g += sc.ncl, ++tc) {
+        const TileCoord c = tile_coord(a, g, sc.rank);
         const int ab = tc % a.acc_bufs;
         if (!wait_or_abort(&s.accempty[ab], ((tc / a.acc_bufs) & 1) ^ 1, a, s.abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -336,16 +362,33 @@ __device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s) {
     mbar_wait(s.drain, 0, DRAIN_TIMEOUT_NS);
 }
 
+__device__ __forceinline__ void store_y(const GemmArgs& a, int m, int n, float v) {
+    const size_t o = static_cast<size_t>(m) * a.N + n;
+    if (a.y_f32) static_cast<float*>(a.y)[o] = v;
+    else static_cast<__nv_bfloat16*>(a.y)[o] = __float2bfloat16_rn(v);
+}
+
 template <int FMT>
-__device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, int warp, int lane) {
+__device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc, int warp,
+                              int lane) {
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const bool first_thread = (warp == WARP_EPI0 && lane == 0);
+    const bool split = a.S > 1;
+    // cluster addresses of every CTA's partial buffer and barriers
+    uint32_t red_at[MAX_SPLITS], ready_at[MAX_SPLITS], freed_at[MAX_SPLITS];
+    if (split) {
+        for (int r = 0; r < a.S; ++r) {
+            red_at[r] = mapa_shared(smem_u32(s.red), r);
+            ready_at[r] = mapa_shared(smem_u32(s.ready), r);
+            freed_at[r] = mapa_shared(smem_u32(s.freed), r);
+        }
+    }
+    const int share = a.BN / a.S;  // tokens of each tile this CTA sums
     int tc = 0;
-    uint32_t sk = 0;  // split-K tiles handled so far (barrier phase)
-    for (int t = blockIdx.x; t < a.total_tiles; t += gridDim.x, ++tc) {
-        const TileCoord c = tile_coord(a, t);
+    for (int g = sc.cid; g < a.tiles_nm; g += sc.ncl, ++tc) {
+        const TileCoord c = tile_coord(a, g, sc.rank);
         const int ab = tc % a.acc_bufs;
         if (!warp_wait_or_abort(&s.accfull[ab], (tc / a.acc_bufs) & 1, a, s.abort_flag)) return;
         tc_fence_after();
@@ -355,9 +398,8 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, i
         const float bn = (a.bias && n_ok) ? bf16_to_f32(a.bias[n]) : 0.0f;
         const bool has_lr = a.lr && c.sp == 0;
         const int m0 = c.mt * a.BN;
-        float* part = (a.S > 1)
-            ? a.partials + ((static_cast<size_t>(c.sp) * a.MT + c.mt) * a.NT + c.nt) * (static_cast<size_t>(a.BN) * 128)
-            : nullptr;
+        // the partial buffer is reused once every CTA of the cluster has read it
+        if (split && tc > 0 && !warp_wait_or_abort(s.freed, (tc - 1) & 1, a, s.abort_flag, true)) return;
         for (int cc = 0; cc < a.BN / 16; ++cc) {
             uint32_t v[16], lv[16];
             tmem_ld16(tbase + ACC_COL0 + ab * a.BN + cc * 16, v);
@@ -370,58 +412,42 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, i
                 float val = __uint_as_float(v[j]) * rf;
                 if constexpr (FMT != FMT_W8) val *= (m < a.M) ? a.xs[m] : 0.0f;
                 if (has_lr) val += __uint_as_float(lv[j]);
-                if (part) {
-                    part[static_cast<size_t>(jm) * 128 + row] = val;
-                } else if (m < a.M && n_ok) {
-                    const size_t o = static_cast<size_t>(m) * a.N + n;
-                    if (a.y_f32) static_cast<float*>(a.y)[o] = val + bn;
-                    else static_cast<__nv_bfloat16*>(a.y)[o] = __float2bfloat16_rn(val + bn);
-                }
+                if (split) s.red[jm * 128 + row] = val;
+                else if (m < a.M && n_ok) store_y(a, m, n, val + bn);
             }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.accempty[ab]);
+        if (!split) continue;
 
-        if (a.S > 1) {
-            // The last split to finish this (nt, mt) tile sums all partials in
-            // split order.  Handshake through two mbarriers (bounded waits):
-            // splitw collects one arrival per epilogue warp once its partials
-            // are globally visible; splitd publishes the counter's verdict.
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s.splitw);
-            const uint32_t par = sk & 1;
-            ++sk;
-            if (first_thread) {
-                int last = 0;
-                if (wait_or_abort(s.splitw, par, a, s.abort_flag)) {
-                    const unsigned prev = atomicAdd(&a.counters[c.mt * a.NT + c.nt], 1u);
-                    last = (prev == static_cast<unsigned>(a.S - 1)) ? 1 : 0;
-                    if (last) a.counters[c.mt * a.NT + c.nt] = 0u;  // ready for the next call
-                }
-                *s.split_last = last;
-                mbar_arrive(s.splitd);
-            }
-            if (!warp_wait_or_abort(s.splitd, par, a, s.abort_flag)) return;
-            if (*s.split_last) {
-                __threadfence();
-                for (int jm = 0; jm < a.BN; ++jm) {
-                    const int m = m0 + jm;
-                    if (m >= a.M) break;
-                    if (!n_ok) continue;
-                    float acc = 0.0f;
-                    for (int sp = 0; sp < a.S; ++sp)
-                        acc += __ldcg(a.partials + ((static_cast<size_t>(sp) * a.MT + c.mt) * a.NT + c.nt) *
-                                                       (static_cast<size_t>(a.BN) * 128) +
-                                      static_cast<size_t>(jm) * 128 + row);
-                    const size_t o = static_cast<size_t>(m) * a.N + n;
-                    if (a.y_f32) static_cast<float*>(a.y)[o] = acc + bn;
-                    else static_cast<__nv_bfloat16*>(a.y)[o] = __float2bfloat16_rn(acc + bn);
-                }
-            }
+        // publish this CTA's partial to the cluster
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s.redw);
+        if (first_thread && wait_or_abort(s.redw, tc & 1, a, s.abort_flag)) {
+            fence_acq_rel_cluster();
+            for (int r = 0; r < a.S; ++r) mbar_arrive_remote(ready_at[r]);
+        }
+        if (!warp_wait_or_abort(s.ready, tc & 1, a, s.abort_flag, true)) return;
+        // sum this CTA's share of the tile's tokens over all partials, in split order
+        const int j0 = sc.rank * share;
+        for (int jm = j0; jm < j0 + share; ++jm) {
+            const int m = m0 + jm;
+            if (m >= a.M) break;
+            const uint32_t off = static_cast<uint32_t>(jm * 128 + row) * 4u;
+            float acc = 0.0f;
+            for (int r = 0; r < a.S; ++r) acc += ld_dsmem_f32(red_at[r] + off);
+            if (n_ok) store_y(a, m, n, acc + bn);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s.readw);
+        if (first_thread && wait_or_abort(s.readw, tc & 1, a, s.abort_flag)) {
+            fence_acq_rel_cluster();
+            for (int r = 0; r < a.S; ++r) mbar_arrive_remote(freed_at[r]);
         }
     }
+    // no CTA of the cluster may still read this CTA's shared memory when it exits
+    if (split && tc > 0) warp_wait_or_abort(s.freed, (tc - 1) & 1, a, s.abort_flag, true);
 }
 
 template <int FMT>
@@ -436,7 +462,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     s.w = s.x + static_cast<size_t>(a.stages) * a.xstage_bytes;
     s.lrA = s.w + static_cast<size_t>(a.stages) * a.wstage_bytes;
     s.lrB = s.lrA + (a.lr ? LR_TILE_A_BYTES : 0);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(s.lrB + (a.lr ? a.xstage_bytes : 0));
+    s.red = reinterpret_cast<float*>(s.lrB + (a.lr ? a.xstage_bytes : 0));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(s.red) + a.red_bytes);
     s.full = bars;
     s.empty = s.full + a.stages;
     s.afull = s.empty + a.stages;
@@ -446,11 +473,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     s.lrfull = s.accempty + 2;
     s.lrempty = s.lrfull + 1;
     s.drain = s.lrempty + 1;
-    s.splitw = s.drain + 1;
-    s.splitd = s.splitw + 1;
-    s.tmem_slot = reinterpret_cast<uint32_t*>(s.splitd + 1);
-    s.split_last = reinterpret_cast<volatile int*>(s.tmem_slot + 1);
-    s.abort_flag = s.split_last + 1;
+    s.redw = s.drain + 1;
+    s.readw = s.redw + 1;
+    s.ready = s.readw + 1;
+    s.freed = s.ready + 1;
+    s.tmem_slot = reinterpret_cast<uint32_t*>(s.freed + 1);
+    s.abort_flag = reinterpret_cast<volatile int*>(s.tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -470,9 +498,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
         mbar_init(s.lrfull, 1);
         mbar_init(s.lrempty, 1);
         mbar_init(s.drain, 1);
-        mbar_init(s.splitw, NUM_EPI_WARPS);
-        mbar_init(s.splitd, 1);
-        *s.split_last = 0;
+        mbar_init(s.redw, NUM_EPI_WARPS);
+        mbar_init(s.readw, NUM_EPI_WARPS);
+        mbar_init(s.ready, a.S);
+        mbar_init(s.freed, a.S);
         *s.abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async();
@@ -488,16 +517,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (a.S > 1) {
+        // every CTA of the cluster has initialised its barriers before any remote arrive
+        asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    }
     const uint32_t tmem = *s.tmem_slot;
+    const Sched sc = sched();
 
     if (warp < NUM_DQ_WARPS) {
-        dequant_role<FMT>(a, tmem, s, warp, lane);
+        dequant_role<FMT>(a, tmem, s, sc, warp, lane);
     } else if (warp < WARP_PRODUCER) {
-        epilogue_role<FMT>(a, tmem, s, warp, lane);
+        epilogue_role<FMT>(a, tmem, s, sc, warp, lane);
     } else if (warp == WARP_PRODUCER) {
-        if (lane == 0) producer_role(a, &tm_x, &tm_t, &tm_l2, s);
+        if (lane == 0) producer_role(a, &tm_x, &tm_t, &tm_l2, s, sc);
     } else if (lane == 0) {
-        mma_role<FMT>(a, tmem, s);
+        mma_role<FMT>(a, tmem, s, sc);
     }
 
     tc_fence_before();

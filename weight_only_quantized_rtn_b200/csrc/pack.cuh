@@ -57,44 +57,41 @@ __global__ void pack_rowfactor_kernel(const float* __restrict__ scales, int64_t 
     }
 }
 
-// One CTA (128 threads, thread = row of the tile) per tile.
+// One CTA (128 threads) per tile.  Codes are read as 8-byte runs (8 inputs of
+// one row; rows start 8-byte aligned because K % 8 == 0), so a warp reads
+// four rows' 64 contiguous bytes each.
 __global__ void __launch_bounds__(128) pack_tiles_kernel(
     const int8_t* __restrict__ codes, const float* __restrict__ scales, int64_t N, int64_t K,
     int64_t G, int fmt, int KT, const float* __restrict__ rowf, uint8_t* __restrict__ packed) {
     const int64_t tile = blockIdx.x;
     const int64_t nt = tile / KT;
     const int kb = static_cast<int>(tile % KT);
+    const int64_t k0 = static_cast<int64_t>(kb) * 64;
+    uint8_t* blk = packed + tile * tile_bytes(fmt);
+    for (int idx = threadIdx.x; idx < 128 * 8; idx += 128) {
+        const int i = idx >> 3, part = idx & 7;
+        const int64_t n = nt * 128 + i, k = k0 + 8 * part;
+        uint2 v = make_uint2(0u, 0u);
+        if (n < N && k < K) v = __ldg(reinterpret_cast<const uint2*>(codes + n * K + k));
+        if (fmt == FMT_W8) {
+            // offset binary q + 128 of a two's-complement byte is q ^ 0x80
+            v.x ^= 0x80808080u;
+            v.y ^= 0x80808080u;
+            *reinterpret_cast<uint2*>(blk + (part >> 1) * 2048 + 16 * i + (part & 1) * 8) = v;
+        } else {
+            const uint32_t b[2] = {v.x, v.y};
+            uint32_t w = 0;
+            for (int t = 0; t < 8; ++t) {
+                const uint32_t u = ((b[t >> 2] >> (8 * (t & 3))) + 8u) & 0xFu;  // (q + 8) mod 16
+                w |= u << (4 * int4_nibble_pos(t));
+            }
+            *reinterpret_cast<uint32_t*>(blk + (part >> 2) * 2048 + 16 * i + 4 * (part & 3)) = w;
+        }
+    }
+    if (fmt == FMT_W8) return;
     const int i = threadIdx.x;
     const int64_t n = nt * 128 + i;
     const bool row_ok = n < N;
-    const int64_t k0 = static_cast<int64_t>(kb) * 64;
-    uint8_t* blk = packed + tile * tile_bytes(fmt);
-    auto code_at = [&](int64_t k) -> int {
-        return (row_ok && k < K) ? static_cast<int>(codes[n * K + k]) : 0;
-    };
-    if (fmt == FMT_W8) {
-        for (int c = 0; c < 4; ++c) {
-            uint32_t w[4];
-            for (int j = 0; j < 4; ++j) {
-                uint32_t v = 0;
-                for (int b = 0; b < 4; ++b)
-                    v |= static_cast<uint32_t>(code_at(k0 + 16 * c + 4 * j + b) + 128) << (8 * b);
-                w[j] = v;
-            }
-            *reinterpret_cast<uint4*>(blk + c * 2048 + 16 * i) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        return;
-    }
-    for (int c = 0; c < 2; ++c) {
-        uint32_t w[4];
-        for (int j = 0; j < 4; ++j) {
-            uint32_t v = 0;
-            for (int t = 0; t < 8; ++t)
-                v |= static_cast<uint32_t>(code_at(k0 + 32 * c + 8 * j + t) + 8) << (4 * int4_nibble_pos(t));
-            w[j] = v;
-        }
-        *reinterpret_cast<uint4*>(blk + c * 2048 + 16 * i) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
     const float rf = row_ok ? rowf[n] : 0.0f;
     const int sh = (rf > 0.0f) ? -ilogbf(rf) : 0;  // s * 2^sh = s / rf exactly
     auto scale16 = [&](int64_t g) -> __half {

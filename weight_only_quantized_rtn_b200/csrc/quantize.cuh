@@ -3,11 +3,13 @@
 // with one scale per output channel, int4 grouped along K with gs 64 / 16).
 //
 // Per group: a = max|W| (exact), s = a / qmax as an IEEE fp32 division, and
-// q = the integer nearest to W / s with ties to even, clamped to +-qmax.  The
-// quotient is estimated in fp64 and then corrected with the exact residual
-// W - k*s (k*s has at most 32 significant bits, so one fp64 fma gives it
-// exactly); the code therefore equals the exact real rounding, independent of
-// how the estimate was rounded.
+// q = the integer nearest to W / s with ties to even, clamped to +-qmax.  An
+// estimate k of the quotient (within one of the answer) is corrected with the
+// exact residual e = W - k*s, compared against s/2: the code therefore equals
+// the rounding of the exact real quotient, whatever rounding the estimate
+// had.  Normal scales take an fp32 path (rtn_byte_f32); subnormal ones an
+// fp64 path (rtn_code), where k*s has at most 32 significant bits and one
+// fp64 fma gives e exactly.
 #pragma once
 #include <cstdint>
 #include "ptx.cuh"
@@ -31,40 +33,94 @@ __device__ __forceinline__ int rtn_code(float w, float s, double inv_s, int qmax
     return static_cast<int>(k);
 }
 
+// The same exact rounding in fp32 for a normal scale (s >= 2^-126).  Adding
+// 1.5 * 2^23 rounds any |t| < 2^22 to an integer, ties to even.  The residual
+// e = w - k*s from one fp32 fma is exact wherever it decides anything: for
+// |e| near s/2 its significand fits in 24 bits (|w| >= s/2 there, so w's last
+// bit is at least half of s's).  Returns the code's two's-complement byte.
+__device__ __forceinline__ uint32_t rtn_byte_f32(float w, float s, float inv, float qmax) {
+    const float kMagic = 12582912.0f;  // 1.5 * 2^23
+    float k = __fsub_rn(__fadd_rn(__fmul_rn(w, inv), kMagic), kMagic);
+    const float e = __fmaf_rn(-k, s, w);
+    const float h = 0.5f * s;
+    if (e > h) {
+        k += 1.0f;
+    } else if (e < -h) {
+        k -= 1.0f;
+    } else if (e == h || e == -h) {  // exact tie: keep the even neighbour
+        if (__float_as_uint(__fadd_rn(k, kMagic)) & 1u) k += (e > 0.0f) ? 1.0f : -1.0f;
+    }
+    k = fminf(fmaxf(k, -qmax), qmax);
+    return __float_as_uint(__fadd_rn(k, kMagic)) & 0xFFu;  // low byte of 0x4B400000 + k
+}
+
 __device__ __forceinline__ float abs_finite_max(float a, float v, bool& bad) {
     bad |= !isfinite(v);
     return fmaxf(a, fabsf(v));
 }
 
-__device__ __forceinline__ uint32_t pack_codes4(float4 v, float s, double inv, int qmax, bool& bad) {
+struct GroupScale {
+    float s;       // fp32(absmax / qmax)
+    float inv;     // fp32 1/s (normal s only)
+    double inv64;  // fp64 1/s
+    bool normal;   // s >= 2^-126: the fp32 path is exact
+};
+
+__device__ __forceinline__ GroupScale group_scale(float a, int qmax) {
+    GroupScale g;
+    g.s = __fdiv_rn(a, static_cast<float>(qmax));
+    g.normal = g.s >= 1.17549435e-38f;
+    g.inv = g.normal ? __frcp_rn(g.s) : 0.0f;
+    g.inv64 = (g.s > 0.0f) ? 1.0 / static_cast<double>(g.s) : 0.0;
+    return g;
+}
+
+__device__ __forceinline__ uint32_t pack_codes4(float4 v, const GroupScale& g, int qmax, bool& bad) {
     const float f[4] = {v.x, v.y, v.z, v.w};
     uint32_t out = 0;
     for (int i = 0; i < 4; ++i) {
-        int q = 0;
-        if (isfinite(f[i])) q = rtn_code(f[i], s, inv, qmax);
-        else bad = true;
-        out |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * i);
+        uint32_t byte = 0;
+        if (!isfinite(f[i])) bad = true;
+        else if (g.normal) byte = rtn_byte_f32(f[i], g.s, g.inv, static_cast<float>(qmax));
+        else byte = static_cast<uint32_t>(rtn_code(f[i], g.s, g.inv64, qmax)) & 0xFFu;
+        out |= byte << (8 * i);
     }
     return out;
 }
 
-// One CTA per row: the group is the whole row (per output channel).
-template <int THREADS>
+// One CTA per row: the group is the whole row (per output channel).  Rows of
+// up to THREADS * VPT float4 stay in registers between the absmax and the
+// rounding; longer rows are read twice (the second read hits L2).
+template <int THREADS, int VPT>
 __global__ void __launch_bounds__(THREADS) quantize_rows_kernel(
     const float* __restrict__ W, int64_t N, int64_t K, int qmax, int8_t* __restrict__ codes,
     float* __restrict__ scales) {
     __shared__ float red[THREADS / 32];
     const int64_t K4 = K / 4;
+    const bool in_regs = K4 <= static_cast<int64_t>(THREADS) * VPT;
     for (int64_t n = blockIdx.x; n < N; n += gridDim.x) {
         const float4* row = reinterpret_cast<const float4*>(W + n * K);
+        float4 cache[VPT];
         float a = 0.0f;
         bool bad = false;
-        for (int64_t i = threadIdx.x; i < K4; i += THREADS) {
-            const float4 v = __ldg(row + i);
-            a = abs_finite_max(a, v.x, bad);
-            a = abs_finite_max(a, v.y, bad);
-            a = abs_finite_max(a, v.z, bad);
-            a = abs_finite_max(a, v.w, bad);
+        if (in_regs) {
+#pragma unroll
+            for (int j = 0; j < VPT; ++j) {
+                const int64_t i = threadIdx.x + static_cast<int64_t>(j) * THREADS;
+                cache[j] = (i < K4) ? __ldcs(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+                a = abs_finite_max(a, cache[j].x, bad);
+                a = abs_finite_max(a, cache[j].y, bad);
+                a = abs_finite_max(a, cache[j].z, bad);
+                a = abs_finite_max(a, cache[j].w, bad);
+            }
+        } else {
+            for (int64_t i = threadIdx.x; i < K4; i += THREADS) {
+                const float4 v = __ldg(row + i);
+                a = abs_finite_max(a, v.x, bad);
+                a = abs_finite_max(a, v.y, bad);
+                a = abs_finite_max(a, v.z, bad);
+                a = abs_finite_max(a, v.w, bad);
+            }
         }
         for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
         if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
@@ -72,12 +128,18 @@ __global__ void __launch_bounds__(THREADS) quantize_rows_kernel(
         a = red[0];
         for (int i = 1; i < THREADS / 32; ++i) a = fmaxf(a, red[i]);
         __syncthreads();
-        const float s = __fdiv_rn(a, static_cast<float>(qmax));
-        const double inv = (s > 0.0f) ? 1.0 / static_cast<double>(s) : 0.0;
-        if (threadIdx.x == 0) scales[n] = s;
+        const GroupScale g = group_scale(a, qmax);
+        if (threadIdx.x == 0) scales[n] = g.s;
         uint32_t* out = reinterpret_cast<uint32_t*>(codes + n * K);
-        for (int64_t i = threadIdx.x; i < K4; i += THREADS)
-            out[i] = pack_codes4(row[i], s, inv, qmax, bad);
+        if (in_regs) {
+#pragma unroll
+            for (int j = 0; j < VPT; ++j) {
+                const int64_t i = threadIdx.x + static_cast<int64_t>(j) * THREADS;
+                if (i < K4) out[i] = pack_codes4(cache[j], g, qmax, bad);
+            }
+        } else {
+            for (int64_t i = threadIdx.x; i < K4; i += THREADS) out[i] = pack_codes4(row[i], g, qmax, bad);
+        }
         if (bad) raise_error(ERRBIT_NONFINITE);
     }
 }
@@ -107,10 +169,9 @@ __global__ void __launch_bounds__(256) quantize_groups_kernel(
         for (int off = lanes_per_group >> 1; off > 0; off >>= 1)
             a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
         if (valid) {
-            const float s = __fdiv_rn(a, static_cast<float>(qmax));
-            const double inv = (s > 0.0f) ? 1.0 / static_cast<double>(s) : 0.0;
-            if ((lane & (lanes_per_group - 1)) == 0) scales[i / lanes_per_group] = s;
-            out[i] = pack_codes4(v, s, inv, qmax, bad);
+            const GroupScale gs = group_scale(a, qmax);
+            if ((lane & (lanes_per_group - 1)) == 0) scales[i / lanes_per_group] = gs.s;
+            out[i] = pack_codes4(v, gs, qmax, bad);
         }
     }
     if (bad) raise_error(ERRBIT_NONFINITE);

@@ -119,15 +119,25 @@ constexpr size_t kSmemLimit = 232448;  // 227 KB opt-in per block on sm_100
 struct Plan {
     int fmt = -1;
     int M = 0, N = 0, K = 0, r = 0;
-    int NT = 0, KT = 0, MT = 0, S = 1, kbps = 0, BN = 0, total_tiles = 0, grid = 0;
+    int NT = 0, KT = 0, MT = 0, S = 1, kbps = 0, BN = 0, tiles_nm = 0, grid = 0;
     int stages = 0, lr_kb = 0, acc_bufs = 1;
-    uint32_t tmem_cols = 0, lr_col0 = 0, wtile = 0, wstage = 0, xstage = 0;
+    uint32_t tmem_cols = 0, lr_col0 = 0, wtile = 0, wstage = 0, xstage = 0, red = 0;
     size_t smem = 0;
-    size_t off_x16 = 0, off_xs = 0, off_thl = 0, off_l2t = 0, off_part = 0, off_cnt = 0, ws = 0;
+    size_t off_x16 = 0, off_xs = 0, off_thl = 0, off_l2t = 0, ws = 0;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+int token_tile(int64_t M, int r) {
+    if (M <= 16) return 16;
+    if (M <= 32) return 32;
+    if (M <= 64) return 64;
+    if (M <= 128 || r) return 128;
+    return 256;
+}
+
+// Launch plan: token tile BN, K split S (a power of two up to 8, the CTAs of
+// one cluster), TMEM columns, shared-memory ring depth, workspace layout.
 bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms) {
     p.fmt = fmt;
     p.M = static_cast<int>(M);
@@ -137,23 +147,26 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     p.NT = static_cast<int>(cdiv(N, 128));
     p.KT = static_cast<int>(cdiv(K, 64));
     p.lr_kb = r ? static_cast<int>(cdiv(2 * r, 64)) : 0;
-    // token tile: the MMA N dimension
-    if (M <= 16) p.BN = 16;
-    else if (M <= 32) p.BN = 32;
-    else if (M <= 64) p.BN = 64;
-    else if (M <= 128 || r) p.BN = 128;
-    else p.BN = 256;
+    p.BN = token_tile(M, r);
     p.MT = static_cast<int>(cdiv(M, p.BN));
-    const int tiles_nm = p.NT * p.MT;
-    // split K so that small problems still cover the SMs
+    // Split K when the output tiles cannot cover half of the SMs.  A split
+    // tile keeps at most 128 tokens (its fp32 partial sits in shared memory).
     int S = 1;
-    if (tiles_nm < sms) S = std::max(1, sms / tiles_nm);
-    S = std::min(S, std::max(1, p.KT / 2));
-    S = std::min(S, 16);
-    p.kbps = static_cast<int>(cdiv(p.KT, S));
-    p.S = static_cast<int>(cdiv(p.KT, p.kbps));
-    p.total_tiles = tiles_nm * p.S;
-    p.grid = std::min(p.total_tiles, sms);
+    if (p.NT * p.MT * 2 <= sms) {
+        if (p.BN > 128) {
+            p.BN = 128;
+            p.MT = static_cast<int>(cdiv(M, p.BN));
+        }
+        while (S * 2 <= wlq::MAX_SPLITS && p.NT * p.MT * S * 2 <= sms && S * 2 <= p.BN && p.KT >= S * 4) S *= 2;
+    }
+    // every split must own at least one K block
+    for (;;) {
+        p.kbps = static_cast<int>(cdiv(p.KT, S));
+        if (S == 1 || static_cast<int64_t>(S - 1) * p.kbps < p.KT) break;
+        S /= 2;
+    }
+    p.S = S;
+    p.tiles_nm = p.NT * p.MT;
     // TMEM: A ring + accumulator(s), double-buffered when they fit
     const uint32_t acc_cols = static_cast<uint32_t>(p.BN) * (r ? 2u : 1u);
     p.acc_bufs = (wlq::ACC_COL0 + 2 * acc_cols <= 512) ? 2 : 1;
@@ -162,15 +175,16 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     p.tmem_cols = 32;
     while (p.tmem_cols < need) p.tmem_cols <<= 1;
     p.lr_col0 = wlq::ACC_COL0 + p.acc_bufs * static_cast<uint32_t>(p.BN);
-    // shared memory ring
+    // shared memory: ring stages + low-rank tiles + split partial + barriers
     p.wtile = wlq::tile_bytes(fmt);
     p.wstage = (p.wtile + 1023u) & ~1023u;
     p.xstage = static_cast<uint32_t>(p.BN) * 128u;
+    p.red = (S > 1) ? static_cast<uint32_t>(p.BN) * 128u * 4u : 0u;
     const size_t lr_bytes = r ? (wlq::LR_TILE_A_BYTES + p.xstage) : 0;
-    const size_t fixed = 1024 /* alignment */ + 512 /* barriers */ + lr_bytes;
+    const size_t fixed = 1024 /* alignment */ + 512 /* barriers */ + lr_bytes + p.red;
     const size_t per_stage = p.xstage + p.wstage;
+    if (fixed + 2 * per_stage > kSmemLimit) return false;
     p.stages = static_cast<int>(std::min<size_t>(16, (kSmemLimit - fixed) / per_stage));
-    if (p.stages < 2) return false;
     p.smem = fixed + p.stages * per_stage;
     // workspace
     size_t off = 0;
@@ -181,10 +195,6 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     if (r) {
         p.off_thl = off; off = align256(off + static_cast<size_t>(M) * p.lr_kb * 64 * 2);
         p.off_l2t = off; off = align256(off + static_cast<size_t>(p.NT) * 128 * p.lr_kb * 64 * 2);
-    }
-    if (p.S > 1) {
-        p.off_part = off; off = align256(off + static_cast<size_t>(p.S) * p.MT * p.NT * p.BN * 128 * 4);
-        p.off_cnt = off;  off = align256(off + static_cast<size_t>(p.MT) * p.NT * 4);
     }
     p.ws = off;
     return true;
@@ -200,16 +210,40 @@ wlq_status check_shape(int64_t N, int64_t K, int bits, int group) {
 }
 
 template <int FMT>
-wlq_status launch_gemm(const Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, const CUtensorMap& tl,
-                       const wlq::GemmArgs& a, DeviceInfo* d, cudaStream_t st) {
+wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, const CUtensorMap& tl,
+                       wlq::GemmArgs& a, DeviceInfo* d, cudaStream_t st) {
+    auto kern = wlq::gemm_kernel<FMT>;
     if (!d->smem_set[FMT]) {
-        cudaError_t e = cudaFuncSetAttribute(wlq::gemm_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(kSmemLimit));
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         d->smem_set[FMT] = true;
     }
-    wlq::gemm_kernel<FMT><<<p.grid, wlq::GEMM_THREADS, p.smem, st>>>(tx, tt, tl, a);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cudaLaunchAttribute attr[1];
+    cfg.blockDim = dim3(wlq::GEMM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = st;
+    int clusters = std::min(p.tiles_nm, d->sms / p.S);
+    if (p.S > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(p.S);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        // persistent clusters: no more than can be resident at once
+        cfg.gridDim = dim3(static_cast<unsigned>(clusters * p.S), 1, 1);
+        int active = 0;
+        if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) == cudaSuccess && active > 0)
+            clusters = std::min(clusters, active);
+        else
+            cudaGetLastError();
+    }
+    cfg.gridDim = dim3(static_cast<unsigned>(clusters * p.S), 1, 1);
+    p.grid = clusters * p.S;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tx, tt, tl, a);
     if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
     return WLQ_OK;
 }
@@ -245,7 +279,7 @@ wlq_status wlq_quantize(const float* W, int64_t N, int64_t K, int bits, int grou
     const int qmax = (1 << (bits - 1)) - 1;
     if (group == 0) {
         const int grid = static_cast<int>(std::min<int64_t>(N, int64_t(d->sms) * 8));
-        wlq::quantize_rows_kernel<256><<<grid, 256, 0, s>>>(W, N, K, qmax, codes, scales);
+        wlq::quantize_rows_kernel<256, 16><<<grid, 256, 0, s>>>(W, N, K, qmax, codes, scales);
     } else {
         const int64_t total4 = N * K / 4;
         wlq::quantize_groups_kernel<<<grid_for(total4, 256, d->sms), 256, 0, s>>>(W, total4, group / 4, qmax,
@@ -271,7 +305,8 @@ wlq_status wlq_pack(const int8_t* codes, const float* scales, int64_t N, int64_t
     if (st != WLQ_OK) return st;
     if (N == 0) return WLQ_OK;
     if (!codes || !scales || !packed) return fail(WLQ_ERR_INVALID_ARG, "null pointer");
-    if (!aligned16(packed)) return fail(WLQ_ERR_ALIGN, "packed must be 16-byte aligned");
+    if (!aligned16(packed) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+        return fail(WLQ_ERR_ALIGN, "packed and codes must be 16-byte aligned, scales 4-byte aligned");
     int dev;
     DeviceInfo* d;
     if ((st = current_device(&dev, &d)) != WLQ_OK) return st;
@@ -395,15 +430,13 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
     a.xs = xs;
     a.bias = static_cast<const uint16_t*>(bias);
     a.y = y;
-    a.partials = p.S > 1 ? reinterpret_cast<float*>(ws + p.off_part) : nullptr;
-    a.counters = p.S > 1 ? reinterpret_cast<unsigned*>(ws + p.off_cnt) : nullptr;
     a.M = p.M; a.N = p.N; a.K = p.K;
     a.NT = p.NT; a.KT = p.KT; a.MT = p.MT; a.S = p.S; a.kbps = p.kbps; a.BN = p.BN;
     a.stages = p.stages; a.lr = r ? 1 : 0; a.lr_kb = p.lr_kb; a.acc_bufs = p.acc_bufs;
     a.y_f32 = (y_dtype == WLQ_OUT_F32) ? 1 : 0;
-    a.total_tiles = p.total_tiles;
+    a.tiles_nm = p.tiles_nm;
     a.tmem_cols = p.tmem_cols; a.lr_col0 = p.lr_col0;
-    a.wtile_bytes = p.wtile; a.wstage_bytes = p.wstage; a.xstage_bytes = p.xstage;
+    a.wtile_bytes = p.wtile; a.wstage_bytes = p.wstage; a.xstage_bytes = p.xstage; a.red_bytes = p.red;
     a.timeout_ns = kDefaultTimeoutNs;
     switch (fmt) {
         case wlq::FMT_W8: return launch_gemm<wlq::FMT_W8>(p, tx, tt, tl, a, d, s);
@@ -464,12 +497,8 @@ wlq_status wlq_linear_noalloc(const void* x, int64_t M, const void* packed, int6
                     p.ws, kStaticScratchBytes);
     void* scratch = nullptr;
     if ((st = static_scratch(dev, &scratch)) != WLQ_OK) return st;
-    if (p.S > 1) {
-        // the split counters must start at zero; the last call may have left anything
-        cudaError_t e = cudaMemsetAsync(static_cast<uint8_t*>(scratch) + p.off_cnt, 0,
-                                        static_cast<size_t>(p.MT) * p.NT * 4, static_cast<cudaStream_t>(stream));
-        if (e != cudaSuccess) return cuda_fail(e, "clear split counters");
-    }
+    // Nothing in the scratch has to start at zero: every region is fully
+    // written by the call's preparation kernels before the GEMM reads it.
     return wlq_linear(x, M, packed, N, K, bits, group, bias, L1, L2, r, y, y_dtype, scratch, kStaticScratchBytes,
                       stream);
 }
