@@ -210,18 +210,20 @@ def run_gpu(args):
     ys = {M: torch.empty((M, N_OUT), dtype=torch.bfloat16, device=dev) for M in MS}
     wss = {M: wlq.new_workspace(M, N_OUT, K_IN, BITS, GROUP, 0, device=dev) for M in MS}
     flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
-    lib, ptr, st = wlq.lib, wlq._ptr, wlq._stream(stream)
+    lib, ptr = wlq.lib, wlq._ptr
 
-    def step(ev=None):
+    def quantize_pack():
+        st = wlq._stream(torch.cuda.current_stream())
         wlq._check(lib.wlq_quantize(ptr(W), N_OUT, K_IN, BITS, GROUP, ptr(codes), ptr(scales), st))
         wlq._check(lib.wlq_pack(ptr(codes), ptr(scales), N_OUT, K_IN, BITS, GROUP, ptr(packed), st))
+
+    def linear(M):
+        wlq.linear_into(ys[M], xs[M], packed, N_OUT, K_IN, BITS, GROUP, bias=b, workspace=wss[M])
+
+    def step():
+        quantize_pack()
         for M in MS:
-            if ev is not None:
-                ev[M][0].record(stream)
-            wlq.linear_into(ys[M], xs[M], packed, N_OUT, K_IN, BITS, GROUP, bias=b, workspace=wss[M],
-                            stream=stream)
-            if ev is not None:
-                ev[M][1].record(stream)
+            linear(M)
 
     launches_per_step = 1 + 2 + len(MS)  # quantize, pack (row factors + tiles), one GEMM per M
 
@@ -229,22 +231,37 @@ def run_gpu(args):
         step()
     torch.cuda.synchronize()
     wlq.check_status()
+
+    # The step runs as CUDA-graph replays (one graph per phase, so that events
+    # between replays time each phase) to keep host launch overhead off the
+    # device timeline.
+    graphs = {}
+    for name, fn in [("qp", quantize_pack)] + [(M, (lambda M=M: linear(M))) for M in MS]:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        graphs[name] = g
+    torch.cuda.synchronize()
+    for _ in range(2):
+        for g in graphs.values():
+            g.replay()
+    torch.cuda.synchronize()
+    wlq.check_status()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
 
+    phases = ["qp"] + list(MS)
     sampler = ClockSampler(local)
     sampler.start()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    inner = [{M: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for M in MS}
-             for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(phases) + 1)] for _ in range(args.steps)]
     for i in range(args.steps):
         flush.zero_()  # evict L2 between steps (outside the timed events)
         torch.cuda.nvtx.range_push("timed_step")
-        starts[i].record(stream)
-        step(inner[i])
-        ends[i].record(stream)
+        evs[i][0].record(stream)
+        for j, ph in enumerate(phases):
+            graphs[ph].replay()
+            evs[i][j + 1].record(stream)
         torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     if dist:
@@ -253,8 +270,9 @@ def run_gpu(args):
     clocks = sampler.stop()
     wlq.check_status()
 
-    ms_step = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
-    per_m_ms = {M: sum(ev[M][0].elapsed_time(ev[M][1]) for ev in inner) / args.steps for M in MS}
+    ms_step = sum(e[0].elapsed_time(e[-1]) for e in evs) / args.steps
+    per_ms = {ph: sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j, ph in enumerate(phases)}
+    per_m_ms = {M: per_ms[M] for M in MS}
     if dist:
         t = torch.tensor([ms_step] + [per_m_ms[M] for M in MS], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -264,17 +282,16 @@ def run_gpu(args):
     # ---- per-M kernels in isolation (L2 flushed before every launch)
     iso = {}
     for M in MS:
-        evs = []
+        pairs = []
         for _ in range(max(5, args.steps)):
             flush.zero_()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            wlq.linear_into(ys[M], xs[M], packed, N_OUT, K_IN, BITS, GROUP, bias=b, workspace=wss[M],
-                            stream=stream)
+            graphs[M].replay()
             e1.record(stream)
-            evs.append((e0, e1))
+            pairs.append((e0, e1))
         torch.cuda.synchronize()
-        iso[M] = statistics.median(a.elapsed_time(c) for a, c in evs)
+        iso[M] = statistics.median(a.elapsed_time(c) for a, c in pairs)
 
     # ---- end to end through the public API with pinned host buffers
     W_h = torch.from_numpy(base["W"]).pin_memory()
@@ -317,7 +334,7 @@ def run_gpu(args):
             "tflops": round(f / t_iso / 1e12, 1), "hbm_gbs": round(byts / t_iso / 1e9, 1),
             "tensor_frac": round(f / t_iso / 1e12 / tc_peak, 4), "hbm_frac": round(byts / t_iso / 1e9 / hbm_peak, 4),
             "algorithmic_bytes": int(byts)}
-    # roofline of the dominant kernel (the M=4096 GEMM), timed live in the step
+    # roofline of the dominant kernel (the M=4096 GEMM, one launch), timed live in the step
     t_dom = per_m_ms[4096] * 1e-3
     achieved = 2.0 * 4096 * N_OUT * K_IN / t_dom / 1e12
     roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tc_peak, "unit": "TFLOP/s",
@@ -332,6 +349,7 @@ def run_gpu(args):
                        "group": "per-channel", "out": "bf16", "parallelism": "replicas x%d" % world,
                        "l2": "flushed between steps (256 MiB write outside the timed events)"},
             "per_m": per_m, "roofline": roof, "clocks": clocks,
+            "quantize_pack_us": round(per_ms["qp"] * 1e3, 2),
             "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                     "ms_per_step": round(e2e_ms, 4)},

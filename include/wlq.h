@@ -166,6 +166,14 @@ wlq_status wlq_get_status(void* stream);
  */
 wlq_status wlq_probe_wait_timeout(uint64_t timeout_ns, void* stream);
 
+/*
+ * Cap the number of CTAs (thread blocks) every later wlq_linear launch uses
+ * on any device; 0 removes the cap.  Host-only, process-wide, not thread
+ * safe against concurrent launches.  For tests that need several output
+ * tiles per CTA, and for tuning; results do not depend on it.
+ */
+void wlq_set_grid_limit(int max_ctas);
+
 /* Human-readable text of the last error returned on this host thread. */
 const char* wlq_last_error(void);
 

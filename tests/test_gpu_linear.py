@@ -73,6 +73,26 @@ def test_parity_low_rank(bits, group, r, M):
 
 
 @pytest.mark.parametrize("bits,group", RECIPES)
+@pytest.mark.parametrize("M,N,K,r,cap", [
+    (40, 1100, 320, 0, 4),     # 9 tiles on 4 CTAs: both accumulator buffers in use
+    (16, 33000, 128, 0, 16),   # 258 tiles of 16 tokens on 16 CTAs
+    (300, 700, 256, 0, 3),     # 128-token tiles, several per CTA
+    (16, 1024, 2048, 0, 16),   # K split over clusters, each cluster several tiles
+    (100, 1024, 512, 32, 4),   # low rank + K split, several tiles per cluster
+    (600, 640, 640, 16, 5),    # low rank, single accumulator buffer, ring wrap-around
+])
+def test_parity_several_tiles_per_cta(bits, group, M, N, K, r, cap):
+    m = wlq()
+    x, W, b, L1, L2 = small_case(M + N + K + r, M, N, K, bits, group, r=r)
+    m.set_grid_limit(cap)
+    try:
+        err, _, _ = linear_case(x, W, bits, group, b, L1, L2)
+    finally:
+        m.set_grid_limit(0)
+    assert err <= TOL, err
+
+
+@pytest.mark.parametrize("bits,group", RECIPES)
 def test_bf16_output_is_rounded_fp32_output(bits, group):
     m = wlq()
     for M in (16, 300):

@@ -25,8 +25,8 @@ STATUS_NAMES = {
     ERR_TIMEOUT: "WLQ_ERR_TIMEOUT", ERR_CUDA: "WLQ_ERR_CUDA",
 }
 EXPORTS = ("wlq_quantize", "wlq_packed_bytes", "wlq_pack", "wlq_unpack", "wlq_linear_workspace",
-           "wlq_linear", "wlq_linear_noalloc", "wlq_get_status", "wlq_probe_wait_timeout", "wlq_last_error",
-           "wlq_version")
+           "wlq_linear", "wlq_linear_noalloc", "wlq_get_status", "wlq_probe_wait_timeout", "wlq_set_grid_limit",
+           "wlq_last_error", "wlq_version")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("libwlq.so is not built; run `python -m weight_only_quantized_rtn_b200._build`")
@@ -44,6 +44,8 @@ lib.wlq_linear.argtypes = [_vp, _i64, _vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp
 lib.wlq_linear_noalloc.argtypes = [_vp, _i64, _vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _vp]
 lib.wlq_get_status.argtypes = [_vp]
 lib.wlq_probe_wait_timeout.argtypes = [_u64, _vp]
+lib.wlq_set_grid_limit.argtypes = [_i32]
+lib.wlq_set_grid_limit.restype = None
 lib.wlq_last_error.restype = ctypes.c_char_p
 lib.wlq_version.restype = ctypes.c_char_p
 for _f in ("wlq_quantize", "wlq_pack", "wlq_unpack", "wlq_linear", "wlq_linear_noalloc", "wlq_get_status",
@@ -158,6 +160,11 @@ def check_status(stream=None):
 
 def probe_wait_timeout(timeout_ns: int, stream=None):
     _check(lib.wlq_probe_wait_timeout(timeout_ns, _stream(stream)))
+
+
+def set_grid_limit(max_ctas: int):
+    """Cap the CTAs of every later wlq_linear launch (0: no cap)."""
+    lib.wlq_set_grid_limit(int(max_ctas))
 
 
 def version() -> str:

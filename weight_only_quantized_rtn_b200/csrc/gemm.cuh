@@ -26,10 +26,16 @@
 // distributed shared memory in split order, so results are bitwise
 // reproducible and no partial sum goes through global memory.
 //
+// Pipeline: one ring of `stages` slots.  Slot i holds an x tile and a packed
+// weight tile in shared memory and an A stage (32 TMEM columns, after the
+// accumulators, which start at column 0) in tensor memory.  The producer refills slot i only after the slot's previous round
+// was released (MMA commit + dequant warps), so a dequant warp that sees slot
+// i full again may overwrite its A stage without a further handshake.
+//
 // Warp roles (448 threads, one CTA per SM, persistent over tiles):
 //   warps 0-7   dequant: warp w handles rows 32(w%4)..+31 and k-half w/4 of
 //               every 64-wide K block; reads codes+scales from smem, converts
-//               in registers, tcgen05.st into a 4-deep ring of A stages.
+//               in registers, tcgen05.st into the slot's A stage.
 //   warps 8-11  epilogue: tcgen05.ld the accumulator (lane = n), scale, add
 //               the low-rank accumulator and the bias, store y (or the split
 //               partial, then the cluster reduction).
@@ -52,9 +58,8 @@ constexpr int WARP_EPI0 = NUM_DQ_WARPS;
 constexpr int WARP_PRODUCER = NUM_DQ_WARPS + NUM_EPI_WARPS;
 constexpr int WARP_MMA = WARP_PRODUCER + 1;
 constexpr int GEMM_THREADS = (WARP_MMA + 1) * 32;
-constexpr int A_STAGES = 4;
 constexpr uint32_t A_STAGE_COLS = 32;  // 128 lanes x 64 16-bit values
-constexpr uint32_t ACC_COL0 = A_STAGES * A_STAGE_COLS;
+constexpr int MAX_STAGES = 16;
 constexpr uint32_t LR_TILE_A_BYTES = 128 * 128;  // 128 rows x 64 bf16
 constexpr uint64_t DRAIN_TIMEOUT_NS = 200ull * 1000 * 1000;
 constexpr int MAX_SPLITS = 8;
@@ -69,7 +74,7 @@ struct GemmArgs {
     int NT, KT, MT, S, kbps, BN;
     int stages, lr, lr_kb, acc_bufs, y_f32;
     int tiles_nm;
-    uint32_t tmem_cols, lr_col0;
+    uint32_t tmem_cols, acc_col0, lr_col0, a_col0;
     uint32_t wtile_bytes, wstage_bytes, xstage_bytes, red_bytes;
     uint64_t timeout_ns;
 };
@@ -94,11 +99,10 @@ struct Smem {
     uint8_t* w;      // stages x wstage_bytes
     uint8_t* lrA;    // 16 KB
     uint8_t* lrB;    // xstage_bytes
-    float* red;      // split partial [BN][128] fp32 (S > 1)
-    uint64_t* full;
-    uint64_t* empty;
-    uint64_t* afull;
-    uint64_t* aempty;
+    float* red;      // split partial [128][BN + 4] fp32 (S > 1)
+    uint64_t* full;    // slot loaded (TMA)
+    uint64_t* empty;   // slot consumed (MMA commit + dequant warps); also frees the slot's A stage
+    uint64_t* afull;   // slot's A stage written to TMEM (dequant warps)
     uint64_t* accfull;
     uint64_t* accempty;
     uint64_t* lrfull;
@@ -114,6 +118,18 @@ struct Smem {
 
 struct Sched {
     int cid, ncl, rank;
+};
+
+// Position in the ring: slot index and the parity of the slot's current round.
+struct Ring {
+    int slot = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void next(int stages) {
+        if (++slot == stages) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
 };
 
 __device__ __forceinline__ Sched sched() {
@@ -227,19 +243,20 @@ __device__ __forceinline__ void nibbles_to_f16x2(uint32_t w, __half2 sig, uint32
 __device__ void producer_role(const GemmArgs& a, const CUtensorMap* tm_x, const CUtensorMap* tm_t,
                               const CUtensorMap* tm_l2, const Smem& s, const Sched& sc) {
     int it = 0, lrit = 0;
+    Ring r;
     bool ok = true;
     for (int g = sc.cid; g < a.tiles_nm && ok; g += sc.ncl) {
         const TileCoord c = tile_coord(a, g, sc.rank);
         for (int kb = c.kb0; kb < c.kb1; ++kb) {
-            const int st = it % a.stages;
-            const uint32_t ph = (it / a.stages) & 1;
-            if (!wait_or_abort(&s.empty[st], ph ^ 1, a, s.abort_flag)) { ok = false; break; }
+            const int st = r.slot;
+            if (!wait_or_abort(&s.empty[st], r.phase ^ 1, a, s.abort_flag)) { ok = false; break; }
             mbar_arrive_expect_tx(&s.full[st], a.xstage_bytes + a.wtile_bytes);
             tma_load_2d(s.x + st * a.xstage_bytes, tm_x, &s.full[st], kb * 64, c.mt * a.BN);
             bulk_load(s.w + st * a.wstage_bytes,
                       a.packed + (static_cast<size_t>(c.nt) * a.KT + kb) * a.wtile_bytes,
                       a.wtile_bytes, &s.full[st]);
             ++it;
+            r.next(a.stages);
         }
         if (ok && a.lr && c.sp == 0) {
             for (int lk = 0; lk < a.lr_kb; ++lk) {
@@ -266,12 +283,12 @@ __device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, co
     const int h = warp >> 2;  // which 32 of the 64 inputs of a K block
     const int row = q * 32 + lane;
     const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    int it = 0;
+    Ring r;
     for (int g = sc.cid; g < a.tiles_nm; g += sc.ncl) {
         const TileCoord c = tile_coord(a, g, sc.rank);
-        for (int kb = c.kb0; kb < c.kb1; ++kb, ++it) {
-            const int st = it % a.stages;
-            if (!warp_wait_or_abort(&s.full[st], (it / a.stages) & 1, a, s.abort_flag)) return;
+        for (int kb = c.kb0; kb < c.kb1; ++kb, r.next(a.stages)) {
+            const int st = r.slot;
+            if (!warp_wait_or_abort(&s.full[st], r.phase, a, s.abort_flag)) return;
             const uint8_t* blk = s.w + st * a.wstage_bytes;
             uint4 c0, c1 = make_uint4(0, 0, 0, 0);
             __half2 sig0, sig1;
@@ -292,9 +309,8 @@ __device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, co
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.empty[st]);
-
-            const int as = it % A_STAGES;
-            if (!warp_wait_or_abort(&s.aempty[as], ((it / A_STAGES) & 1) ^ 1, a, s.abort_flag)) return;
+            // The slot's A stage is free: this round's load was issued only after
+            // the previous round's MMA committed.
             tc_fence_after();
             uint32_t v[16];
             if constexpr (FMT == FMT_W8) {
@@ -305,11 +321,11 @@ __device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, co
                 nibbles_to_f16x2(c0.z, sig1, v + 8);
                 nibbles_to_f16x2(c0.w, sig1, v + 12);
             }
-            tmem_st16(tbase + as * A_STAGE_COLS + h * 16, v);
+            tmem_st16(tbase + a.a_col0 + st * A_STAGE_COLS + h * 16, v);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s.afull[as]);
+            if (lane == 0) mbar_arrive(&s.afull[st]);
         }
     }
 }
@@ -318,27 +334,28 @@ template <int FMT>
 __device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc) {
     const uint32_t idesc = idesc_f16(FMT == FMT_W8 ? 1u : 0u, 128, a.BN);
     const uint32_t idesc_lr = idesc_f16(1u, 128, a.BN);
-    int it = 0, lrit = 0, tc = 0;
+    int lrit = 0, tc = 0;
+    Ring r;
     bool ok = true;
     for (int g = sc.cid; g < a.tiles_nm && ok; g += sc.ncl, ++tc) {
         const TileCoord c = tile_coord(a, g, sc.rank);
         const int ab = tc % a.acc_bufs;
         if (!wait_or_abort(&s.accempty[ab], ((tc / a.acc_bufs) & 1) ^ 1, a, s.abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d = tmem + ACC_COL0 + ab * a.BN;
-        for (int kb = c.kb0; kb < c.kb1 && ok; ++kb, ++it) {
-            const int st = it % a.stages;
-            const int as = it % A_STAGES;
-            if (!wait_or_abort(&s.full[st], (it / a.stages) & 1, a, s.abort_flag) ||
-                !wait_or_abort(&s.afull[as], (it / A_STAGES) & 1, a, s.abort_flag)) { ok = false; break; }
+        const uint32_t d = tmem + a.acc_col0 + ab * a.BN;
+        for (int kb = c.kb0; kb < c.kb1 && ok; ++kb, r.next(a.stages)) {
+            const int st = r.slot;
+            // afull implies full (the dequant warps waited for it), but the
+            // MMA also reads the slot's x tile, so observe full as well
+            if (!wait_or_abort(&s.afull[st], r.phase, a, s.abort_flag) ||
+                !wait_or_abort(&s.full[st], r.phase, a, s.abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint64_t bdesc = smem_desc_sw128(smem_u32(s.x + st * a.xstage_bytes));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_ts(d, tmem + as * A_STAGE_COLS + kk * 8, bdesc + 2 * kk, idesc,
+                mma_ts(d, tmem + a.a_col0 + st * A_STAGE_COLS + kk * 8, bdesc + 2 * kk, idesc,
                        (kb > c.kb0 || kk > 0) ? 1u : 0u);
             mma_commit(&s.empty[st]);
-            mma_commit(&s.aempty[as]);
         }
         if (!ok) break;
         if (a.lr && c.sp == 0) {
@@ -385,7 +402,8 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
             freed_at[r] = mapa_shared(smem_u32(s.freed), r);
         }
     }
-    const int share = a.BN / a.S;  // tokens of each tile this CTA sums
+    const int share = a.BN / a.S;       // tokens of each tile this CTA sums (a multiple of 4)
+    const int red_pitch = a.BN + 4;     // floats per row of the partial buffer (keeps float4 alignment)
     int tc = 0;
     for (int g = sc.cid; g < a.tiles_nm; g += sc.ncl, ++tc) {
         const TileCoord c = tile_coord(a, g, sc.rank);
@@ -402,18 +420,28 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
         if (split && tc > 0 && !warp_wait_or_abort(s.freed, (tc - 1) & 1, a, s.abort_flag, true)) return;
         for (int cc = 0; cc < a.BN / 16; ++cc) {
             uint32_t v[16], lv[16];
-            tmem_ld16(tbase + ACC_COL0 + ab * a.BN + cc * 16, v);
+            tmem_ld16(tbase + a.acc_col0 + ab * a.BN + cc * 16, v);
             if (has_lr) tmem_ld16(tbase + a.lr_col0 + ab * a.BN + cc * 16, lv);
             tmem_wait_ld();
+            float val[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const int jm = cc * 16 + j;
-                const int m = m0 + jm;
-                float val = __uint_as_float(v[j]) * rf;
-                if constexpr (FMT != FMT_W8) val *= (m < a.M) ? a.xs[m] : 0.0f;
-                if (has_lr) val += __uint_as_float(lv[j]);
-                if (split) s.red[jm * 128 + row] = val;
-                else if (m < a.M && n_ok) store_y(a, m, n, val + bn);
+                const int m = m0 + cc * 16 + j;
+                val[j] = __uint_as_float(v[j]) * rf;
+                if constexpr (FMT != FMT_W8) val[j] *= (m < a.M) ? a.xs[m] : 0.0f;
+                if (has_lr) val[j] += __uint_as_float(lv[j]);
+            }
+            if (split) {
+                float4* dst = reinterpret_cast<float4*>(s.red + row * red_pitch + cc * 16);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    dst[j] = make_float4(val[4 * j], val[4 * j + 1], val[4 * j + 2], val[4 * j + 3]);
+            } else if (n_ok) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int m = m0 + cc * 16 + j;
+                    if (m < a.M) store_y(a, m, n, val[j] + bn);
+                }
             }
         }
         tc_fence_before();
@@ -429,15 +457,31 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
             for (int r = 0; r < a.S; ++r) mbar_arrive_remote(ready_at[r]);
         }
         if (!warp_wait_or_abort(s.ready, tc & 1, a, s.abort_flag, true)) return;
-        // sum this CTA's share of the tile's tokens over all partials, in split order
+        // sum this CTA's share of the tile's tokens over all partials, in split
+        // order; four tokens per vector load, all S loads of a quad in flight
         const int j0 = sc.rank * share;
-        for (int jm = j0; jm < j0 + share; ++jm) {
-            const int m = m0 + jm;
-            if (m >= a.M) break;
-            const uint32_t off = static_cast<uint32_t>(jm * 128 + row) * 4u;
-            float acc = 0.0f;
-            for (int r = 0; r < a.S; ++r) acc += ld_dsmem_f32(red_at[r] + off);
-            if (n_ok) store_y(a, m, n, acc + bn);
+        for (int jq = j0; jq < j0 + share; jq += 4) {
+            if (m0 + jq >= a.M) break;
+            const uint32_t off = static_cast<uint32_t>(row * red_pitch + jq) * 4u;
+            float4 part[MAX_SPLITS];
+#pragma unroll
+            for (int r = 0; r < MAX_SPLITS; ++r)
+                if (r < a.S) part[r] = ld_dsmem_f32x4(red_at[r] + off);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int r = 0; r < MAX_SPLITS; ++r)
+                if (r < a.S) {
+                    acc.x += part[r].x;
+                    acc.y += part[r].y;
+                    acc.z += part[r].z;
+                    acc.w += part[r].w;
+                }
+            if (n_ok) {
+                const float o[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (m0 + jq + j < a.M) store_y(a, m0 + jq + j, n, o[j] + bn);
+            }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(s.readw);
@@ -467,8 +511,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     s.full = bars;
     s.empty = s.full + a.stages;
     s.afull = s.empty + a.stages;
-    s.aempty = s.afull + A_STAGES;
-    s.accfull = s.aempty + A_STAGES;
+    s.accfull = s.afull + a.stages;
     s.accempty = s.accfull + 2;
     s.lrfull = s.accempty + 2;
     s.lrempty = s.lrfull + 1;
@@ -486,10 +529,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
         for (int i = 0; i < a.stages; ++i) {
             mbar_init(&s.full[i], 1);
             mbar_init(&s.empty[i], 1 + NUM_DQ_WARPS);
-        }
-        for (int i = 0; i < A_STAGES; ++i) {
             mbar_init(&s.afull[i], NUM_DQ_WARPS);
-            mbar_init(&s.aempty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.accfull[i], 1);

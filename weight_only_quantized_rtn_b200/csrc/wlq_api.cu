@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 #include "../../include/wlq.h"
 #include "gemm.cuh"
@@ -49,6 +50,8 @@ struct DeviceInfo {
     int checked = 0;  // 0 unknown, 1 supported, -1 not
     int sms = 0;
     bool smem_set[3] = {false, false, false};
+    // resident clusters per (format, cluster size, dynamic smem), queried once
+    std::unordered_map<uint64_t, int> max_clusters;
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -121,7 +124,7 @@ struct Plan {
     int M = 0, N = 0, K = 0, r = 0;
     int NT = 0, KT = 0, MT = 0, S = 1, kbps = 0, BN = 0, tiles_nm = 0, grid = 0;
     int stages = 0, lr_kb = 0, acc_bufs = 1;
-    uint32_t tmem_cols = 0, lr_col0 = 0, wtile = 0, wstage = 0, xstage = 0, red = 0;
+    uint32_t tmem_cols = 0, acc_col0 = 0, lr_col0 = 0, a_col0 = 0, wtile = 0, wstage = 0, xstage = 0, red = 0;
     size_t smem = 0;
     size_t off_x16 = 0, off_xs = 0, off_thl = 0, off_l2t = 0, ws = 0;
 };
@@ -157,7 +160,9 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
             p.BN = 128;
             p.MT = static_cast<int>(cdiv(M, p.BN));
         }
-        while (S * 2 <= wlq::MAX_SPLITS && p.NT * p.MT * S * 2 <= sms && S * 2 <= p.BN && p.KT >= S * 4) S *= 2;
+        // each CTA of a split cluster sums BN / S tokens of the tile, four at a
+        // time (vector loads from distributed shared memory): keep BN / S >= 4
+        while (S * 2 <= wlq::MAX_SPLITS && p.NT * p.MT * S * 2 <= sms && S * 8 <= p.BN && p.KT >= S * 4) S *= 2;
     }
     // every split must own at least one K block
     for (;;) {
@@ -166,26 +171,37 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
         S /= 2;
     }
     p.S = S;
+    if (S > 1 && p.BN % (4 * S) != 0) return false;  // the reduction's token quads must not straddle shares
     p.tiles_nm = p.NT * p.MT;
-    // TMEM: A ring + accumulator(s), double-buffered when they fit
+    // TMEM: accumulator(s) first, from column 0, so each starts at a multiple
+    // of its own width (main accumulators at ab*BN, low-rank ones after them);
+    // then one 32-column A stage per ring slot.  The accumulators are
+    // double-buffered when that still leaves room for four slots.
     const uint32_t acc_cols = static_cast<uint32_t>(p.BN) * (r ? 2u : 1u);
-    p.acc_bufs = (wlq::ACC_COL0 + 2 * acc_cols <= 512) ? 2 : 1;
-    if (wlq::ACC_COL0 + acc_cols > 512) return false;
-    const uint32_t need = wlq::ACC_COL0 + p.acc_bufs * acc_cols;
-    p.tmem_cols = 32;
-    while (p.tmem_cols < need) p.tmem_cols <<= 1;
-    p.lr_col0 = wlq::ACC_COL0 + p.acc_bufs * static_cast<uint32_t>(p.BN);
-    // shared memory: ring stages + low-rank tiles + split partial + barriers
+    if (acc_cols + 2 * wlq::A_STAGE_COLS > 512) return false;
+    p.acc_bufs = (2 * acc_cols + 4 * wlq::A_STAGE_COLS <= 512) ? 2 : 1;
+    const uint32_t acc_total = p.acc_bufs * acc_cols;
+    const uint32_t a_col0 = (acc_total + wlq::A_STAGE_COLS - 1) / wlq::A_STAGE_COLS * wlq::A_STAGE_COLS;
+    const int tmem_slots = static_cast<int>((512 - a_col0) / wlq::A_STAGE_COLS);
+    // shared memory: ring slots + low-rank tiles + split partial + barriers
     p.wtile = wlq::tile_bytes(fmt);
     p.wstage = (p.wtile + 1023u) & ~1023u;
     p.xstage = static_cast<uint32_t>(p.BN) * 128u;
-    p.red = (S > 1) ? static_cast<uint32_t>(p.BN) * 128u * 4u : 0u;
+    p.red = (S > 1) ? 128u * static_cast<uint32_t>(p.BN + 4) * 4u : 0u;
     const size_t lr_bytes = r ? (wlq::LR_TILE_A_BYTES + p.xstage) : 0;
-    const size_t fixed = 1024 /* alignment */ + 512 /* barriers */ + lr_bytes + p.red;
+    const size_t fixed = 1024 /* alignment */ + 1024 /* barriers */ + lr_bytes + p.red;
     const size_t per_stage = p.xstage + p.wstage;
     if (fixed + 2 * per_stage > kSmemLimit) return false;
-    p.stages = static_cast<int>(std::min<size_t>(16, (kSmemLimit - fixed) / per_stage));
+    const int smem_slots = static_cast<int>((kSmemLimit - fixed) / per_stage);
+    p.stages = std::min({wlq::MAX_STAGES, tmem_slots, smem_slots});
+    if (p.stages < 2) return false;
     p.smem = fixed + p.stages * per_stage;
+    p.acc_col0 = 0;
+    p.lr_col0 = p.acc_bufs * static_cast<uint32_t>(p.BN);
+    p.a_col0 = a_col0;
+    const uint32_t need = a_col0 + static_cast<uint32_t>(p.stages) * wlq::A_STAGE_COLS;
+    p.tmem_cols = 32;
+    while (p.tmem_cols < need) p.tmem_cols <<= 1;
     // workspace
     size_t off = 0;
     if (fmt != wlq::FMT_W8) {
@@ -209,6 +225,8 @@ wlq_status check_shape(int64_t N, int64_t K, int bits, int group) {
     return WLQ_OK;
 }
 
+int g_grid_limit = 0;  // 0: no cap on the GEMM's CTAs (see wlq_set_grid_limit)
+
 template <int FMT>
 wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, const CUtensorMap& tl,
                        wlq::GemmArgs& a, DeviceInfo* d, cudaStream_t st) {
@@ -225,7 +243,8 @@ wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, co
     cfg.blockDim = dim3(wlq::GEMM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = p.smem;
     cfg.stream = st;
-    int clusters = std::min(p.tiles_nm, d->sms / p.S);
+    const int cta_cap = (g_grid_limit > 0) ? std::min(g_grid_limit, d->sms) : d->sms;
+    int clusters = std::max(1, std::min(p.tiles_nm, cta_cap / p.S));
     if (p.S > 1) {
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = static_cast<unsigned>(p.S);
@@ -234,12 +253,23 @@ wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, co
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         // persistent clusters: no more than can be resident at once
-        cfg.gridDim = dim3(static_cast<unsigned>(clusters * p.S), 1, 1);
+        const uint64_t key = (static_cast<uint64_t>(FMT) << 48) | (static_cast<uint64_t>(p.S) << 32) | p.smem;
         int active = 0;
-        if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) == cudaSuccess && active > 0)
-            clusters = std::min(clusters, active);
-        else
-            cudaGetLastError();
+        {
+            std::lock_guard<std::mutex> lk(g_dev_mu);
+            auto it = d->max_clusters.find(key);
+            if (it != d->max_clusters.end()) active = it->second;
+        }
+        if (active == 0) {
+            cfg.gridDim = dim3(static_cast<unsigned>(clusters * p.S), 1, 1);
+            if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) != cudaSuccess || active <= 0) {
+                cudaGetLastError();
+                active = d->sms / p.S;
+            }
+            std::lock_guard<std::mutex> lk(g_dev_mu);
+            d->max_clusters[key] = active;
+        }
+        clusters = std::min(clusters, active);
     }
     cfg.gridDim = dim3(static_cast<unsigned>(clusters * p.S), 1, 1);
     p.grid = clusters * p.S;
@@ -435,7 +465,7 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
     a.stages = p.stages; a.lr = r ? 1 : 0; a.lr_kb = p.lr_kb; a.acc_bufs = p.acc_bufs;
     a.y_f32 = (y_dtype == WLQ_OUT_F32) ? 1 : 0;
     a.tiles_nm = p.tiles_nm;
-    a.tmem_cols = p.tmem_cols; a.lr_col0 = p.lr_col0;
+    a.tmem_cols = p.tmem_cols; a.acc_col0 = p.acc_col0; a.lr_col0 = p.lr_col0; a.a_col0 = p.a_col0;
     a.wtile_bytes = p.wtile; a.wstage_bytes = p.wstage; a.xstage_bytes = p.xstage; a.red_bytes = p.red;
     a.timeout_ns = kDefaultTimeoutNs;
     switch (fmt) {
@@ -502,6 +532,8 @@ wlq_status wlq_linear_noalloc(const void* x, int64_t M, const void* packed, int6
     return wlq_linear(x, M, packed, N, K, bits, group, bias, L1, L2, r, y, y_dtype, scratch, kStaticScratchBytes,
                       stream);
 }
+
+void wlq_set_grid_limit(int max_ctas) { g_grid_limit = max_ctas > 0 ? max_ctas : 0; }
 
 wlq_status wlq_get_status(void* stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
