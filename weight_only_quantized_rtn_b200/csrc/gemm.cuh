@@ -156,18 +156,22 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, co
     }
 }
 
-// Warp-uniform variant for warps whose lanes all consume the guarded data:
-// every lane polls the barrier, and the decision to give up is taken by lane
-// 0 and broadcast, so lanes never diverge on an abort (no __syncwarp may then
-// wait for a lane that left).  `cluster_scope` acquires at cluster scope, for
-// barriers other CTAs of the cluster arrive on.
+// Warp-uniform wait for warps whose lanes all consume the guarded data:
+// every lane polls the barrier (each lane acquires for itself), and the
+// decision to give up is taken by lane 0 and broadcast, so lanes never
+// diverge on an abort (no __syncwarp may then wait for a lane that left).
+// `cluster_scope` acquires at cluster scope, for barriers other CTAs of the
+// cluster arrive on; `backoff` sleeps between polls, for long waits off the
+// critical path.
 __device__ __forceinline__ bool warp_wait_or_abort(uint64_t* bar, uint32_t parity, const GemmArgs& a,
-                                                   volatile int* abort_flag, bool cluster_scope = false) {
+                                                   volatile int* abort_flag, bool cluster_scope = false,
+                                                   bool backoff = false) {
     const int lane = threadIdx.x & 31;
     uint64_t t0 = 0;
     for (uint32_t spin = 0;; ++spin) {
         const bool done = cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
         if (__all_sync(0xffffffffu, done)) return true;
+        if (backoff && spin > 4) __nanosleep(96);
         int give_up = 0;
         if (lane == 0 && (spin & 63) == 63) {
             if (t0 == 0) t0 = globaltimer_ns();
@@ -345,10 +349,9 @@ __device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const 
         const uint32_t d = tmem + a.acc_col0 + ab * a.BN;
         for (int kb = c.kb0; kb < c.kb1 && ok; ++kb, r.next(a.stages)) {
             const int st = r.slot;
-            // afull implies full (the dequant warps waited for it), but the
-            // MMA also reads the slot's x tile, so observe full as well
-            if (!wait_or_abort(&s.afull[st], r.phase, a, s.abort_flag) ||
-                !wait_or_abort(&s.full[st], r.phase, a, s.abort_flag)) { ok = false; break; }
+            // afull is reached only after every dequant warp observed the slot
+            // full, so it orders the slot's x tile before the MMA as well
+            if (!wait_or_abort(&s.afull[st], r.phase, a, s.abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint64_t bdesc = smem_desc_sw128(smem_u32(s.x + st * a.xstage_bytes));
 #pragma unroll
@@ -408,7 +411,7 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
     for (int g = sc.cid; g < a.tiles_nm; g += sc.ncl, ++tc) {
         const TileCoord c = tile_coord(a, g, sc.rank);
         const int ab = tc % a.acc_bufs;
-        if (!warp_wait_or_abort(&s.accfull[ab], (tc / a.acc_bufs) & 1, a, s.abort_flag)) return;
+        if (!warp_wait_or_abort(&s.accfull[ab], (tc / a.acc_bufs) & 1, a, s.abort_flag, false, true)) return;
         tc_fence_after();
         const int n = c.nt * 128 + row;
         const bool n_ok = n < a.N;

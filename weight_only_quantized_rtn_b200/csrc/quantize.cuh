@@ -88,58 +88,34 @@ __device__ __forceinline__ uint32_t pack_codes4(float4 v, const GroupScale& g, i
     return out;
 }
 
-// One CTA per row: the group is the whole row (per output channel).  Rows of
-// up to THREADS * VPT float4 stay in registers between the absmax and the
-// rounding; longer rows are read twice (the second read hits L2).
-template <int THREADS, int VPT>
-__global__ void __launch_bounds__(THREADS) quantize_rows_kernel(
+// One warp per row: the group is the whole row (per output channel).  Pass 1
+// reads the row for its absmax, pass 2 reads it again (from L2: the row was
+// just read) to round and store the codes; eight loads in flight per lane.
+__global__ void __launch_bounds__(256) quantize_rows_kernel(
     const float* __restrict__ W, int64_t N, int64_t K, int qmax, int8_t* __restrict__ codes,
     float* __restrict__ scales) {
-    __shared__ float red[THREADS / 32];
+    const int lane = threadIdx.x & 31;
+    const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     const int64_t K4 = K / 4;
-    const bool in_regs = K4 <= static_cast<int64_t>(THREADS) * VPT;
-    for (int64_t n = blockIdx.x; n < N; n += gridDim.x) {
+    for (int64_t n = w0; n < N; n += nw) {
         const float4* row = reinterpret_cast<const float4*>(W + n * K);
-        float4 cache[VPT];
         float a = 0.0f;
         bool bad = false;
-        if (in_regs) {
-#pragma unroll
-            for (int j = 0; j < VPT; ++j) {
-                const int64_t i = threadIdx.x + static_cast<int64_t>(j) * THREADS;
-                cache[j] = (i < K4) ? __ldcs(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-                a = abs_finite_max(a, cache[j].x, bad);
-                a = abs_finite_max(a, cache[j].y, bad);
-                a = abs_finite_max(a, cache[j].z, bad);
-                a = abs_finite_max(a, cache[j].w, bad);
-            }
-        } else {
-            for (int64_t i = threadIdx.x; i < K4; i += THREADS) {
-                const float4 v = __ldg(row + i);
-                a = abs_finite_max(a, v.x, bad);
-                a = abs_finite_max(a, v.y, bad);
-                a = abs_finite_max(a, v.z, bad);
-                a = abs_finite_max(a, v.w, bad);
-            }
+#pragma unroll 8
+        for (int64_t i = lane; i < K4; i += 32) {
+            const float4 v = __ldg(row + i);
+            a = abs_finite_max(a, v.x, bad);
+            a = abs_finite_max(a, v.y, bad);
+            a = abs_finite_max(a, v.z, bad);
+            a = abs_finite_max(a, v.w, bad);
         }
         for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
-        __syncthreads();
-        a = red[0];
-        for (int i = 1; i < THREADS / 32; ++i) a = fmaxf(a, red[i]);
-        __syncthreads();
         const GroupScale g = group_scale(a, qmax);
-        if (threadIdx.x == 0) scales[n] = g.s;
+        if (lane == 0) scales[n] = g.s;
         uint32_t* out = reinterpret_cast<uint32_t*>(codes + n * K);
-        if (in_regs) {
-#pragma unroll
-            for (int j = 0; j < VPT; ++j) {
-                const int64_t i = threadIdx.x + static_cast<int64_t>(j) * THREADS;
-                if (i < K4) out[i] = pack_codes4(cache[j], g, qmax, bad);
-            }
-        } else {
-            for (int64_t i = threadIdx.x; i < K4; i += THREADS) out[i] = pack_codes4(row[i], g, qmax, bad);
-        }
+#pragma unroll 8
+        for (int64_t i = lane; i < K4; i += 32) out[i] = pack_codes4(__ldcs(row + i), g, qmax, bad);
         if (bad) raise_error(ERRBIT_NONFINITE);
     }
 }

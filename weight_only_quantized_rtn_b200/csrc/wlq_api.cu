@@ -308,8 +308,7 @@ wlq_status wlq_quantize(const float* W, int64_t N, int64_t K, int bits, int grou
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int qmax = (1 << (bits - 1)) - 1;
     if (group == 0) {
-        const int grid = static_cast<int>(std::min<int64_t>(N, int64_t(d->sms) * 8));
-        wlq::quantize_rows_kernel<256, 16><<<grid, 256, 0, s>>>(W, N, K, qmax, codes, scales);
+        wlq::quantize_rows_kernel<<<grid_for(N * 32, 256, d->sms), 256, 0, s>>>(W, N, K, qmax, codes, scales);
     } else {
         const int64_t total4 = N * K / 4;
         wlq::quantize_groups_kernel<<<grid_for(total4, 256, d->sms), 256, 0, s>>>(W, total4, group / 4, qmax,
