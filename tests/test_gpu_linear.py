@@ -80,6 +80,8 @@ def test_parity_low_rank(bits, group, r, M):
     (16, 1024, 2048, 0, 16),   # K split over clusters, each cluster several tiles
     (100, 1024, 512, 32, 4),   # low rank + K split, several tiles per cluster
     (600, 640, 640, 16, 5),    # low rank, single accumulator buffer, ring wrap-around
+    (600, 4096, 448, 0, 0),    # CTA pairs (256 channels x 256 tokens per MMA), partial last slot
+    (600, 4096, 1024, 0, 6),   # CTA pairs, three pairs for 48 tiles
 ])
 def test_parity_several_tiles_per_cta(bits, group, M, N, K, r, cap):
     m = wlq()

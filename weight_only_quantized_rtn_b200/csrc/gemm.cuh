@@ -19,6 +19,11 @@
 //   low rank          : a second TMEM accumulator gets [Th|Tl] [L2^T|L2^T]^T
 //                       (one MMA K-step per 64 of 2r, bf16, both from smem)
 //
+// CTA pairs (large M): two CTAs of a cluster share each MMA (cta_group::2),
+// M = 256 channels (128 per CTA, each dequantising its own rows into its own
+// TMEM) by BN = 256 tokens (each CTA stages half of the x tile); the first CTA
+// issues the MMAs, which halves the single issuing thread's work per FLOP.
+//
 // Work split: an output tile is 128 channels x BN tokens.  With few tiles the
 // K range is split over the S CTAs of a thread-block cluster (S in 1,2,4,8);
 // each CTA leaves its fp32 partial in its own shared memory and every CTA then
@@ -26,9 +31,12 @@
 // distributed shared memory in split order, so results are bitwise
 // reproducible and no partial sum goes through global memory.
 //
-// Pipeline: one ring of `stages` slots.  Slot i holds an x tile and a packed
-// weight tile in shared memory and an A stage (32 TMEM columns, after the
-// accumulators, which start at column 0) in tensor memory.  The producer refills slot i only after the slot's previous round
+// Pipeline: one ring of `stages` slots.  Slot i covers `ks` consecutive
+// 64-wide K blocks: ks x sub-tiles and ks packed weight tiles (one bulk copy:
+// the tiles of a 128-row band are contiguous) in shared memory, and an A stage
+// of ks * 32 TMEM columns (after the accumulators, which start at column 0)
+// in tensor memory; one handshake per slot amortises the barrier and commit
+// costs over ks blocks.  The producer refills slot i only after the slot's previous round
 // was released (MMA commit + dequant warps), so a dequant warp that sees slot
 // i full again may overwrite its A stage without a further handshake.
 //
@@ -63,6 +71,8 @@ constexpr int MAX_STAGES = 16;
 constexpr uint32_t LR_TILE_A_BYTES = 128 * 128;  // 128 rows x 64 bf16
 constexpr uint64_t DRAIN_TIMEOUT_NS = 200ull * 1000 * 1000;
 constexpr int MAX_SPLITS = 8;
+constexpr int MAX_KS = 4;  // 64-wide K blocks per ring slot, at most
+constexpr uint32_t EPI_STAGE_BYTES = 2048;  // per epilogue warp: 16 tokens x 32 channels (fp32, or bf16 + one pad row)
 
 struct GemmArgs {
     const uint8_t* packed;
@@ -72,10 +82,11 @@ struct GemmArgs {
     void* y;
     int M, N, K;
     int NT, KT, MT, S, kbps, BN;
-    int stages, lr, lr_kb, acc_bufs, y_f32;
+    int stages, ks, lr, lr_kb, acc_bufs, y_f32;  // ks: 64-wide K blocks per ring slot
     int tiles_nm;
     uint32_t tmem_cols, acc_col0, lr_col0, a_col0;
-    uint32_t wtile_bytes, wstage_bytes, xstage_bytes, red_bytes;
+    uint32_t wtile_bytes, wstage_bytes, xsub_bytes, xstage_bytes, red_bytes, stage_bytes;
+    int vec_out;  // unsplit tiles store 16-byte runs of y rows (y 16-byte aligned, rows whole runs)
     uint64_t timeout_ns;
 };
 
@@ -83,14 +94,26 @@ struct TileCoord {
     int nt, mt, sp, kb0, kb1;
 };
 
-// Output tile g of this cluster, K split `rank`.
+// Output tile g of this cluster.  Split clusters: every CTA takes K split
+// `rank` of the same 128-channel tile.  Pairs: CTA `rank` takes channel tile
+// 2 * (g % (NT / 2)) + rank over the whole K range.
+template <bool PAIR>
 __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int g, int rank) {
     TileCoord c;
-    c.nt = g % a.NT;
-    c.mt = g / a.NT;
-    c.sp = rank;
-    c.kb0 = rank * a.kbps;
-    c.kb1 = min(a.KT, c.kb0 + a.kbps);
+    if constexpr (PAIR) {
+        const int ntp = a.NT >> 1;
+        c.nt = (g % ntp) * 2 + rank;
+        c.mt = g / ntp;
+        c.sp = 0;
+        c.kb0 = 0;
+        c.kb1 = a.KT;
+    } else {
+        c.nt = g % a.NT;
+        c.mt = g / a.NT;
+        c.sp = rank;
+        c.kb0 = rank * a.kbps;
+        c.kb1 = min(a.KT, c.kb0 + a.kbps);
+    }
     return c;
 }
 
@@ -98,8 +121,9 @@ struct Smem {
     uint8_t* x;      // stages x xstage_bytes
     uint8_t* w;      // stages x wstage_bytes
     uint8_t* lrA;    // 16 KB
-    uint8_t* lrB;    // xstage_bytes
+    uint8_t* lrB;    // xsub_bytes
     float* red;      // split partial [128][BN + 4] fp32 (S > 1)
+    uint8_t* stage;  // unsplit: per epilogue warp, a 16-token x 32-channel transpose buffer
     uint64_t* full;    // slot loaded (TMA)
     uint64_t* empty;   // slot consumed (MMA commit + dequant warps); also frees the slot's A stage
     uint64_t* afull;   // slot's A stage written to TMEM (dequant warps)
@@ -141,12 +165,13 @@ __device__ __forceinline__ Sched sched() {
 }
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, const GemmArgs& a,
-                                              volatile int* abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
+                                              volatile int* abort_flag, bool cluster_scope = false) {
+    auto ready = [&]() { return cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+    if (ready()) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         for (int i = 0; i < 64; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+            if (ready()) return true;
         if (*abort_flag) return false;
         if (globaltimer_ns() - t0 > a.timeout_ns) {
             raise_error(ERRBIT_TIMEOUT);
@@ -244,28 +269,36 @@ __device__ __forceinline__ void nibbles_to_f16x2(uint32_t w, __half2 sig, uint32
 }
 
 // ------------------------------------------------------------------- roles
+template <bool PAIR>
 __device__ void producer_role(const GemmArgs& a, const CUtensorMap* tm_x, const CUtensorMap* tm_t,
                               const CUtensorMap* tm_l2, const Smem& s, const Sched& sc) {
+    // in a pair each CTA stages its half of the tile's tokens
+    const int row0 = PAIR ? sc.rank * (a.BN >> 1) : 0;
     int it = 0, lrit = 0;
     Ring r;
     bool ok = true;
     for (int g = sc.cid; g < a.tiles_nm && ok; g += sc.ncl) {
-        const TileCoord c = tile_coord(a, g, sc.rank);
-        for (int kb = c.kb0; kb < c.kb1; ++kb) {
+        const TileCoord c = tile_coord<PAIR>(a, g, sc.rank);
+        for (int kb = c.kb0; kb < c.kb1; kb += a.ks) {
+            const int nkb = min(a.ks, c.kb1 - kb);
             const int st = r.slot;
             if (!wait_or_abort(&s.empty[st], r.phase ^ 1, a, s.abort_flag)) { ok = false; break; }
-            mbar_arrive_expect_tx(&s.full[st], a.xstage_bytes + a.wtile_bytes);
-            tma_load_2d(s.x + st * a.xstage_bytes, tm_x, &s.full[st], kb * 64, c.mt * a.BN);
+            // this CTA's x rows and weight tiles land on its own barrier; in a
+            // pair the dequant warps pass both on to the first CTA's MMA
+            mbar_arrive_expect_tx(&s.full[st], nkb * (a.xsub_bytes + a.wtile_bytes));
+            for (int j = 0; j < nkb; ++j)
+                tma_load_2d(s.x + st * a.xstage_bytes + j * a.xsub_bytes, tm_x, &s.full[st], (kb + j) * 64,
+                            c.mt * a.BN + row0);
             bulk_load(s.w + st * a.wstage_bytes,
                       a.packed + (static_cast<size_t>(c.nt) * a.KT + kb) * a.wtile_bytes,
-                      a.wtile_bytes, &s.full[st]);
+                      nkb * a.wtile_bytes, &s.full[st]);
             ++it;
             r.next(a.stages);
         }
         if (ok && a.lr && c.sp == 0) {
             for (int lk = 0; lk < a.lr_kb; ++lk) {
                 if (!wait_or_abort(s.lrempty, (lrit & 1) ^ 1, a, s.abort_flag)) { ok = false; break; }
-                mbar_arrive_expect_tx(s.lrfull, LR_TILE_A_BYTES + a.xstage_bytes);
+                mbar_arrive_expect_tx(s.lrfull, LR_TILE_A_BYTES + a.xsub_bytes);
                 tma_load_2d(s.lrA, tm_l2, s.lrfull, lk * 64, c.nt * 128);
                 tma_load_2d(s.lrB, tm_t, s.lrfull, lk * 64, c.mt * a.BN);
                 ++lrit;
@@ -280,85 +313,112 @@ __device__ void producer_role(const GemmArgs& a, const CUtensorMap* tm_x, const 
     }
 }
 
-template <int FMT>
+template <int FMT, bool PAIR>
 __device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc, int warp,
                              int lane) {
+    // in a pair, the A stage is consumed by the first CTA's MMA: signal there
+    const uint32_t afull_leader = PAIR ? mapa_shared(smem_u32(s.afull), 0) : 0u;
     const int q = warp & 3;   // TMEM lane quarter this warp may access
     const int h = warp >> 2;  // which 32 of the 64 inputs of a K block
     const int row = q * 32 + lane;
     const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
     Ring r;
     for (int g = sc.cid; g < a.tiles_nm; g += sc.ncl) {
-        const TileCoord c = tile_coord(a, g, sc.rank);
-        for (int kb = c.kb0; kb < c.kb1; ++kb, r.next(a.stages)) {
+        const TileCoord c = tile_coord<PAIR>(a, g, sc.rank);
+        for (int kb = c.kb0; kb < c.kb1; kb += a.ks, r.next(a.stages)) {
+            const int nkb = min(a.ks, c.kb1 - kb);
             const int st = r.slot;
             if (!warp_wait_or_abort(&s.full[st], r.phase, a, s.abort_flag)) return;
-            const uint8_t* blk = s.w + st * a.wstage_bytes;
-            uint4 c0, c1 = make_uint4(0, 0, 0, 0);
-            __half2 sig0, sig1;
-            if constexpr (FMT == FMT_W8) {
-                c0 = *reinterpret_cast<const uint4*>(blk + (2 * h) * 2048 + 16 * row);
-                c1 = *reinterpret_cast<const uint4*>(blk + (2 * h + 1) * 2048 + 16 * row);
-            } else {
-                c0 = *reinterpret_cast<const uint4*>(blk + h * 2048 + 16 * row);
-                if constexpr (FMT == FMT_W4G64) {
-                    const __half sg = *reinterpret_cast<const __half*>(blk + 4096 + 2 * row);
-                    sig0 = __half2half2(sg);
-                    sig1 = sig0;
-                } else {
-                    const __half2 sp = *reinterpret_cast<const __half2*>(blk + 4096 + 512 * h + 4 * row);
-                    sig0 = __half2half2(__low2half(sp));
-                    sig1 = __half2half2(__high2half(sp));
+            // The slot's A stage is free: this round's load was issued only after
+            // the previous round's MMA committed.
+            tc_fence_after();
+            const uint32_t acol = tbase + a.a_col0 + st * a.ks * A_STAGE_COLS + h * 16;
+            // read every code (and scale) of the slot first, then release the
+            // weight tiles to the producer before converting
+            constexpr int CW = (FMT == FMT_W8) ? 2 : 1;  // 16-byte code vectors per block per lane
+            uint4 cv[MAX_KS][CW];
+            __half2 sg[MAX_KS][2];
+#pragma unroll
+            for (int j = 0; j < MAX_KS; ++j) {
+                if (j < nkb) {
+                    const uint8_t* blk = s.w + st * a.wstage_bytes + j * a.wtile_bytes;
+                    if constexpr (FMT == FMT_W8) {
+                        cv[j][0] = *reinterpret_cast<const uint4*>(blk + (2 * h) * 2048 + 16 * row);
+                        cv[j][CW - 1] = *reinterpret_cast<const uint4*>(blk + (2 * h + 1) * 2048 + 16 * row);
+                    } else {
+                        cv[j][0] = *reinterpret_cast<const uint4*>(blk + h * 2048 + 16 * row);
+                        if constexpr (FMT == FMT_W4G64) {
+                            sg[j][0] = __half2half2(*reinterpret_cast<const __half*>(blk + 4096 + 2 * row));
+                            sg[j][1] = sg[j][0];
+                        } else {
+                            const __half2 sp = *reinterpret_cast<const __half2*>(blk + 4096 + 512 * h + 4 * row);
+                            sg[j][0] = __half2half2(__low2half(sp));
+                            sg[j][1] = __half2half2(__high2half(sp));
+                        }
+                    }
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.empty[st]);
-            // The slot's A stage is free: this round's load was issued only after
-            // the previous round's MMA committed.
-            tc_fence_after();
-            uint32_t v[16];
-            if constexpr (FMT == FMT_W8) {
-                convert_w8(c0, c1, v);
-            } else {
-                nibbles_to_f16x2(c0.x, sig0, v + 0);
-                nibbles_to_f16x2(c0.y, sig0, v + 4);
-                nibbles_to_f16x2(c0.z, sig1, v + 8);
-                nibbles_to_f16x2(c0.w, sig1, v + 12);
+#pragma unroll
+            for (int j = 0; j < MAX_KS; ++j) {
+                if (j < nkb) {
+                    uint32_t v[16];
+                    if constexpr (FMT == FMT_W8) {
+                        convert_w8(cv[j][0], cv[j][CW - 1], v);
+                    } else {
+                        nibbles_to_f16x2(cv[j][0].x, sg[j][0], v + 0);
+                        nibbles_to_f16x2(cv[j][0].y, sg[j][0], v + 4);
+                        nibbles_to_f16x2(cv[j][0].z, sg[j][1], v + 8);
+                        nibbles_to_f16x2(cv[j][0].w, sg[j][1], v + 12);
+                    }
+                    tmem_st16(acol + j * A_STAGE_COLS, v);
+                }
             }
-            tmem_st16(tbase + a.a_col0 + st * A_STAGE_COLS + h * 16, v);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s.afull[st]);
+            if (lane == 0) {
+                if (PAIR && sc.rank != 0) mbar_arrive_peer(afull_leader + st * 8u);
+                else mbar_arrive(&s.afull[st]);
+            }
         }
     }
 }
 
-template <int FMT>
+template <int FMT, bool PAIR>
 __device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc) {
-    const uint32_t idesc = idesc_f16(FMT == FMT_W8 ? 1u : 0u, 128, a.BN);
+    const uint32_t idesc = idesc_f16(FMT == FMT_W8 ? 1u : 0u, PAIR ? 256 : 128, a.BN);
+    // pair commits signal the same barrier in both CTAs
     const uint32_t idesc_lr = idesc_f16(1u, 128, a.BN);
     int lrit = 0, tc = 0;
     Ring r;
     bool ok = true;
     for (int g = sc.cid; g < a.tiles_nm && ok; g += sc.ncl, ++tc) {
-        const TileCoord c = tile_coord(a, g, sc.rank);
+        const TileCoord c = tile_coord<PAIR>(a, g, sc.rank);
         const int ab = tc % a.acc_bufs;
         if (!wait_or_abort(&s.accempty[ab], ((tc / a.acc_bufs) & 1) ^ 1, a, s.abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem + a.acc_col0 + ab * a.BN;
-        for (int kb = c.kb0; kb < c.kb1 && ok; ++kb, r.next(a.stages)) {
+        for (int kb = c.kb0; kb < c.kb1 && ok; kb += a.ks, r.next(a.stages)) {
+            const int nkb = min(a.ks, c.kb1 - kb);
             const int st = r.slot;
-            // afull is reached only after every dequant warp observed the slot
-            // full, so it orders the slot's x tile before the MMA as well
+            // afull is reached only after every dequant warp (of both CTAs of a
+            // pair) observed its slot full, so it orders the x tiles as well
             if (!wait_or_abort(&s.afull[st], r.phase, a, s.abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const uint64_t bdesc = smem_desc_sw128(smem_u32(s.x + st * a.xstage_bytes));
+            const uint32_t acol = tmem + a.a_col0 + st * a.ks * A_STAGE_COLS;
+            for (int j = 0; j < nkb; ++j) {
+                const uint64_t bdesc = smem_desc_sw128(smem_u32(s.x + st * a.xstage_bytes + j * a.xsub_bytes));
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_ts(d, tmem + a.a_col0 + st * A_STAGE_COLS + kk * 8, bdesc + 2 * kk, idesc,
-                       (kb > c.kb0 || kk > 0) ? 1u : 0u);
-            mma_commit(&s.empty[st]);
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint32_t acc = (kb > c.kb0 || j > 0 || kk > 0) ? 1u : 0u;
+                    if constexpr (PAIR) mma_ts_pair(d, acol + j * A_STAGE_COLS + kk * 8, bdesc + 2 * kk, idesc, acc);
+                    else mma_ts(d, acol + j * A_STAGE_COLS + kk * 8, bdesc + 2 * kk, idesc, acc);
+                }
+            }
+            if constexpr (PAIR) mma_commit_pair_both(&s.empty[st]);
+            else mma_commit(&s.empty[st]);
         }
         if (!ok) break;
         if (a.lr && c.sp == 0) {
@@ -375,10 +435,12 @@ __device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const 
             }
             if (!ok) break;
         }
-        mma_commit(&s.accfull[ab]);
+        if constexpr (PAIR) mma_commit_pair_both(&s.accfull[ab]);
+        else mma_commit(&s.accfull[ab]);
     }
     // make sure no MMA is still reading shared memory or TMEM when the CTA tears down
-    mma_commit(s.drain);
+    if constexpr (PAIR) mma_commit_pair(s.drain);
+    else mma_commit(s.drain);
     mbar_wait(s.drain, 0, DRAIN_TIMEOUT_NS);
 }
 
@@ -388,9 +450,11 @@ __device__ __forceinline__ void store_y(const GemmArgs& a, int m, int n, float v
     else static_cast<__nv_bfloat16*>(a.y)[o] = __float2bfloat16_rn(v);
 }
 
-template <int FMT>
+template <int FMT, bool PAIR>
 __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc, int warp,
                               int lane) {
+    // in a pair the accumulator is released to the first CTA's MMA thread
+    const uint32_t accempty_leader = PAIR ? mapa_shared(smem_u32(s.accempty), 0) : 0u;
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
@@ -409,7 +473,7 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
     const int red_pitch = a.BN + 4;     // floats per row of the partial buffer (keeps float4 alignment)
     int tc = 0;
     for (int g = sc.cid; g < a.tiles_nm; g += sc.ncl, ++tc) {
-        const TileCoord c = tile_coord(a, g, sc.rank);
+        const TileCoord c = tile_coord<PAIR>(a, g, sc.rank);
         const int ab = tc % a.acc_bufs;
         if (!warp_wait_or_abort(&s.accfull[ab], (tc / a.acc_bufs) & 1, a, s.abort_flag, false, true)) return;
         tc_fence_after();
@@ -421,11 +485,9 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
         const int m0 = c.mt * a.BN;
         // the partial buffer is reused once every CTA of the cluster has read it
         if (split && tc > 0 && !warp_wait_or_abort(s.freed, (tc - 1) & 1, a, s.abort_flag, true)) return;
-        for (int cc = 0; cc < a.BN / 16; ++cc) {
-            uint32_t v[16], lv[16];
-            tmem_ld16(tbase + a.acc_col0 + ab * a.BN + cc * 16, v);
-            if (has_lr) tmem_ld16(tbase + a.lr_col0 + ab * a.BN + cc * 16, lv);
-            tmem_wait_ld();
+        // One 16-token chunk of this lane's channel: scale, add the low-rank
+        // term, then store (split partial, staged 16-byte runs, or scalar).
+        auto emit = [&](const uint32_t (&v)[16], const uint32_t (&lv)[16], int cc) {
             float val[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -439,6 +501,52 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     dst[j] = make_float4(val[4 * j], val[4 * j + 1], val[4 * j + 2], val[4 * j + 3]);
+            } else if (a.vec_out) {
+                // Each lane holds one channel for 16 tokens; y is token-major.  Turn
+                // the 16 x 32 block around in shared memory so that every lane stores
+                // whole 16-byte runs of a token's row (channels beyond N hold zeros
+                // and are not stored: N is a multiple of the run length).
+                const int mb = m0 + cc * 16;
+                const int nb = c.nt * 128 + q * 32;
+                uint8_t* stg = s.stage + (warp - WARP_EPI0) * EPI_STAGE_BYTES;
+                if (a.y_f32) {
+                    float* sf = reinterpret_cast<float*>(stg);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) sf[j * 32 + lane] = val[j] + bn;
+                    __syncwarp();
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const int ci = lane + 32 * p, m = mb + (ci >> 3), nn = nb + (ci & 7) * 4;
+                        const float4 v4 = *reinterpret_cast<const float4*>(stg + ci * 16);
+                        if (m < a.M && nn < a.N)
+                            *reinterpret_cast<float4*>(static_cast<float*>(a.y) + static_cast<size_t>(m) * a.N + nn) = v4;
+                    }
+                } else {
+                    // Lane pairs (channels 2i, 2i+1) swap halves so that each lane
+                    // packs both channels of one token into a bf16 pair: even lanes
+                    // take tokens 0-7, odd lanes 8-15.  Token rows are 64 bytes;
+                    // rows 8-15 sit one row further on, so the two halves of a
+                    // warp's stores fall in different banks.
+                    const bool odd = lane & 1;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float mine = (odd ? val[j + 8] : val[j]) + bn;
+                        const float other = __shfl_xor_sync(0xffffffffu, (odd ? val[j] : val[j + 8]) + bn, 1);
+                        const __nv_bfloat162 pr = odd ? __floats2bfloat162_rn(other, mine)
+                                                      : __floats2bfloat162_rn(mine, other);
+                        const int t = odd ? j + 8 : j;
+                        *reinterpret_cast<__nv_bfloat162*>(stg + t * 64 + (t >> 3) * 64 + (lane & ~1) * 2) = pr;
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        const int ci = lane + 32 * p, t = ci >> 2, nn = nb + (ci & 3) * 8, m = mb + t;
+                        const uint4 v4 = *reinterpret_cast<const uint4*>(stg + t * 64 + (t >> 3) * 64 + (ci & 3) * 16);
+                        if (m < a.M && nn < a.N)
+                            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.y) + static_cast<size_t>(m) * a.N + nn) = v4;
+                    }
+                }
+                __syncwarp();
             } else if (n_ok) {
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
@@ -446,10 +554,40 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
                     if (m < a.M) store_y(a, m, n, val[j] + bn);
                 }
             }
+        };
+        const int nch = a.BN / 16;
+        if (has_lr) {
+            for (int cc = 0; cc < nch; ++cc) {
+                uint32_t v[16], lv[16];
+                tmem_ld16(tbase + a.acc_col0 + ab * a.BN + cc * 16, v);
+                tmem_ld16(tbase + a.lr_col0 + ab * a.BN + cc * 16, lv);
+                tmem_wait_ld_pin(v);
+                reg_pin(lv);
+                emit(v, lv, cc);
+            }
+        } else {
+            // two register sets: chunk cc + 1 is read from tensor memory while
+            // chunk cc is stored
+            const uint32_t col = tbase + a.acc_col0 + ab * a.BN;
+            uint32_t va[16], vb[16];
+            tmem_ld16(col, va);
+            tmem_wait_ld_pin(va);
+            for (int cc = 0; cc < nch; cc += 2) {
+                if (cc + 1 < nch) tmem_ld16(col + (cc + 1) * 16, vb);
+                emit(va, va, cc);
+                if (cc + 1 >= nch) break;
+                tmem_wait_ld_pin(vb);
+                if (cc + 2 < nch) tmem_ld16(col + (cc + 2) * 16, va);
+                emit(vb, vb, cc + 1);
+                tmem_wait_ld_pin(va);
+            }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&s.accempty[ab]);
+        if (lane == 0) {
+            if (PAIR && sc.rank != 0) mbar_arrive_peer(accempty_leader + ab * 8u);
+            else mbar_arrive(&s.accempty[ab]);
+        }
         if (!split) continue;
 
         // publish this CTA's partial to the cluster
@@ -497,7 +635,7 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
     if (split && tc > 0) warp_wait_or_abort(s.freed, (tc - 1) & 1, a, s.abort_flag, true);
 }
 
-template <int FMT>
+template <int FMT, bool PAIR>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_t,
             const __grid_constant__ CUtensorMap tm_l2, const GemmArgs a) {
@@ -509,8 +647,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     s.w = s.x + static_cast<size_t>(a.stages) * a.xstage_bytes;
     s.lrA = s.w + static_cast<size_t>(a.stages) * a.wstage_bytes;
     s.lrB = s.lrA + (a.lr ? LR_TILE_A_BYTES : 0);
-    s.red = reinterpret_cast<float*>(s.lrB + (a.lr ? a.xstage_bytes : 0));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(s.red) + a.red_bytes);
+    s.red = reinterpret_cast<float*>(s.lrB + (a.lr ? a.xsub_bytes : 0));
+    s.stage = reinterpret_cast<uint8_t*>(s.red) + a.red_bytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(s.stage + a.stage_bytes);
     s.full = bars;
     s.empty = s.full + a.stages;
     s.afull = s.empty + a.stages;
@@ -532,11 +671,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
         for (int i = 0; i < a.stages; ++i) {
             mbar_init(&s.full[i], 1);
             mbar_init(&s.empty[i], 1 + NUM_DQ_WARPS);
-            mbar_init(&s.afull[i], NUM_DQ_WARPS);
+            mbar_init(&s.afull[i], PAIR ? 2 * NUM_DQ_WARPS : NUM_DQ_WARPS);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.accfull[i], 1);
-            mbar_init(&s.accempty[i], NUM_EPI_WARPS);
+            mbar_init(&s.accempty[i], PAIR ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS);
         }
         mbar_init(s.lrfull, 1);
         mbar_init(s.lrempty, 1);
@@ -556,32 +695,36 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
             prefetch_tensormap(&tm_l2);
         }
     }
-    if (warp == WARP_MMA) tmem_alloc(s.tmem_slot, a.tmem_cols);
+    if (warp == WARP_MMA) {
+        if constexpr (PAIR) tmem_alloc_pair(s.tmem_slot, a.tmem_cols);
+        else tmem_alloc(s.tmem_slot, a.tmem_cols);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (a.S > 1) {
-        // every CTA of the cluster has initialised its barriers before any remote arrive
-        asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-    }
+    // every CTA of the cluster has initialised its barriers before any remote arrive
+    if (PAIR || a.S > 1) cluster_sync_all();
     const uint32_t tmem = *s.tmem_slot;
     const Sched sc = sched();
 
     if (warp < NUM_DQ_WARPS) {
-        dequant_role<FMT>(a, tmem, s, sc, warp, lane);
+        dequant_role<FMT, PAIR>(a, tmem, s, sc, warp, lane);
     } else if (warp < WARP_PRODUCER) {
-        epilogue_role<FMT>(a, tmem, s, sc, warp, lane);
+        epilogue_role<FMT, PAIR>(a, tmem, s, sc, warp, lane);
     } else if (warp == WARP_PRODUCER) {
-        if (lane == 0) producer_role(a, &tm_x, &tm_t, &tm_l2, s, sc);
-    } else if (lane == 0) {
-        mma_role<FMT>(a, tmem, s, sc);
+        if (lane == 0) producer_role<PAIR>(a, &tm_x, &tm_t, &tm_l2, s, sc);
+    } else if (lane == 0 && (!PAIR || sc.rank == 0)) {
+        mma_role<FMT, PAIR>(a, tmem, s, sc);
     }
 
     tc_fence_before();
     __syncthreads();
+    // a pair's CTAs signal each other's barriers and TMEM: neither leaves first
+    if constexpr (PAIR) cluster_sync_all();
     if (warp == WARP_MMA) {
         tc_fence_after();
-        tmem_dealloc(tmem, a.tmem_cols);
+        if constexpr (PAIR) tmem_dealloc_pair(tmem, a.tmem_cols);
+        else tmem_dealloc(tmem, a.tmem_cols);
     }
 }
 

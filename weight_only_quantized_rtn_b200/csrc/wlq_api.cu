@@ -49,7 +49,7 @@ int fmt_of(int bits, int group) {
 struct DeviceInfo {
     int checked = 0;  // 0 unknown, 1 supported, -1 not
     int sms = 0;
-    bool smem_set[3] = {false, false, false};
+    bool smem_set[6] = {false, false, false, false, false, false};
     // resident clusters per (format, cluster size, dynamic smem), queried once
     std::unordered_map<uint64_t, int> max_clusters;
 };
@@ -123,8 +123,9 @@ struct Plan {
     int fmt = -1;
     int M = 0, N = 0, K = 0, r = 0;
     int NT = 0, KT = 0, MT = 0, S = 1, kbps = 0, BN = 0, tiles_nm = 0, grid = 0;
-    int stages = 0, lr_kb = 0, acc_bufs = 1;
-    uint32_t tmem_cols = 0, acc_col0 = 0, lr_col0 = 0, a_col0 = 0, wtile = 0, wstage = 0, xstage = 0, red = 0;
+    int stages = 0, ks = 1, lr_kb = 0, acc_bufs = 1;
+    bool pair = false;  // two CTAs per MMA (cta_group::2)
+    uint32_t tmem_cols = 0, acc_col0 = 0, lr_col0 = 0, a_col0 = 0, wtile = 0, wstage = 0, xsub = 0, xstage = 0, red = 0, stage = 0;
     size_t smem = 0;
     size_t off_x16 = 0, off_xs = 0, off_thl = 0, off_l2t = 0, ws = 0;
 };
@@ -172,34 +173,50 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     }
     p.S = S;
     if (S > 1 && p.BN % (4 * S) != 0) return false;  // the reduction's token quads must not straddle shares
-    p.tiles_nm = p.NT * p.MT;
+    // CTA pairs for large token tiles: two 128-channel tiles share each MMA
+    p.pair = (r == 0 && S == 1 && p.BN == 256 && p.NT % 2 == 0);
+    p.tiles_nm = p.pair ? (p.NT / 2) * p.MT : p.NT * p.MT;
     // TMEM: accumulator(s) first, from column 0, so each starts at a multiple
     // of its own width (main accumulators at ab*BN, low-rank ones after them);
-    // then one 32-column A stage per ring slot.  The accumulators are
-    // double-buffered when that still leaves room for four slots.
+    // then a ks * 32-column A stage per ring slot.  The accumulators are
+    // double-buffered when that still leaves room for four 32-column blocks.
     const uint32_t acc_cols = static_cast<uint32_t>(p.BN) * (r ? 2u : 1u);
     if (acc_cols + 2 * wlq::A_STAGE_COLS > 512) return false;
     p.acc_bufs = (2 * acc_cols + 4 * wlq::A_STAGE_COLS <= 512) ? 2 : 1;
     const uint32_t acc_total = p.acc_bufs * acc_cols;
     const uint32_t a_col0 = (acc_total + wlq::A_STAGE_COLS - 1) / wlq::A_STAGE_COLS * wlq::A_STAGE_COLS;
-    const int tmem_slots = static_cast<int>((512 - a_col0) / wlq::A_STAGE_COLS);
     // shared memory: ring slots + low-rank tiles + split partial + barriers
     p.wtile = wlq::tile_bytes(fmt);
-    p.wstage = (p.wtile + 1023u) & ~1023u;
-    p.xstage = static_cast<uint32_t>(p.BN) * 128u;
+    p.xsub = static_cast<uint32_t>(p.pair ? p.BN / 2 : p.BN) * 128u;  // a pair's CTA stages half the tokens
     p.red = (S > 1) ? 128u * static_cast<uint32_t>(p.BN + 4) * 4u : 0u;
-    const size_t lr_bytes = r ? (wlq::LR_TILE_A_BYTES + p.xstage) : 0;
-    const size_t fixed = 1024 /* alignment */ + 1024 /* barriers */ + lr_bytes + p.red;
-    const size_t per_stage = p.xstage + p.wstage;
-    if (fixed + 2 * per_stage > kSmemLimit) return false;
-    const int smem_slots = static_cast<int>((kSmemLimit - fixed) / per_stage);
-    p.stages = std::min({wlq::MAX_STAGES, tmem_slots, smem_slots});
-    if (p.stages < 2) return false;
-    p.smem = fixed + p.stages * per_stage;
+    const size_t lr_bytes = r ? (wlq::LR_TILE_A_BYTES + p.xsub) : 0;
+    p.stage = (S == 1) ? wlq::NUM_EPI_WARPS * wlq::EPI_STAGE_BYTES : 0u;  // epilogue transpose buffers
+    const size_t fixed = 1024 /* alignment */ + 1024 /* barriers */ + lr_bytes + p.red + p.stage;
+    // K blocks per ring slot: the largest of 4, 2, 1 that still leaves three
+    // slots in both TMEM and shared memory (one handshake per slot)
+    p.ks = 0;
+    for (int ks : {4, 2, 1}) {
+        const uint32_t wstage = (static_cast<uint32_t>(ks) * p.wtile + 1023u) & ~1023u;
+        const uint32_t xstage = static_cast<uint32_t>(ks) * p.xsub;
+        const size_t per_stage = xstage + wstage;
+        if (fixed + 2 * per_stage > kSmemLimit) continue;
+        const int tmem_slots = static_cast<int>((512 - a_col0) / (static_cast<uint32_t>(ks) * wlq::A_STAGE_COLS));
+        const int smem_slots = static_cast<int>((kSmemLimit - fixed) / per_stage);
+        const int stages = std::min({wlq::MAX_STAGES, tmem_slots, smem_slots});
+        if (stages >= 3 || (ks == 1 && stages >= 2)) {
+            p.ks = ks;
+            p.stages = stages;
+            p.wstage = wstage;
+            p.xstage = xstage;
+            p.smem = fixed + stages * per_stage;
+            break;
+        }
+    }
+    if (p.ks == 0) return false;
     p.acc_col0 = 0;
     p.lr_col0 = p.acc_bufs * static_cast<uint32_t>(p.BN);
     p.a_col0 = a_col0;
-    const uint32_t need = a_col0 + static_cast<uint32_t>(p.stages) * wlq::A_STAGE_COLS;
+    const uint32_t need = a_col0 + static_cast<uint32_t>(p.stages * p.ks) * wlq::A_STAGE_COLS;
     p.tmem_cols = 32;
     while (p.tmem_cols < need) p.tmem_cols <<= 1;
     // workspace
@@ -227,16 +244,18 @@ wlq_status check_shape(int64_t N, int64_t K, int bits, int group) {
 
 int g_grid_limit = 0;  // 0: no cap on the GEMM's CTAs (see wlq_set_grid_limit)
 
-template <int FMT>
+template <int FMT, bool PAIR>
 wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, const CUtensorMap& tl,
                        wlq::GemmArgs& a, DeviceInfo* d, cudaStream_t st) {
-    auto kern = wlq::gemm_kernel<FMT>;
-    if (!d->smem_set[FMT]) {
+    auto kern = wlq::gemm_kernel<FMT, PAIR>;
+    const int kid = FMT * 2 + (PAIR ? 1 : 0);
+    if (!d->smem_set[kid]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(kSmemLimit));
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-        d->smem_set[FMT] = true;
+        d->smem_set[kid] = true;
     }
+    const int csize = PAIR ? 2 : p.S;  // CTAs per cluster
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
     cudaLaunchAttribute attr[1];
@@ -244,16 +263,16 @@ wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, co
     cfg.dynamicSmemBytes = p.smem;
     cfg.stream = st;
     const int cta_cap = (g_grid_limit > 0) ? std::min(g_grid_limit, d->sms) : d->sms;
-    int clusters = std::max(1, std::min(p.tiles_nm, cta_cap / p.S));
-    if (p.S > 1) {
+    int clusters = std::max(1, std::min(p.tiles_nm, cta_cap / csize));
+    if (csize > 1) {
         attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = static_cast<unsigned>(p.S);
+        attr[0].val.clusterDim.x = static_cast<unsigned>(csize);
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         // persistent clusters: no more than can be resident at once
-        const uint64_t key = (static_cast<uint64_t>(FMT) << 48) | (static_cast<uint64_t>(p.S) << 32) | p.smem;
+        const uint64_t key = (static_cast<uint64_t>(kid) << 48) | (static_cast<uint64_t>(csize) << 32) | p.smem;
         int active = 0;
         {
             std::lock_guard<std::mutex> lk(g_dev_mu);
@@ -261,18 +280,18 @@ wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, co
             if (it != d->max_clusters.end()) active = it->second;
         }
         if (active == 0) {
-            cfg.gridDim = dim3(static_cast<unsigned>(clusters * p.S), 1, 1);
+            cfg.gridDim = dim3(static_cast<unsigned>(clusters * csize), 1, 1);
             if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) != cudaSuccess || active <= 0) {
                 cudaGetLastError();
-                active = d->sms / p.S;
+                active = d->sms / csize;
             }
             std::lock_guard<std::mutex> lk(g_dev_mu);
             d->max_clusters[key] = active;
         }
         clusters = std::min(clusters, active);
     }
-    cfg.gridDim = dim3(static_cast<unsigned>(clusters * p.S), 1, 1);
-    p.grid = clusters * p.S;
+    cfg.gridDim = dim3(static_cast<unsigned>(clusters * csize), 1, 1);
+    p.grid = clusters * csize;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tx, tt, tl, a);
     if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
     return WLQ_OK;
@@ -447,7 +466,7 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
     CUtensorMap tx, tt, tl;
     std::memset(&tt, 0, sizeof tt);
     std::memset(&tl, 0, sizeof tl);
-    if ((st = make_map_2d(&tx, xin, M, K, p.BN)) != WLQ_OK) return st;
+    if ((st = make_map_2d(&tx, xin, M, K, p.pair ? p.BN / 2 : p.BN)) != WLQ_OK) return st;
     if (r) {
         if ((st = make_map_2d(&tt, thl, M, W, p.BN)) != WLQ_OK) return st;
         if ((st = make_map_2d(&tl, l2t, NT * 128, W, 128)) != WLQ_OK) return st;
@@ -461,16 +480,22 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
     a.y = y;
     a.M = p.M; a.N = p.N; a.K = p.K;
     a.NT = p.NT; a.KT = p.KT; a.MT = p.MT; a.S = p.S; a.kbps = p.kbps; a.BN = p.BN;
-    a.stages = p.stages; a.lr = r ? 1 : 0; a.lr_kb = p.lr_kb; a.acc_bufs = p.acc_bufs;
+    a.stages = p.stages; a.ks = p.ks; a.lr = r ? 1 : 0; a.lr_kb = p.lr_kb; a.acc_bufs = p.acc_bufs;
     a.y_f32 = (y_dtype == WLQ_OUT_F32) ? 1 : 0;
     a.tiles_nm = p.tiles_nm;
     a.tmem_cols = p.tmem_cols; a.acc_col0 = p.acc_col0; a.lr_col0 = p.lr_col0; a.a_col0 = p.a_col0;
-    a.wtile_bytes = p.wtile; a.wstage_bytes = p.wstage; a.xstage_bytes = p.xstage; a.red_bytes = p.red;
+    a.wtile_bytes = p.wtile; a.wstage_bytes = p.wstage; a.xsub_bytes = p.xsub; a.xstage_bytes = p.xstage; a.red_bytes = p.red;
+    a.stage_bytes = p.stage;
+    a.vec_out = (p.S == 1 && (reinterpret_cast<uintptr_t>(y) & 15u) == 0 &&
+                 (y_dtype == WLQ_OUT_F32 ? N % 4 == 0 : N % 8 == 0)) ? 1 : 0;
     a.timeout_ns = kDefaultTimeoutNs;
-    switch (fmt) {
-        case wlq::FMT_W8: return launch_gemm<wlq::FMT_W8>(p, tx, tt, tl, a, d, s);
-        case wlq::FMT_W4G64: return launch_gemm<wlq::FMT_W4G64>(p, tx, tt, tl, a, d, s);
-        default: return launch_gemm<wlq::FMT_W4G16>(p, tx, tt, tl, a, d, s);
+    switch (fmt * 2 + (p.pair ? 1 : 0)) {
+        case 0: return launch_gemm<wlq::FMT_W8, false>(p, tx, tt, tl, a, d, s);
+        case 1: return launch_gemm<wlq::FMT_W8, true>(p, tx, tt, tl, a, d, s);
+        case 2: return launch_gemm<wlq::FMT_W4G64, false>(p, tx, tt, tl, a, d, s);
+        case 3: return launch_gemm<wlq::FMT_W4G64, true>(p, tx, tt, tl, a, d, s);
+        case 4: return launch_gemm<wlq::FMT_W4G16, false>(p, tx, tt, tl, a, d, s);
+        default: return launch_gemm<wlq::FMT_W4G16, true>(p, tx, tt, tl, a, d, s);
     }
 }
 
