@@ -232,17 +232,28 @@ def run_gpu(args):
     torch.cuda.synchronize()
     wlq.check_status()
 
-    # The step runs as CUDA-graph replays (one graph per phase, so that events
-    # between replays time each phase) to keep host launch overhead off the
-    # device timeline.
+    # The step runs as one CUDA-graph replay (host launch overhead off the
+    # device timeline).  Timing events recorded inside the graph split the
+    # replay into its phases; events around the replay time the whole step.
+    phases = ["qp"] + list(MS)
+    inner = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(phases) + 1)]
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step):
+        inner[0].record()
+        quantize_pack()
+        inner[1].record()
+        for j, M in enumerate(MS):
+            linear(M)
+            inner[j + 2].record()
     graphs = {}
-    for name, fn in [("qp", quantize_pack)] + [(M, (lambda M=M: linear(M))) for M in MS]:
+    for M in MS:  # one graph per Linear, for the isolated timings
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            fn()
-        graphs[name] = g
+            linear(M)
+        graphs[M] = g
     torch.cuda.synchronize()
     for _ in range(2):
+        g_step.replay()
         for g in graphs.values():
             g.replay()
     torch.cuda.synchronize()
@@ -251,18 +262,20 @@ def run_gpu(args):
         dist.barrier()
     torch.cuda.synchronize()
 
-    phases = ["qp"] + list(MS)
     sampler = ClockSampler(local)
     sampler.start()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(phases) + 1)] for _ in range(args.steps)]
+    outer = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    phase_ms = {ph: 0.0 for ph in phases}
     for i in range(args.steps):
         flush.zero_()  # evict L2 between steps (outside the timed events)
         torch.cuda.nvtx.range_push("timed_step")
-        evs[i][0].record(stream)
-        for j, ph in enumerate(phases):
-            graphs[ph].replay()
-            evs[i][j + 1].record(stream)
+        outer[i][0].record(stream)
+        g_step.replay()
+        outer[i][1].record(stream)
         torch.cuda.nvtx.range_pop()
+        torch.cuda.synchronize()  # the in-graph events are re-recorded by the next replay
+        for j, ph in enumerate(phases):
+            phase_ms[ph] += inner[j].elapsed_time(inner[j + 1]) / args.steps
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -270,8 +283,8 @@ def run_gpu(args):
     clocks = sampler.stop()
     wlq.check_status()
 
-    ms_step = sum(e[0].elapsed_time(e[-1]) for e in evs) / args.steps
-    per_ms = {ph: sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j, ph in enumerate(phases)}
+    ms_step = sum(a.elapsed_time(c) for a, c in outer) / args.steps
+    per_ms = phase_ms
     per_m_ms = {M: per_ms[M] for M in MS}
     if dist:
         t = torch.tensor([ms_step] + [per_m_ms[M] for M in MS], dtype=torch.float64, device=dev)
@@ -347,7 +360,8 @@ def run_gpu(args):
             "data": "synthetic",
             "config": {"workload": WORKLOAD, "M": list(MS), "N": N_OUT, "K": K_IN, "bits": BITS,
                        "group": "per-channel", "out": "bf16", "parallelism": "replicas x%d" % world,
-                       "l2": "flushed between steps (256 MiB write outside the timed events)"},
+                       "l2": "flushed between steps (256 MiB write outside the timed events)",
+                       "timing": "one CUDA-graph replay per step between CUDA events; phases split by events recorded inside the graph"},
             "per_m": per_m, "roofline": roof, "clocks": clocks,
             "quantize_pack_us": round(per_ms["qp"] * 1e3, 2),
             "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",

@@ -77,7 +77,10 @@ def test_parity_low_rank(bits, group, r, M):
     (40, 1100, 320, 0, 4),     # 9 tiles on 4 CTAs: both accumulator buffers in use
     (16, 33000, 128, 0, 16),   # 258 tiles of 16 tokens on 16 CTAs
     (300, 700, 256, 0, 3),     # 128-token tiles, several per CTA
-    (16, 1024, 2048, 0, 16),   # K split over clusters, each cluster several tiles
+    (16, 1024, 2048, 0, 4),    # K split over clusters, each cluster several tiles
+    (16, 4096, 1024, 0, 8),    # warp-MMA kernel: K split over pairs, eight tiles per cluster
+    (32, 1001, 512, 0, 3),     # warp-MMA kernel: ragged N (scalar stores), one cluster for all tiles
+    (64, 2048, 1024, 0, 8),    # resident-x tensor-core kernel: K split over 4, several tiles per cluster
     (100, 1024, 512, 32, 4),   # low rank + K split, several tiles per cluster
     (600, 640, 640, 16, 5),    # low rank, single accumulator buffer, ring wrap-around
     (600, 4096, 448, 0, 0),    # CTA pairs (256 channels x 256 tokens per MMA), partial last slot

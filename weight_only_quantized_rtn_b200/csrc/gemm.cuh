@@ -67,7 +67,7 @@ constexpr int WARP_PRODUCER = NUM_DQ_WARPS + NUM_EPI_WARPS;
 constexpr int WARP_MMA = WARP_PRODUCER + 1;
 constexpr int GEMM_THREADS = (WARP_MMA + 1) * 32;
 constexpr uint32_t A_STAGE_COLS = 32;  // 128 lanes x 64 16-bit values
-constexpr int MAX_STAGES = 16;
+constexpr int MAX_STAGES = 20;  // ring depth cap (barrier arrays are sized for it)
 constexpr uint32_t LR_TILE_A_BYTES = 128 * 128;  // 128 rows x 64 bf16
 constexpr uint64_t DRAIN_TIMEOUT_NS = 200ull * 1000 * 1000;
 constexpr int MAX_SPLITS = 8;
@@ -83,6 +83,7 @@ struct GemmArgs {
     int M, N, K;
     int NT, KT, MT, S, kbps, BN;
     int stages, ks, lr, lr_kb, acc_bufs, y_f32;  // ks: 64-wide K blocks per ring slot
+    int astages;  // resident-x kernels: depth of the TMEM A-stage ring (stages: weight ring)
     int tiles_nm;
     uint32_t tmem_cols, acc_col0, lr_col0, a_col0;
     uint32_t wtile_bytes, wstage_bytes, xsub_bytes, xstage_bytes, red_bytes, stage_bytes;
@@ -127,6 +128,8 @@ struct Smem {
     uint64_t* full;    // slot loaded (TMA)
     uint64_t* empty;   // slot consumed (MMA commit + dequant warps); also frees the slot's A stage
     uint64_t* afull;   // slot's A stage written to TMEM (dequant warps)
+    uint64_t* aempty;  // resident x: A stage consumed (MMA commit)
+    uint64_t* xfull;   // resident x: the CTA's x rows landed
     uint64_t* accfull;
     uint64_t* accempty;
     uint64_t* lrfull;
@@ -269,7 +272,7 @@ __device__ __forceinline__ void nibbles_to_f16x2(uint32_t w, __half2 sig, uint32
 }
 
 // ------------------------------------------------------------------- roles
-template <bool PAIR>
+template <bool PAIR, bool XRES>
 __device__ void producer_role(const GemmArgs& a, const CUtensorMap* tm_x, const CUtensorMap* tm_t,
                               const CUtensorMap* tm_l2, const Smem& s, const Sched& sc) {
     // in a pair each CTA stages its half of the tile's tokens
@@ -277,18 +280,31 @@ __device__ void producer_role(const GemmArgs& a, const CUtensorMap* tm_x, const 
     int it = 0, lrit = 0;
     Ring r;
     bool ok = true;
+    bool x_issued = false;
     for (int g = sc.cid; g < a.tiles_nm && ok; g += sc.ncl) {
         const TileCoord c = tile_coord<PAIR>(a, g, sc.rank);
+        if (XRES && !x_issued) {
+            // resident x: every tile of this CTA has the same tokens (one token
+            // tile) and the same K range (its split), so x is loaded once
+            mbar_arrive_expect_tx(s.xfull, static_cast<uint32_t>(c.kb1 - c.kb0) * a.xsub_bytes);
+            for (int kb = c.kb0; kb < c.kb1; ++kb)
+                tma_load_2d(s.x + (kb - c.kb0) * a.xsub_bytes, tm_x, s.xfull, kb * 64, 0);
+            x_issued = true;
+        }
         for (int kb = c.kb0; kb < c.kb1; kb += a.ks) {
             const int nkb = min(a.ks, c.kb1 - kb);
             const int st = r.slot;
             if (!wait_or_abort(&s.empty[st], r.phase ^ 1, a, s.abort_flag)) { ok = false; break; }
-            // this CTA's x rows and weight tiles land on its own barrier; in a
-            // pair the dequant warps pass both on to the first CTA's MMA
-            mbar_arrive_expect_tx(&s.full[st], nkb * (a.xsub_bytes + a.wtile_bytes));
-            for (int j = 0; j < nkb; ++j)
-                tma_load_2d(s.x + st * a.xstage_bytes + j * a.xsub_bytes, tm_x, &s.full[st], (kb + j) * 64,
-                            c.mt * a.BN + row0);
+            if constexpr (XRES) {
+                mbar_arrive_expect_tx(&s.full[st], nkb * a.wtile_bytes);
+            } else {
+                // this CTA's x rows and weight tiles land on its own barrier; in a
+                // pair the dequant warps pass both on to the first CTA's MMA
+                mbar_arrive_expect_tx(&s.full[st], nkb * (a.xsub_bytes + a.wtile_bytes));
+                for (int j = 0; j < nkb; ++j)
+                    tma_load_2d(s.x + st * a.xstage_bytes + j * a.xsub_bytes, tm_x, &s.full[st], (kb + j) * 64,
+                                c.mt * a.BN + row0);
+            }
             bulk_load(s.w + st * a.wstage_bytes,
                       a.packed + (static_cast<size_t>(c.nt) * a.KT + kb) * a.wtile_bytes,
                       nkb * a.wtile_bytes, &s.full[st]);
@@ -309,11 +325,12 @@ __device__ void producer_role(const GemmArgs& a, const CUtensorMap* tm_x, const 
         // let every copy already issued land before the CTA can exit
         for (int i = max(0, it - a.stages); i < it; ++i)
             mbar_wait(&s.full[i % a.stages], (i / a.stages) & 1, DRAIN_TIMEOUT_NS);
+        if (XRES && x_issued) mbar_wait(s.xfull, 0, DRAIN_TIMEOUT_NS);
         if (lrit > 0) mbar_wait(s.lrfull, (lrit - 1) & 1, DRAIN_TIMEOUT_NS);
     }
 }
 
-template <int FMT, bool PAIR>
+template <int FMT, bool PAIR, bool XRES>
 __device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc, int warp,
                              int lane) {
     // in a pair, the A stage is consumed by the first CTA's MMA: signal there
@@ -322,17 +339,19 @@ __device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, co
     const int h = warp >> 2;  // which 32 of the 64 inputs of a K block
     const int row = q * 32 + lane;
     const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    Ring r;
+    Ring r, ra;
     for (int g = sc.cid; g < a.tiles_nm; g += sc.ncl) {
         const TileCoord c = tile_coord<PAIR>(a, g, sc.rank);
-        for (int kb = c.kb0; kb < c.kb1; kb += a.ks, r.next(a.stages)) {
+        for (int kb = c.kb0; kb < c.kb1; kb += a.ks, r.next(a.stages), ra.next(a.astages)) {
             const int nkb = min(a.ks, c.kb1 - kb);
             const int st = r.slot;
+            // resident x: the weight ring and the TMEM A-stage ring are separate
+            const int at = XRES ? ra.slot : st;
             if (!warp_wait_or_abort(&s.full[st], r.phase, a, s.abort_flag)) return;
-            // The slot's A stage is free: this round's load was issued only after
-            // the previous round's MMA committed.
+            // Unified ring: the slot's A stage is free, as this round's load was
+            // issued only after the previous round's MMA committed.
             tc_fence_after();
-            const uint32_t acol = tbase + a.a_col0 + st * a.ks * A_STAGE_COLS + h * 16;
+            const uint32_t acol = tbase + a.a_col0 + at * a.ks * A_STAGE_COLS + h * 16;
             // read every code (and scale) of the slot first, then release the
             // weight tiles to the producer before converting
             constexpr int CW = (FMT == FMT_W8) ? 2 : 1;  // 16-byte code vectors per block per lane
@@ -360,6 +379,11 @@ __device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, co
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.empty[st]);
+            if constexpr (XRES) {
+                // the A stage is free once the MMA that read it last has completed
+                if (!warp_wait_or_abort(&s.aempty[at], ra.phase ^ 1, a, s.abort_flag)) return;
+                tc_fence_after();
+            }
 #pragma unroll
             for (int j = 0; j < MAX_KS; ++j) {
                 if (j < nkb) {
@@ -380,13 +404,13 @@ __device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, co
             __syncwarp();
             if (lane == 0) {
                 if (PAIR && sc.rank != 0) mbar_arrive_peer(afull_leader + st * 8u);
-                else mbar_arrive(&s.afull[st]);
+                else mbar_arrive(&s.afull[at]);
             }
         }
     }
 }
 
-template <int FMT, bool PAIR>
+template <int FMT, bool PAIR, bool XRES>
 __device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc) {
     const uint32_t idesc = idesc_f16(FMT == FMT_W8 ? 1u : 0u, PAIR ? 256 : 128, a.BN);
     // pair commits signal the same barrier in both CTAs
@@ -394,22 +418,25 @@ __device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const 
     int lrit = 0, tc = 0;
     Ring r;
     bool ok = true;
+    if (XRES && !wait_or_abort(s.xfull, 0, a, s.abort_flag)) ok = false;
     for (int g = sc.cid; g < a.tiles_nm && ok; g += sc.ncl, ++tc) {
         const TileCoord c = tile_coord<PAIR>(a, g, sc.rank);
         const int ab = tc % a.acc_bufs;
         if (!wait_or_abort(&s.accempty[ab], ((tc / a.acc_bufs) & 1) ^ 1, a, s.abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem + a.acc_col0 + ab * a.BN;
-        for (int kb = c.kb0; kb < c.kb1 && ok; kb += a.ks, r.next(a.stages)) {
+        for (int kb = c.kb0; kb < c.kb1 && ok; kb += a.ks, r.next(XRES ? a.astages : a.stages)) {
             const int nkb = min(a.ks, c.kb1 - kb);
-            const int st = r.slot;
+            const int st = r.slot;  // resident x: the A-stage ring's slot
             // afull is reached only after every dequant warp (of both CTAs of a
             // pair) observed its slot full, so it orders the x tiles as well
             if (!wait_or_abort(&s.afull[st], r.phase, a, s.abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint32_t acol = tmem + a.a_col0 + st * a.ks * A_STAGE_COLS;
             for (int j = 0; j < nkb; ++j) {
-                const uint64_t bdesc = smem_desc_sw128(smem_u32(s.x + st * a.xstage_bytes + j * a.xsub_bytes));
+                const uint8_t* xt = XRES ? s.x + (kb - c.kb0 + j) * a.xsub_bytes
+                                         : s.x + st * a.xstage_bytes + j * a.xsub_bytes;
+                const uint64_t bdesc = smem_desc_sw128(smem_u32(xt));
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint32_t acc = (kb > c.kb0 || j > 0 || kk > 0) ? 1u : 0u;
@@ -418,7 +445,7 @@ __device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const 
                 }
             }
             if constexpr (PAIR) mma_commit_pair_both(&s.empty[st]);
-            else mma_commit(&s.empty[st]);
+            else mma_commit(XRES ? &s.aempty[st] : &s.empty[st]);
         }
         if (!ok) break;
         if (a.lr && c.sp == 0) {
@@ -450,7 +477,71 @@ __device__ __forceinline__ void store_y(const GemmArgs& a, int m, int n, float v
     else static_cast<__nv_bfloat16*>(a.y)[o] = __float2bfloat16_rn(v);
 }
 
-template <int FMT, bool PAIR>
+// Sum this CTA's share of a split tile's tokens over the S partials of the
+// cluster, in split order, and store y.  A warp takes whole token rows: lane l
+// reads channels 4l..4l+3 of a row from every CTA (512 contiguous bytes per
+// warp and CTA) with eight vector loads in flight (8 / S tokens, S splits
+// each), then stores the four adjacent outputs as one vector.
+__device__ __forceinline__ void reduce_share(const GemmArgs& a, const float* red, int pitch, const TileCoord& c,
+                                             const Sched& sc, int m0, int share, int e, int nw, int lane) {
+    const int nq = c.nt * 128 + 4 * lane;
+    float bq[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) bq[i] = (a.bias && nq + i < a.N) ? bf16_to_f32(a.bias[nq + i]) : 0.0f;
+    const int j0 = sc.rank * share;
+    const int lgS = __ffs(a.S) - 1;
+    const uint32_t red_local = smem_u32(red) + static_cast<uint32_t>(4 * lane) * 4u;
+    const int step = nw * (8 >> lgS);  // tokens the nw warps cover per round
+    for (int jt = e; jt < share; jt += step) {
+        float4 part[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int tok = jt + nw * (i >> lgS);
+            if (tok < share && m0 + j0 + tok < a.M)
+                part[i] = ld_dsmem_f32x4(mapa_shared(red_local, i & (a.S - 1)) +
+                                         static_cast<uint32_t>((j0 + tok) * pitch) * 4u);
+        }
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int r = i & (a.S - 1);
+            const int tok = jt + nw * (i >> lgS);
+            if (tok >= share || m0 + j0 + tok >= a.M) break;
+            if (r == 0) {
+                acc = part[i];
+            } else {
+                acc.x += part[i].x;
+                acc.y += part[i].y;
+                acc.z += part[i].z;
+                acc.w += part[i].w;
+            }
+            if (r != a.S - 1) continue;
+            const float o[4] = {acc.x + bq[0], acc.y + bq[1], acc.z + bq[2], acc.w + bq[3]};
+            const int m = m0 + j0 + tok;
+            if (a.vec_out) {
+                if (nq < a.N) {
+                    if (a.y_f32) {
+                        *reinterpret_cast<float4*>(static_cast<float*>(a.y) + static_cast<size_t>(m) * a.N + nq) =
+                            make_float4(o[0], o[1], o[2], o[3]);
+                    } else {
+                        const __nv_bfloat162 lo = __floats2bfloat162_rn(o[0], o[1]);
+                        const __nv_bfloat162 hi = __floats2bfloat162_rn(o[2], o[3]);
+                        uint2 v2;
+                        v2.x = *reinterpret_cast<const uint32_t*>(&lo);
+                        v2.y = *reinterpret_cast<const uint32_t*>(&hi);
+                        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.y) + static_cast<size_t>(m) * a.N + nq) = v2;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (nq + q < a.N) store_y(a, m, nq + q, o[q]);
+            }
+        }
+    }
+}
+
+template <int FMT, bool PAIR, bool XRES>
 __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc, int warp,
                               int lane) {
     // in a pair the accumulator is released to the first CTA's MMA thread
@@ -469,8 +560,7 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
             freed_at[r] = mapa_shared(smem_u32(s.freed), r);
         }
     }
-    const int share = a.BN / a.S;       // tokens of each tile this CTA sums (a multiple of 4)
-    const int red_pitch = a.BN + 4;     // floats per row of the partial buffer (keeps float4 alignment)
+    const int share = a.BN / a.S;       // tokens of each tile this CTA sums (at least 8)
     int tc = 0;
     for (int g = sc.cid; g < a.tiles_nm; g += sc.ncl, ++tc) {
         const TileCoord c = tile_coord<PAIR>(a, g, sc.rank);
@@ -497,10 +587,9 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
                 if (has_lr) val[j] += __uint_as_float(lv[j]);
             }
             if (split) {
-                float4* dst = reinterpret_cast<float4*>(s.red + row * red_pitch + cc * 16);
+                // token-major partial: consecutive lanes write consecutive channels
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    dst[j] = make_float4(val[4 * j], val[4 * j + 1], val[4 * j + 2], val[4 * j + 3]);
+                for (int j = 0; j < 16; ++j) s.red[(cc * 16 + j) * 128 + row] = val[j];
             } else if (a.vec_out) {
                 // Each lane holds one channel for 16 tokens; y is token-major.  Turn
                 // the 16 x 32 block around in shared memory so that every lane stores
@@ -594,48 +683,25 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
         __syncwarp();
         if (lane == 0) mbar_arrive(s.redw);
         if (first_thread && wait_or_abort(s.redw, tc & 1, a, s.abort_flag)) {
+            // the fence orders the partial at cluster scope; the arrives need no
+            // release of their own (a release.cluster arrive costs ~1000 cycles)
             fence_acq_rel_cluster();
-            for (int r = 0; r < a.S; ++r) mbar_arrive_remote(ready_at[r]);
+            for (int r = 0; r < a.S; ++r) mbar_arrive_peer(ready_at[r]);
         }
         if (!warp_wait_or_abort(s.ready, tc & 1, a, s.abort_flag, true)) return;
-        // sum this CTA's share of the tile's tokens over all partials, in split
-        // order; four tokens per vector load, all S loads of a quad in flight
-        const int j0 = sc.rank * share;
-        for (int jq = j0; jq < j0 + share; jq += 4) {
-            if (m0 + jq >= a.M) break;
-            const uint32_t off = static_cast<uint32_t>(row * red_pitch + jq) * 4u;
-            float4 part[MAX_SPLITS];
-#pragma unroll
-            for (int r = 0; r < MAX_SPLITS; ++r)
-                if (r < a.S) part[r] = ld_dsmem_f32x4(red_at[r] + off);
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int r = 0; r < MAX_SPLITS; ++r)
-                if (r < a.S) {
-                    acc.x += part[r].x;
-                    acc.y += part[r].y;
-                    acc.z += part[r].z;
-                    acc.w += part[r].w;
-                }
-            if (n_ok) {
-                const float o[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (m0 + jq + j < a.M) store_y(a, m0 + jq + j, n, o[j] + bn);
-            }
-        }
+        reduce_share(a, s.red, 128, c, sc, m0, share, warp - WARP_EPI0, NUM_EPI_WARPS, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(s.readw);
         if (first_thread && wait_or_abort(s.readw, tc & 1, a, s.abort_flag)) {
             fence_acq_rel_cluster();
-            for (int r = 0; r < a.S; ++r) mbar_arrive_remote(freed_at[r]);
+            for (int r = 0; r < a.S; ++r) mbar_arrive_peer(freed_at[r]);
         }
     }
     // no CTA of the cluster may still read this CTA's shared memory when it exits
     if (split && tc > 0) warp_wait_or_abort(s.freed, (tc - 1) & 1, a, s.abort_flag, true);
 }
 
-template <int FMT, bool PAIR>
+template <int FMT, bool PAIR, bool XRES>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_t,
             const __grid_constant__ CUtensorMap tm_l2, const GemmArgs a) {
@@ -643,17 +709,19 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     Smem s;
-    s.x = base;
-    s.w = s.x + static_cast<size_t>(a.stages) * a.xstage_bytes;
+    s.x = base;  // resident x: kbps x sub-tiles; otherwise stages x xstage_bytes
+    s.w = s.x + (XRES ? static_cast<size_t>(a.kbps) * a.xsub_bytes : static_cast<size_t>(a.stages) * a.xstage_bytes);
     s.lrA = s.w + static_cast<size_t>(a.stages) * a.wstage_bytes;
     s.lrB = s.lrA + (a.lr ? LR_TILE_A_BYTES : 0);
     s.red = reinterpret_cast<float*>(s.lrB + (a.lr ? a.xsub_bytes : 0));
     s.stage = reinterpret_cast<uint8_t*>(s.red) + a.red_bytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(s.stage + a.stage_bytes);
     s.full = bars;
-    s.empty = s.full + a.stages;
-    s.afull = s.empty + a.stages;
-    s.accfull = s.afull + a.stages;
+    s.empty = s.full + MAX_STAGES;
+    s.afull = s.empty + MAX_STAGES;
+    s.aempty = s.afull + MAX_STAGES;
+    s.xfull = s.aempty + MAX_STAGES;
+    s.accfull = s.xfull + 1;
     s.accempty = s.accfull + 2;
     s.lrfull = s.accempty + 2;
     s.lrempty = s.lrfull + 1;
@@ -670,9 +738,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     if (threadIdx.x == 0) {
         for (int i = 0; i < a.stages; ++i) {
             mbar_init(&s.full[i], 1);
-            mbar_init(&s.empty[i], 1 + NUM_DQ_WARPS);
-            mbar_init(&s.afull[i], PAIR ? 2 * NUM_DQ_WARPS : NUM_DQ_WARPS);
+            // resident x: the dequant warps alone release a weight slot
+            mbar_init(&s.empty[i], XRES ? NUM_DQ_WARPS : 1 + NUM_DQ_WARPS);
         }
+        for (int i = 0; i < (XRES ? a.astages : a.stages); ++i) {
+            mbar_init(&s.afull[i], PAIR ? 2 * NUM_DQ_WARPS : NUM_DQ_WARPS);
+            mbar_init(&s.aempty[i], 1);
+        }
+        mbar_init(s.xfull, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.accfull[i], 1);
             mbar_init(&s.accempty[i], PAIR ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS);
@@ -708,13 +781,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     const Sched sc = sched();
 
     if (warp < NUM_DQ_WARPS) {
-        dequant_role<FMT, PAIR>(a, tmem, s, sc, warp, lane);
+        dequant_role<FMT, PAIR, XRES>(a, tmem, s, sc, warp, lane);
     } else if (warp < WARP_PRODUCER) {
-        epilogue_role<FMT, PAIR>(a, tmem, s, sc, warp, lane);
+        epilogue_role<FMT, PAIR, XRES>(a, tmem, s, sc, warp, lane);
     } else if (warp == WARP_PRODUCER) {
-        if (lane == 0) producer_role<PAIR>(a, &tm_x, &tm_t, &tm_l2, s, sc);
+        if (lane == 0) producer_role<PAIR, XRES>(a, &tm_x, &tm_t, &tm_l2, s, sc);
     } else if (lane == 0 && (!PAIR || sc.rank == 0)) {
-        mma_role<FMT, PAIR>(a, tmem, s, sc);
+        mma_role<FMT, PAIR, XRES>(a, tmem, s, sc);
     }
 
     tc_fence_before();

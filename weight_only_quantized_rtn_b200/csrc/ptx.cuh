@@ -250,6 +250,25 @@ __host__ __device__ constexpr uint32_t idesc_f16(uint32_t ab_bf16, uint32_t m, u
            | ((m >> 4) << 24);       // M / 16
 }
 
+// ------------------------------------------------ warp-level MMA (mma.sync)
+// D[16x8] += A[16x16] * B[16x8], fp32 accumulate; A row-major, B column-major.
+__device__ __forceinline__ void mma16816_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma16816_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// Named barrier over the first `threads` threads of the block (id 1..15).
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // ------------------------------------------------------------------ cluster
 // A launch without cluster dimensions is a cluster of one CTA: rank 0,
 // cluster id = blockIdx.x, cluster count = gridDim.x.
@@ -274,12 +293,11 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
     return r;
 }
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-// Arrive on a barrier of another CTA of the pair with the default (CTA-scope)
-// release.  Used where the guarded data are tensor-memory contents ordered by
-// tcgen05 fences on both sides, not plain shared-memory stores.
+// Arrive on a barrier of another CTA of the cluster with the default
+// (CTA-scope) release.  Used where the guarded data are tensor-memory contents
+// ordered by tcgen05 fences on both sides, or right after an explicit
+// fence.acq_rel.cluster that orders plain shared-memory stores; an arrive with
+// release.cluster semantics of its own costs about a thousand cycles.
 __device__ __forceinline__ void mbar_arrive_peer(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }

@@ -13,6 +13,7 @@
 
 #include "../../include/wlq.h"
 #include "gemm.cuh"
+#include "skinny.cuh"
 #include "pack.cuh"
 #include "prep.cuh"
 #include "ptx.cuh"
@@ -49,7 +50,7 @@ int fmt_of(int bits, int group) {
 struct DeviceInfo {
     int checked = 0;  // 0 unknown, 1 supported, -1 not
     int sms = 0;
-    bool smem_set[6] = {false, false, false, false, false, false};
+    bool smem_set[24] = {};
     // resident clusters per (format, cluster size, dynamic smem), queried once
     std::unordered_map<uint64_t, int> max_clusters;
 };
@@ -118,6 +119,7 @@ wlq_status make_map_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64
 // ------------------------------------------------------------------ plan
 constexpr uint64_t kDefaultTimeoutNs = 2ull * 1000 * 1000 * 1000;
 constexpr size_t kSmemLimit = 232448;  // 227 KB opt-in per block on sm_100
+constexpr size_t kXresMaxBytes = 128 * 1024;  // largest resident x block (tokens x K range, bf16)
 
 struct Plan {
     int fmt = -1;
@@ -125,6 +127,9 @@ struct Plan {
     int NT = 0, KT = 0, MT = 0, S = 1, kbps = 0, BN = 0, tiles_nm = 0, grid = 0;
     int stages = 0, ks = 1, lr_kb = 0, acc_bufs = 1;
     bool pair = false;  // two CTAs per MMA (cta_group::2)
+    bool xres = false;  // x resident in shared memory; weight ring released by the dequant warps
+    bool skinny = false;  // one token tile of <= 64 tokens: the warp-MMA streaming kernel
+    int astages = 0;    // resident x: TMEM A-stage ring depth
     uint32_t tmem_cols = 0, acc_col0 = 0, lr_col0 = 0, a_col0 = 0, wtile = 0, wstage = 0, xsub = 0, xstage = 0, red = 0, stage = 0;
     size_t smem = 0;
     size_t off_x16 = 0, off_xs = 0, off_thl = 0, off_l2t = 0, ws = 0;
@@ -172,7 +177,7 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
         S /= 2;
     }
     p.S = S;
-    if (S > 1 && p.BN % (4 * S) != 0) return false;  // the reduction's token quads must not straddle shares
+    if (S > 1 && p.BN % S != 0) return false;  // every CTA of a split cluster sums whole tokens
     // CTA pairs for large token tiles: two 128-channel tiles share each MMA
     p.pair = (r == 0 && S == 1 && p.BN == 256 && p.NT % 2 == 0);
     p.tiles_nm = p.pair ? (p.NT / 2) * p.MT : p.NT * p.MT;
@@ -188,14 +193,75 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     // shared memory: ring slots + low-rank tiles + split partial + barriers
     p.wtile = wlq::tile_bytes(fmt);
     p.xsub = static_cast<uint32_t>(p.pair ? p.BN / 2 : p.BN) * 128u;  // a pair's CTA stages half the tokens
-    p.red = (S > 1) ? 128u * static_cast<uint32_t>(p.BN + 4) * 4u : 0u;
+    p.red = (S > 1) ? static_cast<uint32_t>(p.BN) * 128u * 4u : 0u;  // token-major fp32 partial
     const size_t lr_bytes = r ? (wlq::LR_TILE_A_BYTES + p.xsub) : 0;
     p.stage = (S == 1) ? wlq::NUM_EPI_WARPS * wlq::EPI_STAGE_BYTES : 0u;  // epilogue transpose buffers
     const size_t fixed = 1024 /* alignment */ + 1024 /* barriers */ + lr_bytes + p.red + p.stage;
+    // Resident x (one token tile, small K range): the CTA's x rows stay in
+    // shared memory for the whole K range, the weight ring is released as soon
+    // as the dequant warps hold the codes, and the TMEM A stages form a ring of
+    // their own, so weight loads never wait for the MMA.
+    const size_t xres_bytes = static_cast<size_t>(p.kbps) * p.BN * 128u;
+    p.ks = 0;
+    // Few tokens (at most 32): the skinny kernel (x resident, warp MMAs, no
+    // tensor memory).  At 64 tokens the resident-x tensor-core kernel is faster.
+    p.skinny = !p.pair && r == 0 && p.MT == 1 && p.BN <= 32 && xres_bytes <= kXresMaxBytes;
+    if (p.skinny) {
+        p.red = static_cast<uint32_t>(p.BN) * wlq::SK_PITCH * 4u;  // split partial or output staging
+        p.stage = 0;
+        const size_t sk_fixed = 1024 /* alignment */ + 1024 /* barriers */ + xres_bytes + p.red;
+        {
+            const int ks = wlq::SK_GROUPS;  // one K block per warp group in every slot
+            const uint32_t wstage = (static_cast<uint32_t>(ks) * p.wtile + 1023u) & ~1023u;
+            const int stages = std::min(wlq::MAX_STAGES, static_cast<int>((kSmemLimit - sk_fixed) / wstage));
+            if (sk_fixed + 2 * static_cast<size_t>(wstage) <= kSmemLimit && stages >= 2) {
+                p.ks = ks;
+                p.stages = stages;
+                p.wstage = wstage;
+                p.xstage = 0;
+                p.smem = sk_fixed + stages * static_cast<size_t>(wstage);
+            }
+        }
+        if (p.ks == 0) {
+            p.skinny = false;
+            p.red = (S > 1) ? static_cast<uint32_t>(p.BN) * 128u * 4u : 0u;
+            p.stage = (S == 1) ? wlq::NUM_EPI_WARPS * wlq::EPI_STAGE_BYTES : 0u;
+        } else {
+            p.kbps = (S > 1) ? p.kbps : p.KT;
+            p.tmem_cols = 0;
+            size_t off = 0;
+            if (fmt != wlq::FMT_W8) {
+                p.off_x16 = off; off = align256(off + static_cast<size_t>(M) * K * 2);
+                p.off_xs = off;  off = align256(off + static_cast<size_t>(M) * 4);
+            }
+            p.ws = off;
+            return true;
+        }
+    }
+    p.xres = !p.pair && r == 0 && p.MT == 1 && p.BN <= 64 && xres_bytes <= kXresMaxBytes;
+    if (p.xres) {
+        for (int ks : {4, 2, 1}) {
+            const uint32_t wstage = (static_cast<uint32_t>(ks) * p.wtile + 1023u) & ~1023u;
+            const int astages = static_cast<int>((512 - a_col0) / (static_cast<uint32_t>(ks) * wlq::A_STAGE_COLS));
+            if (fixed + xres_bytes + 2 * wstage > kSmemLimit) continue;
+            const int stages = std::min(wlq::MAX_STAGES, static_cast<int>((kSmemLimit - fixed - xres_bytes) / wstage));
+            const int ast = std::min(wlq::MAX_STAGES, astages);
+            if (stages >= 2 && (ast >= 3 || (ks == 1 && ast >= 2))) {
+                p.ks = ks;
+                p.stages = stages;
+                p.astages = ast;
+                p.wstage = wstage;
+                p.xstage = 0;
+                p.smem = fixed + xres_bytes + stages * static_cast<size_t>(wstage);
+                break;
+            }
+        }
+        if (p.ks == 0) p.xres = false;
+    }
     // K blocks per ring slot: the largest of 4, 2, 1 that still leaves three
     // slots in both TMEM and shared memory (one handshake per slot)
-    p.ks = 0;
     for (int ks : {4, 2, 1}) {
+        if (p.ks) break;
         const uint32_t wstage = (static_cast<uint32_t>(ks) * p.wtile + 1023u) & ~1023u;
         const uint32_t xstage = static_cast<uint32_t>(ks) * p.xsub;
         const size_t per_stage = xstage + wstage;
@@ -216,7 +282,7 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     p.acc_col0 = 0;
     p.lr_col0 = p.acc_bufs * static_cast<uint32_t>(p.BN);
     p.a_col0 = a_col0;
-    const uint32_t need = a_col0 + static_cast<uint32_t>(p.stages * p.ks) * wlq::A_STAGE_COLS;
+    const uint32_t need = a_col0 + static_cast<uint32_t>((p.xres ? p.astages : p.stages) * p.ks) * wlq::A_STAGE_COLS;
     p.tmem_cols = 32;
     while (p.tmem_cols < need) p.tmem_cols <<= 1;
     // workspace
@@ -244,11 +310,11 @@ wlq_status check_shape(int64_t N, int64_t K, int bits, int group) {
 
 int g_grid_limit = 0;  // 0: no cap on the GEMM's CTAs (see wlq_set_grid_limit)
 
-template <int FMT, bool PAIR>
+template <int FMT, bool PAIR, bool XRES>
 wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, const CUtensorMap& tl,
                        wlq::GemmArgs& a, DeviceInfo* d, cudaStream_t st) {
-    auto kern = wlq::gemm_kernel<FMT, PAIR>;
-    const int kid = FMT * 2 + (PAIR ? 1 : 0);
+    auto kern = wlq::gemm_kernel<FMT, PAIR, XRES>;
+    const int kid = FMT * 4 + (PAIR ? 2 : 0) + (XRES ? 1 : 0);
     if (!d->smem_set[kid]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(kSmemLimit));
@@ -295,6 +361,64 @@ wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, co
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tx, tt, tl, a);
     if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
     return WLQ_OK;
+}
+
+template <int FMT, int NB>
+wlq_status launch_skinny(Plan& p, const CUtensorMap& tx, wlq::GemmArgs& a, DeviceInfo* d, cudaStream_t st) {
+    auto kern = wlq::skinny_kernel<FMT, NB>;
+    const int kid = 12 + FMT * 4 + (NB == 2 ? 0 : NB == 4 ? 1 : 2);
+    if (!d->smem_set[kid]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kSmemLimit));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        d->smem_set[kid] = true;
+    }
+    const int csize = p.S;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cudaLaunchAttribute attr[1];
+    cfg.blockDim = dim3(wlq::SK_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = st;
+    const int cta_cap = (g_grid_limit > 0) ? std::min(g_grid_limit, d->sms) : d->sms;
+    int clusters = std::max(1, std::min(p.tiles_nm, cta_cap / csize));
+    if (csize > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(csize);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const uint64_t key = (static_cast<uint64_t>(kid) << 48) | (static_cast<uint64_t>(csize) << 32) | p.smem;
+        int active = 0;
+        {
+            std::lock_guard<std::mutex> lk(g_dev_mu);
+            auto it = d->max_clusters.find(key);
+            if (it != d->max_clusters.end()) active = it->second;
+        }
+        if (active == 0) {
+            cfg.gridDim = dim3(static_cast<unsigned>(clusters * csize), 1, 1);
+            if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) != cudaSuccess || active <= 0) {
+                cudaGetLastError();
+                active = d->sms / csize;
+            }
+            std::lock_guard<std::mutex> lk(g_dev_mu);
+            d->max_clusters[key] = active;
+        }
+        clusters = std::min(clusters, active);
+    }
+    cfg.gridDim = dim3(static_cast<unsigned>(clusters * csize), 1, 1);
+    p.grid = clusters * csize;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tx, a);
+    if (e != cudaSuccess) return cuda_fail(e, "skinny launch");
+    return WLQ_OK;
+}
+
+template <int FMT>
+wlq_status launch_skinny_nb(Plan& p, const CUtensorMap& tx, wlq::GemmArgs& a, DeviceInfo* d, cudaStream_t st) {
+    if (p.BN == 16) return launch_skinny<FMT, 2>(p, tx, a, d, st);
+    if (p.BN == 32) return launch_skinny<FMT, 4>(p, tx, a, d, st);
+    return launch_skinny<FMT, 8>(p, tx, a, d, st);
 }
 
 int grid_for(int64_t work, int per_block, int sms) {
@@ -480,22 +604,36 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
     a.y = y;
     a.M = p.M; a.N = p.N; a.K = p.K;
     a.NT = p.NT; a.KT = p.KT; a.MT = p.MT; a.S = p.S; a.kbps = p.kbps; a.BN = p.BN;
-    a.stages = p.stages; a.ks = p.ks; a.lr = r ? 1 : 0; a.lr_kb = p.lr_kb; a.acc_bufs = p.acc_bufs;
+    a.stages = p.stages; a.astages = p.astages; a.ks = p.ks; a.lr = r ? 1 : 0; a.lr_kb = p.lr_kb; a.acc_bufs = p.acc_bufs;
     a.y_f32 = (y_dtype == WLQ_OUT_F32) ? 1 : 0;
     a.tiles_nm = p.tiles_nm;
     a.tmem_cols = p.tmem_cols; a.acc_col0 = p.acc_col0; a.lr_col0 = p.lr_col0; a.a_col0 = p.a_col0;
     a.wtile_bytes = p.wtile; a.wstage_bytes = p.wstage; a.xsub_bytes = p.xsub; a.xstage_bytes = p.xstage; a.red_bytes = p.red;
     a.stage_bytes = p.stage;
-    a.vec_out = (p.S == 1 && (reinterpret_cast<uintptr_t>(y) & 15u) == 0 &&
-                 (y_dtype == WLQ_OUT_F32 ? N % 4 == 0 : N % 8 == 0)) ? 1 : 0;
+    // vector stores of y: unsplit tiles store 16-byte runs (4 fp32 / 8 bf16
+    // channels), the split reduction 4 adjacent channels (16 / 8 bytes)
+    {
+        const uintptr_t ya = reinterpret_cast<uintptr_t>(y);
+        const bool f32 = y_dtype == WLQ_OUT_F32;
+        if (p.S == 1) a.vec_out = ((ya & 15u) == 0 && N % (f32 ? 4 : 8) == 0) ? 1 : 0;
+        else a.vec_out = ((ya & (f32 ? 15u : 7u)) == 0 && N % 4 == 0) ? 1 : 0;
+    }
     a.timeout_ns = kDefaultTimeoutNs;
-    switch (fmt * 2 + (p.pair ? 1 : 0)) {
-        case 0: return launch_gemm<wlq::FMT_W8, false>(p, tx, tt, tl, a, d, s);
-        case 1: return launch_gemm<wlq::FMT_W8, true>(p, tx, tt, tl, a, d, s);
-        case 2: return launch_gemm<wlq::FMT_W4G64, false>(p, tx, tt, tl, a, d, s);
-        case 3: return launch_gemm<wlq::FMT_W4G64, true>(p, tx, tt, tl, a, d, s);
-        case 4: return launch_gemm<wlq::FMT_W4G16, false>(p, tx, tt, tl, a, d, s);
-        default: return launch_gemm<wlq::FMT_W4G16, true>(p, tx, tt, tl, a, d, s);
+    if (p.skinny) {
+        if (fmt == wlq::FMT_W8) return launch_skinny_nb<wlq::FMT_W8>(p, tx, a, d, s);
+        if (fmt == wlq::FMT_W4G64) return launch_skinny_nb<wlq::FMT_W4G64>(p, tx, a, d, s);
+        return launch_skinny_nb<wlq::FMT_W4G16>(p, tx, a, d, s);
+    }
+    switch (fmt * 3 + (p.pair ? 1 : 0) + (p.xres ? 2 : 0)) {
+        case 0: return launch_gemm<wlq::FMT_W8, false, false>(p, tx, tt, tl, a, d, s);
+        case 1: return launch_gemm<wlq::FMT_W8, true, false>(p, tx, tt, tl, a, d, s);
+        case 2: return launch_gemm<wlq::FMT_W8, false, true>(p, tx, tt, tl, a, d, s);
+        case 3: return launch_gemm<wlq::FMT_W4G64, false, false>(p, tx, tt, tl, a, d, s);
+        case 4: return launch_gemm<wlq::FMT_W4G64, true, false>(p, tx, tt, tl, a, d, s);
+        case 5: return launch_gemm<wlq::FMT_W4G64, false, true>(p, tx, tt, tl, a, d, s);
+        case 6: return launch_gemm<wlq::FMT_W4G16, false, false>(p, tx, tt, tl, a, d, s);
+        case 7: return launch_gemm<wlq::FMT_W4G16, true, false>(p, tx, tt, tl, a, d, s);
+        default: return launch_gemm<wlq::FMT_W4G16, false, true>(p, tx, tt, tl, a, d, s);
     }
 }
 
