@@ -225,7 +225,7 @@ def run_gpu(args):
         for M in MS:
             linear(M)
 
-    launches_per_step = 1 + 2 + len(MS)  # quantize, pack (row factors + tiles), one GEMM per M
+    launches_per_step = 1 + 1 + len(MS)  # quantize, pack (int8: tiles and row factors in one kernel), one GEMM per M
 
     for _ in range(args.warmup):
         step()

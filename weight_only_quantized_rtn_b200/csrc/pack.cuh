@@ -31,7 +31,7 @@ __host__ __device__ constexpr uint32_t tile_bytes(int fmt) {
 
 __device__ __forceinline__ int int4_nibble_pos(int t) { return (t & 1) ? 4 + (t >> 1) : (t >> 1); }
 
-// One warp per padded row: the fp32 factor the epilogue multiplies by.
+// int4: one warp per padded row, the fp32 factor the epilogue multiplies by.
 __global__ void pack_rowfactor_kernel(const float* __restrict__ scales, int64_t N, int64_t G,
                                       int fmt, int64_t N_pad, float* __restrict__ rowf) {
     const int lane = threadIdx.x & 31;
@@ -59,28 +59,38 @@ __global__ void pack_rowfactor_kernel(const float* __restrict__ scales, int64_t 
 
 // One CTA (128 threads) per tile.  Codes are read as 8-byte runs (8 inputs of
 // one row; rows start 8-byte aligned because K % 8 == 0), so a warp reads
-// four rows' 64 contiguous bytes each.
+// four rows' 64 contiguous bytes each; each thread issues all eight of its
+// loads before its first store.  For int8 the K-block-0 CTAs also write the
+// row factors (the channel scales); int4 row factors come from
+// pack_rowfactor_kernel, which runs first.
 __global__ void __launch_bounds__(128) pack_tiles_kernel(
     const int8_t* __restrict__ codes, const float* __restrict__ scales, int64_t N, int64_t K,
-    int64_t G, int fmt, int KT, const float* __restrict__ rowf, uint8_t* __restrict__ packed) {
+    int64_t G, int fmt, int KT, float* __restrict__ rowf, uint8_t* __restrict__ packed) {
     const int64_t tile = blockIdx.x;
     const int64_t nt = tile / KT;
     const int kb = static_cast<int>(tile % KT);
     const int64_t k0 = static_cast<int64_t>(kb) * 64;
     uint8_t* blk = packed + tile * tile_bytes(fmt);
-    for (int idx = threadIdx.x; idx < 128 * 8; idx += 128) {
+    uint2 v[8];
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+        const int idx = threadIdx.x + 128 * it;
         const int i = idx >> 3, part = idx & 7;
         const int64_t n = nt * 128 + i, k = k0 + 8 * part;
-        uint2 v = make_uint2(0u, 0u);
-        if (n < N && k < K) v = __ldg(reinterpret_cast<const uint2*>(codes + n * K + k));
+        v[it] = (n < N && k < K) ? __ldg(reinterpret_cast<const uint2*>(codes + n * K + k)) : make_uint2(0u, 0u);
+    }
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+        const int idx = threadIdx.x + 128 * it;
+        const int i = idx >> 3, part = idx & 7;
         if (fmt == FMT_W8) {
             // offset binary q + 128 of a two's-complement byte is q ^ 0x80
-            v.x ^= 0x80808080u;
-            v.y ^= 0x80808080u;
-            *reinterpret_cast<uint2*>(blk + (part >> 1) * 2048 + 16 * i + (part & 1) * 8) = v;
+            const uint2 o = make_uint2(v[it].x ^ 0x80808080u, v[it].y ^ 0x80808080u);
+            *reinterpret_cast<uint2*>(blk + (part >> 1) * 2048 + 16 * i + (part & 1) * 8) = o;
         } else {
-            const uint32_t b[2] = {v.x, v.y};
+            const uint32_t b[2] = {v[it].x, v[it].y};
             uint32_t w = 0;
+#pragma unroll
             for (int t = 0; t < 8; ++t) {
                 const uint32_t u = ((b[t >> 2] >> (8 * (t & 3))) + 8u) & 0xFu;  // (q + 8) mod 16
                 w |= u << (4 * int4_nibble_pos(t));
@@ -88,10 +98,13 @@ __global__ void __launch_bounds__(128) pack_tiles_kernel(
             *reinterpret_cast<uint32_t*>(blk + (part >> 2) * 2048 + 16 * i + 4 * (part & 3)) = w;
         }
     }
-    if (fmt == FMT_W8) return;
     const int i = threadIdx.x;
     const int64_t n = nt * 128 + i;
     const bool row_ok = n < N;
+    if (fmt == FMT_W8) {
+        if (kb == 0) rowf[n] = row_ok ? scales[n] : 0.0f;
+        return;
+    }
     const float rf = row_ok ? rowf[n] : 0.0f;
     const int sh = (rf > 0.0f) ? -ilogbf(rf) : 0;  // s * 2^sh = s / rf exactly
     auto scale16 = [&](int64_t g) -> __half {

@@ -71,7 +71,7 @@ __device__ __forceinline__ GroupScale group_scale(float a, int qmax) {
     g.s = __fdiv_rn(a, static_cast<float>(qmax));
     g.normal = g.s >= 1.17549435e-38f;
     g.inv = g.normal ? __frcp_rn(g.s) : 0.0f;
-    g.inv64 = (g.s > 0.0f) ? 1.0 / static_cast<double>(g.s) : 0.0;
+    g.inv64 = (!g.normal && g.s > 0.0f) ? 1.0 / static_cast<double>(g.s) : 0.0;  // subnormal path only
     return g;
 }
 
@@ -88,9 +88,10 @@ __device__ __forceinline__ uint32_t pack_codes4(float4 v, const GroupScale& g, i
     return out;
 }
 
-// One warp per row: the group is the whole row (per output channel).  Pass 1
-// reads the row for its absmax, pass 2 reads it again (from L2: the row was
-// just read) to round and store the codes; eight loads in flight per lane.
+// One warp per row, for rows longer than the per-CTA kernel holds: the group
+// is the whole row (per output channel).  Pass 1 reads the row for its absmax,
+// pass 2 reads it again (from L2: the row was just read) to round and store
+// the codes; eight loads in flight per lane.
 __global__ void __launch_bounds__(256) quantize_rows_kernel(
     const float* __restrict__ W, int64_t N, int64_t K, int qmax, int8_t* __restrict__ codes,
     float* __restrict__ scales) {
@@ -120,34 +121,127 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(
     }
 }
 
+// RTN of four weights of one group with a normal fp32 scale (s >= 2^-126),
+// packed as two's-complement bytes: the same arithmetic as rtn_byte_f32,
+// with the exact-tie correction on a branch (a residual of exactly s/2 is
+// rare).  h = s / 2, inv = 1 / s rounded.
+__device__ __forceinline__ uint32_t rtn4_f32(float4 v, float s, float inv, float h, float qmax) {
+    const float kMagic = 12582912.0f;  // 1.5 * 2^23
+    const float w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float k = __fsub_rn(__fadd_rn(__fmul_rn(w[i], inv), kMagic), kMagic);
+        const float e = __fmaf_rn(-k, s, w[i]);
+        k = (e > h) ? k + 1.0f : k;
+        k = (e < -h) ? k - 1.0f : k;
+        if (fabsf(e) == h) {  // exact tie between k and k + sign(e): keep the even one
+            if (__float_as_uint(__fadd_rn(k, kMagic)) & 1u) k += (e > 0.0f) ? 1.0f : -1.0f;
+        }
+        k = fminf(fmaxf(k, -qmax), qmax);
+        out |= (__float_as_uint(__fadd_rn(k, kMagic)) & 0xFFu) << (8 * i);
+    }
+    return out;
+}
+
+// One CTA per row (grid-stride over rows) for rows of up to 32768 inputs: the
+// row is read once, straight into registers (V float4 per thread, all loads
+// in flight together), its absmax is reduced over the CTA, and the codes are
+// computed from the registers.  Every byte of W crosses HBM exactly once.
+// The absmax is taken on the magnitude bit patterns: for non-negative IEEE
+// values the unsigned order is the numeric order, and any NaN or infinity
+// sorts above every finite value, so one compare at the end detects them.
+template <int V>
+__global__ void __launch_bounds__(1024) quantize_rows_cta_kernel(
+    const float* __restrict__ W, int64_t N, int64_t K, int qmax, int8_t* __restrict__ codes,
+    float* __restrict__ scales) {
+    __shared__ uint32_t part[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nwarps = blockDim.x >> 5;
+    const int K4 = static_cast<int>(K / 4);
+    const float fq = static_cast<float>(qmax);
+    bool bad = false;
+    for (int64_t n = blockIdx.x; n < N; n += gridDim.x) {
+        const float4* row = reinterpret_cast<const float4*>(W + n * K);
+        float4 v[V];
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int idx = threadIdx.x + i * blockDim.x;
+            v[i] = idx < K4 ? __ldcs(row + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            m = max(m, __float_as_uint(v[i].x) & 0x7FFFFFFFu);
+            m = max(m, __float_as_uint(v[i].y) & 0x7FFFFFFFu);
+            m = max(m, __float_as_uint(v[i].z) & 0x7FFFFFFFu);
+            m = max(m, __float_as_uint(v[i].w) & 0x7FFFFFFFu);
+        }
+        for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+        if (lane == 0) part[warp] = m;
+        __syncthreads();
+        m = part[0];
+        for (int w = 1; w < nwarps; ++w) m = max(m, part[w]);
+        const bool row_bad = m >= 0x7F800000u;  // NaN or infinity in the row
+        bad |= row_bad;
+        const GroupScale g = group_scale(row_bad ? 0.0f : __uint_as_float(m), qmax);
+        if (threadIdx.x == 0) scales[n] = g.s;
+        uint32_t* out = reinterpret_cast<uint32_t*>(codes + n * K);
+        if (g.normal) {
+            const float h = 0.5f * g.s;
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int idx = threadIdx.x + i * blockDim.x;
+                if (idx < K4) out[idx] = rtn4_f32(v[i], g.s, g.inv, h, fq);
+            }
+        } else {
+            bool unused = false;
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int idx = threadIdx.x + i * blockDim.x;
+                if (idx < K4) out[idx] = pack_codes4(v[i], g, qmax, unused);
+            }
+        }
+        __syncthreads();  // part[] is rewritten for the next row
+    }
+    if (bad) raise_error(ERRBIT_NONFINITE);
+}
+
 // Groups of L = group/4 threads (one float4 each); groups never straddle a
 // warp because L divides 32 and every row holds a whole number of groups.
+// Four float4 per thread are loaded before any is processed; absmax and RTN
+// as in quantize_rows_cta_kernel.
 __global__ void __launch_bounds__(256) quantize_groups_kernel(
     const float* __restrict__ W, int64_t total4, int lanes_per_group, int qmax,
     int8_t* __restrict__ codes, float* __restrict__ scales) {
+    constexpr int U = 4;
     const int lane = threadIdx.x & 31;
     const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     const float4* W4 = reinterpret_cast<const float4*>(W);
     uint32_t* out = reinterpret_cast<uint32_t*>(codes);
+    const float fq = static_cast<float>(qmax);
     bool bad = false;
-    for (int64_t base = warp0 * 32; base < total4; base += nwarps * 32) {
-        const int64_t i = base + lane;
-        const bool valid = i < total4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (valid) v = __ldg(W4 + i);
-        float a = 0.0f;
-        bool b2 = false;
-        a = abs_finite_max(a, v.x, b2);
-        a = abs_finite_max(a, v.y, b2);
-        a = abs_finite_max(a, v.z, b2);
-        a = abs_finite_max(a, v.w, b2);
-        for (int off = lanes_per_group >> 1; off > 0; off >>= 1)
-            a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-        if (valid) {
-            const GroupScale gs = group_scale(a, qmax);
+    for (int64_t base = warp0 * 32 * U; base < total4; base += nwarps * 32 * U) {
+        float4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = base + u * 32 + lane;
+            v[u] = i < total4 ? __ldcs(W4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = base + u * 32 + lane;
+            uint32_t m = max(max(__float_as_uint(v[u].x) & 0x7FFFFFFFu, __float_as_uint(v[u].y) & 0x7FFFFFFFu),
+                             max(__float_as_uint(v[u].z) & 0x7FFFFFFFu, __float_as_uint(v[u].w) & 0x7FFFFFFFu));
+            for (int off = lanes_per_group >> 1; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+            if (i >= total4) continue;
+            const bool gbad = m >= 0x7F800000u;  // NaN or infinity in the group
+            bad |= gbad;
+            const GroupScale gs = group_scale(gbad ? 0.0f : __uint_as_float(m), qmax);
             if ((lane & (lanes_per_group - 1)) == 0) scales[i / lanes_per_group] = gs.s;
-            out[i] = pack_codes4(v, gs, qmax, bad);
+            bool unused = false;
+            out[i] = gs.normal ? rtn4_f32(v[u], gs.s, gs.inv, 0.5f * gs.s, fq) : pack_codes4(v[u], gs, qmax, unused);
         }
     }
     if (bad) raise_error(ERRBIT_NONFINITE);

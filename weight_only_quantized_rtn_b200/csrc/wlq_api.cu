@@ -450,11 +450,17 @@ wlq_status wlq_quantize(const float* W, int64_t N, int64_t K, int bits, int grou
     if ((st = current_device(&dev, &d)) != WLQ_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int qmax = (1 << (bits - 1)) - 1;
-    if (group == 0) {
+    if (group == 0 && K <= 8 * 4 * 1024) {
+        // one CTA per row, the row held in registers (8 float4 per thread)
+        const int64_t per_thread = 8 * 4;
+        const int threads = static_cast<int>(std::min<int64_t>(1024, std::max<int64_t>(32, (cdiv(K, per_thread) + 31) / 32 * 32)));
+        const int grid = static_cast<int>(std::min<int64_t>(N, static_cast<int64_t>(d->sms) * (2048 / threads)));
+        wlq::quantize_rows_cta_kernel<8><<<grid, threads, 0, s>>>(W, N, K, qmax, codes, scales);
+    } else if (group == 0) {
         wlq::quantize_rows_kernel<<<grid_for(N * 32, 256, d->sms), 256, 0, s>>>(W, N, K, qmax, codes, scales);
     } else {
         const int64_t total4 = N * K / 4;
-        wlq::quantize_groups_kernel<<<grid_for(total4, 256, d->sms), 256, 0, s>>>(W, total4, group / 4, qmax,
+        wlq::quantize_groups_kernel<<<grid_for(cdiv(total4, 4), 256, d->sms), 256, 0, s>>>(W, total4, group / 4, qmax,
                                                                                    codes, scales);
     }
     cudaError_t e = cudaGetLastError();
@@ -487,7 +493,8 @@ wlq_status wlq_pack(const int8_t* codes, const float* scales, int64_t N, int64_t
     const int64_t G = group ? K / group : 1;
     uint8_t* base = static_cast<uint8_t*>(packed);
     float* rowf = reinterpret_cast<float*>(base + NT * KT * wlq::tile_bytes(fmt));
-    wlq::pack_rowfactor_kernel<<<grid_for(NT * 128 * 32, 256, d->sms), 256, 0, s>>>(scales, N, G, fmt, NT * 128, rowf);
+    if (fmt != wlq::FMT_W8)  // int8 row factors are written by the tile kernel itself
+        wlq::pack_rowfactor_kernel<<<grid_for(NT * 128 * 32, 256, d->sms), 256, 0, s>>>(scales, N, G, fmt, NT * 128, rowf);
     wlq::pack_tiles_kernel<<<static_cast<unsigned>(NT * KT), 128, 0, s>>>(codes, scales, N, K, G, fmt,
                                                                           static_cast<int>(KT), rowf, base);
     cudaError_t e = cudaGetLastError();
