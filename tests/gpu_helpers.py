@@ -55,7 +55,12 @@ def linear_case(x_bits, W, bits, group, b_bits=None, L1=None, L2=None, rows=None
     b = dev_bf16(b_bits) if b_bits is not None else None
     l1 = dev_bf16(L1) if L1 is not None else None
     l2 = dev_bf16(L2) if L2 is not None else None
-    y = wlq.linear(x, packed, N, K, bits, group, b, l1, l2, out_dtype=out_dtype)
+    # y starts as NaN, so an output the kernel never wrote cannot pass as a
+    # stale copy of an earlier correct result
+    M = x.shape[0]
+    y = torch.full((M, N), float("nan"), dtype=out_dtype, device=x.device)
+    ws = wlq.new_workspace(M, N, K, bits, group, 0 if l1 is None else l1.shape[1], device=x.device)
+    wlq.linear_into(y, x, packed, N, K, bits, group, b, l1, l2, workspace=ws)
     wlq.check_status()
     if rows is None:
         rows = np.arange(x_bits.shape[0])

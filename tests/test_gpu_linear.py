@@ -85,6 +85,9 @@ def test_parity_low_rank(bits, group, r, M):
     (600, 640, 640, 16, 5),    # low rank, single accumulator buffer, ring wrap-around
     (600, 4096, 448, 0, 0),    # CTA pairs (256 channels x 256 tokens per MMA), partial last slot
     (600, 4096, 1024, 0, 6),   # CTA pairs, three pairs for 48 tiles
+    (256, 512, 1024, 0, 16),   # split pairs: K split over four pairs, one tile per 8-CTA cluster
+    (512, 1024, 512, 0, 0),    # split pairs: two 256-token tiles per channel pair, K split over pairs
+    (256, 1920, 1024, 0, 0),   # odd channel-tile count: single-CTA 256-token tiles, K split over 4, partial in the ring
 ])
 def test_parity_several_tiles_per_cta(bits, group, M, N, K, r, cap):
     m = wlq()
@@ -118,7 +121,13 @@ def test_bitwise_reproducible(bits, group):
         codes, scales = m.quantize(dev_f32(W), bits, group)
         packed = m.pack(codes, scales, bits, group)
         args = (dev_bf16(x), packed, 1024, 1024, bits, group, dev_bf16(b), dev_bf16(L1), dev_bf16(L2))
-        ys = [m.linear(*args, out_dtype=torch.float32) for _ in range(3)]
+        ws = m.new_workspace(M, 1024, 1024, bits, group, 32)
+        ys = []
+        for _ in range(3):
+            # NaN never equals itself: an output left unwritten cannot pass
+            y = torch.full((M, 1024), float("nan"), dtype=torch.float32, device="cuda")
+            m.linear_into(y, *args, workspace=ws)
+            ys.append(y)
         assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
 
 

@@ -37,7 +37,7 @@ def test_noalloc_matches_workspace_entry_point_twice(bits, group, M, N, K, r):
     codes, scales = wlq.quantize(dev_f32(W), bits, group)
     packed = wlq.pack(codes, scales, bits, group)
     ws = wlq.new_workspace(M, N, K, bits, group, r)
-    y_ref = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    y_ref = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
     wlq.linear_into(y_ref, x, packed, N, K, bits, group, b, L1, L2, workspace=ws)
     ref = y_ref.cpu().numpy().astype(np.float64)
     for _ in range(2):

@@ -88,6 +88,7 @@ struct GemmArgs {
     uint32_t tmem_cols, acc_col0, lr_col0, a_col0;
     uint32_t wtile_bytes, wstage_bytes, xsub_bytes, xstage_bytes, red_bytes, stage_bytes;
     int vec_out;  // unsplit tiles store 16-byte runs of y rows (y 16-byte aligned, rows whole runs)
+    int red_alias;  // split partial kept in the ring's shared memory (one tile per cluster)
     uint64_t timeout_ns;
 };
 
@@ -96,18 +97,20 @@ struct TileCoord {
 };
 
 // Output tile g of this cluster.  Split clusters: every CTA takes K split
-// `rank` of the same 128-channel tile.  Pairs: CTA `rank` takes channel tile
-// 2 * (g % (NT / 2)) + rank over the whole K range.
+// `rank` of the same 128-channel tile.  Pairs: cluster rank 2p + i (i = 0, 1)
+// takes channel tile 2 * (g % (NT / 2)) + i over K split p (the whole K range
+// when S = 1), and ranks 2p, 2p + 1 share each MMA.
 template <bool PAIR>
 __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int g, int rank) {
     TileCoord c;
     if constexpr (PAIR) {
+        // cluster rank = 2 * split + (CTA within the pair)
         const int ntp = a.NT >> 1;
-        c.nt = (g % ntp) * 2 + rank;
+        c.nt = (g % ntp) * 2 + (rank & 1);
         c.mt = g / ntp;
-        c.sp = 0;
-        c.kb0 = 0;
-        c.kb1 = a.KT;
+        c.sp = rank >> 1;
+        c.kb0 = c.sp * a.kbps;
+        c.kb1 = min(a.KT, c.kb0 + a.kbps);
     } else {
         c.nt = g % a.NT;
         c.mt = g / a.NT;
@@ -276,7 +279,7 @@ template <bool PAIR, bool XRES>
 __device__ void producer_role(const GemmArgs& a, const CUtensorMap* tm_x, const CUtensorMap* tm_t,
                               const CUtensorMap* tm_l2, const Smem& s, const Sched& sc) {
     // in a pair each CTA stages its half of the tile's tokens
-    const int row0 = PAIR ? sc.rank * (a.BN >> 1) : 0;
+    const int row0 = PAIR ? (sc.rank & 1) * (a.BN >> 1) : 0;
     int it = 0, lrit = 0;
     Ring r;
     bool ok = true;
@@ -330,11 +333,15 @@ __device__ void producer_role(const GemmArgs& a, const CUtensorMap* tm_x, const 
     }
 }
 
+template <int FMT, bool PAIR>
+__device__ void crew_split_epilogue(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc, int warp,
+                                    int lane);
+
 template <int FMT, bool PAIR, bool XRES>
 __device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc, int warp,
                              int lane) {
     // in a pair, the A stage is consumed by the first CTA's MMA: signal there
-    const uint32_t afull_leader = PAIR ? mapa_shared(smem_u32(s.afull), 0) : 0u;
+    const uint32_t afull_leader = PAIR ? mapa_shared(smem_u32(s.afull), sc.rank & ~1) : 0u;
     const int q = warp & 3;   // TMEM lane quarter this warp may access
     const int h = warp >> 2;  // which 32 of the 64 inputs of a K block
     const int row = q * 32 + lane;
@@ -403,11 +410,12 @@ __device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, co
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                if (PAIR && sc.rank != 0) mbar_arrive_peer(afull_leader + st * 8u);
+                if (PAIR && (sc.rank & 1)) mbar_arrive_peer(afull_leader + st * 8u);
                 else mbar_arrive(&s.afull[at]);
             }
         }
     }
+    if (a.red_alias) crew_split_epilogue<FMT, PAIR>(a, tmem, s, sc, warp, lane);
 }
 
 template <int FMT, bool PAIR, bool XRES>
@@ -444,7 +452,7 @@ __device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const 
                     else mma_ts(d, acol + j * A_STAGE_COLS + kk * 8, bdesc + 2 * kk, idesc, acc);
                 }
             }
-            if constexpr (PAIR) mma_commit_pair_both(&s.empty[st]);
+            if constexpr (PAIR) mma_commit_pair_both(&s.empty[st], sc.rank);
             else mma_commit(XRES ? &s.aempty[st] : &s.empty[st]);
         }
         if (!ok) break;
@@ -462,7 +470,7 @@ __device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const 
             }
             if (!ok) break;
         }
-        if constexpr (PAIR) mma_commit_pair_both(&s.accfull[ab]);
+        if constexpr (PAIR) mma_commit_pair_both(&s.accfull[ab], sc.rank);
         else mma_commit(&s.accfull[ab]);
     }
     // make sure no MMA is still reading shared memory or TMEM when the CTA tears down
@@ -483,13 +491,16 @@ __device__ __forceinline__ void store_y(const GemmArgs& a, int m, int n, float v
 // warp and CTA) with eight vector loads in flight (8 / S tokens, S splits
 // each), then stores the four adjacent outputs as one vector.
 __device__ __forceinline__ void reduce_share(const GemmArgs& a, const float* red, int pitch, const TileCoord& c,
-                                             const Sched& sc, int m0, int share, int e, int nw, int lane) {
+                                             const Sched& sc, int m0, int share, int e, int nw, int lane,
+                                             bool pair = false) {
     const int nq = c.nt * 128 + 4 * lane;
     float bq[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) bq[i] = (a.bias && nq + i < a.N) ? bf16_to_f32(a.bias[nq + i]) : 0.0f;
-    const int j0 = sc.rank * share;
+    const int j0 = c.sp * share;
     const int lgS = __ffs(a.S) - 1;
+    // split r of these channels lives at cluster rank r (pairs: 2r + this CTA's place in its pair)
+    const int rshift = pair ? 1 : 0, rbase = pair ? (sc.rank & 1) : 0;
     const uint32_t red_local = smem_u32(red) + static_cast<uint32_t>(4 * lane) * 4u;
     const int step = nw * (8 >> lgS);  // tokens the nw warps cover per round
     for (int jt = e; jt < share; jt += step) {
@@ -498,7 +509,7 @@ __device__ __forceinline__ void reduce_share(const GemmArgs& a, const float* red
         for (int i = 0; i < 8; ++i) {
             const int tok = jt + nw * (i >> lgS);
             if (tok < share && m0 + j0 + tok < a.M)
-                part[i] = ld_dsmem_f32x4(mapa_shared(red_local, i & (a.S - 1)) +
+                part[i] = ld_dsmem_f32x4(mapa_shared(red_local, ((i & (a.S - 1)) << rshift) | rbase) +
                                          static_cast<uint32_t>((j0 + tok) * pitch) * 4u);
         }
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -541,23 +552,92 @@ __device__ __forceinline__ void reduce_share(const GemmArgs& a, const float* red
     }
 }
 
+// One tile per cluster with the split partial in the ring (256-token tiles):
+// the dequant warps have nothing left to do once the accumulator is complete,
+// so all twelve non-producer warps finish the tile.  Three warps share each
+// TMEM lane quarter (warp % 4) and take every third 16-token chunk of it to
+// write the partial; then the twelve sum a 1/S share of the tokens over the
+// cluster's partials.  Crew index: epilogue warps 0-3, dequant warps 4-11.
+constexpr int CREW_WARPS = NUM_DQ_WARPS + NUM_EPI_WARPS;
+template <int FMT, bool PAIR>
+__device__ void crew_split_epilogue(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc, int warp,
+                                    int lane) {
+    if (sc.cid >= a.tiles_nm) return;
+    const TileCoord c = tile_coord<PAIR>(a, sc.cid, sc.rank);
+    const bool epi = warp >= WARP_EPI0;
+    const int cw = epi ? warp - WARP_EPI0 : NUM_EPI_WARPS + warp;
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const int k = epi ? 0 : 1 + (warp >> 2);  // which of the quarter's three warps
+    const bool first_thread = (warp == WARP_EPI0 && lane == 0);
+    if (!warp_wait_or_abort(&s.accfull[0], 0, a, s.abort_flag, false, !epi)) return;
+    tc_fence_after();
+    const int n = c.nt * 128 + row;
+    const float rf = n < a.N ? a.rowf[n] : 0.0f;
+    const int m0 = c.mt * a.BN;
+    for (int cc = k; cc < a.BN / 16; cc += 3) {
+        uint32_t v[16];
+        tmem_ld16(tbase + a.acc_col0 + cc * 16, v);
+        tmem_wait_ld_pin(v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            float val = __uint_as_float(v[j]) * rf;
+            if constexpr (FMT != FMT_W8) {
+                const int m = m0 + cc * 16 + j;
+                val *= (m < a.M) ? a.xs[m] : 0.0f;
+            }
+            s.red[(cc * 16 + j) * 128 + row] = val;
+        }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(s.redw);
+    if (first_thread && wait_or_abort(s.redw, 0, a, s.abort_flag)) {
+        // the fence orders the partial at cluster scope; plain arrives follow
+        fence_acq_rel_cluster();
+        for (int r = 0; r < a.S; ++r) {
+            const int rk = PAIR ? (r << 1) | (sc.rank & 1) : r;
+            mbar_arrive_peer(mapa_shared(smem_u32(s.ready), rk));
+        }
+    }
+    if (!warp_wait_or_abort(s.ready, 0, a, s.abort_flag, true)) return;
+    reduce_share(a, s.red, 128, c, sc, m0, a.BN / a.S, cw, CREW_WARPS, lane, PAIR);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(s.readw);
+    if (first_thread && wait_or_abort(s.readw, 0, a, s.abort_flag)) {
+        fence_acq_rel_cluster();
+        for (int r = 0; r < a.S; ++r) {
+            const int rk = PAIR ? (r << 1) | (sc.rank & 1) : r;
+            mbar_arrive_peer(mapa_shared(smem_u32(s.freed), rk));
+        }
+    }
+    // no CTA of the cluster may still read this CTA's shared memory when it exits
+    warp_wait_or_abort(s.freed, 0, a, s.abort_flag, true);
+}
+
 template <int FMT, bool PAIR, bool XRES>
 __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc, int warp,
                               int lane) {
+    if (a.red_alias) {
+        crew_split_epilogue<FMT, PAIR>(a, tmem, s, sc, warp, lane);
+        return;
+    }
     // in a pair the accumulator is released to the first CTA's MMA thread
-    const uint32_t accempty_leader = PAIR ? mapa_shared(smem_u32(s.accempty), 0) : 0u;
+    const uint32_t accempty_leader = PAIR ? mapa_shared(smem_u32(s.accempty), sc.rank & ~1) : 0u;
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const bool first_thread = (warp == WARP_EPI0 && lane == 0);
     const bool split = a.S > 1;
-    // cluster addresses of every CTA's partial buffer and barriers
-    uint32_t red_at[MAX_SPLITS], ready_at[MAX_SPLITS], freed_at[MAX_SPLITS];
+    // cluster addresses of the barriers of every split of these channels
+    // (pairs: cluster rank 2 * split + this CTA's place in its pair)
+    uint32_t ready_at[MAX_SPLITS], freed_at[MAX_SPLITS];
     if (split) {
         for (int r = 0; r < a.S; ++r) {
-            red_at[r] = mapa_shared(smem_u32(s.red), r);
-            ready_at[r] = mapa_shared(smem_u32(s.ready), r);
-            freed_at[r] = mapa_shared(smem_u32(s.freed), r);
+            const int rk = PAIR ? (r << 1) | (sc.rank & 1) : r;
+            ready_at[r] = mapa_shared(smem_u32(s.ready), rk);
+            freed_at[r] = mapa_shared(smem_u32(s.freed), rk);
         }
     }
     const int share = a.BN / a.S;       // tokens of each tile this CTA sums (at least 8)
@@ -674,7 +754,7 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-            if (PAIR && sc.rank != 0) mbar_arrive_peer(accempty_leader + ab * 8u);
+            if (PAIR && (sc.rank & 1)) mbar_arrive_peer(accempty_leader + ab * 8u);
             else mbar_arrive(&s.accempty[ab]);
         }
         if (!split) continue;
@@ -689,7 +769,7 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
             for (int r = 0; r < a.S; ++r) mbar_arrive_peer(ready_at[r]);
         }
         if (!warp_wait_or_abort(s.ready, tc & 1, a, s.abort_flag, true)) return;
-        reduce_share(a, s.red, 128, c, sc, m0, share, warp - WARP_EPI0, NUM_EPI_WARPS, lane);
+        reduce_share(a, s.red, 128, c, sc, m0, share, warp - WARP_EPI0, NUM_EPI_WARPS, lane, PAIR);
         __syncwarp();
         if (lane == 0) mbar_arrive(s.readw);
         if (first_thread && wait_or_abort(s.readw, tc & 1, a, s.abort_flag)) {
@@ -705,6 +785,12 @@ template <int FMT, bool PAIR, bool XRES>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_t,
             const __grid_constant__ CUtensorMap tm_l2, const GemmArgs a) {
+    // a partial kept in the ring needs one tile per cluster (the host plans
+    // it so; refuse anything else)
+    if (a.red_alias && a.tiles_nm > static_cast<int>(cluster_count_x())) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) raise_error(ERRBIT_LAUNCH);
+        return;
+    }
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -716,6 +802,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     s.red = reinterpret_cast<float*>(s.lrB + (a.lr ? a.xsub_bytes : 0));
     s.stage = reinterpret_cast<uint8_t*>(s.red) + a.red_bytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(s.stage + a.stage_bytes);
+    // One tile per cluster: once the tile's accumulator is complete no MMA,
+    // copy or dequant warp touches the ring again, so a [BN][128] fp32 split
+    // partial too large to sit beside the ring reuses the ring's memory.
+    if (a.red_alias) s.red = reinterpret_cast<float*>(s.x);
     s.full = bars;
     s.empty = s.full + MAX_STAGES;
     s.afull = s.empty + MAX_STAGES;
@@ -753,8 +843,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
         mbar_init(s.lrfull, 1);
         mbar_init(s.lrempty, 1);
         mbar_init(s.drain, 1);
-        mbar_init(s.redw, NUM_EPI_WARPS);
-        mbar_init(s.readw, NUM_EPI_WARPS);
+        mbar_init(s.redw, a.red_alias ? CREW_WARPS : NUM_EPI_WARPS);
+        mbar_init(s.readw, a.red_alias ? CREW_WARPS : NUM_EPI_WARPS);
         mbar_init(s.ready, a.S);
         mbar_init(s.freed, a.S);
         *s.abort_flag = 0;
@@ -786,7 +876,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
         epilogue_role<FMT, PAIR, XRES>(a, tmem, s, sc, warp, lane);
     } else if (warp == WARP_PRODUCER) {
         if (lane == 0) producer_role<PAIR, XRES>(a, &tm_x, &tm_t, &tm_l2, s, sc);
-    } else if (lane == 0 && (!PAIR || sc.rank == 0)) {
+    } else if (lane == 0 && (!PAIR || (sc.rank & 1) == 0)) {
         mma_role<FMT, PAIR, XRES>(a, tmem, s, sc);
     }
 

@@ -10,7 +10,7 @@
 namespace wlq {
 
 // Device error word (one per device that loads the library).
-enum : unsigned { ERRBIT_NONFINITE = 1u, ERRBIT_TIMEOUT = 2u };
+enum : unsigned { ERRBIT_NONFINITE = 1u, ERRBIT_TIMEOUT = 2u, ERRBIT_LAUNCH = 4u };
 __device__ unsigned int g_error_word;
 
 __device__ __forceinline__ void raise_error(unsigned bit) { atomicOr(&g_error_word, bit); }
@@ -171,12 +171,14 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
         : "memory");
 }
 // The same completion signalled on the mbarrier at `bar`'s offset in BOTH CTAs
-// of the pair (CTA mask 0b11): a completion notice, not a data copy.
-__device__ __forceinline__ void mma_commit_pair_both(uint64_t* bar) {
+// of the pair (cluster ranks leader_rank and leader_rank + 1): a completion
+// notice, not a data copy.
+__device__ __forceinline__ void mma_commit_pair_both(uint64_t* bar, uint32_t leader_rank) {
+    const uint16_t mask = static_cast<uint16_t>(3u << leader_rank);  // the pair's two cluster ranks
     asm volatile(
-        "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
-            smem_u32(bar))
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(mask)
         : "memory");
 }
 __device__ __forceinline__ void cluster_sync_all() {

@@ -129,6 +129,7 @@ struct Plan {
     bool pair = false;  // two CTAs per MMA (cta_group::2)
     bool xres = false;  // x resident in shared memory; weight ring released by the dequant warps
     bool skinny = false;  // one token tile of <= 64 tokens: the warp-MMA streaming kernel
+    bool red_alias = false;  // split partial in the ring's memory (one tile per cluster)
     int astages = 0;    // resident x: TMEM A-stage ring depth
     uint32_t tmem_cols = 0, acc_col0 = 0, lr_col0 = 0, a_col0 = 0, wtile = 0, wstage = 0, xsub = 0, xstage = 0, red = 0, stage = 0;
     size_t smem = 0;
@@ -145,9 +146,20 @@ int token_tile(int64_t M, int r) {
     return 256;
 }
 
+int g_grid_limit = 0;  // 0: no cap on the GEMM's CTAs (see wlq_set_grid_limit)
+
+// Returned by a launcher when the plan's cluster shape cannot get one tile per
+// cluster on this device; the caller plans again without split pairs.
+constexpr wlq_status kRetryPlan = static_cast<wlq_status>(-100);
+
 // Launch plan: token tile BN, K split S (a power of two up to 8, the CTAs of
 // one cluster), TMEM columns, shared-memory ring depth, workspace layout.
-bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms) {
+// variant 0: CTA pairs may split K (over up to four pairs of a cluster);
+// variant 1: no split pairs, but 256-token tiles may split K (partial in the
+// ring); variant 2: splits use 128-token tiles (partial beside the ring).
+// Variants 0 and 1 need one tile per cluster; the launcher reports
+// kRetryPlan when the device cannot hold that many clusters.
+bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms, int variant = 0) {
     p.fmt = fmt;
     p.M = static_cast<int>(M);
     p.N = static_cast<int>(N);
@@ -158,11 +170,24 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     p.lr_kb = r ? static_cast<int>(cdiv(2 * r, 64)) : 0;
     p.BN = token_tile(M, r);
     p.MT = static_cast<int>(cdiv(M, p.BN));
-    // Split K when the output tiles cannot cover half of the SMs.  A split
-    // tile keeps at most 128 tokens (its fp32 partial sits in shared memory).
+    // Few 256-token tiles: CTA pairs, with the K range split over up to four
+    // pairs of one cluster when plain pairs would leave most SMs idle.  Each
+    // cluster then holds exactly one tile (its partial reuses the ring).
+    const int cap = (g_grid_limit > 0) ? std::min(g_grid_limit, sms) : sms;
     int S = 1;
-    if (p.NT * p.MT * 2 <= sms) {
-        if (p.BN > 128) {
+    bool pair_split = false;
+    if (variant == 0 && r == 0 && p.BN == 256 && p.NT % 2 == 0) {
+        const int64_t tp = static_cast<int64_t>(p.NT / 2) * p.MT;  // pair tiles
+        if (tp * 2 * 2 <= cap) {
+            while (S * 2 <= 4 && tp * 2 * (S * 2) <= cap && p.KT >= S * 2 * 4) S *= 2;
+            pair_split = S > 1;
+        }
+    }
+    // Split K when the output tiles cannot cover half of the SMs.  128-token
+    // split tiles keep their fp32 partial beside the ring; 256-token ones
+    // (variants 0-1, no low-rank term) keep it in the ring's memory.
+    if (!pair_split && p.NT * p.MT * 2 <= sms) {
+        if (p.BN > 128 && (variant == 2 || r != 0)) {
             p.BN = 128;
             p.MT = static_cast<int>(cdiv(M, p.BN));
         }
@@ -179,7 +204,9 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     p.S = S;
     if (S > 1 && p.BN % S != 0) return false;  // every CTA of a split cluster sums whole tokens
     // CTA pairs for large token tiles: two 128-channel tiles share each MMA
-    p.pair = (r == 0 && S == 1 && p.BN == 256 && p.NT % 2 == 0);
+    if (pair_split && S == 1) pair_split = false;  // the K range was too short to split
+    p.pair = (r == 0 && p.BN == 256 && p.NT % 2 == 0) && (S == 1 || pair_split);
+    p.red_alias = S > 1 && p.BN == 256;  // split 256-token tiles: pairs or single CTAs
     p.tiles_nm = p.pair ? (p.NT / 2) * p.MT : p.NT * p.MT;
     // TMEM: accumulator(s) first, from column 0, so each starts at a multiple
     // of its own width (main accumulators at ab*BN, low-rank ones after them);
@@ -193,7 +220,8 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     // shared memory: ring slots + low-rank tiles + split partial + barriers
     p.wtile = wlq::tile_bytes(fmt);
     p.xsub = static_cast<uint32_t>(p.pair ? p.BN / 2 : p.BN) * 128u;  // a pair's CTA stages half the tokens
-    p.red = (S > 1) ? static_cast<uint32_t>(p.BN) * 128u * 4u : 0u;  // token-major fp32 partial
+    // token-major fp32 partial (256-token split tiles: in the ring's memory)
+    p.red = (S > 1 && !p.red_alias) ? static_cast<uint32_t>(p.BN) * 128u * 4u : 0u;
     const size_t lr_bytes = r ? (wlq::LR_TILE_A_BYTES + p.xsub) : 0;
     p.stage = (S == 1) ? wlq::NUM_EPI_WARPS * wlq::EPI_STAGE_BYTES : 0u;  // epilogue transpose buffers
     const size_t fixed = 1024 /* alignment */ + 1024 /* barriers */ + lr_bytes + p.red + p.stage;
@@ -279,6 +307,8 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
         }
     }
     if (p.ks == 0) return false;
+    if (p.red_alias && p.stages * static_cast<size_t>(p.xstage + p.wstage) < static_cast<size_t>(p.BN) * 128u * 4u)
+        return variant < 2 ? make_plan(p, M, N, K, fmt, r, sms, variant + 1) : false;
     p.acc_col0 = 0;
     p.lr_col0 = p.acc_bufs * static_cast<uint32_t>(p.BN);
     p.a_col0 = a_col0;
@@ -308,7 +338,6 @@ wlq_status check_shape(int64_t N, int64_t K, int bits, int group) {
     return WLQ_OK;
 }
 
-int g_grid_limit = 0;  // 0: no cap on the GEMM's CTAs (see wlq_set_grid_limit)
 
 template <int FMT, bool PAIR, bool XRES>
 wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, const CUtensorMap& tl,
@@ -321,7 +350,7 @@ wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, co
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         d->smem_set[kid] = true;
     }
-    const int csize = PAIR ? 2 : p.S;  // CTAs per cluster
+    const int csize = PAIR ? 2 * p.S : p.S;  // CTAs per cluster
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
     cudaLaunchAttribute attr[1];
@@ -356,6 +385,8 @@ wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, co
         }
         clusters = std::min(clusters, active);
     }
+    // a partial kept in the ring needs one tile per cluster
+    if (p.red_alias && clusters < p.tiles_nm) return kRetryPlan;
     cfg.gridDim = dim3(static_cast<unsigned>(clusters * csize), 1, 1);
     p.grid = clusters * csize;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tx, tt, tl, a);
@@ -424,6 +455,63 @@ wlq_status launch_skinny_nb(Plan& p, const CUtensorMap& tx, wlq::GemmArgs& a, De
 int grid_for(int64_t work, int per_block, int sms) {
     const int64_t b = cdiv(std::max<int64_t>(work, 1), per_block);
     return static_cast<int>(std::min<int64_t>(b, int64_t(sms) * 32));
+}
+
+wlq_status launch_linear(Plan& p, int fmt, int64_t M, int64_t N, int64_t K, int r, const void* xin, float* xs,
+                         uint16_t* thl, uint16_t* l2t, int W, const void* packed, const void* bias, void* y,
+                         int y_dtype, DeviceInfo* d, cudaStream_t s) {
+    wlq_status st;
+    const int64_t NT = p.NT, KT = p.KT;
+    // --- descriptors
+    CUtensorMap tx, tt, tl;
+    std::memset(&tt, 0, sizeof tt);
+    std::memset(&tl, 0, sizeof tl);
+    if ((st = make_map_2d(&tx, xin, M, K, p.pair ? p.BN / 2 : p.BN)) != WLQ_OK) return st;
+    if (r) {
+        if ((st = make_map_2d(&tt, thl, M, W, p.BN)) != WLQ_OK) return st;
+        if ((st = make_map_2d(&tl, l2t, NT * 128, W, 128)) != WLQ_OK) return st;
+    }
+    wlq::GemmArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.packed = static_cast<const uint8_t*>(packed);
+    a.rowf = reinterpret_cast<const float*>(a.packed + NT * KT * wlq::tile_bytes(fmt));
+    a.xs = xs;
+    a.bias = static_cast<const uint16_t*>(bias);
+    a.y = y;
+    a.M = p.M; a.N = p.N; a.K = p.K;
+    a.NT = p.NT; a.KT = p.KT; a.MT = p.MT; a.S = p.S; a.kbps = p.kbps; a.BN = p.BN;
+    a.stages = p.stages; a.astages = p.astages; a.ks = p.ks; a.lr = r ? 1 : 0; a.lr_kb = p.lr_kb; a.acc_bufs = p.acc_bufs;
+    a.y_f32 = (y_dtype == WLQ_OUT_F32) ? 1 : 0;
+    a.tiles_nm = p.tiles_nm;
+    a.tmem_cols = p.tmem_cols; a.acc_col0 = p.acc_col0; a.lr_col0 = p.lr_col0; a.a_col0 = p.a_col0;
+    a.wtile_bytes = p.wtile; a.wstage_bytes = p.wstage; a.xsub_bytes = p.xsub; a.xstage_bytes = p.xstage; a.red_bytes = p.red;
+    a.stage_bytes = p.stage;
+    a.red_alias = p.red_alias ? 1 : 0;
+    // vector stores of y: unsplit tiles store 16-byte runs (4 fp32 / 8 bf16
+    // channels), the split reduction 4 adjacent channels (16 / 8 bytes)
+    {
+        const uintptr_t ya = reinterpret_cast<uintptr_t>(y);
+        const bool f32 = y_dtype == WLQ_OUT_F32;
+        if (p.S == 1) a.vec_out = ((ya & 15u) == 0 && N % (f32 ? 4 : 8) == 0) ? 1 : 0;
+        else a.vec_out = ((ya & (f32 ? 15u : 7u)) == 0 && N % 4 == 0) ? 1 : 0;
+    }
+    a.timeout_ns = kDefaultTimeoutNs;
+    if (p.skinny) {
+        if (fmt == wlq::FMT_W8) return launch_skinny_nb<wlq::FMT_W8>(p, tx, a, d, s);
+        if (fmt == wlq::FMT_W4G64) return launch_skinny_nb<wlq::FMT_W4G64>(p, tx, a, d, s);
+        return launch_skinny_nb<wlq::FMT_W4G16>(p, tx, a, d, s);
+    }
+    switch (fmt * 3 + (p.pair ? 1 : 0) + (p.xres ? 2 : 0)) {
+        case 0: return launch_gemm<wlq::FMT_W8, false, false>(p, tx, tt, tl, a, d, s);
+        case 1: return launch_gemm<wlq::FMT_W8, true, false>(p, tx, tt, tl, a, d, s);
+        case 2: return launch_gemm<wlq::FMT_W8, false, true>(p, tx, tt, tl, a, d, s);
+        case 3: return launch_gemm<wlq::FMT_W4G64, false, false>(p, tx, tt, tl, a, d, s);
+        case 4: return launch_gemm<wlq::FMT_W4G64, true, false>(p, tx, tt, tl, a, d, s);
+        case 5: return launch_gemm<wlq::FMT_W4G64, false, true>(p, tx, tt, tl, a, d, s);
+        case 6: return launch_gemm<wlq::FMT_W4G16, false, false>(p, tx, tt, tl, a, d, s);
+        case 7: return launch_gemm<wlq::FMT_W4G16, true, false>(p, tx, tt, tl, a, d, s);
+        default: return launch_gemm<wlq::FMT_W4G16, false, true>(p, tx, tt, tl, a, d, s);
+    }
 }
 
 }  // namespace
@@ -593,56 +681,17 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "prep launch");
 
-    // --- descriptors
-    CUtensorMap tx, tt, tl;
-    std::memset(&tt, 0, sizeof tt);
-    std::memset(&tl, 0, sizeof tl);
-    if ((st = make_map_2d(&tx, xin, M, K, p.pair ? p.BN / 2 : p.BN)) != WLQ_OK) return st;
-    if (r) {
-        if ((st = make_map_2d(&tt, thl, M, W, p.BN)) != WLQ_OK) return st;
-        if ((st = make_map_2d(&tl, l2t, NT * 128, W, 128)) != WLQ_OK) return st;
+    // plans that keep a split partial in the ring need one tile per cluster:
+    // if the device cannot hold that many clusters, take the next variant
+    for (int attempt = 0; attempt < 3; ++attempt) {
+        if (attempt > 0 && !make_plan(p, M, N, K, fmt, r, d->sms, attempt))
+            return fail(WLQ_ERR_UNSUPPORTED, "no launch plan for this shape");
+        st = launch_linear(p, fmt, M, N, K, r, xin, xs, thl, l2t, W, packed, bias, y, y_dtype, d, s);
+        if (st != kRetryPlan) return st;
     }
-    wlq::GemmArgs a;
-    std::memset(&a, 0, sizeof a);
-    a.packed = static_cast<const uint8_t*>(packed);
-    a.rowf = reinterpret_cast<const float*>(a.packed + NT * KT * wlq::tile_bytes(fmt));
-    a.xs = xs;
-    a.bias = static_cast<const uint16_t*>(bias);
-    a.y = y;
-    a.M = p.M; a.N = p.N; a.K = p.K;
-    a.NT = p.NT; a.KT = p.KT; a.MT = p.MT; a.S = p.S; a.kbps = p.kbps; a.BN = p.BN;
-    a.stages = p.stages; a.astages = p.astages; a.ks = p.ks; a.lr = r ? 1 : 0; a.lr_kb = p.lr_kb; a.acc_bufs = p.acc_bufs;
-    a.y_f32 = (y_dtype == WLQ_OUT_F32) ? 1 : 0;
-    a.tiles_nm = p.tiles_nm;
-    a.tmem_cols = p.tmem_cols; a.acc_col0 = p.acc_col0; a.lr_col0 = p.lr_col0; a.a_col0 = p.a_col0;
-    a.wtile_bytes = p.wtile; a.wstage_bytes = p.wstage; a.xsub_bytes = p.xsub; a.xstage_bytes = p.xstage; a.red_bytes = p.red;
-    a.stage_bytes = p.stage;
-    // vector stores of y: unsplit tiles store 16-byte runs (4 fp32 / 8 bf16
-    // channels), the split reduction 4 adjacent channels (16 / 8 bytes)
-    {
-        const uintptr_t ya = reinterpret_cast<uintptr_t>(y);
-        const bool f32 = y_dtype == WLQ_OUT_F32;
-        if (p.S == 1) a.vec_out = ((ya & 15u) == 0 && N % (f32 ? 4 : 8) == 0) ? 1 : 0;
-        else a.vec_out = ((ya & (f32 ? 15u : 7u)) == 0 && N % 4 == 0) ? 1 : 0;
-    }
-    a.timeout_ns = kDefaultTimeoutNs;
-    if (p.skinny) {
-        if (fmt == wlq::FMT_W8) return launch_skinny_nb<wlq::FMT_W8>(p, tx, a, d, s);
-        if (fmt == wlq::FMT_W4G64) return launch_skinny_nb<wlq::FMT_W4G64>(p, tx, a, d, s);
-        return launch_skinny_nb<wlq::FMT_W4G16>(p, tx, a, d, s);
-    }
-    switch (fmt * 3 + (p.pair ? 1 : 0) + (p.xres ? 2 : 0)) {
-        case 0: return launch_gemm<wlq::FMT_W8, false, false>(p, tx, tt, tl, a, d, s);
-        case 1: return launch_gemm<wlq::FMT_W8, true, false>(p, tx, tt, tl, a, d, s);
-        case 2: return launch_gemm<wlq::FMT_W8, false, true>(p, tx, tt, tl, a, d, s);
-        case 3: return launch_gemm<wlq::FMT_W4G64, false, false>(p, tx, tt, tl, a, d, s);
-        case 4: return launch_gemm<wlq::FMT_W4G64, true, false>(p, tx, tt, tl, a, d, s);
-        case 5: return launch_gemm<wlq::FMT_W4G64, false, true>(p, tx, tt, tl, a, d, s);
-        case 6: return launch_gemm<wlq::FMT_W4G16, false, false>(p, tx, tt, tl, a, d, s);
-        case 7: return launch_gemm<wlq::FMT_W4G16, true, false>(p, tx, tt, tl, a, d, s);
-        default: return launch_gemm<wlq::FMT_W4G16, false, true>(p, tx, tt, tl, a, d, s);
-    }
+    return fail(WLQ_ERR_UNSUPPORTED, "no launch plan for this shape");
 }
+
 
 }  // extern "C"
 
@@ -717,6 +766,7 @@ wlq_status wlq_get_status(void* stream) {
     }
     if (word & wlq::ERRBIT_TIMEOUT) return fail(WLQ_ERR_TIMEOUT, "a bounded device wait ran out");
     if (word & wlq::ERRBIT_NONFINITE) return fail(WLQ_ERR_NONFINITE, "non-finite weight");
+    if (word & wlq::ERRBIT_LAUNCH) return fail(WLQ_ERR_CUDA, "a kernel was launched with a shape it cannot run");
     return WLQ_OK;
 }
 
