@@ -88,6 +88,8 @@ def test_parity_low_rank(bits, group, r, M):
     (256, 512, 1024, 0, 16),   # split pairs: K split over four pairs, one tile per 8-CTA cluster
     (512, 1024, 512, 0, 0),    # split pairs: two 256-token tiles per channel pair, K split over pairs
     (256, 1920, 1024, 0, 0),   # odd channel-tile count: single-CTA 256-token tiles, K split over 4, partial in the ring
+    (512, 4096, 512, 0, 12),   # pairs in clusters of two pairs: 30 tiles in full rounds, 2 leftover tiles K-halved
+    (1024, 2048, 1024, 0, 20), # the same with five clusters: 30 full, 2 leftover
 ])
 def test_parity_several_tiles_per_cta(bits, group, M, N, K, r, cap):
     m = wlq()

@@ -72,7 +72,11 @@ constexpr uint32_t LR_TILE_A_BYTES = 128 * 128;  // 128 rows x 64 bf16
 constexpr uint64_t DRAIN_TIMEOUT_NS = 200ull * 1000 * 1000;
 constexpr int MAX_SPLITS = 8;
 constexpr int MAX_KS = 4;  // 64-wide K blocks per ring slot, at most
-constexpr uint32_t EPI_STAGE_BYTES = 2048;  // per epilogue warp: 16 tokens x 32 channels (fp32, or bf16 + one pad row)
+// per epilogue warp: 16 tokens x 32 channels in fp32, or two such chunks in
+// bf16 (16 rows of 64 bytes plus one pad row, 1152 bytes each)
+constexpr int EPI_CHUNKS = 2;
+constexpr uint32_t EPI_STAGE_BYTES = 2304;
+constexpr uint32_t EPI_BF16_CHUNK_BYTES = 1152;
 
 struct GemmArgs {
     const uint8_t* packed;
@@ -88,12 +92,17 @@ struct GemmArgs {
     uint32_t tmem_cols, acc_col0, lr_col0, a_col0;
     uint32_t wtile_bytes, wstage_bytes, xsub_bytes, xstage_bytes, red_bytes, stage_bytes;
     int vec_out;  // unsplit tiles store 16-byte runs of y rows (y 16-byte aligned, rows whole runs)
-    int red_alias;  // split partial kept in the ring's shared memory (one tile per cluster)
+    int red_alias;  // a CTA's last unit may be split, its partial kept in the ring's shared memory
+    int tail;       // pairs in clusters of two pairs: the tiles beyond the last full round are
+                    // each split over the K halves of one cluster's two pairs
+    int tiles_full; // tail: tiles dealt in full rounds (a multiple of 2 x clusters)
+    int S_red;      // CTAs summed by a split unit's reduction
     uint64_t timeout_ns;
 };
 
 struct TileCoord {
     int nt, mt, sp, kb0, kb1;
+    bool split;  // this unit's partial is summed over a cluster reduction
 };
 
 // Output tile g of this cluster.  Split clusters: every CTA takes K split
@@ -103,6 +112,7 @@ struct TileCoord {
 template <bool PAIR>
 __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int g, int rank) {
     TileCoord c;
+    c.split = a.S > 1;
     if constexpr (PAIR) {
         // cluster rank = 2 * split + (CTA within the pair)
         const int ntp = a.NT >> 1;
@@ -168,6 +178,46 @@ __device__ __forceinline__ Sched sched() {
     s.ncl = static_cast<int>(cluster_count_x());
     s.rank = static_cast<int>(cluster_ctarank());
     return s;
+}
+
+// Work unit u of this CTA (u = 0, 1, ...); false once the CTA has no more.
+// Tail mode (pairs in clusters of two pairs, virtual pair v = 2 * cluster +
+// pair): tile v + u * P for P = 2 * clusters while below tiles_full, each over
+// the whole K range; then, for cluster c < tiles_nm - tiles_full, tile
+// tiles_full + c with its K range halved between the cluster's two pairs.
+// Otherwise tile cluster + u * clusters, as tile_coord places it.
+template <bool PAIR>
+__device__ __forceinline__ bool unit_coord(const GemmArgs& a, const Sched& sc, int u, TileCoord& c) {
+    if (PAIR && a.tail) {
+        const int P = 2 * sc.ncl;
+        const int pp = sc.rank >> 1;
+        const int ntp = a.NT >> 1;
+        int g = 2 * sc.cid + pp + u * P;
+        const int rounds = a.tiles_full / P;
+        if (u < rounds) {
+            c.nt = (g % ntp) * 2 + (sc.rank & 1);
+            c.mt = g / ntp;
+            c.sp = 0;
+            c.kb0 = 0;
+            c.kb1 = a.KT;
+            c.split = false;
+            return true;
+        }
+        if (u > rounds || sc.cid >= a.tiles_nm - a.tiles_full) return false;
+        g = a.tiles_full + sc.cid;
+        const int kbh = (a.KT + 1) >> 1;
+        c.nt = (g % ntp) * 2 + (sc.rank & 1);
+        c.mt = g / ntp;
+        c.sp = pp;
+        c.kb0 = pp * kbh;
+        c.kb1 = min(a.KT, c.kb0 + kbh);
+        c.split = true;
+        return true;
+    }
+    const int g = sc.cid + u * sc.ncl;
+    if (g >= a.tiles_nm) return false;
+    c = tile_coord<PAIR>(a, g, sc.rank);
+    return true;
 }
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, const GemmArgs& a,
@@ -284,8 +334,8 @@ __device__ void producer_role(const GemmArgs& a, const CUtensorMap* tm_x, const 
     Ring r;
     bool ok = true;
     bool x_issued = false;
-    for (int g = sc.cid; g < a.tiles_nm && ok; g += sc.ncl) {
-        const TileCoord c = tile_coord<PAIR>(a, g, sc.rank);
+    TileCoord c;
+    for (int u = 0; ok && unit_coord<PAIR>(a, sc, u, c); ++u) {
         if (XRES && !x_issued) {
             // resident x: every tile of this CTA has the same tokens (one token
             // tile) and the same K range (its split), so x is loaded once
@@ -335,7 +385,7 @@ __device__ void producer_role(const GemmArgs& a, const CUtensorMap* tm_x, const 
 
 template <int FMT, bool PAIR>
 __device__ void crew_split_epilogue(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc, int warp,
-                                    int lane);
+                                    int lane, int u, const TileCoord& c);
 
 template <int FMT, bool PAIR, bool XRES>
 __device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc, int warp,
@@ -347,8 +397,9 @@ __device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, co
     const int row = q * 32 + lane;
     const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
     Ring r, ra;
-    for (int g = sc.cid; g < a.tiles_nm; g += sc.ncl) {
-        const TileCoord c = tile_coord<PAIR>(a, g, sc.rank);
+    TileCoord c;
+    int u = 0;
+    for (; unit_coord<PAIR>(a, sc, u, c); ++u) {
         for (int kb = c.kb0; kb < c.kb1; kb += a.ks, r.next(a.stages), ra.next(a.astages)) {
             const int nkb = min(a.ks, c.kb1 - kb);
             const int st = r.slot;
@@ -415,7 +466,9 @@ __device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, co
             }
         }
     }
-    if (a.red_alias) crew_split_epilogue<FMT, PAIR>(a, tmem, s, sc, warp, lane);
+    // a split last unit with its partial in the ring: help finish it
+    if (a.red_alias && u > 0 && unit_coord<PAIR>(a, sc, u - 1, c) && c.split)
+        crew_split_epilogue<FMT, PAIR>(a, tmem, s, sc, warp, lane, u - 1, c);
 }
 
 template <int FMT, bool PAIR, bool XRES>
@@ -427,8 +480,8 @@ __device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const 
     Ring r;
     bool ok = true;
     if (XRES && !wait_or_abort(s.xfull, 0, a, s.abort_flag)) ok = false;
-    for (int g = sc.cid; g < a.tiles_nm && ok; g += sc.ncl, ++tc) {
-        const TileCoord c = tile_coord<PAIR>(a, g, sc.rank);
+    TileCoord c;
+    for (; ok && unit_coord<PAIR>(a, sc, tc, c); ++tc) {
         const int ab = tc % a.acc_bufs;
         if (!wait_or_abort(&s.accempty[ab], ((tc / a.acc_bufs) & 1) ^ 1, a, s.abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -491,14 +544,14 @@ __device__ __forceinline__ void store_y(const GemmArgs& a, int m, int n, float v
 // warp and CTA) with eight vector loads in flight (8 / S tokens, S splits
 // each), then stores the four adjacent outputs as one vector.
 __device__ __forceinline__ void reduce_share(const GemmArgs& a, const float* red, int pitch, const TileCoord& c,
-                                             const Sched& sc, int m0, int share, int e, int nw, int lane,
+                                             const Sched& sc, int m0, int share, int e, int nw, int lane, int S,
                                              bool pair = false) {
     const int nq = c.nt * 128 + 4 * lane;
     float bq[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) bq[i] = (a.bias && nq + i < a.N) ? bf16_to_f32(a.bias[nq + i]) : 0.0f;
     const int j0 = c.sp * share;
-    const int lgS = __ffs(a.S) - 1;
+    const int lgS = __ffs(S) - 1;
     // split r of these channels lives at cluster rank r (pairs: 2r + this CTA's place in its pair)
     const int rshift = pair ? 1 : 0, rbase = pair ? (sc.rank & 1) : 0;
     const uint32_t red_local = smem_u32(red) + static_cast<uint32_t>(4 * lane) * 4u;
@@ -509,13 +562,13 @@ __device__ __forceinline__ void reduce_share(const GemmArgs& a, const float* red
         for (int i = 0; i < 8; ++i) {
             const int tok = jt + nw * (i >> lgS);
             if (tok < share && m0 + j0 + tok < a.M)
-                part[i] = ld_dsmem_f32x4(mapa_shared(red_local, ((i & (a.S - 1)) << rshift) | rbase) +
+                part[i] = ld_dsmem_f32x4(mapa_shared(red_local, ((i & (S - 1)) << rshift) | rbase) +
                                          static_cast<uint32_t>((j0 + tok) * pitch) * 4u);
         }
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const int r = i & (a.S - 1);
+            const int r = i & (S - 1);
             const int tok = jt + nw * (i >> lgS);
             if (tok >= share || m0 + j0 + tok >= a.M) break;
             if (r == 0) {
@@ -526,7 +579,7 @@ __device__ __forceinline__ void reduce_share(const GemmArgs& a, const float* red
                 acc.z += part[i].z;
                 acc.w += part[i].w;
             }
-            if (r != a.S - 1) continue;
+            if (r != S - 1) continue;
             const float o[4] = {acc.x + bq[0], acc.y + bq[1], acc.z + bq[2], acc.w + bq[3]};
             const int m = m0 + j0 + tok;
             if (a.vec_out) {
@@ -561,9 +614,9 @@ __device__ __forceinline__ void reduce_share(const GemmArgs& a, const float* red
 constexpr int CREW_WARPS = NUM_DQ_WARPS + NUM_EPI_WARPS;
 template <int FMT, bool PAIR>
 __device__ void crew_split_epilogue(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc, int warp,
-                                    int lane) {
-    if (sc.cid >= a.tiles_nm) return;
-    const TileCoord c = tile_coord<PAIR>(a, sc.cid, sc.rank);
+                                    int lane, int u, const TileCoord& c) {
+    const int S = a.S_red;
+    const int ab = u % a.acc_bufs;
     const bool epi = warp >= WARP_EPI0;
     const int cw = epi ? warp - WARP_EPI0 : NUM_EPI_WARPS + warp;
     const int q = warp & 3;
@@ -571,14 +624,14 @@ __device__ void crew_split_epilogue(const GemmArgs& a, uint32_t tmem, const Smem
     const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const int k = epi ? 0 : 1 + (warp >> 2);  // which of the quarter's three warps
     const bool first_thread = (warp == WARP_EPI0 && lane == 0);
-    if (!warp_wait_or_abort(&s.accfull[0], 0, a, s.abort_flag, false, !epi)) return;
+    if (!warp_wait_or_abort(&s.accfull[ab], (u / a.acc_bufs) & 1, a, s.abort_flag, false, !epi)) return;
     tc_fence_after();
     const int n = c.nt * 128 + row;
     const float rf = n < a.N ? a.rowf[n] : 0.0f;
     const int m0 = c.mt * a.BN;
     for (int cc = k; cc < a.BN / 16; cc += 3) {
         uint32_t v[16];
-        tmem_ld16(tbase + a.acc_col0 + cc * 16, v);
+        tmem_ld16(tbase + a.acc_col0 + ab * a.BN + cc * 16, v);
         tmem_wait_ld_pin(v);
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -596,18 +649,18 @@ __device__ void crew_split_epilogue(const GemmArgs& a, uint32_t tmem, const Smem
     if (first_thread && wait_or_abort(s.redw, 0, a, s.abort_flag)) {
         // the fence orders the partial at cluster scope; plain arrives follow
         fence_acq_rel_cluster();
-        for (int r = 0; r < a.S; ++r) {
+        for (int r = 0; r < S; ++r) {
             const int rk = PAIR ? (r << 1) | (sc.rank & 1) : r;
             mbar_arrive_peer(mapa_shared(smem_u32(s.ready), rk));
         }
     }
     if (!warp_wait_or_abort(s.ready, 0, a, s.abort_flag, true)) return;
-    reduce_share(a, s.red, 128, c, sc, m0, a.BN / a.S, cw, CREW_WARPS, lane, PAIR);
+    reduce_share(a, s.red, 128, c, sc, m0, a.BN / S, cw, CREW_WARPS, lane, S, PAIR);
     __syncwarp();
     if (lane == 0) mbar_arrive(s.readw);
     if (first_thread && wait_or_abort(s.readw, 0, a, s.abort_flag)) {
         fence_acq_rel_cluster();
-        for (int r = 0; r < a.S; ++r) {
+        for (int r = 0; r < S; ++r) {
             const int rk = PAIR ? (r << 1) | (sc.rank & 1) : r;
             mbar_arrive_peer(mapa_shared(smem_u32(s.freed), rk));
         }
@@ -619,10 +672,6 @@ __device__ void crew_split_epilogue(const GemmArgs& a, uint32_t tmem, const Smem
 template <int FMT, bool PAIR, bool XRES>
 __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc, int warp,
                               int lane) {
-    if (a.red_alias) {
-        crew_split_epilogue<FMT, PAIR>(a, tmem, s, sc, warp, lane);
-        return;
-    }
     // in a pair the accumulator is released to the first CTA's MMA thread
     const uint32_t accempty_leader = PAIR ? mapa_shared(smem_u32(s.accempty), sc.rank & ~1) : 0u;
     const int q = warp & 3;
@@ -642,8 +691,14 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
     }
     const int share = a.BN / a.S;       // tokens of each tile this CTA sums (at least 8)
     int tc = 0;
-    for (int g = sc.cid; g < a.tiles_nm; g += sc.ncl, ++tc) {
-        const TileCoord c = tile_coord<PAIR>(a, g, sc.rank);
+    TileCoord c;
+    for (; unit_coord<PAIR>(a, sc, tc, c); ++tc) {
+        // a split unit with its partial in the ring is always the CTA's last:
+        // the dequant warps help finish it
+        if (c.split && a.red_alias) {
+            crew_split_epilogue<FMT, PAIR>(a, tmem, s, sc, warp, lane, tc, c);
+            return;
+        }
         const int ab = tc % a.acc_bufs;
         if (!warp_wait_or_abort(&s.accfull[ab], (tc / a.acc_bufs) & 1, a, s.abort_flag, false, true)) return;
         tc_fence_after();
@@ -734,6 +789,58 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
                 reg_pin(lv);
                 emit(v, lv, cc);
             }
+        } else if (!split && a.vec_out && !a.y_f32 && nch % EPI_CHUNKS == 0) {
+            // bf16 output, the common case: two 16-token chunks per step (their
+            // conversions and stores are independent, so one warp per SMSP
+            // keeps more in flight)
+            const uint32_t col = tbase + a.acc_col0 + ab * a.BN;
+            const int nb = c.nt * 128 + q * 32;
+            uint8_t* stg = s.stage + (warp - WARP_EPI0) * EPI_STAGE_BYTES;
+            const bool odd = lane & 1;
+            auto emitn = [&](const uint32_t (&vv)[EPI_CHUNKS][16], int cc) {
+#pragma unroll
+                for (int k = 0; k < EPI_CHUNKS; ++k) {
+                    const uint32_t* v = vv[k];
+                    uint8_t* sb = stg + k * EPI_BF16_CHUNK_BYTES;
+                    // lane pairs (channels 2i, 2i+1) swap halves so that each lane
+                    // packs both channels of one token: even lanes tokens 0-7,
+                    // odd lanes 8-15; rows 8-15 sit one row further on
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float lo_t = __uint_as_float(v[j]) * rf + bn;
+                        const float hi_t = __uint_as_float(v[j + 8]) * rf + bn;
+                        const float mine = odd ? hi_t : lo_t;
+                        const float other = __shfl_xor_sync(0xffffffffu, odd ? lo_t : hi_t, 1);
+                        const __nv_bfloat162 pr = odd ? __floats2bfloat162_rn(other, mine)
+                                                      : __floats2bfloat162_rn(mine, other);
+                        const int t = odd ? j + 8 : j;
+                        *reinterpret_cast<__nv_bfloat162*>(sb + t * 64 + (t >> 3) * 64 + (lane & ~1) * 2) = pr;
+                    }
+                }
+                __syncwarp();
+#pragma unroll
+                for (int k = 0; k < EPI_CHUNKS; ++k) {
+                    const uint8_t* sb = stg + k * EPI_BF16_CHUNK_BYTES;
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        const int ci = lane + 32 * p, t = ci >> 2, nn = nb + (ci & 3) * 8;
+                        const int m = m0 + (cc + k) * 16 + t;
+                        const uint4 v4 = *reinterpret_cast<const uint4*>(sb + t * 64 + (t >> 3) * 64 + (ci & 3) * 16);
+                        if (m < a.M && nn < a.N)
+                            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.y) + static_cast<size_t>(m) * a.N + nn) = v4;
+                    }
+                }
+                __syncwarp();
+            };
+            for (int cc = 0; cc < nch; cc += EPI_CHUNKS) {
+                uint32_t vv[EPI_CHUNKS][16];
+#pragma unroll
+                for (int k = 0; k < EPI_CHUNKS; ++k) tmem_ld16(col + (cc + k) * 16, vv[k]);
+                tmem_wait_ld_pin(vv[0]);
+#pragma unroll
+                for (int k = 1; k < EPI_CHUNKS; ++k) reg_pin(vv[k]);
+                emitn(vv, cc);
+            }
         } else {
             // two register sets: chunk cc + 1 is read from tensor memory while
             // chunk cc is stored
@@ -769,7 +876,7 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
             for (int r = 0; r < a.S; ++r) mbar_arrive_peer(ready_at[r]);
         }
         if (!warp_wait_or_abort(s.ready, tc & 1, a, s.abort_flag, true)) return;
-        reduce_share(a, s.red, 128, c, sc, m0, share, warp - WARP_EPI0, NUM_EPI_WARPS, lane, PAIR);
+        reduce_share(a, s.red, 128, c, sc, m0, share, warp - WARP_EPI0, NUM_EPI_WARPS, lane, a.S, PAIR);
         __syncwarp();
         if (lane == 0) mbar_arrive(s.readw);
         if (first_thread && wait_or_abort(s.readw, tc & 1, a, s.abort_flag)) {
@@ -787,7 +894,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
             const __grid_constant__ CUtensorMap tm_l2, const GemmArgs a) {
     // a partial kept in the ring needs one tile per cluster (the host plans
     // it so; refuse anything else)
-    if (a.red_alias && a.tiles_nm > static_cast<int>(cluster_count_x())) {
+    if (a.red_alias && !a.tail && a.tiles_nm > static_cast<int>(cluster_count_x())) {
         if (threadIdx.x == 0 && blockIdx.x == 0) raise_error(ERRBIT_LAUNCH);
         return;
     }
@@ -845,8 +952,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
         mbar_init(s.drain, 1);
         mbar_init(s.redw, a.red_alias ? CREW_WARPS : NUM_EPI_WARPS);
         mbar_init(s.readw, a.red_alias ? CREW_WARPS : NUM_EPI_WARPS);
-        mbar_init(s.ready, a.S);
-        mbar_init(s.freed, a.S);
+        mbar_init(s.ready, a.S_red);
+        mbar_init(s.freed, a.S_red);
         *s.abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async();

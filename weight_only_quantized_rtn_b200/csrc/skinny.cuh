@@ -302,7 +302,7 @@ __device__ void sk_compute(const GemmArgs& a, const SkSmem& s, const Sched& sc, 
             for (int q = 0; q < a.S; ++q) mbar_arrive_peer(mapa_shared(smem_u32(s.ready), q));
         }
         if (!warp_wait_or_abort(s.ready, par, a, s.abort_flag, true)) return;
-        reduce_share(a, s.red, SK_PITCH, c, sc, 0, share, warp, SK_WARPS, lane);
+        reduce_share(a, s.red, SK_PITCH, c, sc, 0, share, warp, SK_WARPS, lane, a.S);
         __syncwarp();
         if (lane == 0) mbar_arrive(s.readw);
         if (first_thread && wait_or_abort(s.readw, par, a, s.abort_flag)) {
@@ -347,8 +347,8 @@ skinny_kernel(const __grid_constant__ CUtensorMap tm_x, const GemmArgs a) {
     else if (i == 66) mbar_init(s.fin, SK_WARPS / 2);
     else if (i == 67) mbar_init(s.cpy, SK_WARPS);
     else if (i == 68) mbar_init(s.readw, SK_WARPS);
-    else if (i == 69) mbar_init(s.ready, a.S);
-    else if (i == 70) mbar_init(s.freed, a.S);
+    else if (i == 69) mbar_init(s.ready, a.S_red);
+    else if (i == 70) mbar_init(s.freed, a.S_red);
     else if (i == 71) *s.abort_flag = 0;
     if (warp == SK_WARPS + 1 && lane == 0) prefetch_tensormap(&tm_x);
     if (i < 72) {

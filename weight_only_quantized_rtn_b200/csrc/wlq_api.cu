@@ -350,7 +350,6 @@ wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, co
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         d->smem_set[kid] = true;
     }
-    const int csize = PAIR ? 2 * p.S : p.S;  // CTAs per cluster
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
     cudaLaunchAttribute attr[1];
@@ -358,15 +357,8 @@ wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, co
     cfg.dynamicSmemBytes = p.smem;
     cfg.stream = st;
     const int cta_cap = (g_grid_limit > 0) ? std::min(g_grid_limit, d->sms) : d->sms;
-    int clusters = std::max(1, std::min(p.tiles_nm, cta_cap / csize));
-    if (csize > 1) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = static_cast<unsigned>(csize);
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        // persistent clusters: no more than can be resident at once
+    // clusters of `csize` CTAs that the device can hold at once (cached)
+    auto resident_clusters = [&](int csize) {
         const uint64_t key = (static_cast<uint64_t>(kid) << 48) | (static_cast<uint64_t>(csize) << 32) | p.smem;
         int active = 0;
         {
@@ -375,15 +367,51 @@ wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, co
             if (it != d->max_clusters.end()) active = it->second;
         }
         if (active == 0) {
-            cfg.gridDim = dim3(static_cast<unsigned>(clusters * csize), 1, 1);
-            if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) != cudaSuccess || active <= 0) {
+            cudaLaunchAttribute at;
+            at.id = cudaLaunchAttributeClusterDimension;
+            at.val.clusterDim.x = static_cast<unsigned>(csize);
+            at.val.clusterDim.y = 1;
+            at.val.clusterDim.z = 1;
+            cudaLaunchConfig_t c2 = cfg;
+            c2.attrs = &at;
+            c2.numAttrs = 1;
+            c2.gridDim = dim3(static_cast<unsigned>((cta_cap / csize) * csize), 1, 1);
+            if (cudaOccupancyMaxActiveClusters(&active, kern, &c2) != cudaSuccess || active <= 0) {
                 cudaGetLastError();
                 active = d->sms / csize;
             }
             std::lock_guard<std::mutex> lk(g_dev_mu);
             d->max_clusters[key] = active;
         }
-        clusters = std::min(clusters, active);
+        return std::min(active, cta_cap / csize);
+    };
+    int csize = PAIR ? 2 * p.S : p.S;  // CTAs per cluster
+    // Pairs over whole K: when the tiles do not fill the last round of pairs,
+    // run clusters of two pairs and split each leftover tile's K range over
+    // one cluster's two pairs (a half-length last round).
+    a.tail = 0;
+    if (PAIR && p.S == 1 && p.stages * static_cast<size_t>(p.xstage + p.wstage) >= static_cast<size_t>(p.BN) * 512u) {
+        const int c4 = resident_clusters(4);
+        const int P = 2 * c4;
+        const int rem = (P > 0) ? p.tiles_nm % P : 0;
+        if (c4 > 0 && p.tiles_nm > P && rem > 0 && rem <= c4) {
+            csize = 4;
+            a.tail = 1;
+            a.tiles_full = p.tiles_nm - rem;
+            a.red_alias = 1;
+            a.S_red = 2;
+        }
+    }
+    int clusters = std::max(1, std::min(a.tail ? resident_clusters(4) : p.tiles_nm, cta_cap / csize));
+    if (csize > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(csize);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        // persistent clusters: no more than can be resident at once
+        clusters = std::min(clusters, resident_clusters(csize));
     }
     // a partial kept in the ring needs one tile per cluster
     if (p.red_alias && clusters < p.tiles_nm) return kRetryPlan;
@@ -487,6 +515,7 @@ wlq_status launch_linear(Plan& p, int fmt, int64_t M, int64_t N, int64_t K, int 
     a.wtile_bytes = p.wtile; a.wstage_bytes = p.wstage; a.xsub_bytes = p.xsub; a.xstage_bytes = p.xstage; a.red_bytes = p.red;
     a.stage_bytes = p.stage;
     a.red_alias = p.red_alias ? 1 : 0;
+    a.S_red = p.S;
     // vector stores of y: unsplit tiles store 16-byte runs (4 fp32 / 8 bf16
     // channels), the split reduction 4 adjacent channels (16 / 8 bytes)
     {
