@@ -51,6 +51,31 @@ def test_quantize_edge_cases(bits, group):
     assert_codes_equal(cg, sg, co, so)
 
 
+@pytest.mark.parametrize("bits,group", [(8, 0), (4, 64), (4, 16)])
+def test_quantize_quotients_near_half_integers(bits, group):
+    """Weights at (k + 1/2 + d) * s for small d, on both sides of the tie and on
+    it: the estimate W * (1/s) may round either way there, so the exact
+    residual decides (both the fast and the corrected branch run)."""
+    g = np.random.default_rng(123 + bits + group)
+    qmax = 127 if bits == 8 else 7
+    N, K = 64, 256
+    gsz = K if group == 0 else group
+    W = np.zeros((N, K), dtype=np.float32)
+    deltas = np.array([0.0, 2.0**-12, -2.0**-12, 2.0**-14, -2.0**-14, 2.0**-17, -2.0**-17, 2.0**-21, -2.0**-21, 1e-3])
+    for n in range(N):
+        for g0 in range(0, K, gsz):
+            a = np.float32(g.uniform(0.01, 3.0))
+            s = np.float32(a / np.float32(qmax))  # the group's fp32 scale (division correctly rounded)
+            k = g.integers(-qmax, qmax, gsz)
+            d = deltas[g.integers(0, len(deltas), gsz)]
+            w = ((k + 0.5 + d) * np.float64(s)).astype(np.float32)
+            w = np.clip(w, -a, a)
+            w[0] = a  # the group's absmax
+            W[n, g0:g0 + gsz] = w
+    cg, sg, co, so = quantize_both(W, bits, group)
+    assert_codes_equal(cg, sg, co, so)
+
+
 def test_quantize_ragged_and_single_row():
     for N, K in [(1, 8), (3, 24), (129, 1000), (257, 4104)]:
         W = wi.weight(21, N, N, K)

@@ -122,25 +122,44 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(
 }
 
 // RTN of four weights of one group with a normal fp32 scale (s >= 2^-126),
-// packed as two's-complement bytes: the same arithmetic as rtn_byte_f32,
-// with the exact-tie correction on a branch (a residual of exactly s/2 is
-// rare).  h = s / 2, inv = 1 / s rounded.
-__device__ __forceinline__ uint32_t rtn4_f32(float4 v, float s, float inv, float h, float qmax) {
+// packed as two's-complement bytes, bit-identical to rtn_byte_f32.
+//  - t = W * (1/s) (two roundings) is within 2^-15 of the exact quotient W/s
+//    for |W/s| <= 128, so k = rint(t) is the answer unless t lies within
+//    2^-12 of a half-integer.  Such rare weights (and exact ties) take the
+//    exact path: residual e = W - k*s from one fma, compared with s/2.
+//  - No clamp: s = RN(a/qmax) and |W| <= a give |W/s| < qmax + 1/2, so the
+//    code never leaves [-qmax, qmax].
+//  - k + 1.5*2^23 holds k in its low bits; byte permutes gather the four
+//    low bytes.  h = s / 2, inv = 1 / s rounded.
+__device__ __forceinline__ uint32_t rtn4_f32(float4 v, float s, float inv, float h) {
     const float kMagic = 12582912.0f;  // 1.5 * 2^23
     const float w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t out = 0;
+    float km[4];
+    bool near_half = false;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        float k = __fsub_rn(__fadd_rn(__fmul_rn(w[i], inv), kMagic), kMagic);
-        const float e = __fmaf_rn(-k, s, w[i]);
-        k = (e > h) ? k + 1.0f : k;
-        k = (e < -h) ? k - 1.0f : k;
-        if (fabsf(e) == h) {  // exact tie between k and k + sign(e): keep the even one
-            if (__float_as_uint(__fadd_rn(k, kMagic)) & 1u) k += (e > 0.0f) ? 1.0f : -1.0f;
-        }
-        k = fminf(fmaxf(k, -qmax), qmax);
-        out |= (__float_as_uint(__fadd_rn(k, kMagic)) & 0xFFu) << (8 * i);
+        const float t = __fmul_rn(w[i], inv);
+        km[i] = __fadd_rn(t, kMagic);
+        const float d = __fsub_rn(t, __fsub_rn(km[i], kMagic));
+        near_half |= fabsf(d) > 0.499755859375f;  // 1/2 - 2^-12
     }
+    if (near_half) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float k = __fsub_rn(km[i], kMagic);
+            const float e = __fmaf_rn(-k, s, w[i]);
+            k = (e > h) ? k + 1.0f : k;
+            k = (e < -h) ? k - 1.0f : k;
+            if (fabsf(e) == h) {  // exact tie between k and k + sign(e): keep the even one
+                if (__float_as_uint(__fadd_rn(k, kMagic)) & 1u) k += (e > 0.0f) ? 1.0f : -1.0f;
+            }
+            km[i] = __fadd_rn(k, kMagic);
+        }
+    }
+    uint32_t lo, hi, out;
+    asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(lo) : "r"(__float_as_uint(km[0])), "r"(__float_as_uint(km[1])));
+    asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(hi) : "r"(__float_as_uint(km[2])), "r"(__float_as_uint(km[3])));
+    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(out) : "r"(lo), "r"(hi));
     return out;
 }
 
@@ -159,7 +178,6 @@ __global__ void __launch_bounds__(1024) quantize_rows_cta_kernel(
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nwarps = blockDim.x >> 5;
     const int K4 = static_cast<int>(K / 4);
-    const float fq = static_cast<float>(qmax);
     bool bad = false;
     for (int64_t n = blockIdx.x; n < N; n += gridDim.x) {
         const float4* row = reinterpret_cast<const float4*>(W + n * K);
@@ -192,7 +210,7 @@ __global__ void __launch_bounds__(1024) quantize_rows_cta_kernel(
 #pragma unroll
             for (int i = 0; i < V; ++i) {
                 const int idx = threadIdx.x + i * blockDim.x;
-                if (idx < K4) out[idx] = rtn4_f32(v[i], g.s, g.inv, h, fq);
+                if (idx < K4) out[idx] = rtn4_f32(v[i], g.s, g.inv, h);
             }
         } else {
             bool unused = false;
@@ -220,7 +238,6 @@ __global__ void __launch_bounds__(256) quantize_groups_kernel(
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     const float4* W4 = reinterpret_cast<const float4*>(W);
     uint32_t* out = reinterpret_cast<uint32_t*>(codes);
-    const float fq = static_cast<float>(qmax);
     bool bad = false;
     for (int64_t base = warp0 * 32 * U; base < total4; base += nwarps * 32 * U) {
         float4 v[U];
@@ -241,7 +258,7 @@ __global__ void __launch_bounds__(256) quantize_groups_kernel(
             const GroupScale gs = group_scale(gbad ? 0.0f : __uint_as_float(m), qmax);
             if ((lane & (lanes_per_group - 1)) == 0) scales[i / lanes_per_group] = gs.s;
             bool unused = false;
-            out[i] = gs.normal ? rtn4_f32(v[u], gs.s, gs.inv, 0.5f * gs.s, fq) : pack_codes4(v[u], gs, qmax, unused);
+            out[i] = gs.normal ? rtn4_f32(v[u], gs.s, gs.inv, 0.5f * gs.s) : pack_codes4(v[u], gs, qmax, unused);
         }
     }
     if (bad) raise_error(ERRBIT_NONFINITE);
