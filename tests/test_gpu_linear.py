@@ -55,6 +55,47 @@ def test_parity_shapes(bits, group, N, K):
     assert err <= TOL, err
 
 
+@pytest.mark.parametrize("bits,group", RECIPES)
+@pytest.mark.parametrize("M,N,K", [
+    (1, 4096, 4096),    # direct-load kernel: one token
+    (5, 1000, 576),     # ragged tokens and channels (not a multiple of 32)
+    (9, 33, 2048),      # 9..16 tokens: two 8-token MMA columns; one partial 32-channel CTA
+    (16, 2080, 4096),   # 16 tokens, 65 CTAs
+    (16, 512, 16384),   # x too large for shared memory: the warp-MMA streaming kernel instead
+])
+def test_parity_few_tokens(bits, group, M, N, K):
+    x, W, b, _, _ = small_case(60 + M, M, N, K, bits, group)
+    err, _, _ = linear_case(x, W, bits, group, b)
+    assert err <= TOL, err
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 512, 16384), (32, 512, 16384), (16, 1024, 12288)])
+def test_ring_reuse_after_reads_complete(M, N, K):
+    """Warp-MMA kernel with a large resident x and 4-8 CTA clusters: its weight
+    ring slots are refilled as soon as all warps release them, so every read
+    of a slot must have completed first.  These shapes once lost that race
+    (a band of channels wrong in one CTA per run); five runs, all exact repeats
+    and within tolerance."""
+    m = wlq()
+    x, W, b, _, _ = small_case(70 + M, M, N, K, 8, 0)
+    codes, scales = m.quantize(dev_f32(W), 8, 0)
+    packed = m.pack(codes, scales, 8, 0)
+    co, so = oracle.quantize(W, 8, 0)
+    ref = oracle.linear(x, co, so, 0, b, None, None)
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    xd, bd = dev_bf16(x), dev_bf16(b)
+    first = None
+    for _ in range(5):
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        m.linear_into(y, xd, packed, N, K, 8, 0, bd)
+        m.check_status()
+        yh = y.cpu().numpy()
+        assert float(np.max(np.abs(yh - ref))) <= TOL * rms
+        if first is None:
+            first = yh
+        assert np.array_equal(yh, first)
+
+
 def test_parity_k_not_multiple_of_64():
     # int8 per channel only needs K % 8 == 0: the last K block is partial
     for K in (8, 72, 200):

@@ -97,6 +97,7 @@ struct GemmArgs {
                     // each split over the K halves of one cluster's two pairs
     int tiles_full; // tail: tiles dealt in full rounds (a multiple of 2 x clusters)
     int S_red;      // CTAs summed by a split unit's reduction
+    const void* xg;  // x in global memory (the direct-load few-token kernel)
     uint64_t timeout_ns;
 };
 
@@ -434,6 +435,18 @@ __device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, co
                         }
                     }
                 }
+            }
+            {
+                uint32_t held = 0;
+#pragma unroll
+                for (int j = 0; j < MAX_KS; ++j) {
+                    if (j < nkb) {
+                        held ^= cv[j][0].x ^ cv[j][0].y ^ cv[j][0].z ^ cv[j][0].w;
+                        if constexpr (FMT == FMT_W8) held ^= cv[j][CW - 1].x ^ cv[j][CW - 1].y ^ cv[j][CW - 1].z ^ cv[j][CW - 1].w;
+                        else held ^= h2u(sg[j][0]) ^ h2u(sg[j][1]);
+                    }
+                }
+                loads_done_before_release(held);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.empty[st]);

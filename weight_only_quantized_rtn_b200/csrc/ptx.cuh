@@ -266,6 +266,17 @@ __device__ __forceinline__ void mma16816_f16(float (&d)[4], uint32_t a0, uint32_
                  : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
                  : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+// A shared-memory slot whose reads are handed back for a TMA refill (async
+// proxy) must have those reads complete first: an issued ld.shared that has
+// not returned is not ordered against the refill.  `held` combines every
+// word the lane loaded (any instruction reading them waits for the loads);
+// the proxy fence then orders the generic-proxy reads before the async-proxy
+// writes that follow the release.
+__device__ __forceinline__ void loads_done_before_release(uint32_t held) {
+    asm volatile("" ::"r"(held) : "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Named barrier over the first `threads` threads of the block (id 1..15).
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");

@@ -196,7 +196,13 @@ __device__ void sk_compute(const GemmArgs& a, const SkSmem& s, const Sched& sc, 
             const bool mine = kb + grp < c.kb1;
             if (!warp_wait_or_abort(&s.full[st], r.phase, a, s.abort_flag)) return;
             SkCodes<FMT> cv;
-            if (mine) cv = sk_load_codes<FMT>(s.w + st * a.wstage_bytes + grp * a.wtile_bytes, row0, t);
+            uint32_t held = 0;
+            if (mine) {
+                cv = sk_load_codes<FMT>(s.w + st * a.wstage_bytes + grp * a.wtile_bytes, row0, t);
+                held = cv.r0.x ^ cv.r0.y ^ cv.r0.z ^ cv.r0.w ^ cv.r1.x ^ cv.r1.y ^ cv.r1.z ^ cv.r1.w;
+                if constexpr (FMT != FMT_W8) held ^= h2u(cv.s0) ^ h2u(cv.s1);
+            }
+            loads_done_before_release(held);
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.empty[st]);
             if (!mine) continue;

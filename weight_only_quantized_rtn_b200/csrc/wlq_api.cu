@@ -14,6 +14,7 @@
 #include "../../include/wlq.h"
 #include "gemm.cuh"
 #include "skinny.cuh"
+#include "gemv.cuh"
 #include "pack.cuh"
 #include "prep.cuh"
 #include "ptx.cuh"
@@ -50,7 +51,7 @@ int fmt_of(int bits, int group) {
 struct DeviceInfo {
     int checked = 0;  // 0 unknown, 1 supported, -1 not
     int sms = 0;
-    bool smem_set[24] = {};
+    bool smem_set[32] = {};
     // resident clusters per (format, cluster size, dynamic smem), queried once
     std::unordered_map<uint64_t, int> max_clusters;
 };
@@ -129,6 +130,7 @@ struct Plan {
     bool pair = false;  // two CTAs per MMA (cta_group::2)
     bool xres = false;  // x resident in shared memory; weight ring released by the dequant warps
     bool skinny = false;  // one token tile of <= 64 tokens: the warp-MMA streaming kernel
+    bool gemv = false;    // <= 16 tokens, x small enough for shared memory: the direct-load kernel
     bool red_alias = false;  // split partial in the ring's memory (one tile per cluster)
     int astages = 0;    // resident x: TMEM A-stage ring depth
     uint32_t tmem_cols = 0, acc_col0 = 0, lr_col0 = 0, a_col0 = 0, wtile = 0, wstage = 0, xsub = 0, xstage = 0, red = 0, stage = 0;
@@ -231,6 +233,25 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     // their own, so weight loads never wait for the MMA.
     const size_t xres_bytes = static_cast<size_t>(p.kbps) * p.BN * 128u;
     p.ks = 0;
+    // At most 16 tokens, no low rank, x (zero-padded) fits in shared memory:
+    // the direct-load kernel (no weight ring, no K split across CTAs).
+    {
+        const int nb = (M <= 8) ? 1 : 2;
+        const size_t need = 128 + static_cast<size_t>(nb * 8) * wlq::gv_x_pitch(p.KT) +
+                            static_cast<size_t>(wlq::GV_SLICES) * 2 * 32 * nb * 4 * 4;
+        if (r == 0 && M <= 16 && need <= kSmemLimit - 1024) {
+            p.gemv = true;
+            p.smem = need;
+            p.grid = static_cast<int>(cdiv(N, wlq::GV_ROWS));
+            size_t off = 0;
+            if (fmt != wlq::FMT_W8) {
+                p.off_x16 = off; off = align256(off + static_cast<size_t>(M) * K * 2);
+                p.off_xs = off;  off = align256(off + static_cast<size_t>(M) * 4);
+            }
+            p.ws = off;
+            return true;
+        }
+    }
     // Few tokens (at most 32): the skinny kernel (x resident, warp MMAs, no
     // tensor memory).  At 64 tokens the resident-x tensor-core kernel is faster.
     p.skinny = !p.pair && r == 0 && p.MT == 1 && p.BN <= 32 && xres_bytes <= kXresMaxBytes;
@@ -425,7 +446,7 @@ wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, co
 template <int FMT, int NB>
 wlq_status launch_skinny(Plan& p, const CUtensorMap& tx, wlq::GemmArgs& a, DeviceInfo* d, cudaStream_t st) {
     auto kern = wlq::skinny_kernel<FMT, NB>;
-    const int kid = 12 + FMT * 4 + (NB == 2 ? 0 : NB == 4 ? 1 : 2);
+    const int kid = 12 + FMT * 3 + (NB == 2 ? 0 : NB == 4 ? 1 : 2);  // 12..20 (gemm: 0..11, gemv: 21..26)
     if (!d->smem_set[kid]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(kSmemLimit));
@@ -473,6 +494,29 @@ wlq_status launch_skinny(Plan& p, const CUtensorMap& tx, wlq::GemmArgs& a, Devic
     return WLQ_OK;
 }
 
+template <int FMT, int NB>
+wlq_status launch_gemv(Plan& p, wlq::GemmArgs& a, DeviceInfo* d, cudaStream_t st) {
+    auto kern = wlq::gemv_kernel<FMT, NB>;
+    const int kid = 21 + FMT * 2 + (NB == 1 ? 0 : 1);
+    if (!d->smem_set[kid]) {
+        // the kernel also holds a little static shared memory (its barrier)
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kSmemLimit - 1024));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        d->smem_set[kid] = true;
+    }
+    kern<<<static_cast<unsigned>(p.grid), wlq::GV_THREADS, p.smem, st>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "gemv launch");
+    return WLQ_OK;
+}
+
+template <int FMT>
+wlq_status launch_gemv_nb(Plan& p, wlq::GemmArgs& a, DeviceInfo* d, cudaStream_t st) {
+    if (p.M <= 8) return launch_gemv<FMT, 1>(p, a, d, st);
+    return launch_gemv<FMT, 2>(p, a, d, st);
+}
+
 template <int FMT>
 wlq_status launch_skinny_nb(Plan& p, const CUtensorMap& tx, wlq::GemmArgs& a, DeviceInfo* d, cudaStream_t st) {
     if (p.BN == 16) return launch_skinny<FMT, 2>(p, tx, a, d, st);
@@ -494,7 +538,8 @@ wlq_status launch_linear(Plan& p, int fmt, int64_t M, int64_t N, int64_t K, int 
     CUtensorMap tx, tt, tl;
     std::memset(&tt, 0, sizeof tt);
     std::memset(&tl, 0, sizeof tl);
-    if ((st = make_map_2d(&tx, xin, M, K, p.pair ? p.BN / 2 : p.BN)) != WLQ_OK) return st;
+    std::memset(&tx, 0, sizeof tx);
+    if (!p.gemv && (st = make_map_2d(&tx, xin, M, K, p.pair ? p.BN / 2 : p.BN)) != WLQ_OK) return st;
     if (r) {
         if ((st = make_map_2d(&tt, thl, M, W, p.BN)) != WLQ_OK) return st;
         if ((st = make_map_2d(&tl, l2t, NT * 128, W, 128)) != WLQ_OK) return st;
@@ -525,6 +570,12 @@ wlq_status launch_linear(Plan& p, int fmt, int64_t M, int64_t N, int64_t K, int 
         else a.vec_out = ((ya & (f32 ? 15u : 7u)) == 0 && N % 4 == 0) ? 1 : 0;
     }
     a.timeout_ns = kDefaultTimeoutNs;
+    a.xg = xin;
+    if (p.gemv) {
+        if (fmt == wlq::FMT_W8) return launch_gemv_nb<wlq::FMT_W8>(p, a, d, s);
+        if (fmt == wlq::FMT_W4G64) return launch_gemv_nb<wlq::FMT_W4G64>(p, a, d, s);
+        return launch_gemv_nb<wlq::FMT_W4G16>(p, a, d, s);
+    }
     if (p.skinny) {
         if (fmt == wlq::FMT_W8) return launch_skinny_nb<wlq::FMT_W8>(p, tx, a, d, s);
         if (fmt == wlq::FMT_W4G64) return launch_skinny_nb<wlq::FMT_W4G64>(p, tx, a, d, s);
