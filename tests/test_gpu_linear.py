@@ -59,9 +59,9 @@ def test_parity_shapes(bits, group, N, K):
 @pytest.mark.parametrize("M,N,K", [
     (1, 4096, 4096),    # direct-load kernel: one token
     (5, 1000, 576),     # ragged tokens and channels (not a multiple of 32)
-    (9, 33, 2048),      # 9..16 tokens: two 8-token MMA columns; one partial 32-channel CTA
-    (16, 2080, 4096),   # 16 tokens, 65 CTAs
-    (16, 512, 16384),   # x too large for shared memory: the warp-MMA streaming kernel instead
+    (9, 33, 2048),      # 9..16 tokens: two 8-token MMA columns; one ragged channel tile
+    (16, 2080, 4096),   # 16 tokens, 17 tiles on 8-CTA clusters
+    (16, 512, 16384),   # direct-load kernel: K split over an 8-CTA cluster
 ])
 def test_parity_few_tokens(bits, group, M, N, K):
     x, W, b, _, _ = small_case(60 + M, M, N, K, bits, group)
@@ -69,7 +69,20 @@ def test_parity_few_tokens(bits, group, M, N, K):
     assert err <= TOL, err
 
 
-@pytest.mark.parametrize("M,N,K", [(16, 512, 16384), (32, 512, 16384), (16, 1024, 12288)])
+@pytest.mark.parametrize("bits,group,M,N,K", [
+    (8, 0, 3, 200, 200),      # one K split, three whole K blocks and 8 inputs
+    (8, 0, 12, 700, 4040),    # 8-CTA clusters, the last split ends in a ragged block
+    (4, 16, 16, 300, 1232),   # int4 groups of 16, ragged last block
+])
+def test_parity_few_tokens_ragged_k(bits, group, M, N, K):
+    """Direct-load kernel with K not a multiple of 64: the inputs of the last
+    K block beyond K must read as zero (their codes are 0)."""
+    x, W, b, _, _ = small_case(80 + M, M, N, K, bits, group)
+    err, _, _ = linear_case(x, W, bits, group, b)
+    assert err <= TOL, err
+
+
+@pytest.mark.parametrize("M,N,K", [(24, 512, 16384), (32, 512, 16384), (20, 1024, 12288)])
 def test_ring_reuse_after_reads_complete(M, N, K):
     """Warp-MMA kernel with a large resident x and 4-8 CTA clusters: its weight
     ring slots are refilled as soon as all warps release them, so every read
@@ -119,7 +132,9 @@ def test_parity_low_rank(bits, group, r, M):
     (16, 33000, 128, 0, 16),   # 258 tiles of 16 tokens on 16 CTAs
     (300, 700, 256, 0, 3),     # 128-token tiles, several per CTA
     (16, 1024, 2048, 0, 4),    # K split over clusters, each cluster several tiles
-    (16, 4096, 1024, 0, 8),    # warp-MMA kernel: K split over pairs, eight tiles per cluster
+    (16, 4096, 1024, 0, 8),    # direct-load kernel on 8 CTAs: four tiles each
+    (16, 4096, 16384, 0, 8),   # direct-load kernel: x needs 4-CTA clusters, sixteen tiles per cluster
+    (24, 4096, 1024, 0, 8),    # warp-MMA kernel: K split over a cluster, several tiles per cluster
     (32, 1001, 512, 0, 3),     # warp-MMA kernel: ragged N (scalar stores), one cluster for all tiles
     (64, 2048, 1024, 0, 8),    # resident-x tensor-core kernel: K split over 4, several tiles per cluster
     (100, 1024, 512, 32, 4),   # low rank + K split, several tiles per cluster

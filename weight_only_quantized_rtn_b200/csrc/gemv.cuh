@@ -1,27 +1,46 @@
-// gemv.cuh -- the weight-only quantized Linear for at most 16 tokens with a
-// small x ("Joy-face_change_optimized" model card, files table: weight-only
-// Linear; "Nunchaku Lite", how it works: 4-bit weights, 16-bit activations).
+// gemv.cuh -- the weight-only quantized Linear for at most 16 tokens
+// ("Joy-face_change_optimized" model card, files table: weight-only Linear;
+// "Nunchaku Lite", how it works: 4-bit weights, 16-bit activations).
 //
 //   y[m,n] = rowf[n] * xs[m] * sum_k xin[m,k] * w16[n,k]  +  b[n]
 //
 // Same packed operand, row factors and x (bf16, or the fp16 x16 of the int4
 // formats) as the other engines.  Here streaming the packed weights from HBM
-// is the whole cost, so nothing stands between the weight bytes and the MMAs:
+// is the whole cost, so the kernel is built around that stream:
 //
-//  - one CTA per 32 output channels, no cluster, no K split across CTAs;
-//  - 16 warps: warp w takes rows 16 (w % 2)..+15 of the CTA's 32 and K slice
-//    w / 2 of 8; each lane loads its codes straight from global memory into
-//    registers (four K blocks in flight), dequantises them and runs m16n8k16
-//    warp MMAs (fp32 accumulate) against x fragments read from shared memory;
-//  - x ([M][K], zero-padded to 8 or 16 tokens and to whole K blocks) is copied
-//    to shared memory once per CTA by bulk copies, while the first weight
-//    loads are in flight;
-//  - the 8 K slices of each row are summed in slice order (deterministic) in
-//    shared memory, then scaled, biased and stored.
+//  - a cluster of S CTAs takes one 128-channel tile of the packed operand, CTA
+//    (cluster rank) q its K split q of kbps 64-wide blocks; clusters are
+//    persistent over tiles;
+//  - one producer thread (a warp of its own) streams the split's packed
+//    blocks, four per ring slot
+//    (one contiguous bulk copy of 17-32 KB: a bulk copy costs a fixed
+//    ~0.2 us of the SM's copy engine, so small copies cannot keep up);
+//  - all 16 compute warps work on the same landed block: int8, warp w takes
+//    rows 32 (w % 4)..+31 and MMA K step w / 4 (16 inputs); int4, warp w takes
+//    rows 16 (w % 8)..+15 and 32-input half w / 8.  Codes reach registers by
+//    ldmatrix (8 rows x 16 bytes per matrix: conflict-free), are dequantised
+//    in registers and feed m16n8k16 warp MMAs (fp32 accumulate) against x
+//    fragments read from shared memory once per block;
+//  - the CTA's x rows ([M][its K range]) are copied to shared memory once, by
+//    16-byte asynchronous copies from the compute threads; token rows >= M
+//    are never read back into an output;
+//  - the warps' partial sums are staged in shared memory and added in K-part
+//    order; each thread then sends four adjacent rows of one token of the sum
+//    to the CTA that owns them (rows [q' 128/S, (q'+1) 128/S) belong to CTA
+//    q') with one 16-byte distributed-shared-memory store; one cluster
+//    barrier later CTA q' adds the S partials of its rows in split order,
+//    scales, biases and stores them.  The summation order is fixed: results
+//    are reproducible.
 //
-// The input renumbering inside a 64-wide K block is the one of the skinny
-// kernel: lane (g, t) takes inputs 16t..16t+15 of its rows, the run of 16
-// codes the packed tile holds contiguously, and reads x the same way.
+// Inputs inside a 64-wide K block are renumbered for the MMA (the dot
+// products are unchanged; x is read with the same renumbering):
+//   int8: step s (inputs 16s..16s+15 of the block, packed chunk s): lane
+//         (g, t) holds inputs 16s + 4t + {0, 1} as fragment columns 2t, 2t+1
+//         and 16s + 4t + {2, 3} as columns 2t+8, 2t+9 -- the four bytes
+//         ldmatrix hands lane (g, t) from a 16-byte row;
+//   int4: half h (inputs 32h..32h+31, packed chunk h), sub-step j = 0, 1:
+//         lane (g, t) holds inputs 32h + 8t + 4j + {0, 1} and + {2, 3} -- the
+//         32-bit word t of the 16-byte row, eight nibbles.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -29,134 +48,265 @@
 #include "ptx.cuh"
 #include "pack.cuh"
 #include "gemm.cuh"
-#include "skinny.cuh"
 
 namespace wlq {
 
-constexpr int GV_SLICES = 8;                      // K slices per CTA
-constexpr int GV_WARPS = 2 * GV_SLICES;           // x 2 row groups of 16
-constexpr int GV_THREADS = GV_WARPS * 32;
-constexpr int GV_ROWS = 32;                       // output channels per CTA
-constexpr int GV_U = 4;                           // K blocks of codes in flight per warp
+constexpr int GV_WARPS = 16;                      // compute warps
+constexpr int GV_THREADS = (GV_WARPS + 1) * 32;   // + the producer warp
+constexpr int GV_SLOT_KB = 4;                     // K blocks per ring slot (one bulk copy)
+constexpr int GV_MAX_STAGES = 8;
+constexpr int GV_MAX_SPLITS = 8;                  // portable cluster size
 
-__host__ __device__ constexpr uint32_t gv_x_pitch(int KT) { return static_cast<uint32_t>(KT) * 128u + 16u; }
+// partials summed per output row and CTA of the cluster: int8 four K steps,
+// int4 two K halves
+__host__ __device__ constexpr int gv_parts(int fmt) { return fmt == FMT_W8 ? 4 : 2; }
+// bytes per token row of the CTA's x (its K range + a skew that keeps the
+// fragment reads conflict-free: 32 bytes for int8, 64 for int4)
+__host__ __device__ constexpr uint32_t gv_x_pitch(int kbps, int fmt) {
+    return static_cast<uint32_t>(kbps) * 128u + (fmt == FMT_W8 ? 32u : 64u);
+}
+__host__ __device__ constexpr uint32_t gv_slot_bytes(int fmt) { return GV_SLOT_KB * tile_bytes(fmt); }
+// dynamic shared memory: alignment + barriers + token scales + x rows +
+// staging (parts x NB*8 tokens x 128 rows, fp32) + the cluster's partials of
+// this CTA's rows (S x NB*8 x 128/S, fp32) + ring
+__host__ __device__ constexpr size_t gv_smem_bytes(int fmt, int nb, int kbps, int stages) {
+    return 128 + 256 + 64 + static_cast<size_t>(nb * 8) * gv_x_pitch(kbps, fmt) +
+           static_cast<size_t>(gv_parts(fmt) + 1) * (nb * 8) * 128u * 4u + static_cast<size_t>(stages) * gv_slot_bytes(fmt);
+}
+
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void st_dsmem_v4(uint32_t cluster_addr, float4 v) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(v.x), "f"(v.y), "f"(v.z),
+                 "f"(v.w)
+                 : "memory");
+}
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&d)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]) : "r"(addr) : "memory");
+}
+__device__ __forceinline__ void ldmatrix_x2(uint32_t addr, uint32_t (&d)[2]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+                 : "=r"(d[0]), "=r"(d[1]) : "r"(addr) : "memory");
+}
 
 template <int FMT, int NB>
 __global__ void __launch_bounds__(GV_THREADS, 1) gemv_kernel(const GemmArgs a) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
-    uint8_t* xsm = smem_raw + (((raw + 127u) & ~127u) - raw);      // [NB*8][pitch]
-    const uint32_t pitch = gv_x_pitch(a.KT);
-    float* red = reinterpret_cast<float*>(xsm + NB * 8 * pitch);   // [slices][2][32][NB*4]
-    __shared__ uint64_t xbar;
+    uint8_t* base = smem_raw + (((raw + 127u) & ~127u) - raw);
+    uint64_t* full = reinterpret_cast<uint64_t*>(base);            // [GV_MAX_STAGES]
+    uint64_t* empty = full + GV_MAX_STAGES;                          // [GV_MAX_STAGES]
+    float* xs_sm = reinterpret_cast<float*>(base + 256);            // [16]
+    uint8_t* xsm = base + 256 + 64;                                  // [NB*8][pitch]
+    const uint32_t pitch = gv_x_pitch(a.kbps, FMT);
+    constexpr int P = gv_parts(FMT);
+    float* stage = reinterpret_cast<float*>(xsm + NB * 8 * pitch);  // [P][NB*8][128]
+    float* red = stage + P * NB * 8 * 128;                           // [S][NB*8][128/S]
+    uint8_t* ring = reinterpret_cast<uint8_t*>(red + NB * 8 * 128);  // [stages][slot]
+    constexpr uint32_t SLOT = gv_slot_bytes(FMT);
+    constexpr uint32_t TB = tile_bytes(FMT);
+    const int stages = a.stages;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int rg = warp & 1, slice = warp >> 1;
-    const int nt = blockIdx.x >> 2;                        // 128-channel tile of the packed operand
-    const int row0 = (blockIdx.x & 3) * GV_ROWS + rg * 16 + g;  // rows row0, row0 + 8 of that tile
-    const int kb_lo = slice * a.KT / GV_SLICES, kb_hi = (slice + 1) * a.KT / GV_SLICES;
+    const int S = a.S;
+    const int q = (S > 1) ? static_cast<int>(cluster_ctarank()) : 0;
+    const int cid = (S > 1) ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+    const int ncl = (S > 1) ? static_cast<int>(cluster_count_x()) : static_cast<int>(gridDim.x);
+    const int kb0 = q * a.kbps, kb1 = min(a.KT, kb0 + a.kbps);
+    const int nkb = kb1 - kb0;
+    const int nslots = (nkb + GV_SLOT_KB - 1) / GV_SLOT_KB;  // ring slots per tile
     const int Mv = min(a.M, NB * 8);
+    const int rows_per = 128 / S;  // rows of each tile this CTA sums and stores
 
-    // x: zero what the copies do not cover (token rows >= M, inputs >= K),
-    // then one bulk copy per token row
-    if (threadIdx.x == 0) {
-        mbar_init(&xbar, 1);
-        fence_barrier_init();
+    if (threadIdx.x < GV_MAX_STAGES) {
+        mbar_init(&full[threadIdx.x], 1);
+        mbar_init(&empty[threadIdx.x], GV_WARPS);
     }
-    const uint32_t row_bytes = static_cast<uint32_t>(a.K) * 2u;
-    for (uint32_t i = threadIdx.x; i < static_cast<uint32_t>(NB * 8) * (pitch / 16u); i += GV_THREADS) {
-        const uint32_t m = i / (pitch / 16u), off = (i % (pitch / 16u)) * 16u;
-        if (static_cast<int>(m) >= Mv || off >= row_bytes)
-            *reinterpret_cast<uint4*>(xsm + m * pitch + off) = make_uint4(0u, 0u, 0u, 0u);
-    }
+    if (threadIdx.x == 0) fence_barrier_init();
     __syncthreads();
-    if (threadIdx.x == 0) {
-        mbar_arrive_expect_tx(&xbar, static_cast<uint32_t>(Mv) * row_bytes);
-        for (int m = 0; m < Mv; ++m)
-            bulk_load(xsm + m * pitch, reinterpret_cast<const uint8_t*>(a.xg) + static_cast<size_t>(m) * row_bytes,
-                      row_bytes, &xbar);
+
+    if (warp < GV_WARPS) {
+        // ---- x rows m < M over this CTA's K range; inputs beyond K (a ragged
+        // last K block) are zeroed, as their codes are 0
+        const uint32_t chunks = static_cast<uint32_t>(nkb) * 8u;  // 16-byte chunks per row
+        const int kin = min(a.K, kb1 * 64) - kb0 * 64;            // real inputs of the range
+        const uint8_t* xg = static_cast<const uint8_t*>(a.xg);
+        for (uint32_t i = threadIdx.x; i < static_cast<uint32_t>(Mv) * chunks; i += GV_WARPS * 32) {
+            const uint32_t m = i / chunks, c = i % chunks;
+            uint8_t* dst = xsm + m * pitch + c * 16u;
+            if (static_cast<int>(c) * 8 < kin)
+                cp_async_16(smem_u32(dst), xg + (static_cast<size_t>(m) * a.K + kb0 * 64) * 2 + c * 16u);
+            else
+                *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        if (threadIdx.x < NB * 8)
+            xs_sm[threadIdx.x] = (FMT != FMT_W8 && static_cast<int>(threadIdx.x) < a.M) ? a.xs[threadIdx.x] : 1.0f;
+        cp_async_wait_all();
+        named_sync(1, GV_WARPS * 32);  // x in shared memory for every compute warp
     }
 
-    float acc[NB][4];
-#pragma unroll
-    for (int j = 0; j < NB; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
-    const uint8_t* band = a.packed + static_cast<size_t>(nt) * a.KT * a.wtile_bytes;
-    bool have_x = false, bad = false;
-    for (int kb = kb_lo; kb < kb_hi; kb += GV_U) {
-        SkCodes<FMT> cv[GV_U];
-#pragma unroll
-        for (int j = 0; j < GV_U; ++j)
-            if (kb + j < kb_hi) cv[j] = sk_load_codes<FMT>(band + static_cast<size_t>(kb + j) * a.wtile_bytes, row0, t);
-        if (!have_x) {
-            // bounded: on a timeout the error bit is set and the (garbage) sums
-            // still flow to the end, so every thread reaches the barriers below
-            if (!mbar_wait(&xbar, 0, a.timeout_ns)) bad = true;
-            have_x = true;
-        }
-#pragma unroll
-        for (int j = 0; j < GV_U; ++j) {
-            if (kb + j >= kb_hi) break;
-            uint32_t p0[8], p1[8];
-            sk_convert<FMT>(cv[j], p0, p1);
-            const uint8_t* xk = xsm + (kb + j) * 128 + 32 * t;
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                const uint8_t* xr = xk + (nb * 8 + g) * pitch;
-                const uint4 u0 = *reinterpret_cast<const uint4*>(xr);
-                const uint4 u1 = *reinterpret_cast<const uint4*>(xr + 16);
-                const uint32_t b[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    if constexpr (FMT == FMT_W8)
-                        mma16816_bf16(acc[nb], p0[2 * k4], p1[2 * k4], p0[2 * k4 + 1], p1[2 * k4 + 1], b[2 * k4],
-                                      b[2 * k4 + 1]);
-                    else
-                        mma16816_f16(acc[nb], p0[2 * k4], p1[2 * k4], p0[2 * k4 + 1], p1[2 * k4 + 1], b[2 * k4],
-                                     b[2 * k4 + 1]);
+    int it = 0;
+    for (int tile = cid; tile < a.NT; tile += ncl) {
+        // epilogue operands of this thread's output row, fetched early
+        const int n_out = tile * 128 + q * rows_per + static_cast<int>(threadIdx.x) % rows_per;
+        const float rf = (warp < GV_WARPS && n_out < a.N) ? a.rowf[n_out] : 0.0f;
+        const float bias = (warp < GV_WARPS && a.bias && n_out < a.N) ? bf16_to_f32(a.bias[n_out]) : 0.0f;
+
+        if (warp == GV_WARPS) {
+            // ---- producer: this tile's blocks of the split, four per slot
+            if (lane == 0) {
+                const uint8_t* src = a.packed + (static_cast<size_t>(tile) * a.KT + kb0) * TB;
+                for (int i = 0; i < nslots; ++i, ++it) {
+                    const int st = it % stages;
+                    // bounded: on a timeout the error bit is set and the copy is
+                    // issued anyway (the data are then garbage, never a fault)
+                    mbar_wait(&empty[st], ((it / stages) & 1) ^ 1, a.timeout_ns);
+                    const uint32_t bytes = static_cast<uint32_t>(min(GV_SLOT_KB, nkb - i * GV_SLOT_KB)) * TB;
+                    mbar_arrive_expect_tx(&full[st], bytes);
+                    bulk_load(ring + st * SLOT, src + static_cast<size_t>(i) * SLOT, bytes, &full[st]);
                 }
             }
-        }
-    }
-    if (!have_x && !mbar_wait(&xbar, 0, a.timeout_ns)) bad = true;  // a slice with no K blocks
-    if (bad && lane == 0) raise_error(ERRBIT_TIMEOUT);
+            __syncwarp();
+        } else {
+            // int8: rows 32 rb + {0..31} (two 16-row MMA blocks), K step ks;
+            // int4: rows 16 rb + {0..15}, K half ks
+            const int rb = (FMT == FMT_W8) ? (warp & 3) : (warp & 7);
+            const int ks = (FMT == FMT_W8) ? (warp >> 2) : (warp >> 3);
+            constexpr int RB = (FMT == FMT_W8) ? 2 : 1;  // 16-row MMA blocks per warp
+            float acc[RB][NB][4];
+#pragma unroll
+            for (int b = 0; b < RB; ++b)
+#pragma unroll
+                for (int j = 0; j < NB; ++j) acc[b][j][0] = acc[b][j][1] = acc[b][j][2] = acc[b][j][3] = 0.0f;
+            // ldmatrix row address of this lane inside a block's tile
+            uint32_t lm_off;
+            if constexpr (FMT == FMT_W8) {
+                // matrices: (block 0, rows 0-7), (block 0, rows 8-15), (block 1, ...), (block 1, ...)
+                const int row = 32 * rb + 16 * (lane >> 4) + 8 * ((lane >> 3) & 1) + (lane & 7);
+                lm_off = static_cast<uint32_t>(ks * 2048 + 16 * row);
+            } else {
+                const int row = 16 * rb + 8 * ((lane >> 3) & 1) + (lane & 7);  // lanes 16-31: ignored
+                lm_off = static_cast<uint32_t>(ks * 2048 + 16 * row);
+            }
+            const int row_g = (FMT == FMT_W8) ? 32 * rb + g : 16 * rb + g;  // this lane's first row
+            for (int i = 0; i < nslots; ++i, ++it) {
+                const int st = it % stages;
+                mbar_wait(&full[st], (it / stages) & 1, a.timeout_ns);  // bounded (error bit on timeout)
+                const uint8_t* slot = ring + st * SLOT;
+                const int nk = min(GV_SLOT_KB, nkb - i * GV_SLOT_KB);
+                uint32_t held = 0;
+                for (int j = 0; j < nk; ++j) {
+                    const uint8_t* blk = slot + j * TB;
+                    const int kx = (i * GV_SLOT_KB + j) * 128;  // byte offset of the block in an x row
+                    if constexpr (FMT == FMT_W8) {
+                        uint32_t d[4];
+                        ldmatrix_x4(smem_u32(blk) + lm_off, d);
+                        held ^= d[0] ^ d[1] ^ d[2] ^ d[3];
+                        uint32_t b[NB][2];
+#pragma unroll
+                        for (int nb = 0; nb < NB; ++nb) {
+                            const uint2 u = *reinterpret_cast<const uint2*>(xsm + (nb * 8 + g) * pitch + kx + 32 * ks + 8 * t);
+                            b[nb][0] = u.x;
+                            b[nb][1] = u.y;
+                        }
+#pragma unroll
+                        for (int bk = 0; bk < RB; ++bk) {
+                            const uint32_t lo0 = bytes_to_bf16x2(d[2 * bk], 0x7440u, 0x7441u);
+                            const uint32_t hi0 = bytes_to_bf16x2(d[2 * bk], 0x7442u, 0x7443u);
+                            const uint32_t lo1 = bytes_to_bf16x2(d[2 * bk + 1], 0x7440u, 0x7441u);
+                            const uint32_t hi1 = bytes_to_bf16x2(d[2 * bk + 1], 0x7442u, 0x7443u);
+#pragma unroll
+                            for (int nb = 0; nb < NB; ++nb)
+                                mma16816_bf16(acc[bk][nb], lo0, lo1, hi0, hi1, b[nb][0], b[nb][1]);
+                        }
+                    } else {
+                        uint32_t d[2];
+                        ldmatrix_x2(smem_u32(blk) + lm_off, d);
+                        uint16_t h0, h1;
+                        if constexpr (FMT == FMT_W4G64) {
+                            h0 = *reinterpret_cast<const uint16_t*>(blk + 4096 + 2 * row_g);
+                            h1 = *reinterpret_cast<const uint16_t*>(blk + 4096 + 2 * (row_g + 8));
+                        } else {  // group of inputs 32 ks + 8t..+7: 2 ks + t / 2
+                            h0 = *reinterpret_cast<const uint16_t*>(blk + 4096 + 512 * ks + 4 * row_g + 2 * (t >> 1));
+                            h1 = *reinterpret_cast<const uint16_t*>(blk + 4096 + 512 * ks + 4 * (row_g + 8) + 2 * (t >> 1));
+                        }
+                        held ^= d[0] ^ d[1] ^ h0 ^ h1;
+                        uint32_t f0[4], f1[4];
+                        nibbles_to_f16x2(d[0], __half2half2(__ushort_as_half(h0)), f0);
+                        nibbles_to_f16x2(d[1], __half2half2(__ushort_as_half(h1)), f1);
+#pragma unroll
+                        for (int nb = 0; nb < NB; ++nb) {
+                            const uint4 u = *reinterpret_cast<const uint4*>(xsm + (nb * 8 + g) * pitch + kx + 64 * ks + 16 * t);
+                            mma16816_f16(acc[0][nb], f0[0], f1[0], f0[1], f1[1], u.x, u.y);
+                            mma16816_f16(acc[0][nb], f0[2], f1[2], f0[3], f1[3], u.z, u.w);
+                        }
+                    }
+                }
+                // the slot's codes are in registers: hand it back to the producer
+                loads_done_before_release(held);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[st]);
+            }
 
-    // sum the slices in order, scale, add the bias, store
-    float* mine = red + ((slice * 2 + rg) * 32 + lane) * (NB * 4);
+            // stage this warp's partial: stage[ks][m][row]
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb)
+            for (int bk = 0; bk < RB; ++bk)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) mine[nb * 4 + e] = acc[nb][e];
-    __syncthreads();
-    if (slice != 0) return;
-    float sum[NB][4];
+                for (int h = 0; h < 2; ++h)
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb)
+                    for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) sum[nb][e] = 0.0f;
-    for (int sl = 0; sl < GV_SLICES; ++sl) {
-        const float* p = red + ((sl * 2 + rg) * 32 + lane) * (NB * 4);
+                        for (int e = 0; e < 2; ++e)
+                            stage[(ks * NB * 8 + nb * 8 + 2 * t + e) * 128 + row_g + 16 * bk + 8 * h] =
+                                acc[bk][nb][2 * h + e];
+            named_sync(2, GV_WARPS * 32);
+            // sum the P parts of four adjacent rows of one token, in part order,
+            // and send them to the owner of the rows: slot q of its buffer
+            for (int i = static_cast<int>(threadIdx.x); i < Mv * 32; i += GV_WARPS * 32) {
+                const int m = i >> 5, r4 = 4 * (i & 31);
+                float4 v = *reinterpret_cast<const float4*>(stage + m * 128 + r4);
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sum[nb][e] += p[nb * 4 + e];
-    }
-    const int n0 = nt * 128 + row0, n1 = n0 + 8;
-    const float rf0 = n0 < a.N ? a.rowf[n0] : 0.0f, rf1 = n1 < a.N ? a.rowf[n1] : 0.0f;
-    const float b0 = (a.bias && n0 < a.N) ? bf16_to_f32(a.bias[n0]) : 0.0f;
-    const float b1 = (a.bias && n1 < a.N) ? bf16_to_f32(a.bias[n1]) : 0.0f;
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int m = nb * 8 + 2 * t + (e & 1);
-            const int n = (e < 2) ? n0 : n1;
-            if (m >= a.M || n >= a.N) continue;
-            float v = sum[nb][e] * ((e < 2) ? rf0 : rf1);
-            if constexpr (FMT != FMT_W8) v *= a.xs[m];
-            store_y(a, m, n, v + ((e < 2) ? b0 : b1));
+                for (int pp = 1; pp < P; ++pp) {
+                    const float4 u = *reinterpret_cast<const float4*>(stage + (pp * NB * 8 + m) * 128 + r4);
+                    v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+                }
+                const int owner = r4 / rows_per;
+                const uint32_t addr =
+                    smem_u32(red) + static_cast<uint32_t>((q * NB * 8 + m) * rows_per + r4 % rows_per) * 4u;
+                if (S > 1) st_dsmem_v4(mapa_shared(addr, static_cast<uint32_t>(owner)), v);
+                else *reinterpret_cast<float4*>(smem_raw + (addr - raw)) = v;
+            }
+        }
+        // every partial of this CTA's rows has landed in its buffer
+        if (S > 1) cluster_sync_all();
+        else __syncthreads();
+
+        // sum the S partials of each of this CTA's rows in split order, scale,
+        // bias, store.  Thread i takes row i % rows_per and tokens
+        // i / rows_per + k (512 / rows_per).
+        if (warp < GV_WARPS) {
+            const int rl = static_cast<int>(threadIdx.x) % rows_per;
+            for (int m = static_cast<int>(threadIdx.x) / rows_per; m < Mv; m += GV_WARPS * 32 / rows_per) {
+                float v = red[m * rows_per + rl];
+                for (int sp = 1; sp < S; ++sp) v += red[(sp * NB * 8 + m) * rows_per + rl];
+                if (n_out < a.N) store_y(a, m, n_out, v * rf * xs_sm[m] + bias);
+            }
+        }
+        // the buffers are rewritten by the next tile: every CTA of the cluster
+        // must have read them first
+        if (tile + ncl < a.NT) {
+            if (S > 1) cluster_sync_all();
+            else __syncthreads();
         }
     }
+    // nothing may land in shared memory after the CTA has exited (every copy
+    // has landed unless a wait above timed out)
+    if (warp == GV_WARPS && lane == 0)
+        for (int i = max(0, it - stages); i < it; ++i) mbar_wait(&full[i % stages], (i / stages) & 1, DRAIN_TIMEOUT_NS);
 }
 
 }  // namespace wlq

@@ -13,9 +13,11 @@
 // the ring slot back at once, dequantises in registers and feeds warp-level
 // MMAs (m16n8k16, fp32 accumulate); the two groups' sums are added (in a fixed
 // order) at the end of the tile.  No MMA-issuing thread, no tensor memory and
-// no hand-off between warps sits between the weight stream and the math: a
-// single tcgen05.mma issues no faster than about one per 46 cycles, which at
-// 16 tokens is ten times the tensor work it carries.
+// no hand-off between warps sits between the weight stream and the math.  (A
+// tcgen05.mma issues no faster than about one per 46 cycles: at 16 tokens
+// that is ~1400 FLOP/clk/SM, below the ~2000 of m16n8k16 warp MMAs; at 32
+// tokens it would be ~2800, but here the weight stream, not the MMA rate,
+// bounds the kernel.)
 //
 // Inputs inside a 64-wide K block are renumbered for the MMA: lane (g, t) of
 // a warp (g = lane / 4, t = lane % 4) takes inputs 16t..16t+15 of its rows

@@ -233,16 +233,34 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     // their own, so weight loads never wait for the MMA.
     const size_t xres_bytes = static_cast<size_t>(p.kbps) * p.BN * 128u;
     p.ks = 0;
-    // At most 16 tokens, no low rank, x (zero-padded) fits in shared memory:
-    // the direct-load kernel (no weight ring, no K split across CTAs).
-    {
+    // At most 16 tokens, no low rank: the direct-load kernel.  A cluster of
+    // S CTAs splits each 128-channel tile's K range; S grows while the tiles
+    // times S fit on the SMs (and every split keeps two K blocks), then while
+    // the CTA's x rows and a two-slot weight ring do not fit in shared memory.
+    // The ring takes what shared memory is left, up to eight slots.
+    if (r == 0 && M <= 16) {
         const int nb = (M <= 8) ? 1 : 2;
-        const size_t need = 128 + static_cast<size_t>(nb * 8) * wlq::gv_x_pitch(p.KT) +
-                            static_cast<size_t>(wlq::GV_SLICES) * 2 * 32 * nb * 4 * 4;
-        if (r == 0 && M <= 16 && need <= kSmemLimit - 1024) {
+        const size_t lim = kSmemLimit - 1024;
+        int gs = 1;
+        while (gs * 2 <= wlq::GV_MAX_SPLITS && static_cast<int64_t>(p.NT) * gs * 2 <= cap && p.KT >= gs * 2 * 2)
+            gs *= 2;
+        auto kbps_of = [&](int s_) { return static_cast<int>(cdiv(p.KT, s_)); };
+        while (wlq::gv_smem_bytes(fmt, nb, kbps_of(gs), 2) > lim && gs * 2 <= wlq::GV_MAX_SPLITS && p.KT >= gs * 2)
+            gs *= 2;
+        // every split owns at least one K block
+        while (gs > 1 && static_cast<int64_t>(gs - 1) * kbps_of(gs) >= p.KT) gs /= 2;
+        const size_t fixed = wlq::gv_smem_bytes(fmt, nb, kbps_of(gs), 0);
+        const int st = (fixed < lim) ? static_cast<int>(std::min<size_t>(wlq::GV_MAX_STAGES,
+                                                                          (lim - fixed) / wlq::gv_slot_bytes(fmt)))
+                                     : 0;
+        if (st >= 2) {
             p.gemv = true;
-            p.smem = need;
-            p.grid = static_cast<int>(cdiv(N, wlq::GV_ROWS));
+            p.S = gs;
+            p.kbps = kbps_of(gs);
+            p.stages = st;
+            p.smem = wlq::gv_smem_bytes(fmt, nb, p.kbps, st);
+            p.tiles_nm = p.NT;
+            p.grid = static_cast<int>(std::min<int64_t>(p.NT, std::max(1, cap / gs))) * gs;  // persistent over tiles
             size_t off = 0;
             if (fmt != wlq::FMT_W8) {
                 p.off_x16 = off; off = align256(off + static_cast<size_t>(M) * K * 2);
@@ -497,16 +515,50 @@ wlq_status launch_skinny(Plan& p, const CUtensorMap& tx, wlq::GemmArgs& a, Devic
 template <int FMT, int NB>
 wlq_status launch_gemv(Plan& p, wlq::GemmArgs& a, DeviceInfo* d, cudaStream_t st) {
     auto kern = wlq::gemv_kernel<FMT, NB>;
-    const int kid = 21 + FMT * 2 + (NB == 1 ? 0 : 1);
+    const int kid = 21 + FMT * 2 + (NB == 1 ? 0 : 1);  // 21..26
     if (!d->smem_set[kid]) {
-        // the kernel also holds a little static shared memory (its barrier)
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(kSmemLimit - 1024));
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         d->smem_set[kid] = true;
     }
-    kern<<<static_cast<unsigned>(p.grid), wlq::GV_THREADS, p.smem, st>>>(a);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cudaLaunchAttribute attr[1];
+    cfg.blockDim = dim3(wlq::GV_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = st;
+    const int csize = p.S;
+    int clusters = p.grid / csize;
+    if (csize > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(csize);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        // clusters are persistent over tiles: launch no more than fit at once
+        const uint64_t key = (static_cast<uint64_t>(kid) << 48) | (static_cast<uint64_t>(csize) << 32) | p.smem;
+        int active = 0;
+        {
+            std::lock_guard<std::mutex> lk(g_dev_mu);
+            auto it = d->max_clusters.find(key);
+            if (it != d->max_clusters.end()) active = it->second;
+        }
+        if (active == 0) {
+            cfg.gridDim = dim3(static_cast<unsigned>(clusters * csize), 1, 1);
+            if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) != cudaSuccess || active <= 0) {
+                cudaGetLastError();
+                active = d->sms / csize;
+            }
+            std::lock_guard<std::mutex> lk(g_dev_mu);
+            d->max_clusters[key] = active;
+        }
+        clusters = std::max(1, std::min(clusters, active));
+    }
+    cfg.gridDim = dim3(static_cast<unsigned>(clusters * csize), 1, 1);
+    p.grid = clusters * csize;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a);
     if (e != cudaSuccess) return cuda_fail(e, "gemv launch");
     return WLQ_OK;
 }
