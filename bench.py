@@ -3,7 +3,8 @@
 Workload (seeded, synthetic): W [4096, 4096] ~ N(0, 0.02) fp32 with 1% of the
 input columns x20, RTN int8 per output channel; x bf16 [M, 4096] ~ N(0, 1)
 for M in {16, 256, 4096}; bias [4096] ~ N(0, 0.01).  One step is one pass of
-the whole path: quantize W, pack it, then the Linear at M = 16, 256 and 4096
+the whole path: quantize W and pack it (one fused pass), then the Linear at
+M = 16, 256 and 4096
 (inputs already in HBM; L2 flushed between steps).  value = total Linear
 FLOPs (2 M N K) of all ranks / the max over ranks of the device time.
 
@@ -36,7 +37,7 @@ MS = (16, 256, 4096)
 METRIC = "quantized-linear TFLOP/s and HBM GB/s vs B200 roofline, M=16..4096"
 WORKLOAD = ("DiT attention projection W8A16: W[4096,4096] fp32 N(0,0.02), 1% input columns x20, "
             "RTN int8 per output channel; x bf16 [M,4096] N(0,1), M in {16,256,4096}; bias N(0,0.01); "
-            "step = quantize + pack + Linear at the three M")
+            "step = quantize + pack (one fused pass over W) + Linear at the three M")
 PROFILE = os.path.join(ROOT, "profiles", "gemm_w8_attn_m4096.txt")
 
 
@@ -204,7 +205,6 @@ def run_gpu(args):
     W = torch.from_numpy(base["W"]).to(dev)
     b = torch.from_numpy(base["b"].view(np.int16)).to(dev).view(torch.bfloat16)
     xs = {M: torch.from_numpy(wi.attn_w8(M)["x"].view(np.int16)).to(dev).view(torch.bfloat16) for M in MS}
-    codes = torch.empty((N_OUT, K_IN), dtype=torch.int8, device=dev)
     scales = torch.empty((N_OUT, 1), dtype=torch.float32, device=dev)
     packed = torch.empty(wlq.packed_bytes(N_OUT, K_IN, BITS, GROUP), dtype=torch.uint8, device=dev)
     ys = {M: torch.empty((M, N_OUT), dtype=torch.bfloat16, device=dev) for M in MS}
@@ -220,9 +220,9 @@ def run_gpu(args):
         flush.view(torch.float32).sum()
 
     def quantize_pack():
+        # RTN quantization straight into the packed operand (one pass over W)
         st = wlq._stream(torch.cuda.current_stream())
-        wlq._check(lib.wlq_quantize(ptr(W), N_OUT, K_IN, BITS, GROUP, ptr(codes), ptr(scales), st))
-        wlq._check(lib.wlq_pack(ptr(codes), ptr(scales), N_OUT, K_IN, BITS, GROUP, ptr(packed), st))
+        wlq._check(lib.wlq_quantize_pack(ptr(W), N_OUT, K_IN, BITS, GROUP, ptr(scales), ptr(packed), st))
 
     def linear(M):
         wlq.linear_into(ys[M], xs[M], packed, N_OUT, K_IN, BITS, GROUP, bias=b, workspace=wss[M])
@@ -232,7 +232,7 @@ def run_gpu(args):
         for M in MS:
             linear(M)
 
-    launches_per_step = 1 + 1 + len(MS)  # quantize, pack (int8: tiles and row factors in one kernel), one GEMM per M
+    launches_per_step = 1 + len(MS)  # quantize-and-pack, one GEMM per M
 
     for _ in range(args.warmup):
         step()

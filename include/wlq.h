@@ -93,6 +93,21 @@ size_t wlq_packed_bytes(int64_t N, int64_t K, int bits, int group);
 wlq_status wlq_pack(const int8_t* codes, const float* scales, int64_t N, int64_t K,
                     int bits, int group, void* packed, void* stream);
 
+/*
+ * wlq_quantize followed by wlq_pack in one pass over W (the same two steps
+ * of the pages: RTN quantization, then the loader's layout), without the
+ * int8 [N, K] codes: W is read once and the packed operand written once.
+ * The packed bytes and the scales are bit-identical to those of
+ * wlq_pack(wlq_quantize(W)) for the same recipe.
+ * W      : fp32 [N, K], 16-byte aligned, K <= 32768 (else WLQ_ERR_SHAPE)
+ * scales : fp32 [N, K / g] (as wlq_quantize), 4-byte aligned
+ * packed : wlq_packed_bytes(N, K, bits, group) bytes, 16-byte aligned
+ * Recipes (8, 0), (4, 64), (4, 16).  A non-finite weight sets
+ * WLQ_ERR_NONFINITE in the device error word, as wlq_quantize does.
+ */
+wlq_status wlq_quantize_pack(const float* W, int64_t N, int64_t K, int bits, int group,
+                             float* scales, void* packed, void* stream);
+
 /* Inverse of the code part of wlq_pack: packed -> codes int8 [N, K]. */
 wlq_status wlq_unpack(const void* packed, int64_t N, int64_t K, int bits, int group,
                       int8_t* codes, void* stream);

@@ -114,6 +114,13 @@ def test_argument_errors_before_any_device_access(lib):
     assert lib.wlq_quantize(None, 0, 64, 8, 0, None, None, None) == 0          # N == 0: no-op
     assert lib.wlq_quantize(vp(16), 4, 64, 8, 0, vp(17), vp(16), None) == 3    # alignment
     assert b"16-byte" in lib.wlq_last_error()
+    lib.wlq_quantize_pack.argtypes = [vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int, vp, vp, vp]
+    assert lib.wlq_quantize_pack(None, 4, 64, 8, 64, None, None, None) == 4     # no packed layout for (8, 64)
+    assert lib.wlq_quantize_pack(None, 4, 60, 8, 0, None, None, None) == 2      # K % 8
+    assert lib.wlq_quantize_pack(None, 4, 40960, 8, 0, None, None, None) == 2   # row longer than the registers hold
+    assert lib.wlq_quantize_pack(None, 4, 64, 8, 0, None, None, None) == 1      # null
+    assert lib.wlq_quantize_pack(None, 0, 64, 8, 0, None, None, None) == 0      # N == 0: no-op
+    assert lib.wlq_quantize_pack(vp(16), 4, 64, 8, 0, vp(16), vp(40), None) == 3  # packed misaligned
     # M == 0 is a no-op
     assert lib.wlq_linear(None, 0, None, 64, 64, 8, 0, None, None, None, 0, None, 0, None, 0, None) == 0
     assert lib.wlq_linear(None, 4, None, 64, 64, 4, 0, None, None, None, 0, None, 0, None, 0, None) == 4

@@ -119,3 +119,68 @@ def test_wait_probe_times_out_and_device_stays_usable():
     W = wi.weight(24, 1, 16, 64)
     cg, sg, co, so = quantize_both(W, 8, 0)
     assert_codes_equal(cg, sg, co, so)
+
+
+def _pack_reference(W, bits, group):
+    """quantize then pack, the two-kernel path, on the device."""
+    m = wlq()
+    codes, scales = m.quantize(dev_f32(W), bits, group)
+    return scales, m.pack(codes, scales, bits, group)
+
+
+@pytest.mark.parametrize("bits,group", [(8, 0), (4, 64), (4, 16)])
+@pytest.mark.parametrize("N,K", [(37, 384), (300, 448), (129, 2112), (1, 64), (256, 4096)])
+def test_quantize_pack_equals_quantize_then_pack(bits, group, N, K):
+    """The fused pass writes the same packed bytes and scales as quantize
+    followed by pack, on edge-case rows (zero, ties, subnormal, huge, a lone
+    outlier, constant) and ragged N; ragged K for the recipes that allow it."""
+    g = np.random.default_rng(7 * N + K + bits)
+    W = (g.standard_normal((N, K)) * 0.02).astype(np.float32)
+    if N > 6:
+        W[0] = 0.0
+        W[1] = g.integers(-9, 10, K).astype(np.float32) * 0.5
+        W[2] *= 1e-38
+        W[3] *= 1e36
+        W[4, 5] = -50.0
+        W[5, :] = 3.0
+    m = wlq()
+    s_ref, p_ref = _pack_reference(W, bits, group)
+    s_f, p_f = m.quantize_pack(dev_f32(W), bits, group)
+    torch.cuda.synchronize()
+    m.check_status()
+    assert torch.equal(s_f, s_ref)
+    assert p_f.numel() == p_ref.numel()
+    assert torch.equal(p_f, p_ref)
+
+
+@pytest.mark.parametrize("bits,group,K", [(8, 0, 200), (8, 0, 4040), (4, 16, 1232)])
+def test_quantize_pack_ragged_k(bits, group, K):
+    """K not a multiple of 64: the last tile's inputs beyond K are code 0 (and
+    their int4 group scales 0), as pack writes them."""
+    g = np.random.default_rng(K)
+    W = (g.standard_normal((150, K)) * 0.05).astype(np.float32)
+    m = wlq()
+    s_ref, p_ref = _pack_reference(W, bits, group)
+    s_f, p_f = m.quantize_pack(dev_f32(W), bits, group)
+    torch.cuda.synchronize()
+    assert torch.equal(s_f, s_ref)
+    assert torch.equal(p_f, p_ref)
+
+
+@pytest.mark.parametrize("bits,group", [(8, 0), (4, 64), (4, 16)])
+def test_quantize_pack_nonfinite_flags_and_zeroes(bits, group):
+    """A NaN or infinity sets the non-finite error bit; its group (row) gets
+    scale 0 and codes 0, exactly as the two-kernel path."""
+    g = np.random.default_rng(5)
+    W = (g.standard_normal((140, 256)) * 0.02).astype(np.float32)
+    W[3, 17] = np.nan
+    W[130, 200] = np.inf
+    m = wlq()
+    m.check_status()
+    s_f, p_f = m.quantize_pack(dev_f32(W), bits, group)
+    torch.cuda.synchronize()
+    assert m.get_status() == m.ERR_NONFINITE
+    s_ref, p_ref = _pack_reference(W, bits, group)
+    assert m.get_status() == m.ERR_NONFINITE  # the two-kernel path flags it too (and clears the word)
+    assert torch.equal(s_f, s_ref)
+    assert torch.equal(p_f, p_ref)

@@ -38,6 +38,7 @@ lib.wlq_packed_bytes.argtypes = [_i64, _i64, _i32, _i32]
 lib.wlq_packed_bytes.restype = _sz
 lib.wlq_pack.argtypes = [_vp, _vp, _i64, _i64, _i32, _i32, _vp, _vp]
 lib.wlq_unpack.argtypes = [_vp, _i64, _i64, _i32, _i32, _vp, _vp]
+lib.wlq_quantize_pack.argtypes = [_vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp]
 lib.wlq_linear_workspace.argtypes = [_i64, _i64, _i64, _i32, _i32, _i32]
 lib.wlq_linear_workspace.restype = _sz
 lib.wlq_linear.argtypes = [_vp, _i64, _vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _sz, _vp]
@@ -48,7 +49,7 @@ lib.wlq_set_grid_limit.argtypes = [_i32]
 lib.wlq_set_grid_limit.restype = None
 lib.wlq_last_error.restype = ctypes.c_char_p
 lib.wlq_version.restype = ctypes.c_char_p
-for _f in ("wlq_quantize", "wlq_pack", "wlq_unpack", "wlq_linear", "wlq_linear_noalloc", "wlq_get_status",
+for _f in ("wlq_quantize", "wlq_quantize_pack", "wlq_pack", "wlq_unpack", "wlq_linear", "wlq_linear_noalloc", "wlq_get_status",
            "wlq_probe_wait_timeout"):
     getattr(lib, _f).restype = ctypes.c_int
 
@@ -99,6 +100,19 @@ def pack(codes: torch.Tensor, scales: torch.Tensor, bits: int, group: int, strea
     out = torch.empty(nbytes, dtype=torch.uint8, device=codes.device)
     _check(lib.wlq_pack(_ptr(codes), _ptr(scales), N, K, bits, group, _ptr(out), _stream(stream)))
     return out
+
+
+def quantize_pack(W: torch.Tensor, bits: int, group: int, stream=None):
+    """quantize then pack in one pass: fp32 W [N, K] -> (scales fp32 [N,G], packed uint8)."""
+    assert W.dtype == torch.float32 and W.is_cuda and W.is_contiguous()
+    N, K = W.shape
+    nbytes = packed_bytes(N, K, bits, group)
+    if nbytes == 0:
+        raise WlqError(ERR_UNSUPPORTED, "no packed layout for bits=%d group=%d K=%d" % (bits, group, K))
+    scales = torch.empty((N, groups(K, group)), dtype=torch.float32, device=W.device)
+    out = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    _check(lib.wlq_quantize_pack(_ptr(W), N, K, bits, group, _ptr(scales), _ptr(out), _stream(stream)))
+    return scales, out
 
 
 def unpack(packed: torch.Tensor, N: int, K: int, bits: int, group: int, stream=None) -> torch.Tensor:

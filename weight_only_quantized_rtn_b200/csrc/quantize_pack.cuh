@@ -1,0 +1,155 @@
+// quantize_pack.cuh -- RTN quantization written straight into the packed
+// operand ("Joy-face_change_optimized" model card, files table and tools row:
+// int8 with one scale per output channel, int4 grouped along K with gs 64 /
+// 16; the "loader" step lays the codes out for the GEMM).
+//
+// The result is bit-identical to quantize (quantize.cuh) followed by pack
+// (pack.cuh): same absmax, same scale, same exactly rounded codes, same
+// offset-binary bytes and nibble order, same fp16 scale normalisation and row
+// factors, same zero fill beyond N and K.  The int8 [N, K] code array is never
+// written or read back: W is read once and the packed operand written once.
+#pragma once
+#include <cstdint>
+#include <cuda_fp16.h>
+#include "ptx.cuh"
+#include "quantize.cuh"
+#include "pack.cuh"
+
+namespace wlq {
+
+// One CTA per padded output row (grid-stride over ceil(N/128)*128 rows).  The
+// row's ceil(K/64)*64 inputs (zeros past K and for rows >= N) are held in
+// registers: thread j takes float4 j + i*blockDim (i < V), so the lanes of a
+// warp hold consecutive inputs and a group of g inputs is g/4 adjacent lanes.
+//  - int8: the row's absmax is reduced over the CTA (magnitude bit patterns,
+//    as in quantize_rows_cta_kernel); each float4 becomes one 32-bit word of
+//    four offset-binary bytes at its place in the row's 16-byte run.
+//  - int4: each group's absmax is reduced over its lanes; the row's largest
+//    group scale (over the CTA) fixes the fp16 normalisation 2^e_n and the
+//    row factor 2^-e_n; two adjacent lanes merge their four nibbles each into
+//    one 32-bit word of eight.
+template <int FMT, int V>
+__global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
+    const float* __restrict__ W, int64_t N, int64_t K, int KT, int64_t rows, int qmax,
+    float* __restrict__ scales, float* __restrict__ rowf, uint8_t* __restrict__ packed) {
+    constexpr uint32_t TB = tile_bytes(FMT);
+    constexpr int L = (FMT == FMT_W4G64) ? 16 : 4;  // int4: lanes per group (group / 4)
+    constexpr int GS = 4 * L;                        // int4: group size
+    __shared__ uint32_t part[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nwarps = blockDim.x >> 5;
+    const int K4 = static_cast<int>(K / 4);
+    const int KP4 = KT * 16;  // float4s of the padded row
+    const int64_t G = (FMT == FMT_W8) ? 1 : K / GS;
+    bool bad = false;
+    for (int64_t n = blockIdx.x; n < rows; n += gridDim.x) {
+        const bool row_ok = n < N;
+        const int i_row = static_cast<int>(n & 127);
+        uint8_t* tiles = packed + static_cast<size_t>(n >> 7) * KT * TB;
+        const float4* row = reinterpret_cast<const float4*>(W + (row_ok ? n : 0) * K);
+        float4 v[V];
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int idx = threadIdx.x + i * blockDim.x;
+            v[i] = (row_ok && idx < K4) ? __ldcs(row + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if constexpr (FMT == FMT_W8) {
+            uint32_t m = 0;
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                m = max(m, __float_as_uint(v[i].x) & 0x7FFFFFFFu);
+                m = max(m, __float_as_uint(v[i].y) & 0x7FFFFFFFu);
+                m = max(m, __float_as_uint(v[i].z) & 0x7FFFFFFFu);
+                m = max(m, __float_as_uint(v[i].w) & 0x7FFFFFFFu);
+            }
+            for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+            if (lane == 0) part[warp] = m;
+            __syncthreads();
+            m = part[0];
+            for (int w = 1; w < nwarps; ++w) m = max(m, part[w]);
+            const bool row_bad = m >= 0x7F800000u;  // NaN or infinity in the row
+            bad |= row_bad;
+            const GroupScale g = group_scale(row_bad ? 0.0f : __uint_as_float(m), qmax);
+            if (threadIdx.x == 0) {
+                if (row_ok) scales[n] = g.s;
+                rowf[n] = row_ok ? g.s : 0.0f;
+            }
+            const float h = 0.5f * g.s;
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int idx = threadIdx.x + i * blockDim.x;
+                if (idx >= KP4) continue;
+                bool unused = false;
+                const uint32_t c4 = g.normal ? rtn4_f32(v[i], g.s, g.inv, h) : pack_codes4(v[i], g, qmax, unused);
+                const int k = 4 * idx;  // inputs k..k+3 of block k/64, run (k%64)/16
+                *reinterpret_cast<uint32_t*>(tiles + (k >> 6) * TB + ((k >> 4) & 3) * 2048 + 16 * i_row + (k & 15)) =
+                    c4 ^ 0x80808080u;  // offset binary q + 128
+            }
+            __syncthreads();  // part[] is rewritten for the next row
+        } else {
+            // group absmax (per group of L lanes; 0 for a group holding a NaN
+            // or infinity) and the row's largest group scale over the CTA
+            // (scales are non-negative floats: their bit patterns order them)
+            float ga[V];
+            uint32_t smax = 0;
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                uint32_t m = max(max(__float_as_uint(v[i].x) & 0x7FFFFFFFu, __float_as_uint(v[i].y) & 0x7FFFFFFFu),
+                                 max(__float_as_uint(v[i].z) & 0x7FFFFFFFu, __float_as_uint(v[i].w) & 0x7FFFFFFFu));
+                for (int off = L >> 1; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+                const bool gbad = m >= 0x7F800000u;
+                bad |= gbad;
+                ga[i] = gbad ? 0.0f : __uint_as_float(m);
+                smax = max(smax, __float_as_uint(__fdiv_rn(ga[i], static_cast<float>(qmax))));
+            }
+            for (int off = 16; off > 0; off >>= 1) smax = max(smax, __shfl_xor_sync(0xffffffffu, smax, off));
+            if (lane == 0) part[warp] = smax;
+            __syncthreads();
+            smax = part[0];
+            for (int w = 1; w < nwarps; ++w) smax = max(smax, part[w]);
+            const float S = __uint_as_float(smax);
+            float rf = 0.0f;
+            if (row_ok && S > 0.0f) {
+                int ex;
+                frexpf(S, &ex);             // S in [2^(ex-1), 2^ex)
+                rf = ldexpf(1.0f, ex - 9);  // 2^-e_n with e_n = 9 - ex
+            }
+            if (threadIdx.x == 0) rowf[n] = rf;
+            const int sh = (rf > 0.0f) ? -ilogbf(rf) : 0;  // s * 2^sh = s / rf exactly
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int idx = threadIdx.x + i * blockDim.x;
+                const int k = 4 * idx;
+                bool unused = false;
+                const GroupScale gs = group_scale(ga[i], qmax);
+                const uint32_t c4 = gs.normal ? rtn4_f32(v[i], gs.s, gs.inv, 0.5f * gs.s) : pack_codes4(v[i], gs, qmax, unused);
+                // four nibbles (q + 8) at their places among the eight of the word
+                uint32_t w = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t u = ((c4 >> (8 * j)) + 8u) & 0xFu;
+                    w |= u << (4 * int4_nibble_pos(4 * (idx & 1) + j));
+                }
+                w |= __shfl_xor_sync(0xffffffffu, w, 1);
+                if (idx >= KP4) continue;
+                uint8_t* blk = tiles + (k >> 6) * TB;
+                if ((idx & 1) == 0)  // word (k%32)/8 of run (k%64)/32
+                    *reinterpret_cast<uint32_t*>(blk + ((k >> 5) & 1) * 2048 + 16 * i_row + 4 * ((k >> 3) & 3)) = w;
+                if ((idx & (L - 1)) == 0) {  // first lane of the group: its scales
+                    const int64_t gi = k / GS;
+                    const bool real = row_ok && gi < G;
+                    if (real) scales[n * G + gi] = gs.s;
+                    const __half h16 = (real && rf != 0.0f) ? __float2half_rn(ldexpf(gs.s, sh)) : __float2half_rn(0.0f);
+                    if constexpr (FMT == FMT_W4G64)
+                        *reinterpret_cast<__half*>(blk + 4096 + 2 * i_row) = h16;
+                    else  // group (k%64)/16: half ((k%64)/32), slot ((k%32)/16)
+                        *reinterpret_cast<__half*>(blk + 4096 + 512 * ((k >> 5) & 1) + 4 * i_row + 2 * ((k >> 4) & 1)) = h16;
+                }
+            }
+            __syncthreads();  // part[] is rewritten for the next row
+        }
+    }
+    if (bad) raise_error(ERRBIT_NONFINITE);
+}
+
+}  // namespace wlq

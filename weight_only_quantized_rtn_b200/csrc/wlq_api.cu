@@ -15,6 +15,7 @@
 #include "gemm.cuh"
 #include "skinny.cuh"
 #include "gemv.cuh"
+#include "quantize_pack.cuh"
 #include "pack.cuh"
 #include "prep.cuh"
 #include "ptx.cuh"
@@ -685,6 +686,44 @@ wlq_status wlq_quantize(const float* W, int64_t N, int64_t K, int bits, int grou
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+    return WLQ_OK;
+}
+
+wlq_status wlq_quantize_pack(const float* W, int64_t N, int64_t K, int bits, int group, float* scales,
+                             void* packed, void* stream) {
+    const int fmt = fmt_of(bits, group);
+    if (fmt < 0) return fail(WLQ_ERR_UNSUPPORTED, "quantize_pack supports (8,0), (4,64) and (4,16)");
+    wlq_status st = check_shape(N, K, bits, group);
+    if (st != WLQ_OK) return st;
+    if (N == 0) return WLQ_OK;
+    if (K > 8 * 4 * 1024) return fail(WLQ_ERR_SHAPE, "quantize_pack holds a row in registers: K <= 32768");
+    if (!W || !scales || !packed) return fail(WLQ_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(W) || !aligned16(packed) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+        return fail(WLQ_ERR_ALIGN, "W and packed must be 16-byte aligned, scales 4-byte aligned");
+    int dev;
+    DeviceInfo* d;
+    if ((st = current_device(&dev, &d)) != WLQ_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t NT = cdiv(N, 128), KT = cdiv(K, 64);
+    uint8_t* base = static_cast<uint8_t*>(packed);
+    float* rowf = reinterpret_cast<float*>(base + NT * KT * wlq::tile_bytes(fmt));
+    const int qmax = (1 << (bits - 1)) - 1;
+    // one CTA per padded row, the row in registers: 8 float4 per thread
+    const int64_t kp4 = KT * 16;
+    const int threads = static_cast<int>(std::min<int64_t>(1024, std::max<int64_t>(32, (cdiv(kp4, 8) + 31) / 32 * 32)));
+    const int64_t rows = NT * 128;
+    const int grid = static_cast<int>(std::min<int64_t>(rows, static_cast<int64_t>(d->sms) * (2048 / threads)));
+    if (fmt == wlq::FMT_W8)
+        wlq::quantize_pack_rows_kernel<wlq::FMT_W8, 8><<<grid, threads, 0, s>>>(W, N, K, static_cast<int>(KT), rows,
+                                                                               qmax, scales, rowf, base);
+    else if (fmt == wlq::FMT_W4G64)
+        wlq::quantize_pack_rows_kernel<wlq::FMT_W4G64, 8><<<grid, threads, 0, s>>>(W, N, K, static_cast<int>(KT), rows,
+                                                                                  qmax, scales, rowf, base);
+    else
+        wlq::quantize_pack_rows_kernel<wlq::FMT_W4G16, 8><<<grid, threads, 0, s>>>(W, N, K, static_cast<int>(KT), rows,
+                                                                                  qmax, scales, rowf, base);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "quantize_pack launch");
     return WLQ_OK;
 }
 
