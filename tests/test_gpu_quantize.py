@@ -129,7 +129,7 @@ def _pack_reference(W, bits, group):
 
 
 @pytest.mark.parametrize("bits,group", [(8, 0), (4, 64), (4, 16)])
-@pytest.mark.parametrize("N,K", [(37, 384), (300, 448), (129, 2112), (1, 64), (256, 4096)])
+@pytest.mark.parametrize("N,K", [(37, 384), (300, 448), (129, 2112), (1, 64), (256, 4096), (70, 12288)])
 def test_quantize_pack_equals_quantize_then_pack(bits, group, N, K):
     """The fused pass writes the same packed bytes and scales as quantize
     followed by pack, on edge-case rows (zero, ties, subnormal, huge, a lone
