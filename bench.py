@@ -125,7 +125,7 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
-def cpu_baseline(n_rows_per_m=(16, 64, 944)):
+def cpu_baseline(n_rows_per_m=(48, 192, 2832)):
     """The oracle as it stands on this host's cores: quantize the whole W, then
     the Linear for a bounded sample of rows of each M batch."""
     import oracle
