@@ -905,6 +905,7 @@ template <int FMT, bool PAIR, bool XRES>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_t,
             const __grid_constant__ CUtensorMap tm_l2, const GemmArgs a) {
+    grid_dependency_sync();
     // a partial kept in the ring needs one tile per cluster (the host plans
     // it so; refuse anything else)
     if (a.red_alias && !a.tail && a.tiles_nm > static_cast<int>(cluster_count_x())) {
@@ -1013,6 +1014,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
 
 // Exercise the bounded wait alone: nothing ever arrives on this barrier.
 __global__ void wait_probe_kernel(uint64_t timeout_ns) {
+    grid_dependency_sync();
     __shared__ uint64_t bar;
     if (threadIdx.x == 0) {
         mbar_init(&bar, 1);

@@ -34,6 +34,7 @@ __device__ __forceinline__ int int4_nibble_pos(int t) { return (t & 1) ? 4 + (t 
 // int4: one warp per padded row, the fp32 factor the epilogue multiplies by.
 __global__ void pack_rowfactor_kernel(const float* __restrict__ scales, int64_t N, int64_t G,
                                       int fmt, int64_t N_pad, float* __restrict__ rowf) {
+    grid_dependency_sync();
     const int lane = threadIdx.x & 31;
     const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -66,6 +67,7 @@ __global__ void pack_rowfactor_kernel(const float* __restrict__ scales, int64_t 
 __global__ void __launch_bounds__(128) pack_tiles_kernel(
     const int8_t* __restrict__ codes, const float* __restrict__ scales, int64_t N, int64_t K,
     int64_t G, int fmt, int KT, float* __restrict__ rowf, uint8_t* __restrict__ packed) {
+    grid_dependency_sync();
     const int64_t tile = blockIdx.x;
     const int64_t nt = tile / KT;
     const int kb = static_cast<int>(tile % KT);
@@ -125,6 +127,7 @@ __global__ void __launch_bounds__(128) pack_tiles_kernel(
 __global__ void __launch_bounds__(128) unpack_tiles_kernel(const uint8_t* __restrict__ packed,
                                                            int64_t N, int64_t K, int fmt, int KT,
                                                            int8_t* __restrict__ codes) {
+    grid_dependency_sync();
     const int64_t tile = blockIdx.x;
     const int64_t nt = tile / KT;
     const int kb = static_cast<int>(tile % KT);

@@ -23,6 +23,7 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as
 // One warp per row.
 __global__ void __launch_bounds__(256) prep_x16_kernel(const uint16_t* __restrict__ x, int M, int K,
                                                        __half* __restrict__ x16, float* __restrict__ xs) {
+    grid_dependency_sync();
     const int lane = threadIdx.x & 31;
     const int w0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nw = (gridDim.x * blockDim.x) >> 5;
@@ -88,6 +89,7 @@ constexpr int LR_PITCH = LR_KC + 8;  // smem row pitch in bf16 elements (144 byt
 __global__ void __launch_bounds__(128) prep_lr_t_kernel(const uint16_t* __restrict__ x,
                                                         const uint16_t* __restrict__ L1, int M, int K,
                                                         int r, int W, uint16_t* __restrict__ thl) {
+    grid_dependency_sync();
     __shared__ __align__(16) uint16_t xt[LR_ROWS * LR_PITCH];
     __shared__ __align__(16) uint16_t lt[64 * LR_PITCH];  // [j][k]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -147,6 +149,7 @@ __global__ void __launch_bounds__(128) prep_lr_t_kernel(const uint16_t* __restri
 // L2t[n][c] = L2[c mod r][n] for c < 2r, zero beyond 2r or N.
 __global__ void prep_lr_l2t_kernel(const uint16_t* __restrict__ L2, int N, int N_pad, int r, int W,
                                    uint16_t* __restrict__ l2t) {
+    grid_dependency_sync();
     const int64_t total = static_cast<int64_t>(N_pad) * W;
     for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
          idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {

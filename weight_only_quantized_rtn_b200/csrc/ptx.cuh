@@ -21,6 +21,15 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// Programmatic dependent launch: every kernel of this library may be
+// launched while the previous grid on its stream is still finishing.  Its
+// first action waits until that grid has completed and its memory writes are
+// visible (a no-op for a normally ordered launch), then lets the next grid be
+// scheduled as soon as every CTA of this one is running.
+__device__ __forceinline__ void grid_dependency_sync() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

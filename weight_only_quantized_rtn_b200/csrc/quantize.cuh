@@ -95,6 +95,7 @@ __device__ __forceinline__ uint32_t pack_codes4(float4 v, const GroupScale& g, i
 __global__ void __launch_bounds__(256) quantize_rows_kernel(
     const float* __restrict__ W, int64_t N, int64_t K, int qmax, int8_t* __restrict__ codes,
     float* __restrict__ scales) {
+    grid_dependency_sync();
     const int lane = threadIdx.x & 31;
     const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -174,6 +175,7 @@ template <int V>
 __global__ void __launch_bounds__(1024) quantize_rows_cta_kernel(
     const float* __restrict__ W, int64_t N, int64_t K, int qmax, int8_t* __restrict__ codes,
     float* __restrict__ scales) {
+    grid_dependency_sync();
     __shared__ uint32_t part[32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nwarps = blockDim.x >> 5;
@@ -232,6 +234,7 @@ __global__ void __launch_bounds__(1024) quantize_rows_cta_kernel(
 __global__ void __launch_bounds__(256) quantize_groups_kernel(
     const float* __restrict__ W, int64_t total4, int lanes_per_group, int qmax,
     int8_t* __restrict__ codes, float* __restrict__ scales) {
+    grid_dependency_sync();
     constexpr int U = 4;
     const int lane = threadIdx.x & 31;
     const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;

@@ -32,6 +32,7 @@ template <int FMT, int V>
 __global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
     const float* __restrict__ W, int64_t N, int64_t K, int KT, int64_t rows, int qmax,
     float* __restrict__ scales, float* __restrict__ rowf, uint8_t* __restrict__ packed) {
+    grid_dependency_sync();
     constexpr uint32_t TB = tile_bytes(FMT);
     constexpr int L = (FMT == FMT_W4G64) ? 16 : 4;  // int4: lanes per group (group / 4)
     constexpr int GS = 4 * L;                        // int4: group size

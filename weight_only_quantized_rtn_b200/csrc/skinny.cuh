@@ -325,6 +325,7 @@ __device__ void sk_compute(const GemmArgs& a, const SkSmem& s, const Sched& sc, 
 template <int FMT, int NB>
 __global__ void __launch_bounds__(SK_THREADS, 1)
 skinny_kernel(const __grid_constant__ CUtensorMap tm_x, const GemmArgs a) {
+    grid_dependency_sync();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);

@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <utility>
 #include <mutex>
 #include <unordered_map>
 
@@ -379,6 +380,18 @@ wlq_status check_shape(int64_t N, int64_t K, int bits, int group) {
 }
 
 
+// Adds programmatic dependent launch to a configuration (keeping its cluster
+// attribute, if any): see launch_k.
+void add_pdl(cudaLaunchConfig_t& cfg, cudaLaunchAttribute (&all)[2]) {
+    int na = 0;
+    if (cfg.numAttrs > 0) all[na++] = cfg.attrs[0];
+    all[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    all[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+    cfg.attrs = all;
+    cfg.numAttrs = static_cast<unsigned>(na);
+}
+
 template <int FMT, bool PAIR, bool XRES>
 wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, const CUtensorMap& tl,
                        wlq::GemmArgs& a, DeviceInfo* d, cudaStream_t st) {
@@ -457,6 +470,8 @@ wlq_status launch_gemm(Plan& p, const CUtensorMap& tx, const CUtensorMap& tt, co
     if (p.red_alias && clusters < p.tiles_nm) return kRetryPlan;
     cfg.gridDim = dim3(static_cast<unsigned>(clusters * csize), 1, 1);
     p.grid = clusters * csize;
+    cudaLaunchAttribute all_attrs[2];
+    add_pdl(cfg, all_attrs);
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tx, tt, tl, a);
     if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
     return WLQ_OK;
@@ -508,6 +523,8 @@ wlq_status launch_skinny(Plan& p, const CUtensorMap& tx, wlq::GemmArgs& a, Devic
     }
     cfg.gridDim = dim3(static_cast<unsigned>(clusters * csize), 1, 1);
     p.grid = clusters * csize;
+    cudaLaunchAttribute all_attrs[2];
+    add_pdl(cfg, all_attrs);
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tx, a);
     if (e != cudaSuccess) return cuda_fail(e, "skinny launch");
     return WLQ_OK;
@@ -559,6 +576,8 @@ wlq_status launch_gemv(Plan& p, wlq::GemmArgs& a, DeviceInfo* d, cudaStream_t st
     }
     cfg.gridDim = dim3(static_cast<unsigned>(clusters * csize), 1, 1);
     p.grid = clusters * csize;
+    cudaLaunchAttribute all_attrs[2];
+    add_pdl(cfg, all_attrs);
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a);
     if (e != cudaSuccess) return cuda_fail(e, "gemv launch");
     return WLQ_OK;
@@ -575,6 +594,26 @@ wlq_status launch_skinny_nb(Plan& p, const CUtensorMap& tx, wlq::GemmArgs& a, De
     if (p.BN == 16) return launch_skinny<FMT, 2>(p, tx, a, d, st);
     if (p.BN == 32) return launch_skinny<FMT, 4>(p, tx, a, d, st);
     return launch_skinny<FMT, 8>(p, tx, a, d, st);
+}
+
+// Every launch allows programmatic dependent launch: the kernel may start
+// while the previous grid on the stream finishes; each kernel's first action
+// is griddepcontrol.wait (ptx.cuh, grid_dependency_sync), which blocks until
+// that grid has completed and its memory is visible.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 int grid_for(int64_t work, int per_block, int sms) {
@@ -676,12 +715,12 @@ wlq_status wlq_quantize(const float* W, int64_t N, int64_t K, int bits, int grou
         const int64_t per_thread = 8 * 4;
         const int threads = static_cast<int>(std::min<int64_t>(1024, std::max<int64_t>(32, (cdiv(K, per_thread) + 31) / 32 * 32)));
         const int grid = static_cast<int>(std::min<int64_t>(N, static_cast<int64_t>(d->sms) * (2048 / threads)));
-        wlq::quantize_rows_cta_kernel<8><<<grid, threads, 0, s>>>(W, N, K, qmax, codes, scales);
+        launch_k(wlq::quantize_rows_cta_kernel<8>, grid, threads, 0, s, W, N, K, qmax, codes, scales);
     } else if (group == 0) {
-        wlq::quantize_rows_kernel<<<grid_for(N * 32, 256, d->sms), 256, 0, s>>>(W, N, K, qmax, codes, scales);
+        launch_k(wlq::quantize_rows_kernel, grid_for(N * 32, 256, d->sms), 256, 0, s, W, N, K, qmax, codes, scales);
     } else {
         const int64_t total4 = N * K / 4;
-        wlq::quantize_groups_kernel<<<grid_for(cdiv(total4, 4), 256, d->sms), 256, 0, s>>>(W, total4, group / 4, qmax,
+        launch_k(wlq::quantize_groups_kernel, grid_for(cdiv(total4, 4), 256, d->sms), 256, 0, s, W, total4, group / 4, qmax,
                                                                                    codes, scales);
     }
     cudaError_t e = cudaGetLastError();
@@ -714,13 +753,13 @@ wlq_status wlq_quantize_pack(const float* W, int64_t N, int64_t K, int bits, int
     const int64_t rows = NT * 128;
     const int grid = static_cast<int>(std::min<int64_t>(rows, static_cast<int64_t>(d->sms) * (2048 / threads)));
     if (fmt == wlq::FMT_W8)
-        wlq::quantize_pack_rows_kernel<wlq::FMT_W8, 8><<<grid, threads, 0, s>>>(W, N, K, static_cast<int>(KT), rows,
+        launch_k(wlq::quantize_pack_rows_kernel<wlq::FMT_W8, 8>, grid, threads, 0, s, W, N, K, static_cast<int>(KT), rows,
                                                                                qmax, scales, rowf, base);
     else if (fmt == wlq::FMT_W4G64)
-        wlq::quantize_pack_rows_kernel<wlq::FMT_W4G64, 8><<<grid, threads, 0, s>>>(W, N, K, static_cast<int>(KT), rows,
+        launch_k(wlq::quantize_pack_rows_kernel<wlq::FMT_W4G64, 8>, grid, threads, 0, s, W, N, K, static_cast<int>(KT), rows,
                                                                                   qmax, scales, rowf, base);
     else
-        wlq::quantize_pack_rows_kernel<wlq::FMT_W4G16, 8><<<grid, threads, 0, s>>>(W, N, K, static_cast<int>(KT), rows,
+        launch_k(wlq::quantize_pack_rows_kernel<wlq::FMT_W4G16, 8>, grid, threads, 0, s, W, N, K, static_cast<int>(KT), rows,
                                                                                   qmax, scales, rowf, base);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "quantize_pack launch");
@@ -753,8 +792,8 @@ wlq_status wlq_pack(const int8_t* codes, const float* scales, int64_t N, int64_t
     uint8_t* base = static_cast<uint8_t*>(packed);
     float* rowf = reinterpret_cast<float*>(base + NT * KT * wlq::tile_bytes(fmt));
     if (fmt != wlq::FMT_W8)  // int8 row factors are written by the tile kernel itself
-        wlq::pack_rowfactor_kernel<<<grid_for(NT * 128 * 32, 256, d->sms), 256, 0, s>>>(scales, N, G, fmt, NT * 128, rowf);
-    wlq::pack_tiles_kernel<<<static_cast<unsigned>(NT * KT), 128, 0, s>>>(codes, scales, N, K, G, fmt,
+        launch_k(wlq::pack_rowfactor_kernel, grid_for(NT * 128 * 32, 256, d->sms), 256, 0, s, scales, N, G, fmt, NT * 128, rowf);
+    launch_k(wlq::pack_tiles_kernel, static_cast<unsigned>(NT * KT), 128, 0, s, codes, scales, N, K, G, fmt,
                                                                           static_cast<int>(KT), rowf, base);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "pack launch");
@@ -774,7 +813,7 @@ wlq_status wlq_unpack(const void* packed, int64_t N, int64_t K, int bits, int gr
     DeviceInfo* d;
     if ((st = current_device(&dev, &d)) != WLQ_OK) return st;
     const int64_t NT = cdiv(N, 128), KT = cdiv(K, 64);
-    wlq::unpack_tiles_kernel<<<static_cast<unsigned>(NT * KT), 128, 0, static_cast<cudaStream_t>(stream)>>>(
+    launch_k(wlq::unpack_tiles_kernel, static_cast<unsigned>(NT * KT), 128, 0, static_cast<cudaStream_t>(stream), 
         static_cast<const uint8_t*>(packed), N, K, fmt, static_cast<int>(KT), codes);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "unpack launch");
@@ -826,7 +865,7 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
     if (workspace && !aligned16(workspace)) return fail(WLQ_ERR_ALIGN, "workspace must be 16-byte aligned");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    const int64_t NT = p.NT, KT = p.KT;
+    const int64_t NT = p.NT;
 
     // --- operand preparation
     const void* xin = x;
@@ -834,7 +873,7 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
     if (fmt != wlq::FMT_W8) {
         __half* x16 = reinterpret_cast<__half*>(ws + p.off_x16);
         xs = reinterpret_cast<float*>(ws + p.off_xs);
-        wlq::prep_x16_kernel<<<grid_for(M * 32, 256, d->sms), 256, 0, s>>>(static_cast<const uint16_t*>(x), p.M,
+        launch_k(wlq::prep_x16_kernel, grid_for(M * 32, 256, d->sms), 256, 0, s, static_cast<const uint16_t*>(x), p.M,
                                                                           p.K, x16, xs);
         xin = x16;
     }
@@ -844,9 +883,9 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
     if (r) {
         thl = reinterpret_cast<uint16_t*>(ws + p.off_thl);
         l2t = reinterpret_cast<uint16_t*>(ws + p.off_l2t);
-        wlq::prep_lr_t_kernel<<<static_cast<unsigned>(cdiv(M, wlq::LR_ROWS)), 128, 0, s>>>(
+        launch_k(wlq::prep_lr_t_kernel, static_cast<unsigned>(cdiv(M, wlq::LR_ROWS)), 128, 0, s, 
             static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(L1), p.M, p.K, r, W, thl);
-        wlq::prep_lr_l2t_kernel<<<grid_for(NT * 128 * W, 256, d->sms), 256, 0, s>>>(
+        launch_k(wlq::prep_lr_l2t_kernel, grid_for(NT * 128 * W, 256, d->sms), 256, 0, s, 
             static_cast<const uint16_t*>(L2), p.N, static_cast<int>(NT * 128), r, W, l2t);
     }
     cudaError_t e = cudaGetLastError();
@@ -947,7 +986,7 @@ wlq_status wlq_probe_wait_timeout(uint64_t timeout_ns, void* stream) {
     wlq_status st = current_device(&dev, &d);
     if (st != WLQ_OK) return st;
     const uint64_t cap = 10ull * 1000 * 1000 * 1000;
-    wlq::wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(std::min(timeout_ns, cap));
+    launch_k(wlq::wait_probe_kernel, 1, 32, 0, static_cast<cudaStream_t>(stream), std::min(timeout_ns, cap));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "probe launch");
     return WLQ_OK;
