@@ -905,10 +905,10 @@ template <int FMT, bool PAIR, bool XRES>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_t,
             const __grid_constant__ CUtensorMap tm_l2, const GemmArgs a) {
-    grid_dependency_sync();
     // a partial kept in the ring needs one tile per cluster (the host plans
     // it so; refuse anything else)
     if (a.red_alias && !a.tail && a.tiles_nm > static_cast<int>(cluster_count_x())) {
+        grid_dependency_sync();
         if (threadIdx.x == 0 && blockIdx.x == 0) raise_error(ERRBIT_LAUNCH);
         return;
     }
@@ -990,6 +990,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     if (PAIR || a.S > 1) cluster_sync_all();
     const uint32_t tmem = *s.tmem_slot;
     const Sched sc = sched();
+    // the set-up above touches no global memory: it overlaps the previous
+    // kernel's tail when launched as a programmatic dependent
+    grid_dependency_sync();
 
     if (warp < NUM_DQ_WARPS) {
         dequant_role<FMT, PAIR, XRES>(a, tmem, s, sc, warp, lane);

@@ -94,7 +94,6 @@ __device__ __forceinline__ void ldmatrix_x2(uint32_t addr, uint32_t (&d)[2]) {
 
 template <int FMT, int NB>
 __global__ void __launch_bounds__(GV_THREADS, 1) gemv_kernel(const GemmArgs a) {
-    grid_dependency_sync();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* base = smem_raw + (((raw + 127u) & ~127u) - raw);
@@ -129,6 +128,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1) gemv_kernel(const GemmArgs a) {
     }
     if (threadIdx.x == 0) fence_barrier_init();
     __syncthreads();
+    grid_dependency_sync();  // nothing above touches global memory
 
     if (warp < GV_WARPS) {
         // ---- x rows m < M over this CTA's K range; inputs beyond K (a ragged

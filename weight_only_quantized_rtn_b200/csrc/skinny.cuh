@@ -325,7 +325,6 @@ __device__ void sk_compute(const GemmArgs& a, const SkSmem& s, const Sched& sc, 
 template <int FMT, int NB>
 __global__ void __launch_bounds__(SK_THREADS, 1)
 skinny_kernel(const __grid_constant__ CUtensorMap tm_x, const GemmArgs a) {
-    grid_dependency_sync();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -367,6 +366,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tm_x, const GemmArgs a) {
     __syncthreads();
     // every CTA of the cluster has initialised its barriers before any remote arrive
     if (a.S > 1) cluster_sync_all();
+    grid_dependency_sync();  // nothing above touches global memory
     const Sched sc = sched();
     if (warp < SK_WARPS) sk_compute<FMT, NB>(a, s, sc, warp, lane);
     else if (warp == SK_WARPS && lane == 0) sk_producer(a, s, sc);
