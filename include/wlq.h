@@ -53,6 +53,8 @@ typedef enum {
 } wlq_status;
 
 typedef enum { WLQ_OUT_BF16 = 0, WLQ_OUT_F32 = 1 } wlq_out_dtype;
+typedef enum { WLQ_IN_F32 = 0, WLQ_IN_BF16 = 1 } wlq_in_dtype;
+typedef enum { WLQ_SCALE_F32 = 0, WLQ_SCALE_F16 = 1, WLQ_SCALE_BF16 = 2 } wlq_scale_dtype;
 
 /*
  * RTN symmetric quantization ("Joy-face_change_optimized", files table and
@@ -107,6 +109,39 @@ wlq_status wlq_pack(const int8_t* codes, const float* scales, int64_t N, int64_t
  */
 wlq_status wlq_quantize_pack(const float* W, int64_t N, int64_t K, int bits, int group,
                              float* scales, void* packed, void* stream);
+
+/*
+ * RTN symmetric quantization for any width of 2..8 bits, from fp32 or bf16,
+ * with fp32, fp16 or bf16 stored scales ("Joy-face_change_optimized" model
+ * card: tools row, RTN per channel or per group; section 1, the KV-dtype
+ * setting: image K/V cached as int8 with one scale per token and head -- a
+ * [tokens*heads, head_dim] input with group = head_dim; section 2: a 5-bit
+ * MLP).  qmax = 2^(bits-1) - 1.  Per group (the row when group == 0):
+ *   a = max |W|;  s = the value of the scale format nearest to a / qmax;
+ *   q = clamp(round_half_even(W / s), -qmax, qmax) exactly, with that s.
+ * W      : [N, K] fp32 or bf16 (w_dtype), 16-byte aligned
+ * codes  : int8 [N, K], 4-byte aligned
+ * scales : [N, K / g] in scale_dtype, aligned to its type
+ * group  : 0 or a multiple of 4 dividing K; K % 8 == 0.
+ * bits = 8, group and fp32 scales as in wlq_quantize give the same result.
+ * A NaN or infinity in a group, or a 16-bit scale that overflows, sets
+ * WLQ_ERR_NONFINITE in the device error word; that group gets s = 0, codes 0.
+ */
+wlq_status wlq_quantize_ex(const void* W, int w_dtype, int64_t N, int64_t K, int bits, int group,
+                           int scale_dtype, int8_t* codes, void* scales, void* stream);
+
+/*
+ * fp8 block quantization ("Joy-face_change_optimized" model card, section
+ * 1.1: DiT blocks quantized to fp8 on the GPU for small cards).  Format e4m3
+ * (no infinity, largest finite 448).  Per group of g inputs of a row (the row
+ * when group == 0): s = fp32(max|W| / 448); code = e4m3 nearest to
+ * fp32(W / s), ties to an even significand, saturated to +-448; s = 0 gives
+ * codes 0.
+ * W: [N, K] fp32 or bf16, 16-byte aligned; codes: uint8 [N, K] e4m3 bit
+ * patterns; scales: fp32 [N, K / g].  Non-finite weights as wlq_quantize_ex.
+ */
+wlq_status wlq_quantize_fp8(const void* W, int w_dtype, int64_t N, int64_t K, int group,
+                            uint8_t* codes, float* scales, void* stream);
 
 /* Inverse of the code part of wlq_pack: packed -> codes int8 [N, K]. */
 wlq_status wlq_unpack(const void* packed, int64_t N, int64_t K, int bits, int group,

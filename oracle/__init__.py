@@ -46,7 +46,10 @@ def bind(path: str):
     lib.oracle_quantize.argtypes = [vp, i64, i64, i32, i32, vp, vp]
     lib.oracle_dequantize.argtypes = [vp, vp, i64, i64, i32, vp]
     lib.oracle_linear.argtypes = [vp, i64, i64, vp, vp, i64, i32, vp, vp, vp, i32, vp]
-    for f in (lib.oracle_quantize, lib.oracle_dequantize, lib.oracle_linear):
+    lib.oracle_quantize_ex.argtypes = [vp, i32, i64, i64, i32, i32, i32, vp, vp]
+    lib.oracle_quantize_fp8.argtypes = [vp, i32, i64, i64, i32, vp, vp]
+    for f in (lib.oracle_quantize, lib.oracle_dequantize, lib.oracle_linear, lib.oracle_quantize_ex,
+              lib.oracle_quantize_fp8):
         f.restype = ctypes.c_int
     return lib
 
@@ -123,3 +126,39 @@ def linear(x_bits: np.ndarray, codes: np.ndarray, scales: np.ndarray, group: int
     _check(_load().oracle_linear(_p(x_bits), M, K, _p(codes), _p(scales), N, group,
                                  _p(bias_bits), _p(L1_bits), _p(L2_bits), r, _p(y)))
     return y
+
+
+SCALE_F32, SCALE_F16, SCALE_BF16 = 0, 1, 2
+
+
+def quantize_ex(W: np.ndarray, bits: int, group: int, scale_dtype: int = SCALE_F32):
+    """RTN for 2..8 bits with a 32- or 16-bit stored scale.
+
+    W: fp32 array, or uint16 bf16 bit patterns.  Returns (codes int8 [N,K],
+    scale values fp32 [N,G]: the stored scales, exactly)."""
+    if W.dtype == np.uint16:
+        W = np.ascontiguousarray(W)
+        w_dtype = 1
+    else:
+        W = np.ascontiguousarray(W, dtype=np.float32)
+        w_dtype = 0
+    N, K = W.shape
+    codes = np.empty((N, K), np.int8)
+    scales = np.empty((N, groups_of(K, group)), np.float32)
+    _check(_load().oracle_quantize_ex(_p(W), w_dtype, N, K, bits, group, scale_dtype, _p(codes), _p(scales)))
+    return codes, scales
+
+
+def quantize_fp8(W: np.ndarray, group: int):
+    """fp8 e4m3 block quantization: returns (codes uint8 e4m3 bits [N,K], scales fp32 [N,G])."""
+    if W.dtype == np.uint16:
+        W = np.ascontiguousarray(W)
+        w_dtype = 1
+    else:
+        W = np.ascontiguousarray(W, dtype=np.float32)
+        w_dtype = 0
+    N, K = W.shape
+    codes = np.empty((N, K), np.uint8)
+    scales = np.empty((N, groups_of(K, group)), np.float32)
+    _check(_load().oracle_quantize_fp8(_p(W), w_dtype, N, K, group, _p(codes), _p(scales)))
+    return codes, scales

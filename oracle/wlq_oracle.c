@@ -115,6 +115,163 @@ int oracle_quantize(const float* W, int64_t N, int64_t K, int bits, int group,
     return ORACLE_OK;
 }
 
+/*
+ * Round a non-negative real held exactly in fp64 to the nearest value of a
+ * binary floating-point format with `p` significand bits (implicit bit
+ * included) and minimum normal exponent `emin` (subnormals below 2^emin with
+ * the fixed spacing 2^(emin - p + 1)), ties to even.  Returns +inf when the
+ * rounded value exceeds `maxv`.  The spacing is a power of two, so x / spacing
+ * is exact and the rounding is a single one.
+ */
+static double round_to_format(double x, int p, int emin, double maxv) {
+    if (x == 0.0) return 0.0;
+    int E;
+    frexp(x, &E); /* x in [2^(E-1), 2^E) */
+    int lead = E - 1;
+    if (lead < emin) lead = emin;
+    const double spacing = ldexp(1.0, lead - (p - 1));
+    const double r = round_half_even(x / spacing) * spacing;
+    return (r > maxv) ? INFINITY : r;
+}
+
+/* a weight of an fp32 or bf16 input array, exactly */
+static double in_value(const void* W, int w_dtype, int64_t i) {
+    if (w_dtype == 0) return (double)((const float*)W)[i];
+    return bf16_value(((const uint16_t*)W)[i]);
+}
+
+/*
+ * RTN symmetric quantization for any width of 2..8 bits, an fp32 or bf16
+ * input, and a 32- or 16-bit stored scale ([JFC] tools row and files table:
+ * RTN with per-channel or grouped scales; [JFC] section 1, the KV-dtype
+ * setting: cached image K/V held as int8 with one scale per token and head,
+ * i.e. one group per (token, head) row of head_dim inputs; [JFC] section 2:
+ * a 5-bit MLP proposed as a further width).
+ * w_dtype     : 0 fp32, 1 bf16 (bit patterns)
+ * bits        : 2..8, qmax = 2^(bits-1) - 1
+ * group       : 0 = whole row, else the group size along K
+ * scale_dtype : 0 fp32, 1 fp16, 2 bf16 -- the stored scale is the value of
+ *               that format nearest to a / qmax (ties to even); the codes are
+ *               RTN of W / s with that stored s, clamped to +-qmax (a 16-bit
+ *               scale may round below a / qmax)
+ * codes       : int8 [N, K];  scale_values : fp32 [N, K / g], the stored
+ *               scales' values (16-bit values are exact in fp32)
+ * A stored scale that overflows its format is reported as non-finite.
+ */
+int oracle_quantize_ex(const void* W, int w_dtype, int64_t N, int64_t K, int bits, int group,
+                       int scale_dtype, int8_t* codes, float* scale_values) {
+    if (N < 0 || K <= 0 || bits < 2 || bits > 8 || group < 0 || w_dtype < 0 || w_dtype > 1 ||
+        scale_dtype < 0 || scale_dtype > 2)
+        return ORACLE_ERR_ARG;
+    const int64_t g = (group == 0) ? K : group;
+    if (K % g != 0) return ORACLE_ERR_ARG;
+    const int64_t G = K / g;
+    const double qmax = ldexp(1.0, bits - 1) - 1.0;
+    for (int64_t i = 0; i < N * K; ++i)
+        if (!isfinite(in_value(W, w_dtype, i))) return ORACLE_ERR_NONFINITE;
+    int overflow = 0;
+#pragma omp parallel for schedule(static) reduction(| : overflow)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t gi = 0; gi < G; ++gi) {
+            double a = 0.0;
+            for (int64_t k = 0; k < g; ++k) {
+                double v = fabs(in_value(W, w_dtype, n * K + gi * g + k));
+                if (v > a) a = v;
+            }
+            /* the stored scale: nearest value of the format to a / qmax (the
+             * fp64 quotient is within 2^-53 relative of a / qmax, and a, qmax
+             * are short enough that no tie of a 24-bit or shorter format lies
+             * that close unless the quotient is exact) */
+            const double qd = a / qmax;
+            double s;
+            if (scale_dtype == 0) s = (double)(float)qd;
+            else if (scale_dtype == 1) s = round_to_format(qd, 11, -14, 65504.0);
+            else s = round_to_format(qd, 8, -126, ldexp(255.0, 127 - 7));
+            if (isinf(s)) { overflow = 1; s = 0.0; }
+            scale_values[n * G + gi] = (float)s;
+            for (int64_t k = 0; k < g; ++k) {
+                double c = 0.0;
+                if (s != 0.0) {
+                    /* s is exactly an fp32 value; as in oracle_quantize the
+                     * fp64 quotient rounds like the exact real */
+                    c = round_half_even(in_value(W, w_dtype, n * K + gi * g + k) / s);
+                    if (c > qmax) c = qmax;
+                    if (c < -qmax) c = -qmax;
+                }
+                codes[n * K + gi * g + k] = (int8_t)c;
+            }
+        }
+    }
+    return overflow ? ORACLE_ERR_NONFINITE : ORACLE_OK;
+}
+
+/*
+ * fp8 (e4m3, the "fn" variant: no infinity, largest finite 448) block
+ * quantization along K ([JFC] section 1.1: DiT blocks streamed to 8 GB cards
+ * in fp8, quantized on the GPU, the card noting that a CPU rounding differed
+ * from CUDA's on a small fraction of elements -- here both sides round once,
+ * to nearest even, from the same fp32 quotient).  The scale granularity is
+ * not given; the reading is one fp32 scale per group of g inputs of a row
+ * (g = K: per row): per group, s = fp32(a / 448); each
+ * weight becomes the e4m3 value nearest to t = fp32(W / s) (ties to an even
+ * significand), saturated to +-448; an all-zero group has s = 0 and codes 0.
+ * codes : uint8 [N, K] e4m3 bit patterns (sign, 4 exponent bits with bias 7,
+ *         3 significand bits; exponent field 0 = subnormals of spacing 2^-9)
+ * scales: fp32 [N, K / g]
+ */
+static uint8_t e4m3_encode(double t) {
+    const int neg = signbit(t) ? 1 : 0;
+    double x = fabs(t);
+    /* nearest e4m3 magnitude, ties to even: spacing 2^-9 below 2^-6, else
+     * 2^(exponent - 3) */
+    double r = round_to_format(x, 4, -6, 448.0);
+    if (isinf(r)) r = 448.0; /* saturate */
+    uint8_t bits;
+    if (r < ldexp(1.0, -6)) {
+        bits = (uint8_t)(r / ldexp(1.0, -9)); /* subnormal (or zero): m / 8 * 2^-6 */
+    } else {
+        int E;
+        const double m = frexp(r, &E); /* r = m 2^E, m in [0.5, 1) */
+        const int e = (E - 1) + 7;     /* biased exponent */
+        const int man = (int)((m * 2.0 - 1.0) * 8.0);
+        bits = (uint8_t)((e << 3) | man);
+    }
+    return (uint8_t)(bits | (neg << 7));
+}
+
+int oracle_quantize_fp8(const void* W, int w_dtype, int64_t N, int64_t K, int group, uint8_t* codes,
+                        float* scales) {
+    if (N < 0 || K <= 0 || group < 0 || w_dtype < 0 || w_dtype > 1) return ORACLE_ERR_ARG;
+    const int64_t g = (group == 0) ? K : group;
+    if (K % g != 0) return ORACLE_ERR_ARG;
+    const int64_t G = K / g;
+    for (int64_t i = 0; i < N * K; ++i)
+        if (!isfinite(in_value(W, w_dtype, i))) return ORACLE_ERR_NONFINITE;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t gi = 0; gi < G; ++gi) {
+            double a = 0.0;
+            for (int64_t k = 0; k < g; ++k) {
+                double v = fabs(in_value(W, w_dtype, n * K + gi * g + k));
+                if (v > a) a = v;
+            }
+            const float s = (float)(a / 448.0);
+            scales[n * G + gi] = s;
+            for (int64_t k = 0; k < g; ++k) {
+                uint8_t c = 0;
+                if (s != 0.0f) {
+                    /* t = the fp32 nearest to W / s: the fp64 quotient of two
+                     * fp32 values rounds to fp32 like the exact one */
+                    const float t = (float)(in_value(W, w_dtype, n * K + gi * g + k) / (double)s);
+                    c = e4m3_encode((double)t);
+                }
+                codes[n * K + gi * g + k] = c;
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
 /* Dequantized weights, exact in fp64: deq[n,k] = q[n,k] * s[n, k / g]. */
 int oracle_dequantize(const int8_t* codes, const float* scales, int64_t N, int64_t K,
                       int group, double* deq) {

@@ -121,6 +121,20 @@ def test_argument_errors_before_any_device_access(lib):
     assert lib.wlq_quantize_pack(None, 4, 64, 8, 0, None, None, None) == 1      # null
     assert lib.wlq_quantize_pack(None, 0, 64, 8, 0, None, None, None) == 0      # N == 0: no-op
     assert lib.wlq_quantize_pack(vp(16), 4, 64, 8, 0, vp(16), vp(40), None) == 3  # packed misaligned
+    i64, i32 = ctypes.c_int64, ctypes.c_int
+    lib.wlq_quantize_ex.argtypes = [vp, i32, i64, i64, i32, i32, i32, vp, vp, vp]
+    assert lib.wlq_quantize_ex(None, 0, 4, 64, 9, 0, 0, None, None, None) == 4    # bits 2..8
+    assert lib.wlq_quantize_ex(None, 0, 4, 64, 1, 0, 0, None, None, None) == 4
+    assert lib.wlq_quantize_ex(None, 2, 4, 64, 8, 0, 0, None, None, None) == 4    # input dtype
+    assert lib.wlq_quantize_ex(None, 0, 4, 64, 8, 0, 3, None, None, None) == 4    # scale dtype
+    assert lib.wlq_quantize_ex(None, 0, 4, 64, 8, 6, 0, None, None, None) == 2    # group % 4
+    assert lib.wlq_quantize_ex(None, 1, 4, 64, 5, 16, 1, None, None, None) == 1   # null
+    assert lib.wlq_quantize_ex(vp(16), 1, 4, 64, 5, 16, 1, vp(16), vp(17), None) == 3  # fp16 scales 2-byte aligned
+    lib.wlq_quantize_fp8.argtypes = [vp, i32, i64, i64, i32, vp, vp, vp]
+    assert lib.wlq_quantize_fp8(None, 0, 4, 64, 10, None, None, None) == 2        # group % 4
+    assert lib.wlq_quantize_fp8(None, 0, 4, 60, 0, None, None, None) == 2         # K % 8
+    assert lib.wlq_quantize_fp8(None, 0, 4, 64, 32, None, None, None) == 1        # null
+    assert lib.wlq_quantize_fp8(None, 0, 0, 64, 32, None, None, None) == 0        # N == 0
     # M == 0 is a no-op
     assert lib.wlq_linear(None, 0, None, 64, 64, 8, 0, None, None, None, 0, None, 0, None, 0, None) == 0
     assert lib.wlq_linear(None, 4, None, 64, 64, 4, 0, None, None, None, 0, None, 0, None, 0, None) == 4

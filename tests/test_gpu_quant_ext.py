@@ -1,0 +1,129 @@
+"""GPU RTN at other widths / inputs / scale formats and fp8 e4m3 block
+quantization against the oracle: codes and stored scales bit-exact; the
+int8 KV-cache shape (one group per token and head) timed."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.gpu_helpers import dev_f32
+
+pytestmark = pytest.mark.gpu
+
+
+def wlq():
+    import weight_only_quantized_rtn_b200 as m
+    return m
+
+
+def _bf16_bits(x: np.ndarray) -> np.ndarray:
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    return (((u + 0x7FFF + ((u >> 16) & 1)) >> 16) & 0xFFFF).astype(np.uint16)
+
+
+def _dev(W: np.ndarray, bf16: bool) -> torch.Tensor:
+    if bf16:
+        return torch.from_numpy(_bf16_bits(W).view(np.int16)).cuda().view(torch.bfloat16)
+    return dev_f32(W)
+
+
+def _host_in(W: np.ndarray, bf16: bool) -> np.ndarray:
+    return _bf16_bits(W) if bf16 else W
+
+
+def _edge_weights(seed, N, K):
+    g = np.random.default_rng(seed)
+    W = (g.standard_normal((N, K)) * np.exp(g.uniform(-4, 4, (N, 1)))).astype(np.float32)
+    W[0] = 0.0                                            # all-zero row
+    W[1] = g.integers(-9, 10, K).astype(np.float32) * 0.5  # many halves
+    W[2] *= 1e-36                                         # tiny
+    W[3, 7] = -40.0                                       # a lone outlier
+    W[4] = 3.0                                            # constant
+    return W
+
+
+@pytest.mark.parametrize("bits", [2, 3, 5, 8])
+@pytest.mark.parametrize("group", [0, 16, 128])
+@pytest.mark.parametrize("scale_dtype", [0, 1, 2])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_quantize_ex_bit_exact(bits, group, scale_dtype, bf16):
+    m = wlq()
+    W = _edge_weights(bits * 31 + group + scale_dtype, 37, 384)
+    if scale_dtype == 1:
+        W[2] = 0.001  # keep fp16 scales inside their range (the tiny row would be 0 there anyway)
+    co, so = oracle.quantize_ex(_host_in(W, bf16), bits, group, scale_dtype)
+    cg, sg = m.quantize_ex(_dev(W, bf16), bits, group, scale_dtype)
+    torch.cuda.synchronize()
+    m.check_status()
+    np.testing.assert_array_equal(cg.cpu().numpy(), co)
+    np.testing.assert_array_equal(sg.float().cpu().numpy(), so)
+
+
+def test_quantize_ex_eight_bit_fp32_equals_quantize():
+    m = wlq()
+    W = _edge_weights(3, 64, 512)
+    for group, bits in ((0, 8), (64, 4), (16, 4)):
+        c0, s0 = m.quantize(dev_f32(W), bits, group)
+        c1, s1 = m.quantize_ex(dev_f32(W), bits, group, 0)
+        torch.cuda.synchronize()
+        assert torch.equal(c0, c1) and torch.equal(s0, s1)
+
+
+def test_quantize_ex_nonfinite_and_fp16_overflow_flag():
+    m = wlq()
+    m.check_status()
+    W = (np.random.default_rng(1).standard_normal((8, 64)) * 0.1).astype(np.float32)
+    W[2, 3] = np.nan
+    c, s = m.quantize_ex(dev_f32(W), 8, 32, 0)
+    assert m.get_status() == m.ERR_NONFINITE
+    assert float(s[2, 0]) == 0.0 and not c[2, :32].any()
+    W[2, 3] = 0.0
+    W[5, 40] = 1e7  # 1e7 / 127 overflows fp16
+    c, s = m.quantize_ex(dev_f32(W), 8, 32, 1)
+    assert m.get_status() == m.ERR_NONFINITE
+    assert float(s[5, 1]) == 0.0 and not c[5, 32:].any()
+    c, s = m.quantize_ex(dev_f32(W), 8, 32, 2)  # bf16 holds it
+    assert m.get_status() == m.OK
+
+
+@pytest.mark.parametrize("group", [0, 32, 128])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_quantize_fp8_bit_exact(group, bf16):
+    m = wlq()
+    W = _edge_weights(77 + group, 41, 512)
+    co, so = oracle.quantize_fp8(_host_in(W, bf16), group)
+    cg, sg = m.quantize_fp8(_dev(W, bf16), group)
+    torch.cuda.synchronize()
+    m.check_status()
+    np.testing.assert_array_equal(sg.cpu().numpy(), so)
+    np.testing.assert_array_equal(cg.cpu().numpy(), co)
+
+
+def test_kv_cache_int8_per_token_head_timed():
+    """K/V of 4096 tokens x 32 heads x head_dim 128 in bf16, one int8 scale
+    group per (token, head), fp16 scales: bit-exact on a slice, and timed
+    (HBM-bound: 2 B read + 1 B + 2/128 B written per element)."""
+    m = wlq()
+    T, H, D = 4096, 32, 128
+    g = np.random.default_rng(12)
+    kv = (g.standard_normal((T * H, D)) * 0.5).astype(np.float32)
+    x = _dev(kv, True)
+    codes, scales = m.quantize_ex(x, 8, D, 1)
+    torch.cuda.synchronize()
+    co, so = oracle.quantize_ex(_bf16_bits(kv[:2048]), 8, D, 1)
+    np.testing.assert_array_equal(codes[:2048].cpu().numpy(), co)
+    np.testing.assert_array_equal(scales[:2048].float().cpu().numpy(), so)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    ts = []
+    for _ in range(10):
+        flush.zero_()
+        flush.view(torch.float32).sum()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        m.quantize_ex(x, 8, D, 1)
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    us = sorted(ts)[len(ts) // 2]
+    nbytes = T * H * D * (2 + 1) + T * H * 2
+    print("\nKV int8 per (token, head): %d x %d x %d bf16 -> %.1f us, %.0f GB/s" % (T, H, D, us, nbytes / us / 1e3))

@@ -11,6 +11,7 @@ import tempfile
 import pytest
 
 import oracle
+import tests.test_oracle_ext_pins as ext
 import tests.test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "wlq_oracle.c")
@@ -25,6 +26,11 @@ MUTATIONS = {
     "group_index": ("(double)scales[n * G + k / g];\n                acc",
                     "(double)scales[n * G + k % G];\n                acc"),
     "signed_max": ("double v = fabs((double)w[k]);", "double v = (double)w[k];"),
+    "format_rounds_down": ("const double r = round_half_even(x / spacing) * spacing;",
+                           "const double r = floor(x / spacing) * spacing;"),
+    "sixteen_bit_scale_kept_fp32": ("if (scale_dtype == 0) s = (double)(float)qd;",
+                                    "if (scale_dtype >= 0) s = (double)(float)qd;"),
+    "fp8_max_off": ("const float s = (float)(a / 448.0);", "const float s = (float)(a / 480.0);"),
 }
 
 PIN_TESTS = [
@@ -37,6 +43,10 @@ PIN_TESTS = [
     lambda: pins.test_linear_matches_numpy_matmul(4, 16),
     lambda: pins.test_linear_matches_numpy_matmul(8, 0),
     lambda: pins.test_linear_low_rank_only_and_plain_only(),
+    lambda: ext.test_codes_are_the_brute_force_nearest_with_the_stored_scale(5, oracle.SCALE_F16),
+    lambda: ext.test_codes_are_the_brute_force_nearest_with_the_stored_scale(3, oracle.SCALE_BF16),
+    lambda: ext.test_fp8_codes_are_the_nearest_e4m3_ties_to_even_saturated(),
+    lambda: ext.test_fp8_codes_match_torch_e4m3fn_conversion(),
 ]
 
 

@@ -39,6 +39,8 @@ lib.wlq_packed_bytes.restype = _sz
 lib.wlq_pack.argtypes = [_vp, _vp, _i64, _i64, _i32, _i32, _vp, _vp]
 lib.wlq_unpack.argtypes = [_vp, _i64, _i64, _i32, _i32, _vp, _vp]
 lib.wlq_quantize_pack.argtypes = [_vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp]
+lib.wlq_quantize_ex.argtypes = [_vp, _i32, _i64, _i64, _i32, _i32, _i32, _vp, _vp, _vp]
+lib.wlq_quantize_fp8.argtypes = [_vp, _i32, _i64, _i64, _i32, _vp, _vp, _vp]
 lib.wlq_linear_workspace.argtypes = [_i64, _i64, _i64, _i32, _i32, _i32]
 lib.wlq_linear_workspace.restype = _sz
 lib.wlq_linear.argtypes = [_vp, _i64, _vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _sz, _vp]
@@ -49,7 +51,7 @@ lib.wlq_set_grid_limit.argtypes = [_i32]
 lib.wlq_set_grid_limit.restype = None
 lib.wlq_last_error.restype = ctypes.c_char_p
 lib.wlq_version.restype = ctypes.c_char_p
-for _f in ("wlq_quantize", "wlq_quantize_pack", "wlq_pack", "wlq_unpack", "wlq_linear", "wlq_linear_noalloc", "wlq_get_status",
+for _f in ("wlq_quantize", "wlq_quantize_pack", "wlq_quantize_ex", "wlq_quantize_fp8", "wlq_pack", "wlq_unpack", "wlq_linear", "wlq_linear_noalloc", "wlq_get_status",
            "wlq_probe_wait_timeout"):
     getattr(lib, _f).restype = ctypes.c_int
 
@@ -85,6 +87,39 @@ def quantize(W: torch.Tensor, bits: int, group: int, stream=None):
     codes = torch.empty((N, K), dtype=torch.int8, device=W.device)
     scales = torch.empty((N, groups(K, group)), dtype=torch.float32, device=W.device)
     _check(lib.wlq_quantize(_ptr(W), N, K, bits, group, _ptr(codes), _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+SCALE_F32, SCALE_F16, SCALE_BF16 = 0, 1, 2
+_SCALE_TORCH = {SCALE_F32: torch.float32, SCALE_F16: torch.float16, SCALE_BF16: torch.bfloat16}
+
+
+def _in_dtype(W: torch.Tensor) -> int:
+    if W.dtype == torch.float32:
+        return 0
+    if W.dtype == torch.bfloat16:
+        return 1
+    raise WlqError(ERR_UNSUPPORTED, "input must be fp32 or bf16")
+
+
+def quantize_ex(W: torch.Tensor, bits: int, group: int, scale_dtype: int = SCALE_F32, stream=None):
+    """RTN for 2..8 bits from fp32 or bf16 W [N, K] -> (codes int8 [N,K], scales [N,G] in scale_dtype)."""
+    assert W.is_cuda and W.is_contiguous()
+    N, K = W.shape
+    codes = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    scales = torch.empty((N, groups(K, group)), dtype=_SCALE_TORCH[scale_dtype], device=W.device)
+    _check(lib.wlq_quantize_ex(_ptr(W), _in_dtype(W), N, K, bits, group, scale_dtype, _ptr(codes), _ptr(scales),
+                               _stream(stream)))
+    return codes, scales
+
+
+def quantize_fp8(W: torch.Tensor, group: int, stream=None):
+    """fp8 e4m3 block quantization of fp32 or bf16 W [N, K] -> (codes uint8 [N,K], scales fp32 [N,G])."""
+    assert W.is_cuda and W.is_contiguous()
+    N, K = W.shape
+    codes = torch.empty((N, K), dtype=torch.uint8, device=W.device)
+    scales = torch.empty((N, groups(K, group)), dtype=torch.float32, device=W.device)
+    _check(lib.wlq_quantize_fp8(_ptr(W), _in_dtype(W), N, K, group, _ptr(codes), _ptr(scales), _stream(stream)))
     return codes, scales
 
 

@@ -1,0 +1,148 @@
+// quantize_ext.cuh -- RTN for other widths, inputs and scale formats, and fp8
+// block quantization ("Joy-face_change_optimized" model card: tools row, RTN
+// per channel or per group; section 1, the KV-dtype setting: image K/V cached
+// as int8 with one scale per token and head; section 2, a 5-bit MLP; section
+// 1.1, DiT blocks quantized to fp8 on the GPU).
+//
+// quantize_ex_kernel: for each group (g inputs of a row), a = max|W| exactly,
+// the stored scale s = the value of the scale format nearest to a / qmax
+// (fp32: IEEE division; fp16 / bf16: the fp64 quotient rounded once to the
+// 16-bit format, which equals the correctly rounded one), and
+// q = clamp(RTN(W / s), +-qmax) computed exactly with that stored s (a 16-bit
+// s may lie below a / qmax, so the clamp can act).  A group holding a NaN or
+// an infinity, or whose 16-bit scale overflows, gets s = 0 and codes 0 and
+// sets the non-finite error bit.
+//
+// quantize_fp8_kernel: s = fp32(a / 448); each weight becomes
+// e4m3(RN(fp32(W / s))) saturated to +-448 (one rounding from the fp32
+// quotient, cvt.rn.satfinite); an all-zero group has s = 0 and codes 0.
+//
+// One warp per group (grid-stride); a lane takes four adjacent inputs at a
+// time (groups are multiples of 4 inputs).  Pass 1 reduces the absmax, pass 2
+// re-reads the group (from L1 / L2) and writes the codes.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include "ptx.cuh"
+#include "quantize.cuh"
+
+namespace wlq {
+
+enum ScaleFmt : int { SCALE_F32 = 0, SCALE_F16 = 1, SCALE_BF16 = 2 };
+
+template <bool IN_BF16>
+__device__ __forceinline__ float4 load4(const void* W, int64_t i4) {
+    if constexpr (IN_BF16) {
+        const uint2 u = reinterpret_cast<const uint2*>(W)[i4];
+        return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                           __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+    } else {
+        return reinterpret_cast<const float4*>(W)[i4];
+    }
+}
+
+__device__ __forceinline__ uint32_t absbits_max4(float4 v) {
+    return max(max(__float_as_uint(v.x) & 0x7FFFFFFFu, __float_as_uint(v.y) & 0x7FFFFFFFu),
+               max(__float_as_uint(v.z) & 0x7FFFFFFFu, __float_as_uint(v.w) & 0x7FFFFFFFu));
+}
+
+template <bool IN_BF16, int SF>
+__global__ void __launch_bounds__(256) quantize_ex_kernel(const void* __restrict__ W, int64_t groups, int g4,
+                                                          int qmax, int8_t* __restrict__ codes,
+                                                          void* __restrict__ scales) {
+    grid_dependency_sync();
+    const int lane = threadIdx.x & 31;
+    const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    bool bad = false;
+    for (int64_t gi = w0; gi < groups; gi += nw) {
+        const int64_t base = gi * g4;  // first float4 of the group
+        uint32_t m = 0;
+        for (int j = lane; j < g4; j += 32) m = max(m, absbits_max4(load4<IN_BF16>(W, base + j)));
+        for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+        bool gbad = m >= 0x7F800000u;  // NaN or infinity in the group
+        const float a = gbad ? 0.0f : __uint_as_float(m);
+        float s;
+        if constexpr (SF == SCALE_F32) {
+            s = __fdiv_rn(a, static_cast<float>(qmax));
+        } else if constexpr (SF == SCALE_F16) {
+            const __half h = __double2half(static_cast<double>(a) / static_cast<double>(qmax));
+            s = __half2float(h);
+        } else {
+            const __nv_bfloat16 h = __double2bfloat16(static_cast<double>(a) / static_cast<double>(qmax));
+            s = __bfloat162float(h);
+        }
+        if (isinf(s)) {  // the 16-bit scale overflowed
+            gbad = true;
+            s = 0.0f;
+        }
+        bad |= gbad;
+        if (lane == 0) {
+            if constexpr (SF == SCALE_F32) static_cast<float*>(scales)[gi] = s;
+            else if constexpr (SF == SCALE_F16) static_cast<__half*>(scales)[gi] = __float2half_rn(s);
+            else static_cast<__nv_bfloat16*>(scales)[gi] = __float2bfloat16_rn(s);
+        }
+        GroupScale gs;
+        gs.s = s;
+        gs.normal = s >= 1.17549435e-38f;
+        gs.inv = gs.normal ? __frcp_rn(s) : 0.0f;
+        gs.inv64 = (!gs.normal && s > 0.0f) ? 1.0 / static_cast<double>(s) : 0.0;
+        uint32_t* out = reinterpret_cast<uint32_t*>(codes);
+        for (int j = lane; j < g4; j += 32) {
+            const float4 v = load4<IN_BF16>(W, base + j);
+            uint32_t c = 0;
+            if (gs.normal) {
+                const float w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    c |= rtn_byte_f32(w[e], gs.s, gs.inv, static_cast<float>(qmax)) << (8 * e);
+            } else {
+                bool unused = false;
+                c = pack_codes4(v, gs, qmax, unused);  // s == 0 (and non-finite weights) give code 0
+            }
+            out[base + j] = c;
+        }
+    }
+    if (bad) raise_error(ERRBIT_NONFINITE);
+}
+
+__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+template <bool IN_BF16>
+__global__ void __launch_bounds__(256) quantize_fp8_kernel(const void* __restrict__ W, int64_t groups, int g4,
+                                                           uint8_t* __restrict__ codes, float* __restrict__ scales) {
+    grid_dependency_sync();
+    const int lane = threadIdx.x & 31;
+    const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    bool bad = false;
+    for (int64_t gi = w0; gi < groups; gi += nw) {
+        const int64_t base = gi * g4;
+        uint32_t m = 0;
+        for (int j = lane; j < g4; j += 32) m = max(m, absbits_max4(load4<IN_BF16>(W, base + j)));
+        for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+        const bool gbad = m >= 0x7F800000u;
+        bad |= gbad;
+        const float s = gbad ? 0.0f : __fdiv_rn(__uint_as_float(m), 448.0f);
+        if (lane == 0) scales[gi] = s;
+        uint32_t* out = reinterpret_cast<uint32_t*>(codes);
+        for (int j = lane; j < g4; j += 32) {
+            uint32_t c = 0;
+            if (s != 0.0f) {
+                const float4 v = load4<IN_BF16>(W, base + j);
+                const uint32_t lo = cvt_e4m3x2(__fdiv_rn(v.x, s), __fdiv_rn(v.y, s));
+                const uint32_t hi = cvt_e4m3x2(__fdiv_rn(v.z, s), __fdiv_rn(v.w, s));
+                c = lo | (hi << 16);
+            }
+            out[base + j] = c;
+        }
+    }
+    if (bad) raise_error(ERRBIT_NONFINITE);
+}
+
+}  // namespace wlq

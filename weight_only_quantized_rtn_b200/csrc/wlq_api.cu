@@ -17,6 +17,7 @@
 #include "skinny.cuh"
 #include "gemv.cuh"
 #include "quantize_pack.cuh"
+#include "quantize_ext.cuh"
 #include "pack.cuh"
 #include "prep.cuh"
 #include "ptx.cuh"
@@ -763,6 +764,65 @@ wlq_status wlq_quantize_pack(const float* W, int64_t N, int64_t K, int bits, int
                                                                                   qmax, scales, rowf, base);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "quantize_pack launch");
+    return WLQ_OK;
+}
+
+wlq_status wlq_quantize_ex(const void* W, int w_dtype, int64_t N, int64_t K, int bits, int group, int scale_dtype,
+                           int8_t* codes, void* scales, void* stream) {
+    if (bits < 2 || bits > 8) return fail(WLQ_ERR_UNSUPPORTED, "bits must be 2..8");
+    if (w_dtype != WLQ_IN_F32 && w_dtype != WLQ_IN_BF16) return fail(WLQ_ERR_UNSUPPORTED, "input must be fp32 or bf16");
+    if (scale_dtype < WLQ_SCALE_F32 || scale_dtype > WLQ_SCALE_BF16)
+        return fail(WLQ_ERR_UNSUPPORTED, "scales must be fp32, fp16 or bf16");
+    if (group < 0 || (group && group % 4)) return fail(WLQ_ERR_SHAPE, "group must be 0 or a positive multiple of 4");
+    wlq_status st = check_shape(N, K, bits, group);
+    if (st != WLQ_OK) return st;
+    if (N == 0) return WLQ_OK;
+    if (!W || !codes || !scales) return fail(WLQ_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(W) || (reinterpret_cast<uintptr_t>(codes) & 3u) ||
+        (reinterpret_cast<uintptr_t>(scales) & (scale_dtype == WLQ_SCALE_F32 ? 3u : 1u)))
+        return fail(WLQ_ERR_ALIGN, "W must be 16-byte aligned, codes 4-byte, scales aligned to their type");
+    int dev;
+    DeviceInfo* d;
+    if ((st = current_device(&dev, &d)) != WLQ_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t g = group ? group : K;
+    const int64_t groups = N * (K / g);
+    const int g4 = static_cast<int>(g / 4);
+    const int qmax = (1 << (bits - 1)) - 1;
+    const int grid = grid_for(groups * 32, 256, d->sms);
+#define WLQ_QX(B, F) launch_k(wlq::quantize_ex_kernel<B, F>, grid, 256, 0, s, W, groups, g4, qmax, codes, scales)
+    const bool bf = (w_dtype == WLQ_IN_BF16);
+    if (scale_dtype == WLQ_SCALE_F32) { if (bf) WLQ_QX(true, wlq::SCALE_F32); else WLQ_QX(false, wlq::SCALE_F32); }
+    else if (scale_dtype == WLQ_SCALE_F16) { if (bf) WLQ_QX(true, wlq::SCALE_F16); else WLQ_QX(false, wlq::SCALE_F16); }
+    else { if (bf) WLQ_QX(true, wlq::SCALE_BF16); else WLQ_QX(false, wlq::SCALE_BF16); }
+#undef WLQ_QX
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "quantize_ex launch");
+    return WLQ_OK;
+}
+
+wlq_status wlq_quantize_fp8(const void* W, int w_dtype, int64_t N, int64_t K, int group, uint8_t* codes,
+                            float* scales, void* stream) {
+    if (w_dtype != WLQ_IN_F32 && w_dtype != WLQ_IN_BF16) return fail(WLQ_ERR_UNSUPPORTED, "input must be fp32 or bf16");
+    if (group < 0 || (group && group % 4)) return fail(WLQ_ERR_SHAPE, "group must be 0 or a positive multiple of 4");
+    wlq_status st = check_shape(N, K, 8, group);
+    if (st != WLQ_OK) return st;
+    if (N == 0) return WLQ_OK;
+    if (!W || !codes || !scales) return fail(WLQ_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(W) || (reinterpret_cast<uintptr_t>(codes) & 3u) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+        return fail(WLQ_ERR_ALIGN, "W must be 16-byte aligned, codes and scales 4-byte aligned");
+    int dev;
+    DeviceInfo* d;
+    if ((st = current_device(&dev, &d)) != WLQ_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t g = group ? group : K;
+    const int64_t groups = N * (K / g);
+    const int g4 = static_cast<int>(g / 4);
+    const int grid = grid_for(groups * 32, 256, d->sms);
+    if (w_dtype == WLQ_IN_BF16) launch_k(wlq::quantize_fp8_kernel<true>, grid, 256, 0, s, W, groups, g4, codes, scales);
+    else launch_k(wlq::quantize_fp8_kernel<false>, grid, 256, 0, s, W, groups, g4, codes, scales);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "quantize_fp8 launch");
     return WLQ_OK;
 }
 
