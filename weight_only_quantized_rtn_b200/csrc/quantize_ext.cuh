@@ -19,7 +19,8 @@
 //
 // One warp per group (grid-stride); a lane takes four adjacent inputs at a
 // time (groups are multiples of 4 inputs).  Pass 1 reduces the absmax, pass 2
-// re-reads the group (from L1 / L2) and writes the codes.
+// re-reads the group (from L1 / L2) and writes the codes.  Groups of at most
+// 128 inputs whose g / 4 divides 32 take quantize_ex_short_kernel instead.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -102,6 +103,79 @@ __global__ void __launch_bounds__(256) quantize_ex_kernel(const void* __restrict
                 c = pack_codes4(v, gs, qmax, unused);  // s == 0 (and non-finite weights) give code 0
             }
             out[base + j] = c;
+        }
+    }
+    if (bad) raise_error(ERRBIT_NONFINITE);
+}
+
+// Short groups (g / 4 divides 32: g <= 128), one pass: a warp takes 32 / L
+// groups at once, L = g / 4 lanes each (one float4 per lane), and U such
+// warp-rounds are loaded before any is quantized.  Same arithmetic as
+// quantize_ex_kernel, from registers.
+template <bool IN_BF16, int SF, int L>
+__global__ void __launch_bounds__(256) quantize_ex_short_kernel(const void* __restrict__ W, int64_t groups,
+                                                                int qmax, int8_t* __restrict__ codes,
+                                                                void* __restrict__ scales) {
+    grid_dependency_sync();
+    constexpr int U = 4;
+    constexpr int GPW = 32 / L;  // groups per warp-round
+    const int lane = threadIdx.x & 31;
+    const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    const int64_t total4 = groups * L;
+    uint32_t* out = reinterpret_cast<uint32_t*>(codes);
+    bool bad = false;
+    for (int64_t r0 = w0 * U; r0 * GPW < groups; r0 += nw * U) {
+        float4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i4 = (r0 + u) * 32 + lane;  // float4 index: group (r0+u)*GPW + lane / L
+            v[u] = i4 < total4 ? load4<IN_BF16>(W, i4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i4 = (r0 + u) * 32 + lane;
+            uint32_t m = absbits_max4(v[u]);
+#pragma unroll
+            for (int off = L >> 1; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+            if (i4 >= total4) continue;
+            bool gbad = m >= 0x7F800000u;
+            const float a = gbad ? 0.0f : __uint_as_float(m);
+            float s;
+            if constexpr (SF == SCALE_F32) {
+                s = __fdiv_rn(a, static_cast<float>(qmax));
+            } else if constexpr (SF == SCALE_F16) {
+                s = __half2float(__double2half(static_cast<double>(a) / static_cast<double>(qmax)));
+            } else {
+                s = __bfloat162float(__double2bfloat16(static_cast<double>(a) / static_cast<double>(qmax)));
+            }
+            if (isinf(s)) {
+                gbad = true;
+                s = 0.0f;
+            }
+            bad |= gbad;
+            if ((lane & (L - 1)) == 0) {
+                const int64_t gi = i4 / L;
+                if constexpr (SF == SCALE_F32) static_cast<float*>(scales)[gi] = s;
+                else if constexpr (SF == SCALE_F16) static_cast<__half*>(scales)[gi] = __float2half_rn(s);
+                else static_cast<__nv_bfloat16*>(scales)[gi] = __float2bfloat16_rn(s);
+            }
+            uint32_t c = 0;
+            if (s >= 1.17549435e-38f) {
+                const float inv = __frcp_rn(s);
+                const float w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) c |= rtn_byte_f32(w[e], s, inv, static_cast<float>(qmax)) << (8 * e);
+            } else if (s > 0.0f) {
+                GroupScale gs;
+                gs.s = s;
+                gs.normal = false;
+                gs.inv = 0.0f;
+                gs.inv64 = 1.0 / static_cast<double>(s);
+                bool unused = false;
+                c = pack_codes4(v[u], gs, qmax, unused);
+            }
+            out[i4] = c;
         }
     }
     if (bad) raise_error(ERRBIT_NONFINITE);

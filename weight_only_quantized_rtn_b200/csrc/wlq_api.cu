@@ -789,13 +789,34 @@ wlq_status wlq_quantize_ex(const void* W, int w_dtype, int64_t N, int64_t K, int
     const int64_t groups = N * (K / g);
     const int g4 = static_cast<int>(g / 4);
     const int qmax = (1 << (bits - 1)) - 1;
-    const int grid = grid_for(groups * 32, 256, d->sms);
-#define WLQ_QX(B, F) launch_k(wlq::quantize_ex_kernel<B, F>, grid, 256, 0, s, W, groups, g4, qmax, codes, scales)
     const bool bf = (w_dtype == WLQ_IN_BF16);
-    if (scale_dtype == WLQ_SCALE_F32) { if (bf) WLQ_QX(true, wlq::SCALE_F32); else WLQ_QX(false, wlq::SCALE_F32); }
-    else if (scale_dtype == WLQ_SCALE_F16) { if (bf) WLQ_QX(true, wlq::SCALE_F16); else WLQ_QX(false, wlq::SCALE_F16); }
-    else { if (bf) WLQ_QX(true, wlq::SCALE_BF16); else WLQ_QX(false, wlq::SCALE_BF16); }
+    if (g4 <= 32 && 32 % g4 == 0) {
+        // short groups: one pass from registers, 32 / g4 groups per warp, four rounds in flight
+        const int64_t rounds = cdiv(groups * g4, 32);
+        const int grid = grid_for(cdiv(rounds, 4) * 32, 256, d->sms);
+#define WLQ_QS(B, F, L) launch_k(wlq::quantize_ex_short_kernel<B, F, L>, grid, 256, 0, s, W, groups, qmax, codes, scales)
+#define WLQ_QSL(B, F)                                                    \
+    switch (g4) {                                                        \
+        case 1: WLQ_QS(B, F, 1); break;                                  \
+        case 2: WLQ_QS(B, F, 2); break;                                  \
+        case 4: WLQ_QS(B, F, 4); break;                                  \
+        case 8: WLQ_QS(B, F, 8); break;                                  \
+        case 16: WLQ_QS(B, F, 16); break;                                \
+        default: WLQ_QS(B, F, 32); break;                                \
+    }
+        if (scale_dtype == WLQ_SCALE_F32) { if (bf) { WLQ_QSL(true, wlq::SCALE_F32) } else { WLQ_QSL(false, wlq::SCALE_F32) } }
+        else if (scale_dtype == WLQ_SCALE_F16) { if (bf) { WLQ_QSL(true, wlq::SCALE_F16) } else { WLQ_QSL(false, wlq::SCALE_F16) } }
+        else { if (bf) { WLQ_QSL(true, wlq::SCALE_BF16) } else { WLQ_QSL(false, wlq::SCALE_BF16) } }
+#undef WLQ_QSL
+#undef WLQ_QS
+    } else {
+        const int grid = grid_for(groups * 32, 256, d->sms);
+#define WLQ_QX(B, F) launch_k(wlq::quantize_ex_kernel<B, F>, grid, 256, 0, s, W, groups, g4, qmax, codes, scales)
+        if (scale_dtype == WLQ_SCALE_F32) { if (bf) WLQ_QX(true, wlq::SCALE_F32); else WLQ_QX(false, wlq::SCALE_F32); }
+        else if (scale_dtype == WLQ_SCALE_F16) { if (bf) WLQ_QX(true, wlq::SCALE_F16); else WLQ_QX(false, wlq::SCALE_F16); }
+        else { if (bf) WLQ_QX(true, wlq::SCALE_BF16); else WLQ_QX(false, wlq::SCALE_BF16); }
 #undef WLQ_QX
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "quantize_ex launch");
     return WLQ_OK;
