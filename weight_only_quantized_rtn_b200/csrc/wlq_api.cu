@@ -792,8 +792,9 @@ wlq_status wlq_quantize_ex(const void* W, int w_dtype, int64_t N, int64_t K, int
     const bool bf = (w_dtype == WLQ_IN_BF16);
     if (g4 <= 32 && 32 % g4 == 0) {
         // short groups: one pass from registers, 32 / g4 groups per warp, four rounds in flight
+        // persistent: the CTAs that fit at once (8 per SM) loop over the rounds
         const int64_t rounds = cdiv(groups * g4, 32);
-        const int grid = grid_for(cdiv(rounds, 4) * 32, 256, d->sms);
+        const int grid = static_cast<int>(std::min<int64_t>(cdiv(cdiv(rounds, 4), 8), static_cast<int64_t>(d->sms) * 8));
 #define WLQ_QS(B, F, L) launch_k(wlq::quantize_ex_short_kernel<B, F, L>, grid, 256, 0, s, W, groups, qmax, codes, scales)
 #define WLQ_QSL(B, F)                                                    \
     switch (g4) {                                                        \
@@ -810,7 +811,7 @@ wlq_status wlq_quantize_ex(const void* W, int w_dtype, int64_t N, int64_t K, int
 #undef WLQ_QSL
 #undef WLQ_QS
     } else {
-        const int grid = grid_for(groups * 32, 256, d->sms);
+        const int grid = static_cast<int>(std::min<int64_t>(cdiv(groups, 8), static_cast<int64_t>(d->sms) * 8));
 #define WLQ_QX(B, F) launch_k(wlq::quantize_ex_kernel<B, F>, grid, 256, 0, s, W, groups, g4, qmax, codes, scales)
         if (scale_dtype == WLQ_SCALE_F32) { if (bf) WLQ_QX(true, wlq::SCALE_F32); else WLQ_QX(false, wlq::SCALE_F32); }
         else if (scale_dtype == WLQ_SCALE_F16) { if (bf) WLQ_QX(true, wlq::SCALE_F16); else WLQ_QX(false, wlq::SCALE_F16); }
@@ -839,7 +840,7 @@ wlq_status wlq_quantize_fp8(const void* W, int w_dtype, int64_t N, int64_t K, in
     const int64_t g = group ? group : K;
     const int64_t groups = N * (K / g);
     const int g4 = static_cast<int>(g / 4);
-    const int grid = grid_for(groups * 32, 256, d->sms);
+    const int grid = static_cast<int>(std::min<int64_t>(cdiv(groups, 8), static_cast<int64_t>(d->sms) * 8));
     if (w_dtype == WLQ_IN_BF16) launch_k(wlq::quantize_fp8_kernel<true>, grid, 256, 0, s, W, groups, g4, codes, scales);
     else launch_k(wlq::quantize_fp8_kernel<false>, grid, 256, 0, s, W, groups, g4, codes, scales);
     cudaError_t e = cudaGetLastError();
