@@ -146,6 +146,23 @@ def cpu_baseline(n_rows_per_m=(48, 192, 2832)):
                       % ("/".join(map(str, n_rows_per_m)), "/".join(map(str, MS)))}
 
 
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Each value's maximum over all ranks: a job's time is its slowest rank's.
+    Every rank must call it with the same number of values (one collective)."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def job_tflops(world, flops_per_rank, ms):
+    """Whole-job throughput of independent replicas (weak scaling): the work
+    of all ranks over the slowest rank's time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -304,11 +321,9 @@ def run_gpu(args):
     ms_step = sum(a.elapsed_time(c) for a, c in outer) / args.steps
     per_ms = phase_ms
     per_m_ms = {M: per_ms[M] for M in MS}
-    if dist:
-        t = torch.tensor([ms_step] + [per_m_ms[M] for M in MS], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t[0])
-        per_m_ms = {M: float(t[1 + i]) for i, M in enumerate(MS)}
+    red = max_over_ranks([ms_step] + [per_m_ms[M] for M in MS], dist, dev)
+    ms_step = red[0]
+    per_m_ms = {M: red[1 + i] for i, M in enumerate(MS)}
 
     # ---- per-M kernels in isolation (L2 flushed before every launch)
     iso = {}
@@ -386,15 +401,12 @@ def run_gpu(args):
         if not torch.equal(y_h[M], y_first[M]):
             raise RuntimeError("pipelined end-to-end steps changed the output at M=%d" % M)
     e2e_ms = e_start.elapsed_time(e_end) / e2e_steps
-    if dist:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
+    e2e_ms = max_over_ranks([e2e_ms], dist, dev)[0]
     wlq.check_status()
 
     hbm_peak, tc_peak, tc_sust, peak_src = measured_peaks()
     flops = linear_flops()
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = job_tflops(world, flops, ms_step)
     per_m = {}
     for M in MS:
         f = 2.0 * M * N_OUT * K_IN
@@ -422,7 +434,7 @@ def run_gpu(args):
                        "timing": "one CUDA-graph replay per step between CUDA events (kernels chained by programmatic dependent launch); phases from replays of a second graph of the step with events between its phases"},
             "per_m": per_m, "roofline": roof, "clocks": clocks,
             "quantize_pack_us": round(per_ms["qp"] * 1e3, 2),
-            "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "e2e": {"value": round(job_tflops(world, flops, e2e_ms), 3), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                     "ms_per_step": round(e2e_ms, 4),
                     "schedule": "steps back to back on three streams (uploads, compute, downloads overlap across steps); outputs checked equal to a plain step's"},
