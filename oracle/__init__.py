@@ -162,3 +162,55 @@ def quantize_fp8(W: np.ndarray, group: int):
     scales = np.empty((N, groups_of(K, group)), np.float32)
     _check(_load().oracle_quantize_fp8(_p(W), w_dtype, N, K, group, _p(codes), _p(scales)))
     return codes, scales
+
+
+def _bf16_rne_bits(x: np.ndarray) -> np.ndarray:
+    """fp64 -> bf16 bit patterns, round to nearest even in one step (via the
+    exact fp64 value: scale to 8 significant bits and round half to even)."""
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros(x.shape, np.uint16)
+    flat, of = x.ravel(), out.ravel()
+    for i, v in enumerate(flat):
+        if v == 0.0:
+            of[i] = 0x8000 if np.signbit(v) else 0
+            continue
+        m, e = np.frexp(abs(v))                  # |v| = m 2^e, m in [0.5, 1)
+        lead = max(e - 1, -126)                  # bf16 normals from 2^-126, subnormals below
+        spacing = np.ldexp(1.0, lead - 7)
+        q = abs(v) / spacing                     # exact: spacing is a power of two
+        f = np.floor(q)
+        d = q - f
+        r = f + 1.0 if (d > 0.5 or (d == 0.5 and f % 2 == 1)) else f
+        f32 = np.float32(r * spacing)            # exact: at most 8 significant bits
+        bits = int(np.array([f32], np.float32).view(np.uint32)[0] >> 16)
+        of[i] = bits | (0x8000 if v < 0 else 0)
+    return out
+
+
+def _bf16_value(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def lowrank_split(W: np.ndarray, r: int):
+    """Top-r SVD split before quantizing the residual ("Nunchaku Lite" article,
+    why it matters / how it works: the hardest part of the weights goes to a
+    16-bit low-rank branch, the rest is quantized).
+
+    With W [N, K] and the Linear y = x W^T, the branch is y += (x L1) L2 with
+    L1 [K, r], L2 [r, N], so L1 L2 approximates W^T:  W^T = U S V^T (fp64
+    SVD), L1 = U_r S_r^(1/2), L2 = S_r^(1/2) V_r^T.  L1 and L2 are stored in
+    bf16 (round to nearest even); the residual R = W - (bf16(L1) bf16(L2))^T
+    is formed in fp64 and rounded to fp32 for quantization.
+
+    Returns dict(L1 [K,r] fp64, L2 [r,N] fp64, L1_bits, L2_bits (bf16 bit
+    patterns), R [N,K] fp32, sigma (all singular values, descending)).  The
+    factors are unique only up to the sign of each component (their product
+    is unique when the singular values are distinct)."""
+    W = np.asarray(W, dtype=np.float64)
+    U, S, Vt = np.linalg.svd(W.T, full_matrices=False)
+    sq = np.sqrt(S[:r])
+    L1 = U[:, :r] * sq[None, :]
+    L2 = sq[:, None] * Vt[:r, :]
+    L1b, L2b = _bf16_rne_bits(L1), _bf16_rne_bits(L2)
+    R = (W - (_bf16_value(L1b) @ _bf16_value(L2b)).T).astype(np.float32)
+    return dict(L1=L1, L2=L2, L1_bits=L1b, L2_bits=L2b, R=R, sigma=S)
