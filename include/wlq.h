@@ -12,6 +12,10 @@
  *    section "why it matters": the hard part of the weights is carried by a
  *    16-bit low-rank correction; section "how it works": the W4A16 kernels
  *    keep activations in 16 bits.
+ *  - The same model card, section 1 (the KV-dtype setting: cached K/V in int8
+ *    with one scale per token and head), section 1.1 (DiT blocks quantized to
+ *    fp8 on the GPU) and section 2 (a 5-bit MLP): the wider quantizers
+ *    wlq_quantize_ex and wlq_quantize_fp8.
  *
  * Conventions shared by every call:
  *  - W is [N, K] row-major (N outputs, K inputs); x is [M, K] and y is [M, N],
@@ -24,6 +28,10 @@
  *    returned before anything is enqueued; faults detected on the device
  *    (non-finite weights, a bounded wait that ran out) are recorded in the
  *    device error word and returned by wlq_get_status().
+ *  - Every kernel is launched with programmatic dependent launch: it may be
+ *    scheduled while the previous kernel on the stream is finishing, but it
+ *    touches no global memory before that kernel has completed and its writes
+ *    are visible, so stream order holds as for a plain launch.
  *  - Supported recipes (bits, group): (8, 0) = int8 per output channel;
  *    (4, 64) and (4, 16) = int4 grouped along K.  wlq_quantize also accepts
  *    (8, g) and (4, 0) for g in {16, 32, 64, 128}.
