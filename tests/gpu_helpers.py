@@ -69,9 +69,18 @@ def linear_case(x_bits, W, bits, group, b_bits=None, L1=None, L2=None, rows=None
     return rel_err(yg, y_ref), yg, y_ref
 
 
-def sample_rows(M: int, n: int = 12, seed: int = 0) -> np.ndarray:
-    if M <= n:
+def sample_rows(M: int, n: int = 12, seed: int = 0, block: int = 128) -> np.ndarray:
+    """Rows checked at full size: every row up to 64 tokens; beyond that the
+    first and last row of every `block`-token block (so each token tile of
+    every plan, 64 to 256 tokens, has at least two checked rows, and each CTA
+    of a CTA pair, which stages 128 of a 256-token tile, has its own), plus
+    one row at an offset that moves by 37 from block to block (so the
+    checked rows fall on every position inside a tile), plus `n` random rows."""
+    if M <= 64:
         return np.arange(M)
     g = np.random.default_rng(seed)
-    r = set(g.choice(M, n - 2, replace=False).tolist()) | {0, M - 1}
+    r = set(g.choice(M, min(n, M), replace=False).tolist())
+    for i, b0 in enumerate(range(0, M, block)):
+        end = min(M, b0 + block)
+        r |= {b0, end - 1, min(end - 1, b0 + (37 * i) % block)}
     return np.array(sorted(r))

@@ -143,3 +143,29 @@ def test_argument_errors_before_any_device_access(lib):
     assert lib.wlq_linear(None, 4, None, 64, 64, 8, 0, None, None, None, 0, None, 7, None, 0, None) == 1
     # misaligned x is rejected before any device access
     assert lib.wlq_linear(vp(18), 4, vp(32), 64, 64, 8, 0, None, None, None, 0, vp(64), 0, None, 0, None) == 3
+
+
+def test_noalloc_argument_errors_match_the_workspace_entry_point(lib):
+    """wlq_linear_noalloc makes wlq_linear's argument checks before it plans or
+    sizes its scratch: a bad rank with a large M is a shape error, not a
+    scratch-size or no-plan error, and every status comes before any device
+    access (this machine has no GPU)."""
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.wlq_linear.argtypes = [vp, i64, vp, i64, i64, i32, i32, vp, vp, vp, i32, vp, i32, vp, ctypes.c_size_t, vp]
+    lib.wlq_linear_noalloc.argtypes = [vp, i64, vp, i64, i64, i32, i32, vp, vp, vp, i32, vp, i32, vp]
+    big = 1 << 20
+    cases = [
+        # x, M, packed, N, K, bits, group, bias, L1, L2, r, y, y_dtype -> status
+        ((vp(16), big, vp(16), 4096, 4096, 4, 64, None, vp(16), vp(16), 8, vp(16), 0), 2),   # bad rank, large M
+        ((vp(16), (1 << 30) + 1, vp(16), 64, 64, 8, 0, None, None, None, 0, vp(16), 0), 2),  # M > 2^30
+        ((vp(16), -1, vp(16), 64, 64, 8, 0, None, None, None, 0, vp(16), 0), 1),             # M < 0
+        ((vp(16), 4, vp(16), 64, 64, 4, 0, None, None, None, 0, vp(16), 0), 4),              # no packed layout
+        ((vp(16), 4, vp(16), 64, 64, 8, 0, None, None, None, 16, vp(16), 0), 1),             # r > 0 without L1, L2
+        ((vp(16), 4, vp(16), 64, 64, 8, 0, None, None, None, 0, vp(16), 5), 1),              # bad y dtype
+        ((None, 4, vp(16), 64, 64, 8, 0, None, None, None, 0, vp(16), 0), 1),                # null x
+        ((vp(18), 4, vp(16), 64, 64, 8, 0, None, None, None, 0, vp(16), 0), 3),              # misaligned x
+        ((None, 0, None, 64, 64, 8, 0, None, None, None, 0, None, 0), 0),                    # M == 0: no-op
+    ]
+    for args, want in cases:
+        assert lib.wlq_linear(*args, None, 0, None) == want, args
+        assert lib.wlq_linear_noalloc(*args, None) == want, args

@@ -14,7 +14,7 @@ import torch
 
 import oracle
 import wlq_inputs as wi
-from tests.gpu_helpers import TOL, dev_bf16, dev_f32, linear_case, rel_err, sample_rows
+from tests.gpu_helpers import TOL, assert_codes_equal, dev_bf16, dev_f32, linear_case, rel_err, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -127,7 +127,26 @@ def test_parity_low_rank(bits, group, r, M):
 
 
 @pytest.mark.parametrize("bits,group", RECIPES)
+@pytest.mark.parametrize("r", [16, 32, 64])
+@pytest.mark.parametrize("M", [16, 300, 600])
+def test_parity_low_rank_zero_weight_rows(bits, group, r, M):
+    """All-zero weight rows (scale 0, row factor 0) still carry their low-rank
+    term: the branch shares the main accumulator, so such a row's operand is
+    left unscaled and the epilogue scales it by 1."""
+    x, W, b, L1, L2 = small_case(900 + r + M, M, 512, 512, bits, group, r=r)
+    W[[0, 3, 130, 511]] = 0.0
+    err, y, y_ref = linear_case(x, W, bits, group, b, L1, L2)
+    assert err <= TOL, err
+    assert np.abs(y_ref[:, 3]).max() > 0  # the low-rank term of a zero row is not zero
+
+
+@pytest.mark.parametrize("bits,group", RECIPES)
 @pytest.mark.parametrize("M,N,K,r,cap", [
+    (600, 4096, 1024, 32, 0),  # low rank on CTA pairs (256-token tiles, the term in the pair's accumulator)
+    (512, 1024, 512, 32, 0),   # low rank on split pairs: the term on K split 0 only
+    (256, 1920, 1024, 64, 0),  # low rank, 256-token tiles on single CTAs with the partial in the ring
+    (1024, 2048, 1024, 16, 20),# low rank on pairs, several tiles per pair
+
     (40, 1100, 320, 0, 4),     # 9 tiles on 4 CTAs: both accumulator buffers in use
     (16, 33000, 128, 0, 16),   # 258 tiles of 16 tokens on 16 CTAs
     (300, 700, 256, 0, 3),     # 128-token tiles, several per CTA
@@ -159,16 +178,29 @@ def test_parity_several_tiles_per_cta(bits, group, M, N, K, r, cap):
 
 
 @pytest.mark.parametrize("bits,group", RECIPES)
-def test_bf16_output_is_rounded_fp32_output(bits, group):
+@pytest.mark.parametrize("M,N,K", [
+    (16, 384, 512),     # few-token kernel
+    (300, 384, 512),    # K split over a cluster (partial in shared memory)
+    (300, 16384, 512),  # unsplit 256-token tiles, CTA pairs: the bf16 fast epilogue
+    (1560, 4096, 1024), # pairs with a tail round, ragged last token tile
+    (600, 4096, 448),   # pairs, partial last ring slot
+    (64, 4096, 1024),   # resident-x tensor-core kernel
+    (100, 1000, 512),   # ragged N: scalar stores
+])
+def test_bf16_output_is_rounded_fp32_output(bits, group, M, N, K):
+    """The bf16 output is the fp32 output rounded to nearest even, bit for
+    bit, on every engine and epilogue variant (the int4 row factor of x
+    included)."""
     m = wlq()
-    for M in (16, 300):
-        x, W, b, _, _ = small_case(5, M, 384, 512, bits, group)
-        codes, scales = m.quantize(dev_f32(W), bits, group)
-        packed = m.pack(codes, scales, bits, group)
-        xd, bd = dev_bf16(x), dev_bf16(b)
-        y32 = m.linear(xd, packed, 384, 512, bits, group, bd, out_dtype=torch.float32)
-        y16 = m.linear(xd, packed, 384, 512, bits, group, bd, out_dtype=torch.bfloat16)
-        assert torch.equal(y16, y32.to(torch.bfloat16))
+    x, W, b, _, _ = small_case(5 + M, M, N, K, bits, group)
+    codes, scales = m.quantize(dev_f32(W), bits, group)
+    packed = m.pack(codes, scales, bits, group)
+    xd, bd = dev_bf16(x), dev_bf16(b)
+    y32 = m.linear(xd, packed, N, K, bits, group, bd, out_dtype=torch.float32)
+    y16 = m.linear(xd, packed, N, K, bits, group, bd, out_dtype=torch.bfloat16)
+    m.check_status()
+    assert not torch.isnan(y32).any()
+    assert torch.equal(y16, y32.to(torch.bfloat16))
 
 
 @pytest.mark.parametrize("bits,group", RECIPES)
@@ -238,18 +270,88 @@ def test_full_mlp_w4_gs64(which, M):
     _check_full(d["x"], d["W"], 4, 64, d["b"])
 
 
-_MIXED = {}
+def _bf16_close(y_bf16_rows: np.ndarray, ref: np.ndarray):
+    """A bf16 output against the fp64 oracle: the parity bound plus the bf16
+    rounding of each value (half a bf16 unit in the last place, at most
+    2^-8 of the value)."""
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    bad = np.abs(y_bf16_rows.astype(np.float64) - ref) > TOL * rms + 2.0 ** -8 * np.abs(ref)
+    assert not bad.any(), "%d bf16 outputs outside the bound" % int(bad.sum())
 
 
-@pytest.mark.parametrize("name", [n for n, *_ in wi.MIXED_LAYERS])
-def test_full_mixed_block(name):
-    if not _MIXED:
-        _MIXED.update(wi.mixed_block(4096))
-    blk = _MIXED
-    layer = blk["layers"][name]
-    K = layer["W"].shape[1]
-    x = blk["x"] if K == wi.HIDDEN else wi.activations(3, 99, 4096, K)
-    _check_full(x, layer["W"], layer["bits"], layer["group"], layer["b"])
+def _oracle_chain(x_rows, up_q, up_b, down_q, down_b, group):
+    """The oracle's chained pair on the same rows: up in fp64, handed on as
+    bf16 (rounded to nearest even, as the product hands on its bf16 output),
+    then down in fp64."""
+    y_up = oracle.linear(x_rows, up_q[0], up_q[1], group, up_b)
+    y_dn = oracle.linear(oracle._bf16_rne_bits(y_up), down_q[0], down_q[1], group, down_b)
+    return y_up, y_dn
+
+
+@pytest.mark.parametrize("M", [16, 1560, 6240])
+def test_full_mlp_chained_up_then_down(M):
+    """The MLP workload as configured: a GELU-free chained pair, down
+    consuming up's bf16 output on the same stream, with both weights
+    quantized by the fused quantize-pack pass (its codes and scales checked
+    against the oracle too)."""
+    m = wlq()
+    up, dn = wi.mlp_w4(M, "up"), wi.mlp_w4(M, "down")
+    N1, K1 = up["W"].shape
+    N2, K2 = dn["W"].shape
+    s_up, p_up = m.quantize_pack(dev_f32(up["W"]), 4, 64)
+    s_dn, p_dn = m.quantize_pack(dev_f32(dn["W"]), 4, 64)
+    q_up, q_dn = oracle.quantize(up["W"], 4, 64), oracle.quantize(dn["W"], 4, 64)
+    assert_codes_equal(m.unpack(p_up, N1, K1, 4, 64), s_up, *q_up)
+    assert_codes_equal(m.unpack(p_dn, N2, K2, 4, 64), s_dn, *q_dn)
+    x = dev_bf16(up["x"])
+    y_up = torch.full((M, N1), float("nan"), dtype=torch.bfloat16, device="cuda")
+    y_dn = torch.full((M, N2), float("nan"), dtype=torch.float32, device="cuda")
+    m.linear_into(y_up, x, p_up, N1, K1, 4, 64, dev_bf16(up["b"]),
+                  workspace=m.new_workspace(M, N1, K1, 4, 64))
+    m.linear_into(y_dn, y_up, p_dn, N2, K2, 4, 64, dev_bf16(dn["b"]),
+                  workspace=m.new_workspace(M, N2, K2, 4, 64))
+    m.check_status()
+    rows = sample_rows(M, 12, seed=M)
+    ref_up, ref_dn = _oracle_chain(up["x"][rows], q_up, up["b"], q_dn, dn["b"], 64)
+    _bf16_close(y_up.float().cpu().numpy()[rows], ref_up)
+    err = rel_err(y_dn.cpu().numpy()[rows], ref_dn)
+    assert err <= TOL, err
+
+
+def test_full_mixed_block_back_to_back():
+    """The mixed-precision block as configured: q, k, v, o (int8 per channel)
+    and up (int4 gs16) on x, then down (int4 gs16) on up's bf16 output -- six
+    launches back to back on one stream, nothing synchronised between them."""
+    m = wlq()
+    M = 4096
+    blk = wi.mixed_block(M)
+    x_bits = blk["x"]
+    x = dev_bf16(x_bits)
+    dev_layers, outs = {}, {}
+    for name, N, K, bits, group in wi.MIXED_LAYERS:
+        L = blk["layers"][name]
+        s, p = m.quantize_pack(dev_f32(L["W"]), bits, group)
+        dev_layers[name] = (p, dev_bf16(L["b"]), m.new_workspace(M, N, K, bits, group))
+        dt = torch.bfloat16 if name == "up" else torch.float32
+        outs[name] = torch.full((M, N), float("nan"), dtype=dt, device="cuda")
+    torch.cuda.synchronize()
+    for name, N, K, bits, group in wi.MIXED_LAYERS:
+        p, b, ws = dev_layers[name]
+        inp = outs["up"] if name == "down" else x
+        m.linear_into(outs[name], inp, p, N, K, bits, group, b, workspace=ws)
+    m.check_status()
+    rows = sample_rows(M, 12, seed=3)
+    q = {name: oracle.quantize(blk["layers"][name]["W"], bits, group)
+         for name, N, K, bits, group in wi.MIXED_LAYERS}
+    for name in ("q", "k", "v", "o"):
+        ref = oracle.linear(x_bits[rows], *q[name], 0, blk["layers"][name]["b"])
+        err = rel_err(outs[name].cpu().numpy()[rows], ref)
+        assert err <= TOL, (name, err)
+    ref_up, ref_dn = _oracle_chain(x_bits[rows], q["up"], blk["layers"]["up"]["b"], q["down"],
+                                   blk["layers"]["down"]["b"], 16)
+    _bf16_close(outs["up"].float().cpu().numpy()[rows], ref_up)
+    err = rel_err(outs["down"].cpu().numpy()[rows], ref_dn)
+    assert err <= TOL, ("down", err)
 
 
 @pytest.mark.parametrize("M", [256, 4096])

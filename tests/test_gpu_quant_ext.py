@@ -127,3 +127,46 @@ def test_kv_cache_int8_per_token_head_timed():
     us = sorted(ts)[len(ts) // 2]
     nbytes = T * H * D * (2 + 1) + T * H * 2
     print("\nKV int8 per (token, head): %d x %d x %d bf16 -> %.1f us, %.0f GB/s" % (T, H, D, us, nbytes / us / 1e3))
+
+
+def _scale_edge_weights(scale_dtype, qmax, seed):
+    """Groups of 16 whose absmax a makes a / qmax land exactly on, or one fp32
+    step beside, the midpoint of two neighbouring 16-bit values (where rounding
+    the fp32 quotient again would be wrong), plus, for fp16, absmaxes whose
+    scale is subnormal in fp16 (where the scale can round far below a / qmax
+    and the clamp to +-qmax acts)."""
+    g = np.random.default_rng(seed)
+    if scale_dtype == 1:
+        lo = g.integers(0x1000, 0x5000, 200).astype(np.uint16)          # normal fp16 values
+        v = lo.view(np.float16).astype(np.float64)
+        nxt = (lo + 1).view(np.float16).astype(np.float64)
+    else:
+        lo = g.integers(0x3000, 0x4300, 200).astype(np.uint16)          # bf16 values
+        v = (lo.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        nxt = ((lo.astype(np.uint32) + 1) << 16).view(np.float32).astype(np.float64)
+    mids = (v + nxt) / 2                                                 # exact in fp64
+    a0 = (mids * qmax).astype(np.float32)                                # exact: <= 19 significant bits
+    a = np.concatenate([a0, np.nextafter(a0, np.float32(np.inf)), np.nextafter(a0, np.float32(0))])
+    if scale_dtype == 1:
+        sub = (g.integers(1, 1024, 150) * 2.0 ** -24 * qmax * g.uniform(0.9, 1.1, 150)).astype(np.float32)
+        a = np.concatenate([a, sub])
+    a = a[np.isfinite(a) & (a > 0)]
+    a = a[: len(a) // 4 * 4]  # four groups of 16 per row of 64
+    G = len(a)
+    W = (g.uniform(-1, 1, (G, 16)) * a[:, None]).astype(np.float32)
+    W[np.arange(G), g.integers(0, 16, G)] = a * np.where(g.random(G) < 0.5, -1, 1)
+    return W.reshape(-1, 64)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 5, 8])
+@pytest.mark.parametrize("scale_dtype", [1, 2])
+def test_quantize_ex_scale_midpoints_and_subnormal_scales(bits, scale_dtype):
+    m = wlq()
+    qmax = (1 << (bits - 1)) - 1
+    W = _scale_edge_weights(scale_dtype, qmax, 17 * bits + scale_dtype)
+    co, so = oracle.quantize_ex(W, bits, 16, scale_dtype)
+    cg, sg = m.quantize_ex(dev_f32(W), bits, 16, scale_dtype)
+    torch.cuda.synchronize()
+    m.check_status()
+    np.testing.assert_array_equal(sg.float().cpu().numpy(), so)
+    np.testing.assert_array_equal(cg.cpu().numpy(), co)

@@ -35,6 +35,18 @@ def test_quantize_bit_exact_on_workload_weights(case):
     assert_codes_equal(cg, sg, co, so)
 
 
+@pytest.mark.parametrize("case", list(range(11)))
+def test_quantize_pack_bit_exact_on_workload_weights(case):
+    """The fused quantize-pack pass (the benchmark's first launch) against the
+    oracle on every workload weight: unpacked codes and fp32 scales bit-exact."""
+    name, W, bits, group = list(_workload_weights())[case]
+    m = wlq()
+    s_f, p_f = m.quantize_pack(dev_f32(W), bits, group)
+    m.check_status()
+    co, so = oracle.quantize(W, bits, group)
+    assert_codes_equal(m.unpack(p_f, W.shape[0], W.shape[1], bits, group), s_f, co, so)
+
+
 @pytest.mark.parametrize("bits,group", [(8, 0), (4, 64), (4, 16), (8, 64), (4, 0), (8, 16), (4, 32), (4, 128)])
 def test_quantize_edge_cases(bits, group):
     g = np.random.default_rng(99)
@@ -151,6 +163,9 @@ def test_quantize_pack_equals_quantize_then_pack(bits, group, N, K):
     assert torch.equal(s_f, s_ref)
     assert p_f.numel() == p_ref.numel()
     assert torch.equal(p_f, p_ref)
+    # and against the oracle directly: the packed codes and the scales
+    co, so = oracle.quantize(W, bits, group)
+    assert_codes_equal(m.unpack(p_f, N, K, bits, group), s_f, co, so)
 
 
 @pytest.mark.parametrize("bits,group,K", [(8, 0, 200), (8, 0, 4040), (4, 16, 1232)])
@@ -165,6 +180,8 @@ def test_quantize_pack_ragged_k(bits, group, K):
     torch.cuda.synchronize()
     assert torch.equal(s_f, s_ref)
     assert torch.equal(p_f, p_ref)
+    co, so = oracle.quantize(W, bits, group)
+    assert_codes_equal(m.unpack(p_f, W.shape[0], K, bits, group), s_f, co, so)
 
 
 @pytest.mark.parametrize("bits,group", [(8, 0), (4, 64), (4, 16)])
