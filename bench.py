@@ -170,6 +170,158 @@ def dist_env():
     return world, rank, local
 
 
+# ---------------------------------------------------------------------------
+# Every configured workload, timed in the launch configuration of a model's
+# layer sequence: a CUDA graph of back-to-back units (one unit = the
+# workload's Linear calls), kernels chained by programmatic dependent launch,
+# the units rotating over enough copies of the packed weights that every unit
+# reads its weights from HBM, not from L2 (L2 is also flushed before each
+# replay).  Per unit: device time, TFLOP/s, algorithmic GB/s and both roofline
+# fractions against the measured peaks.
+# ---------------------------------------------------------------------------
+L2_BYTES = 126 * 2 ** 20
+
+
+def workload_entries():
+    """(key, M, layers, wiring) for every configured workload.  layers:
+    (name, N, K, bits, group, r); wiring: 'each' (every layer on x), 'chain'
+    (down on up's bf16 output) or 'block' (q, k, v, o and up on x, down on
+    up's bf16 output)."""
+    H, F = wi.HIDDEN, wi.MLP
+    out = [("tiny_w8_m64", 64, [("lin", 512, 256, 8, 0, 0)], "each")]
+    for M in (16, 256, 4096):
+        out.append(("attn_w8_m%d" % M, M, [("proj", H, H, 8, 0, 0)], "each"))
+    for M in (16, 1560, 6240):
+        out.append(("mlp_w4g64_up_m%d" % M, M, [("up", F, H, 4, 64, 0)], "each"))
+        out.append(("mlp_w4g64_down_m%d" % M, M, [("down", H, F, 4, 64, 0)], "each"))
+        out.append(("mlp_w4g64_chained_m%d" % M, M, [("up", F, H, 4, 64, 0), ("down", H, F, 4, 64, 0)], "chain"))
+    out.append(("mixed_block_m4096", 4096, [(n, N, K, b, g, 0) for n, N, K, b, g in wi.MIXED_LAYERS], "block"))
+    for M in (256, 4096):
+        out.append(("svdq_w4g64_lr32_m%d" % M, M, [("lr", H, H, 4, 64, wi.RANK)], "each"))
+    return out
+
+
+def _layer_weight(key, name, N, K):
+    """The workload's seeded fp32 weight for this layer (timing only needs its
+    shape and value range; the recipe is the parity tests')."""
+    if key.startswith("tiny"):
+        return wi.tiny_w8()["W"]
+    if key.startswith("attn"):
+        return wi.attn_w8(1)["W"]
+    if key.startswith("mlp"):
+        return wi.mlp_w4(1, name)["W"]
+    if key.startswith("mixed"):
+        i = [n for n, *_ in wi.MIXED_LAYERS].index(name)
+        return wi.weight(3, 10 * (i + 1), N, K)
+    return wi.svdq_w4_lr(1)["W"]
+
+
+def time_workloads(wlq, torch, dev, evict_l2, hbm_peak, tc_peak, reps=3):
+    res = {}
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+    for key, M, layers, wiring in workload_entries():
+        K0 = layers[0][2]
+        x = bf(wi.activations(5, 1, M, K0))
+        wbytes = sum(wlq.packed_bytes(N, K, b, g) for _, N, K, b, g, _ in layers)
+        copies = int(min(16, max(1, -(-3 * L2_BYTES // wbytes))))
+        units = max(8, copies)
+        L = []
+        for name, N, K, bits, group, r in layers:
+            W = torch.from_numpy(_layer_weight(key, name, N, K)).to(dev)
+            _, p = wlq.quantize_pack(W, bits, group)
+            del W
+            ps = [p] + [p.clone() for _ in range(copies - 1)]
+            b = bf(wi.bias(5, 2, N))
+            L1 = bf(wi.normal_bf16(wi.rng(5, 3), (K, r), 0.05)) if r else None
+            L2 = bf(wi.normal_bf16(wi.rng(5, 4), (r, N), 0.05)) if r else None
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ws = wlq.new_workspace(M, N, K, bits, group, r, device=dev)
+            L.append(dict(name=name, N=N, K=K, bits=bits, group=group, r=r, ps=ps, b=b, L1=L1, L2=L2, y=y, ws=ws))
+
+        def unit(i):
+            for j, l in enumerate(L):
+                inp = x
+                if wiring == "chain" and j == 1:
+                    inp = L[0]["y"]
+                if wiring == "block" and l["name"] == "down":
+                    inp = [u for u in L if u["name"] == "up"][0]["y"]
+                wlq.linear_into(l["y"], inp, l["ps"][i % copies], l["N"], l["K"], l["bits"], l["group"], l["b"],
+                                l["L1"], l["L2"], workspace=l["ws"])
+
+        for i in range(3):
+            unit(i)
+        torch.cuda.synchronize()
+        wlq.check_status()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(units):
+                unit(i)
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            evict_l2()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e-3 / units)
+        wlq.check_status()
+        t = statistics.median(ts)
+        flops = sum(2.0 * M * l["N"] * l["K"] + (2.0 * M * l["r"] * (l["K"] + l["N"]) if l["r"] else 0.0) for l in L)
+        byts = sum(wlq.packed_bytes(l["N"], l["K"], l["bits"], l["group"]) + 2 * M * l["K"] + 2 * M * l["N"] + 2 * l["N"]
+                   + (2 * l["r"] * (l["K"] + l["N"]) if l["r"] else 0) for l in L)
+        res[key] = {"M": M, "layers": ["%s %dx%d int%d %s%s" % (l["name"], l["N"], l["K"], l["bits"],
+                                                                "gs%d" % l["group"] if l["group"] else "per-channel",
+                                                                " r=%d" % l["r"] if l["r"] else "") for l in L],
+                    "wiring": wiring, "us": round(t * 1e6, 2), "tflops": round(flops / t / 1e12, 1),
+                    "hbm_gbs": round(byts / t / 1e9, 1), "tensor_frac": round(flops / t / 1e12 / tc_peak, 4),
+                    "hbm_frac": round(byts / t / 1e9 / hbm_peak, 4), "algorithmic_bytes": int(byts),
+                    "flops": flops, "weight_copies": copies, "units_per_replay": units}
+        del L, g
+        torch.cuda.empty_cache()
+    return res
+
+
+def time_lowrank_producer(wlq, torch, dev, evict_l2, reps=3):
+    """The step before the low-rank branch on the SVDQuant workload's weight
+    (W = (L1 L2)^T + R, [4096, 4096], r = 32): the GPU top-r split (sketch of
+    64 columns, two power passes), the residual R = W - (L1 L2)^T and its
+    quantize-pack (int4 gs64), each timed alone after an L2 flush."""
+    d = wi.svdq_w4_lr(1)
+    l1p = (d["L1"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    l2p = (d["L2"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    W = torch.from_numpy(((l1p @ l2p).T + d["W"].astype(np.float64)).astype(np.float32)).to(dev)
+    N, K = W.shape
+    omega = torch.from_numpy(wi.normal_f32(wi.rng(9, 2), (N, 64), 1.0)).to(dev)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            evict_l2()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            out = fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        wlq.check_status()
+        return statistics.median(ts), out
+
+    t_split, (L1, L2, _) = timed(lambda: wlq.lowrank_split(W, 32, omega, power_iters=2))
+    t_res, R = timed(lambda: wlq.lowrank_residual(W, L1, L2))
+    t_qp, _ = timed(lambda: wlq.quantize_pack(R, 4, 64))
+    return {"workload": "SVDQuant-style weight W = (L1 L2)^T + R, [4096, 4096], r = 32 (planted N(0,0.05) bf16 "
+                        "factors, R ~ N(0, 0.02)); sketch l = 64, 2 power passes",
+            "split_us": round(t_split, 1), "residual_us": round(t_res, 1), "quantize_pack_us": round(t_qp, 1),
+            "residual_gbs": round(2 * N * K * 4 / t_res / 1e3, 1),  # W read + R written
+            "timing": "each call alone, L2 flushed before, CUDA events, median of %d" % reps}
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
@@ -439,6 +591,12 @@ def run_gpu(args):
                     "ms_per_step": round(e2e_ms, 4),
                     "schedule": "steps back to back on three streams (uploads, compute, downloads overlap across steps); outputs checked equal to a plain step's"},
             "gpu_launches": launches_per_step * args.steps}
+    if not args.no_configs:
+        line["configs"] = time_workloads(wlq, torch, dev, evict_l2, hbm_peak, tc_peak)
+        line["lowrank_producer"] = time_lowrank_producer(wlq, torch, dev, evict_l2)
+        line["configs_timing"] = ("per unit = one CUDA-graph replay of back-to-back units / units; units rotate over "
+                                  "weight copies totalling >= 3x L2 and L2 is flushed before each replay; "
+                                  "median of 3 replays; bf16 outputs")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:
@@ -456,6 +614,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-workload timings")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
     if args.impl == "reference":

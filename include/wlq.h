@@ -83,7 +83,9 @@ wlq_status wlq_quantize(const float* W, int64_t N, int64_t K, int bits, int grou
 
 /*
  * Bytes of the packed operand produced by wlq_pack (0 for an unsupported
- * recipe or a bad shape).  Host-only, no device access.
+ * recipe or a bad shape).  Host-only, no device access.  No passage of the
+ * pages defines it: a sizing helper for the layout below, which is this
+ * library's own (the pages name the loader step, not its layout).
  * Layout: ceil(N/128) * ceil(K/64) tiles of 128 outputs x 64 inputs, each
  * holding the codes (int8: 8192 B; int4: 4096 B) followed, for int4, by the
  * tile's group scales in fp16 (gs64: 256 B; gs16: 1024 B), then one fp32
@@ -151,13 +153,18 @@ wlq_status wlq_quantize_ex(const void* W, int w_dtype, int64_t N, int64_t K, int
 wlq_status wlq_quantize_fp8(const void* W, int w_dtype, int64_t N, int64_t K, int group,
                             uint8_t* codes, float* scales, void* stream);
 
-/* Inverse of the code part of wlq_pack: packed -> codes int8 [N, K]. */
+/*
+ * Inverse of the code part of wlq_pack: packed -> codes int8 [N, K].  No
+ * passage of the pages defines it: a layout helper that lets a caller (and
+ * the tests) read the packed codes back.
+ */
 wlq_status wlq_unpack(const void* packed, int64_t N, int64_t K, int bits, int group,
                       int8_t* codes, void* stream);
 
 /*
  * Workspace bytes wlq_linear needs for this shape (host-only; 0 when it
- * needs none: int8 weights without the low-rank branch).  The contents need
+ * needs none: int8 weights without the low-rank branch).  No passage of the
+ * pages defines it: a sizing helper for the caller-owned scratch.  The contents need
  * no initialisation.  A workspace must not be shared by calls that may run
  * concurrently.
  */
@@ -171,7 +178,8 @@ size_t wlq_linear_workspace(int64_t M, int64_t N, int64_t K, int bits, int group
  * x      : bf16 [M, K]
  * packed : output of wlq_pack for (N, K, bits, group)
  * bias   : bf16 [N] or NULL
- * L1, L2 : bf16 [K, r] and [r, N], or NULL with r == 0; r in {0, 16, 32, 64}
+ * L1, L2 : bf16 [K, r] (16-byte aligned) and [r, N], or NULL with r == 0;
+ *          r in {0, 16, 32, 64}
  * y      : [M, N] in y_dtype (WLQ_OUT_BF16 or WLQ_OUT_F32)
  * workspace / ws_bytes : at least wlq_linear_workspace(M, N, K, bits, group, r)
  *                        bytes (may be NULL when that is 0)
@@ -210,8 +218,56 @@ wlq_status wlq_linear_noalloc(const void* x, int64_t M, const void* packed, int6
                               int r, void* y, int y_dtype, void* stream);
 
 /*
+ * Workspace bytes wlq_lowrank_split needs (host-only; 0 for an unsupported
+ * shape).  No passage of the pages defines it: a sizing helper.
+ */
+size_t wlq_lowrank_workspace(int64_t N, int64_t K, int r, int l);
+
+/*
+ * Low-rank split of a weight before it is quantized ("Nunchaku Lite", section
+ * "why it matters": the hardest part of the weights is carried by a 16-bit
+ * low-rank correction and only the rest is quantized).  The best rank-r part
+ * of W^T [K, N] (its top r singular triplets), split evenly:
+ *   W^T ~ U_r S_r V_r^T,   L1 = U_r S_r^(1/2) [K, r],   L2 = S_r^(1/2) V_r^T [r, N]
+ * found by randomized subspace iteration with l sketch columns and
+ * power_iters passes of W W^T (each followed by a re-orthonormalisation),
+ * then an fp64 eigen-solve of the l x l projected problem.  Like any SVD,
+ * each component's sign is arbitrary; the product L1 L2 is not.  The error
+ * against the exact split shrinks with the gap between the r-th and the
+ * (l+1)-th singular values, like (s_(l+1) / s_r)^(2 power_iters + 1).
+ * W      : fp32 [N, K], 16-byte aligned
+ * omega  : fp32 [N, l], a test matrix drawn by the caller (e.g. independent
+ *          standard normals), 16-byte aligned
+ * L1, L2 : bf16 [K, r] and [r, N] (round to nearest even), 16-byte aligned
+ * sigma  : fp32 [r] estimated singular values, descending, or NULL
+ * workspace / ws_bytes : at least wlq_lowrank_workspace(N, K, r, l) bytes
+ * r in {16, 32, 64}; l in {32, 64}, l >= r; 0 <= power_iters <= 8; N, K >= l.
+ * Asynchronous on `stream`; deterministic run to run.
+ */
+wlq_status wlq_lowrank_split(const float* W, int64_t N, int64_t K, int r, int l, int power_iters,
+                             const float* omega, void* L1, void* L2, float* sigma, void* workspace,
+                             size_t ws_bytes, void* stream);
+
+/*
+ * The part of W the low-rank branch leaves for quantization (same passage):
+ *   R[n][k] = fp32( W[n][k] - sum_{j<r} L1[k][j] L2[j][n] )
+ * the sum taken in fp64 over j in increasing order (products and additions
+ * rounded one by one, no fused multiply-add), then one rounding to fp32.
+ * Quantize R with wlq_quantize / wlq_quantize_pack and give (L1, L2) to
+ * wlq_linear.  W, R: fp32 [N, K] (4-byte aligned; R must not overlap W);
+ * L1: bf16 [K, r]; L2: bf16 [r, N]; r in {16, 32, 64}.
+ */
+wlq_status wlq_lowrank_residual(const float* W, const void* L1, const void* L2, int64_t N, int64_t K, int r,
+                                float* R, void* stream);
+
+/*
  * Synchronise `stream`, then read and clear this device's error word:
  * WLQ_OK, WLQ_ERR_NONFINITE or WLQ_ERR_TIMEOUT (or WLQ_ERR_CUDA).
+ * The error path follows "Nunchaku Lite", section "hardware and precision
+ * support": the quantizer checks the GPU's compute capability when it loads
+ * and raises a clear error on a mismatch.  Here every call returns
+ * WLQ_ERR_UNSUPPORTED on a device other than sm_100, and errors found on the
+ * device are kept until this call reads them.
  */
 wlq_status wlq_get_status(void* stream);
 
@@ -232,7 +288,10 @@ wlq_status wlq_probe_wait_timeout(uint64_t timeout_ns, void* stream);
  */
 void wlq_set_grid_limit(int max_ctas);
 
-/* Human-readable text of the last error returned on this host thread. */
+/*
+ * Human-readable text of the last error returned on this host thread (the
+ * clear error of "Nunchaku Lite", section "hardware and precision support").
+ */
 const char* wlq_last_error(void);
 
 /* Library version, e.g. "0.1.0". */

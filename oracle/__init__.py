@@ -48,8 +48,9 @@ def bind(path: str):
     lib.oracle_linear.argtypes = [vp, i64, i64, vp, vp, i64, i32, vp, vp, vp, i32, vp]
     lib.oracle_quantize_ex.argtypes = [vp, i32, i64, i64, i32, i32, i32, vp, vp]
     lib.oracle_quantize_fp8.argtypes = [vp, i32, i64, i64, i32, vp, vp]
+    lib.oracle_lowrank_residual.argtypes = [vp, vp, vp, i64, i64, i32, vp]
     for f in (lib.oracle_quantize, lib.oracle_dequantize, lib.oracle_linear, lib.oracle_quantize_ex,
-              lib.oracle_quantize_fp8):
+              lib.oracle_quantize_fp8, lib.oracle_lowrank_residual):
         f.restype = ctypes.c_int
     return lib
 
@@ -166,25 +167,20 @@ def quantize_fp8(W: np.ndarray, group: int):
 
 def _bf16_rne_bits(x: np.ndarray) -> np.ndarray:
     """fp64 -> bf16 bit patterns, round to nearest even in one step (via the
-    exact fp64 value: scale to 8 significant bits and round half to even)."""
+    exact fp64 value: scale to 8 significant bits and round half to even).
+    Element by element, written with whole-array operations."""
     x = np.asarray(x, dtype=np.float64)
-    out = np.zeros(x.shape, np.uint16)
-    flat, of = x.ravel(), out.ravel()
-    for i, v in enumerate(flat):
-        if v == 0.0:
-            of[i] = 0x8000 if np.signbit(v) else 0
-            continue
-        m, e = np.frexp(abs(v))                  # |v| = m 2^e, m in [0.5, 1)
-        lead = max(e - 1, -126)                  # bf16 normals from 2^-126, subnormals below
-        spacing = np.ldexp(1.0, lead - 7)
-        q = abs(v) / spacing                     # exact: spacing is a power of two
-        f = np.floor(q)
-        d = q - f
-        r = f + 1.0 if (d > 0.5 or (d == 0.5 and f % 2 == 1)) else f
-        f32 = np.float32(r * spacing)            # exact: at most 8 significant bits
-        bits = int(np.array([f32], np.float32).view(np.uint32)[0] >> 16)
-        of[i] = bits | (0x8000 if v < 0 else 0)
-    return out
+    a = np.abs(x)
+    _, e = np.frexp(a)                           # |x| = m 2^e, m in [0.5, 1) (e = 0 for x = 0)
+    lead = np.maximum(e - 1, -126)               # bf16 normals from 2^-126, subnormals below
+    spacing = np.ldexp(1.0, lead - 7)            # bf16 spacing in that binade
+    q = a / spacing                              # exact: spacing is a power of two
+    f = np.floor(q)
+    d = q - f
+    r = np.where((d > 0.5) | ((d == 0.5) & (np.fmod(f, 2.0) == 1.0)), f + 1.0, f)
+    f32 = (r * spacing).astype(np.float32)       # exact: at most 8 significant bits
+    bits = (f32.view(np.uint32) >> 16).astype(np.uint16)
+    return bits | np.where(np.signbit(x), np.uint16(0x8000), np.uint16(0)).astype(np.uint16)
 
 
 def _bf16_value(bits: np.ndarray) -> np.ndarray:
@@ -214,3 +210,19 @@ def lowrank_split(W: np.ndarray, r: int):
     L1b, L2b = _bf16_rne_bits(L1), _bf16_rne_bits(L2)
     R = (W - (_bf16_value(L1b) @ _bf16_value(L2b)).T).astype(np.float32)
     return dict(L1=L1, L2=L2, L1_bits=L1b, L2_bits=L2b, R=R, sigma=S)
+
+
+def lowrank_residual(W: np.ndarray, L1_bits: np.ndarray, L2_bits: np.ndarray) -> np.ndarray:
+    """R = fp32(W - (L1 L2)^T): the part of W the low-rank branch leaves for
+    quantization ("Nunchaku Lite" article, why it matters), for given bf16
+    factors (bit patterns L1 [K, r], L2 [r, N]).  The sum over the rank is
+    taken in fp64 in increasing j, then rounded once to fp32 (``wlq_oracle.c``)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    L1_bits = np.ascontiguousarray(L1_bits, dtype=np.uint16)
+    L2_bits = np.ascontiguousarray(L2_bits, dtype=np.uint16)
+    N, K = W.shape
+    r = L1_bits.shape[1]
+    assert L1_bits.shape == (K, r) and L2_bits.shape == (r, N)
+    R = np.empty((N, K), np.float32)
+    _check(_load().oracle_lowrank_residual(_p(W), _p(L1_bits), _p(L2_bits), N, K, r, _p(R)))
+    return R

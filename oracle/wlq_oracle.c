@@ -333,3 +333,31 @@ int oracle_linear(const uint16_t* x, int64_t M, int64_t K,
     }
     return ORACLE_OK;
 }
+
+/*
+ * Residual of the low-rank split [NL "why it matters": the hard part of W is
+ * carried by the 16-bit low-rank branch, the rest R is quantized].  With the
+ * Linear y = x W^T and the branch y += (x L1) L2, L1 [K, r] and L2 [r, N]
+ * stand for W^T's best rank-r part, so
+ *   R[n][k] = fp32( W[n][k] - sum_{j=0}^{r-1} L1[k][j] * L2[j][n] )
+ * with the sum taken in fp64 over j in increasing order (each product and
+ * each addition rounded on its own), then one rounding to fp32.
+ * W: fp32 [N, K]; L1, L2: bf16 bits; R: fp32 [N, K].
+ */
+int oracle_lowrank_residual(const float* W, const uint16_t* L1, const uint16_t* L2,
+                            int64_t N, int64_t K, int r, float* R) {
+    if (N < 0 || K <= 0 || r < 0 || (r > 0 && (L1 == 0 || L2 == 0))) return ORACLE_ERR_ARG;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            double p = 0.0;
+            for (int j = 0; j < r; ++j) {
+                const double prod = bf16_value(L1[k * r + j]) * bf16_value(L2[(int64_t)j * N + n]);
+                p = p + prod;
+            }
+            const double d = (double)W[n * K + k] - p;
+            R[n * K + k] = (float)d;
+        }
+    }
+    return ORACLE_OK;
+}

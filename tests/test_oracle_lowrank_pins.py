@@ -62,3 +62,71 @@ def test_bf16_storage_is_round_to_nearest_even():
     exact = x32.astype(np.float64) == x
     ref = torch.from_numpy(x32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     np.testing.assert_array_equal(bits[exact], ref[exact])
+
+
+def test_bf16_rounding_of_fp64_values_is_nearest_with_ties_to_even():
+    """fp64 values that fp32 cannot hold (where rounding through fp32 first
+    could differ): the chosen bf16 is at least as near as both neighbours,
+    and an exact midpoint goes to the even significand."""
+    g = np.random.default_rng(8)
+    x = g.standard_normal(20000) * np.exp(g.uniform(-30, 30, 20000))
+    # exact midpoints between bf16 neighbours, and values just off them
+    base = (g.integers(128, 256, 2000) * 2.0 ** g.integers(-20, 20, 2000)).astype(np.float64)
+    ulp = 2.0 ** (np.floor(np.log2(base)) - 7)
+    mids = base + ulp / 2
+    x = np.concatenate([x, mids, -mids, mids + ulp * 2.0 ** -30, mids - ulp * 2.0 ** -30])
+    bits = oracle._bf16_rne_bits(x)
+    v = oracle._bf16_value(bits)
+    up = oracle._bf16_value((bits.astype(np.int64) + 1).astype(np.uint16))
+    dn = oracle._bf16_value((bits.astype(np.int64) - 1).astype(np.uint16))
+    d0, d1, d2 = np.abs(x - v), np.abs(x - up), np.abs(x - dn)
+    assert np.all(d0 <= d1) and np.all(d0 <= d2)
+    tie = (d0 == d1) | (d0 == d2)
+    assert tie.sum() >= 4000
+    assert np.all(bits[tie] % 2 == 0)
+    assert np.all(np.sign(v[x != 0]) == np.sign(x[x != 0]))
+
+
+def _bf16_of(x):
+    return oracle._bf16_rne_bits(np.asarray(x, np.float64))
+
+
+def test_residual_with_zero_factors_is_w():
+    g = np.random.default_rng(11)
+    W = g.standard_normal((37, 24)).astype(np.float32)
+    R = oracle.lowrank_residual(W, np.zeros((24, 8), np.uint16), np.zeros((8, 37), np.uint16))
+    np.testing.assert_array_equal(R, W)
+
+
+def test_residual_equals_fp64_matmul_when_every_sum_is_exact():
+    """Small-integer factors and weights: every product and partial sum is an
+    exact integer, so the result must equal numpy's fp64 matmul bit for bit,
+    whatever order it sums in.  N != K != r, so a transposed or swapped index
+    changes the answer."""
+    g = np.random.default_rng(12)
+    N, K, r = 23, 17, 5
+    L1 = g.integers(-8, 9, (K, r)).astype(np.float64)
+    L2 = g.integers(-8, 9, (r, N)).astype(np.float64)
+    W = g.integers(-500, 501, (N, K)).astype(np.float32)
+    R = oracle.lowrank_residual(W, _bf16_of(L1), _bf16_of(L2))
+    np.testing.assert_array_equal(R, (W.astype(np.float64) - (L1 @ L2).T).astype(np.float32))
+
+
+def test_residual_rounds_once_to_fp32():
+    """W - p with p exact in fp64 but W - p not representable in fp32: one
+    rounding of the exact difference (not of an fp32 product)."""
+    W = np.array([[1.0]], np.float32)
+    L1 = _bf16_of([[2.0 ** -30]])
+    L2 = _bf16_of([[1.0 + 2.0 ** -7]])
+    R = oracle.lowrank_residual(W, L1, L2)
+    exact = 1.0 - 2.0 ** -30 * (1.0 + 2.0 ** -7)
+    assert R[0, 0] == np.float32(exact)
+    assert R[0, 0] == np.float32(1.0)  # the difference is far below fp32's half ulp of 1
+
+
+def test_split_residual_is_the_split_formula():
+    g = np.random.default_rng(13)
+    W = g.standard_normal((40, 30)).astype(np.float32)
+    out = oracle.lowrank_split(W, 6)
+    R = oracle.lowrank_residual(W, out["L1_bits"], out["L2_bits"])
+    np.testing.assert_allclose(R, out["R"], rtol=0, atol=1e-6)

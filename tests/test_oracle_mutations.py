@@ -12,6 +12,7 @@ import pytest
 
 import oracle
 import tests.test_oracle_ext_pins as ext
+import tests.test_oracle_lowrank_pins as lr
 import tests.test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "wlq_oracle.c")
@@ -31,6 +32,11 @@ MUTATIONS = {
     "sixteen_bit_scale_kept_fp32": ("if (scale_dtype == 0) s = (double)(float)qd;",
                                     "if (scale_dtype >= 0) s = (double)(float)qd;"),
     "fp8_max_off": ("const float s = (float)(a / 448.0);", "const float s = (float)(a / 480.0);"),
+    "residual_l1_transposed": ("bf16_value(L1[k * r + j]) * bf16_value(L2[(int64_t)j * N + n]);",
+                               "bf16_value(L1[(int64_t)j * K + k]) * bf16_value(L2[(int64_t)j * N + n]);"),
+    "residual_last_rank_dropped": ("for (int j = 0; j < r; ++j) {\n                const double prod",
+                                   "for (int j = 0; j < r - 1; ++j) {\n                const double prod"),
+    "residual_sign": ("const double d = (double)W[n * K + k] - p;", "const double d = (double)W[n * K + k] + p;"),
 }
 
 PIN_TESTS = [
@@ -47,6 +53,7 @@ PIN_TESTS = [
     lambda: ext.test_codes_are_the_brute_force_nearest_with_the_stored_scale(3, oracle.SCALE_BF16),
     lambda: ext.test_fp8_codes_are_the_nearest_e4m3_ties_to_even_saturated(),
     lambda: ext.test_fp8_codes_match_torch_e4m3fn_conversion(),
+    lambda: lr.test_residual_equals_fp64_matmul_when_every_sum_is_exact(),
 ]
 
 

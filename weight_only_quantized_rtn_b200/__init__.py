@@ -24,9 +24,10 @@ STATUS_NAMES = {
     ERR_NONFINITE: "WLQ_ERR_NONFINITE", ERR_WORKSPACE: "WLQ_ERR_WORKSPACE",
     ERR_TIMEOUT: "WLQ_ERR_TIMEOUT", ERR_CUDA: "WLQ_ERR_CUDA",
 }
-EXPORTS = ("wlq_quantize", "wlq_packed_bytes", "wlq_pack", "wlq_unpack", "wlq_linear_workspace",
-           "wlq_linear", "wlq_linear_noalloc", "wlq_get_status", "wlq_probe_wait_timeout", "wlq_set_grid_limit",
-           "wlq_last_error", "wlq_version")
+EXPORTS = ("wlq_quantize", "wlq_quantize_pack", "wlq_quantize_ex", "wlq_quantize_fp8", "wlq_packed_bytes",
+           "wlq_pack", "wlq_unpack", "wlq_linear_workspace", "wlq_linear", "wlq_linear_noalloc",
+           "wlq_lowrank_workspace", "wlq_lowrank_split", "wlq_lowrank_residual", "wlq_get_status",
+           "wlq_probe_wait_timeout", "wlq_set_grid_limit", "wlq_last_error", "wlq_version")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("libwlq.so is not built; run `python -m weight_only_quantized_rtn_b200._build`")
@@ -45,14 +46,18 @@ lib.wlq_linear_workspace.argtypes = [_i64, _i64, _i64, _i32, _i32, _i32]
 lib.wlq_linear_workspace.restype = _sz
 lib.wlq_linear.argtypes = [_vp, _i64, _vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _sz, _vp]
 lib.wlq_linear_noalloc.argtypes = [_vp, _i64, _vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _vp]
+lib.wlq_lowrank_workspace.argtypes = [_i64, _i64, _i32, _i32]
+lib.wlq_lowrank_workspace.restype = _sz
+lib.wlq_lowrank_split.argtypes = [_vp, _i64, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+lib.wlq_lowrank_residual.argtypes = [_vp, _vp, _vp, _i64, _i64, _i32, _vp, _vp]
 lib.wlq_get_status.argtypes = [_vp]
 lib.wlq_probe_wait_timeout.argtypes = [_u64, _vp]
 lib.wlq_set_grid_limit.argtypes = [_i32]
 lib.wlq_set_grid_limit.restype = None
 lib.wlq_last_error.restype = ctypes.c_char_p
 lib.wlq_version.restype = ctypes.c_char_p
-for _f in ("wlq_quantize", "wlq_quantize_pack", "wlq_quantize_ex", "wlq_quantize_fp8", "wlq_pack", "wlq_unpack", "wlq_linear", "wlq_linear_noalloc", "wlq_get_status",
-           "wlq_probe_wait_timeout"):
+for _f in ("wlq_quantize", "wlq_quantize_pack", "wlq_quantize_ex", "wlq_quantize_fp8", "wlq_pack", "wlq_unpack", "wlq_linear",
+           "wlq_linear_noalloc", "wlq_lowrank_split", "wlq_lowrank_residual", "wlq_get_status", "wlq_probe_wait_timeout"):
     getattr(lib, _f).restype = ctypes.c_int
 
 
@@ -196,6 +201,34 @@ def linear_noalloc_into(y, x, packed, N, K, bits, group, bias=None, L1=None, L2=
     _check(lib.wlq_linear_noalloc(_ptr(x), M, _ptr(packed), N, K, bits, group, _ptr(bias), _ptr(L1), _ptr(L2), r,
                                   _ptr(y), out, _stream(stream)))
     return y
+
+
+def lowrank_split(W: torch.Tensor, r: int, omega: torch.Tensor, power_iters: int = 2, stream=None):
+    """Top-r split of W's transpose for the low-rank branch: fp32 W [N, K] and a
+    caller-drawn test matrix omega fp32 [N, l] -> (L1 bf16 [K, r], L2 bf16
+    [r, N], sigma fp32 [r])."""
+    assert W.dtype == torch.float32 and W.is_cuda and W.is_contiguous()
+    N, K = W.shape
+    l = omega.shape[1]
+    L1 = torch.empty((K, r), dtype=torch.bfloat16, device=W.device)
+    L2 = torch.empty((r, N), dtype=torch.bfloat16, device=W.device)
+    sigma = torch.empty(r, dtype=torch.float32, device=W.device)
+    n = int(lib.wlq_lowrank_workspace(N, K, r, l))
+    if n == 0:
+        raise WlqError(ERR_SHAPE, "no low-rank split for N=%d K=%d r=%d l=%d" % (N, K, r, l))
+    ws = torch.empty(n, dtype=torch.uint8, device=W.device)
+    _check(lib.wlq_lowrank_split(_ptr(W), N, K, r, l, power_iters, _ptr(omega), _ptr(L1), _ptr(L2), _ptr(sigma),
+                                 _ptr(ws), n, _stream(stream)))
+    return L1, L2, sigma
+
+
+def lowrank_residual(W: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor, stream=None) -> torch.Tensor:
+    """R = fp32(W - (L1 L2)^T), the part left for quantization."""
+    N, K = W.shape
+    r = L1.shape[1]
+    R = torch.empty_like(W)
+    _check(lib.wlq_lowrank_residual(_ptr(W), _ptr(L1), _ptr(L2), N, K, r, _ptr(R), _stream(stream)))
+    return R
 
 
 def get_status(stream=None) -> int:

@@ -16,8 +16,11 @@
 //   int8, per channel : A = bf16(q) exactly (|q| <= 127), rowf[n] = s[n], xs = 1
 //   int4, gs 64 / 16  : A = fp16(q * fp16(s 2^e_n)), rowf[n] = 2^-e_n,
 //                       B = x16 = fp16(x 2^f_m), xs[m] = 2^-f_m
-//   low rank          : a second TMEM accumulator gets [Th|Tl] [L2^T|L2^T]^T
-//                       (one MMA K-step per 64 of 2r, bf16, both from smem)
+//   low rank          : the same accumulator first gets [T'h|T'l|T'h] [L2'h|
+//                       L2'h|L2'l]^T with T' = T / xs, L2' = L2 / rowf (bf16
+//                       MMAs from shared memory, one K-step per 64 of 3r; the
+//                       operands come pre-divided, so the epilogue's rowf xs
+//                       scaling restores them), ahead of the tile's K loop
 //
 // CTA pairs (large M): two CTAs of a cluster share each MMA (cta_group::2),
 // M = 256 channels (128 per CTA, each dequantising its own rows into its own
@@ -69,6 +72,7 @@ constexpr int GEMM_THREADS = (WARP_MMA + 1) * 32;
 constexpr uint32_t A_STAGE_COLS = 32;  // 128 lanes x 64 16-bit values
 constexpr int MAX_STAGES = 20;  // ring depth cap (barrier arrays are sized for it)
 constexpr uint32_t LR_TILE_A_BYTES = 128 * 128;  // 128 rows x 64 bf16
+constexpr int MAX_LR_KB = 3;  // low-rank K blocks (3r <= 192), each with its own buffer
 constexpr uint64_t DRAIN_TIMEOUT_NS = 200ull * 1000 * 1000;
 constexpr int MAX_SPLITS = 8;
 constexpr int MAX_KS = 4;  // 64-wide K blocks per ring slot, at most
@@ -135,8 +139,7 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int g, int ra
 struct Smem {
     uint8_t* x;      // stages x xstage_bytes
     uint8_t* w;      // stages x wstage_bytes
-    uint8_t* lrA;    // 16 KB
-    uint8_t* lrB;    // xsub_bytes
+    uint8_t* lr;     // lr_kb buffers: A (16 KB: L2'' for 128 channels) then B (xsub_bytes: T'' rows)
     float* red;      // split partial [128][BN + 4] fp32 (S > 1)
     uint8_t* stage;  // unsplit: per epilogue warp, a 16-token x 32-channel transpose buffer
     uint64_t* full;    // slot loaded (TMA)
@@ -146,8 +149,9 @@ struct Smem {
     uint64_t* xfull;   // resident x: the CTA's x rows landed
     uint64_t* accfull;
     uint64_t* accempty;
-    uint64_t* lrfull;
-    uint64_t* lrempty;
+    uint64_t* lrfull;   // [MAX_LR_KB] low-rank block landed (TMA)
+    uint64_t* lrempty;  // [MAX_LR_KB] low-rank block consumed (MMA commit)
+    uint64_t* lrpeer;   // [MAX_LR_KB] pairs: the second CTA's half of the block landed
     uint64_t* drain;
     uint64_t* redw;   // local: every epilogue warp wrote its part of red
     uint64_t* readw;  // local: every epilogue warp finished reading the cluster's partials
@@ -331,12 +335,26 @@ __device__ void producer_role(const GemmArgs& a, const CUtensorMap* tm_x, const 
                               const CUtensorMap* tm_l2, const Smem& s, const Sched& sc) {
     // in a pair each CTA stages its half of the tile's tokens
     const int row0 = PAIR ? (sc.rank & 1) * (a.BN >> 1) : 0;
-    int it = 0, lrit = 0;
+    int it = 0, lru = 0;  // lru: units with a low-rank term so far (each flips every LR buffer once)
     Ring r;
     bool ok = true;
     bool x_issued = false;
     TileCoord c;
     for (int u = 0; ok && unit_coord<PAIR>(a, sc, u, c); ++u) {
+        // the unit's low-rank blocks first (the MMA consumes them ahead of its K
+        // loop); each has its own buffer, so they are fetched while the
+        // previous unit's K loop runs
+        if (a.lr && c.sp == 0) {
+            for (int lk = 0; lk < a.lr_kb; ++lk) {
+                if (!wait_or_abort(&s.lrempty[lk], (lru & 1) ^ 1, a, s.abort_flag)) { ok = false; break; }
+                uint8_t* buf = s.lr + static_cast<size_t>(lk) * (LR_TILE_A_BYTES + a.xsub_bytes);
+                mbar_arrive_expect_tx(&s.lrfull[lk], LR_TILE_A_BYTES + a.xsub_bytes);
+                tma_load_2d(buf, tm_l2, &s.lrfull[lk], lk * 64, c.nt * 128);
+                tma_load_2d(buf + LR_TILE_A_BYTES, tm_t, &s.lrfull[lk], lk * 64, c.mt * a.BN + row0);
+            }
+            if (!ok) break;
+            ++lru;
+        }
         if (XRES && !x_issued) {
             // resident x: every tile of this CTA has the same tokens (one token
             // tile) and the same K range (its split), so x is loaded once
@@ -365,22 +383,14 @@ __device__ void producer_role(const GemmArgs& a, const CUtensorMap* tm_x, const 
             ++it;
             r.next(a.stages);
         }
-        if (ok && a.lr && c.sp == 0) {
-            for (int lk = 0; lk < a.lr_kb; ++lk) {
-                if (!wait_or_abort(s.lrempty, (lrit & 1) ^ 1, a, s.abort_flag)) { ok = false; break; }
-                mbar_arrive_expect_tx(s.lrfull, LR_TILE_A_BYTES + a.xsub_bytes);
-                tma_load_2d(s.lrA, tm_l2, s.lrfull, lk * 64, c.nt * 128);
-                tma_load_2d(s.lrB, tm_t, s.lrfull, lk * 64, c.mt * a.BN);
-                ++lrit;
-            }
-        }
     }
     if (!ok) {
         // let every copy already issued land before the CTA can exit
         for (int i = max(0, it - a.stages); i < it; ++i)
             mbar_wait(&s.full[i % a.stages], (i / a.stages) & 1, DRAIN_TIMEOUT_NS);
         if (XRES && x_issued) mbar_wait(s.xfull, 0, DRAIN_TIMEOUT_NS);
-        if (lrit > 0) mbar_wait(s.lrfull, (lrit - 1) & 1, DRAIN_TIMEOUT_NS);
+        if (lru > 0)
+            for (int lk = 0; lk < a.lr_kb; ++lk) mbar_wait(&s.lrfull[lk], (lru - 1) & 1, DRAIN_TIMEOUT_NS);
     }
 }
 
@@ -487,9 +497,9 @@ __device__ void dequant_role(const GemmArgs& a, uint32_t tmem, const Smem& s, co
 template <int FMT, bool PAIR, bool XRES>
 __device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const Sched& sc) {
     const uint32_t idesc = idesc_f16(FMT == FMT_W8 ? 1u : 0u, PAIR ? 256 : 128, a.BN);
-    // pair commits signal the same barrier in both CTAs
-    const uint32_t idesc_lr = idesc_f16(1u, 128, a.BN);
-    int lrit = 0, tc = 0;
+    // the low-rank blocks are bf16 on both sides
+    const uint32_t idesc_lr = idesc_f16(1u, PAIR ? 256 : 128, a.BN);
+    int lru = 0, tc = 0;
     Ring r;
     bool ok = true;
     if (XRES && !wait_or_abort(s.xfull, 0, a, s.abort_flag)) ok = false;
@@ -499,6 +509,30 @@ __device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const 
         if (!wait_or_abort(&s.accempty[ab], ((tc / a.acc_bufs) & 1) ^ 1, a, s.abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem + a.acc_col0 + ab * a.BN;
+        // low-rank blocks first, into the same accumulator (K split 0 only);
+        // in a pair both CTAs' halves must have landed (the second CTA's MMA
+        // warp forwards its arrival)
+        const bool has_lr = a.lr && c.sp == 0;
+        if (has_lr) {
+            for (int lk = 0; lk < a.lr_kb; ++lk) {
+                if (!wait_or_abort(&s.lrfull[lk], lru & 1, a, s.abort_flag)) { ok = false; break; }
+                if (PAIR && !wait_or_abort(&s.lrpeer[lk], lru & 1, a, s.abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint8_t* buf = s.lr + static_cast<size_t>(lk) * (LR_TILE_A_BYTES + a.xsub_bytes);
+                const uint64_t adesc = smem_desc_sw128(smem_u32(buf));
+                const uint64_t bdesc = smem_desc_sw128(smem_u32(buf + LR_TILE_A_BYTES));
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint32_t acc = (lk > 0 || kk > 0) ? 1u : 0u;
+                    if constexpr (PAIR) mma_ss_pair(d, adesc + 2 * kk, bdesc + 2 * kk, idesc_lr, acc);
+                    else mma_ss(d, adesc + 2 * kk, bdesc + 2 * kk, idesc_lr, acc);
+                }
+                if constexpr (PAIR) mma_commit_pair_both(&s.lrempty[lk], sc.rank);
+                else mma_commit(&s.lrempty[lk]);
+            }
+            if (!ok) break;
+            ++lru;
+        }
         for (int kb = c.kb0; kb < c.kb1 && ok; kb += a.ks, r.next(XRES ? a.astages : a.stages)) {
             const int nkb = min(a.ks, c.kb1 - kb);
             const int st = r.slot;  // resident x: the A-stage ring's slot
@@ -513,7 +547,7 @@ __device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const 
                 const uint64_t bdesc = smem_desc_sw128(smem_u32(xt));
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint32_t acc = (kb > c.kb0 || j > 0 || kk > 0) ? 1u : 0u;
+                    const uint32_t acc = (has_lr || kb > c.kb0 || j > 0 || kk > 0) ? 1u : 0u;
                     if constexpr (PAIR) mma_ts_pair(d, acol + j * A_STAGE_COLS + kk * 8, bdesc + 2 * kk, idesc, acc);
                     else mma_ts(d, acol + j * A_STAGE_COLS + kk * 8, bdesc + 2 * kk, idesc, acc);
                 }
@@ -522,20 +556,6 @@ __device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const 
             else mma_commit(XRES ? &s.aempty[st] : &s.empty[st]);
         }
         if (!ok) break;
-        if (a.lr && c.sp == 0) {
-            const uint32_t dl = tmem + a.lr_col0 + ab * a.BN;
-            for (int lk = 0; lk < a.lr_kb; ++lk, ++lrit) {
-                if (!wait_or_abort(s.lrfull, lrit & 1, a, s.abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                const uint64_t adesc = smem_desc_sw128(smem_u32(s.lrA));
-                const uint64_t bdesc = smem_desc_sw128(smem_u32(s.lrB));
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ss(dl, adesc + 2 * kk, bdesc + 2 * kk, idesc_lr, (lk > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(s.lrempty);
-            }
-            if (!ok) break;
-        }
         if constexpr (PAIR) mma_commit_pair_both(&s.accfull[ab], sc.rank);
         else mma_commit(&s.accfull[ab]);
     }
@@ -543,6 +563,32 @@ __device__ void mma_role(const GemmArgs& a, uint32_t tmem, const Smem& s, const 
     if constexpr (PAIR) mma_commit_pair(s.drain);
     else mma_commit(s.drain);
     mbar_wait(s.drain, 0, DRAIN_TIMEOUT_NS);
+}
+
+// Second CTA of a pair, low rank: its half of every low-rank block lands on
+// its own barrier; the first CTA's MMA thread (which reads both halves) is
+// told by one remote arrive per block, after this thread saw it land.
+template <bool PAIR>
+__device__ void lr_forward_role(const GemmArgs& a, const Smem& s, const Sched& sc) {
+    const uint32_t leader = static_cast<uint32_t>(sc.rank & ~1);
+    int lru = 0;
+    TileCoord c;
+    for (int u = 0; unit_coord<PAIR>(a, sc, u, c); ++u) {
+        if (!(a.lr && c.sp == 0)) continue;
+        for (int lk = 0; lk < a.lr_kb; ++lk) {
+            if (!wait_or_abort(&s.lrfull[lk], lru & 1, a, s.abort_flag)) return;
+            mbar_arrive_peer(mapa_shared(smem_u32(&s.lrpeer[lk]), leader));
+        }
+        ++lru;
+    }
+}
+
+// The factor the epilogue scales a channel's accumulator by.  With a
+// low-rank term, a channel whose row factor is 0 (an all-zero weight row:
+// its main sum is 0) has its low-rank operand left unscaled, so it is scaled
+// by 1 here.
+__device__ __forceinline__ float epi_row_factor(const GemmArgs& a, float rf) {
+    return (a.lr && rf == 0.0f) ? 1.0f : rf;
 }
 
 __device__ __forceinline__ void store_y(const GemmArgs& a, int m, int n, float v) {
@@ -640,7 +686,7 @@ __device__ void crew_split_epilogue(const GemmArgs& a, uint32_t tmem, const Smem
     if (!warp_wait_or_abort(&s.accfull[ab], (u / a.acc_bufs) & 1, a, s.abort_flag, false, !epi)) return;
     tc_fence_after();
     const int n = c.nt * 128 + row;
-    const float rf = n < a.N ? a.rowf[n] : 0.0f;
+    const float rf = n < a.N ? epi_row_factor(a, a.rowf[n]) : 0.0f;
     const int m0 = c.mt * a.BN;
     for (int cc = k; cc < a.BN / 16; cc += 3) {
         uint32_t v[16];
@@ -717,9 +763,8 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
         tc_fence_after();
         const int n = c.nt * 128 + row;
         const bool n_ok = n < a.N;
-        const float rf = n_ok ? a.rowf[n] : 0.0f;
+        const float rf = n_ok ? epi_row_factor(a, a.rowf[n]) : 0.0f;
         const float bn = (a.bias && n_ok) ? bf16_to_f32(a.bias[n]) : 0.0f;
-        const bool has_lr = a.lr && c.sp == 0;
         const int m0 = c.mt * a.BN;
         // the partial buffer is reused once every CTA of the cluster has read it
         if (split && tc > 0 && !warp_wait_or_abort(s.freed, (tc - 1) & 1, a, s.abort_flag, true)) return;
@@ -732,7 +777,6 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
                 const int m = m0 + cc * 16 + j;
                 val[j] = __uint_as_float(v[j]) * rf;
                 if constexpr (FMT != FMT_W8) val[j] *= (m < a.M) ? a.xs[m] : 0.0f;
-                if (has_lr) val[j] += __uint_as_float(lv[j]);
             }
             if (split) {
                 // token-major partial: consecutive lanes write consecutive channels
@@ -793,16 +837,7 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
             }
         };
         const int nch = a.BN / 16;
-        if (has_lr) {
-            for (int cc = 0; cc < nch; ++cc) {
-                uint32_t v[16], lv[16];
-                tmem_ld16(tbase + a.acc_col0 + ab * a.BN + cc * 16, v);
-                tmem_ld16(tbase + a.lr_col0 + ab * a.BN + cc * 16, lv);
-                tmem_wait_ld_pin(v);
-                reg_pin(lv);
-                emit(v, lv, cc);
-            }
-        } else if (!split && a.vec_out && !a.y_f32 && nch % EPI_CHUNKS == 0) {
+        if (!split && a.vec_out && !a.y_f32 && nch % EPI_CHUNKS == 0) {
             // bf16 output, the common case: two 16-token chunks per step (their
             // conversions and stores are independent, so one warp per SMSP
             // keeps more in flight)
@@ -810,7 +845,9 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
             const int nb = c.nt * 128 + q * 32;
             uint8_t* stg = s.stage + (warp - WARP_EPI0) * EPI_STAGE_BYTES;
             const bool odd = lane & 1;
-            auto emitn = [&](const uint32_t (&vv)[EPI_CHUNKS][16], int cc) {
+            // int4: the x16 row factors of the step's 32 tokens, one per lane,
+            // read once (before any store of the step) and passed by shuffle
+            auto emitn = [&](const uint32_t (&vv)[EPI_CHUNKS][16], int cc, float xv) {
 #pragma unroll
                 for (int k = 0; k < EPI_CHUNKS; ++k) {
                     const uint32_t* v = vv[k];
@@ -820,8 +857,15 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
                     // odd lanes 8-15; rows 8-15 sit one row further on
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        const float lo_t = __uint_as_float(v[j]) * rf + bn;
-                        const float hi_t = __uint_as_float(v[j + 8]) * rf + bn;
+                        float lo_t = __uint_as_float(v[j]) * rf;
+                        float hi_t = __uint_as_float(v[j + 8]) * rf;
+                        if constexpr (FMT != FMT_W8) {
+                            // int4: undo the x16 row scaling of tokens j and j + 8
+                            lo_t *= __shfl_sync(0xffffffffu, xv, k * 16 + j);
+                            hi_t *= __shfl_sync(0xffffffffu, xv, k * 16 + j + 8);
+                        }
+                        lo_t += bn;
+                        hi_t += bn;
                         const float mine = odd ? hi_t : lo_t;
                         const float other = __shfl_xor_sync(0xffffffffu, odd ? lo_t : hi_t, 1);
                         const __nv_bfloat162 pr = odd ? __floats2bfloat162_rn(other, mine)
@@ -845,14 +889,20 @@ __device__ void epilogue_role(const GemmArgs& a, uint32_t tmem, const Smem& s, c
                 }
                 __syncwarp();
             };
+            static_assert(EPI_CHUNKS * 16 == 32, "one row factor per lane");
             for (int cc = 0; cc < nch; cc += EPI_CHUNKS) {
+                float xv = 1.0f;
+                if constexpr (FMT != FMT_W8) {
+                    const int mx = m0 + cc * 16 + lane;
+                    xv = (mx < a.M) ? __ldg(a.xs + mx) : 0.0f;
+                }
                 uint32_t vv[EPI_CHUNKS][16];
 #pragma unroll
                 for (int k = 0; k < EPI_CHUNKS; ++k) tmem_ld16(col + (cc + k) * 16, vv[k]);
                 tmem_wait_ld_pin(vv[0]);
 #pragma unroll
                 for (int k = 1; k < EPI_CHUNKS; ++k) reg_pin(vv[k]);
-                emitn(vv, cc);
+                emitn(vv, cc, xv);
             }
         } else {
             // two register sets: chunk cc + 1 is read from tensor memory while
@@ -918,9 +968,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     Smem s;
     s.x = base;  // resident x: kbps x sub-tiles; otherwise stages x xstage_bytes
     s.w = s.x + (XRES ? static_cast<size_t>(a.kbps) * a.xsub_bytes : static_cast<size_t>(a.stages) * a.xstage_bytes);
-    s.lrA = s.w + static_cast<size_t>(a.stages) * a.wstage_bytes;
-    s.lrB = s.lrA + (a.lr ? LR_TILE_A_BYTES : 0);
-    s.red = reinterpret_cast<float*>(s.lrB + (a.lr ? a.xsub_bytes : 0));
+    s.lr = s.w + static_cast<size_t>(a.stages) * a.wstage_bytes;
+    s.red = reinterpret_cast<float*>(s.lr + (a.lr ? static_cast<size_t>(a.lr_kb) * (LR_TILE_A_BYTES + a.xsub_bytes) : 0));
     s.stage = reinterpret_cast<uint8_t*>(s.red) + a.red_bytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(s.stage + a.stage_bytes);
     // One tile per cluster: once the tile's accumulator is complete no MMA,
@@ -935,8 +984,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     s.accfull = s.xfull + 1;
     s.accempty = s.accfull + 2;
     s.lrfull = s.accempty + 2;
-    s.lrempty = s.lrfull + 1;
-    s.drain = s.lrempty + 1;
+    s.lrempty = s.lrfull + MAX_LR_KB;
+    s.lrpeer = s.lrempty + MAX_LR_KB;
+    s.drain = s.lrpeer + MAX_LR_KB;
     s.redw = s.drain + 1;
     s.readw = s.redw + 1;
     s.ready = s.readw + 1;
@@ -961,8 +1011,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
             mbar_init(&s.accfull[i], 1);
             mbar_init(&s.accempty[i], PAIR ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS);
         }
-        mbar_init(s.lrfull, 1);
-        mbar_init(s.lrempty, 1);
+        for (int i = 0; i < MAX_LR_KB; ++i) {
+            mbar_init(&s.lrfull[i], 1);
+            mbar_init(&s.lrempty[i], 1);
+            mbar_init(&s.lrpeer[i], 1);
+        }
         mbar_init(s.drain, 1);
         mbar_init(s.redw, a.red_alias ? CREW_WARPS : NUM_EPI_WARPS);
         mbar_init(s.readw, a.red_alias ? CREW_WARPS : NUM_EPI_WARPS);
@@ -1002,6 +1055,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
         if (lane == 0) producer_role<PAIR, XRES>(a, &tm_x, &tm_t, &tm_l2, s, sc);
     } else if (lane == 0 && (!PAIR || (sc.rank & 1) == 0)) {
         mma_role<FMT, PAIR, XRES>(a, tmem, s, sc);
+    } else if (PAIR && lane == 0 && a.lr) {
+        lr_forward_role<PAIR>(a, s, sc);
     }
 
     tc_fence_before();

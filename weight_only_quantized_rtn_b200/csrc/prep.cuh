@@ -7,14 +7,21 @@
 //    significand fits fp16's 11 bits, so x16 * 2^-f_m == x except for values
 //    below 2^-23 of the row maximum.  xs[m] = 2^-f_m is undone in the epilogue.
 //  * low-rank branch ("Nunchaku Lite", why it matters: a 16-bit low-rank
-//    correction): T = x L1 in fp32 on the tensor cores, stored as a bf16
-//    pair T = Th + Tl (hi, lo) so the second GEMM T L2 sees T to ~2^-17;
-//    L2 is transposed into a K-major [N_pad, 2r] operand [L2^T | L2^T] so
-//    that one extra MMA K-step computes Th L2 + Tl L2.
+//    correction), folded into the GEMM's own accumulator.  The GEMM's
+//    epilogue multiplies its accumulator by rowf[n] xs[m], so the branch is
+//    fed pre-divided by those factors: T' = (x L1)[m] / xs[m] (a power of
+//    two: exact) and L2' = L2[n] / rowf[n] (exact for int4, whose row
+//    factors are powers of two; one fp32 rounding for int8's channel scales).
+//    Each is carried as a bf16 pair hi + lo (~2^-17 relative) and the GEMM
+//    adds [T'h | T'l | T'h] [L2'h | L2'h | L2'l]^T = T'L2' - T'l L2'l over 3r
+//    extra inputs (bf16 MMAs into the same fp32 accumulator).  A row whose
+//    factor is 0 (an all-zero weight row) keeps L2 unscaled, and the epilogue
+//    then scales that row by 1 instead.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include "ptx.cuh"
 
 namespace wlq {
 
@@ -62,6 +69,76 @@ __global__ void __launch_bounds__(256) prep_x16_kernel(const uint16_t* __restric
     }
 }
 
+// The same conversion with one CTA per row (grid-stride over rows) and the
+// row held in registers: PER 16-byte chunks per thread, K <= 8 * PER * THREADS.
+// Row maximum over bf16 magnitude bit patterns (NaN ignored, as fmaxf does;
+// an infinity leaves the row unscaled), then the same ldexpf / round to
+// nearest fp16 per element as prep_x16_kernel: the outputs are identical.
+// MINB > 1 caps the registers (65536 / (threads * MINB) per thread) so that a
+// CTA of this kernel can run beside a streaming CTA on the same SM.
+template <int PER, int THREADS, int MINB>
+__global__ void __launch_bounds__(THREADS, MINB) prep_x16_rows_kernel(const uint16_t* __restrict__ x, int M, int K,
+                                                                     __half* __restrict__ x16, float* __restrict__ xs) {
+    grid_dependency_sync();
+    __shared__ uint32_t wmax[32];
+    __shared__ int fsh;
+    const int K8 = K / 8;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int m = blockIdx.x; m < M; m += gridDim.x) {
+        const uint4* row = reinterpret_cast<const uint4*>(x + static_cast<size_t>(m) * K);
+        uint4 v[PER];
+        uint32_t amax = 0;
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const int i = threadIdx.x + j * blockDim.x;
+            v[j] = (i < K8) ? __ldg(row + i) : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint32_t lo = w[e] & 0x7FFFu, hi = (w[e] >> 16) & 0x7FFFu;
+                amax = max(amax, lo > 0x7F80u ? 0u : lo);  // a NaN does not count
+                amax = max(amax, hi > 0x7F80u ? 0u : hi);
+            }
+        }
+        for (int off = 16; off > 0; off >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        if (lane == 0) wmax[warp] = amax;
+        __syncthreads();
+        if (warp == 0) {
+            uint32_t a = (lane < static_cast<int>((blockDim.x + 31) >> 5)) ? wmax[lane] : 0u;
+            for (int off = 16; off > 0; off >>= 1) a = max(a, __shfl_xor_sync(0xffffffffu, a, off));
+            if (lane == 0) {
+                const float fa = bf16_bits_to_f32(a);
+                int f = 0;
+                if (fa > 0.0f && isfinite(fa)) {
+                    int ex;
+                    frexpf(fa, &ex);  // fa in [2^(ex-1), 2^ex)
+                    f = 9 - ex;
+                }
+                fsh = f;
+                xs[m] = ldexpf(1.0f, -f);
+            }
+        }
+        __syncthreads();
+        const int f = fsh;
+        uint4* out = reinterpret_cast<uint4*>(x16 + static_cast<size_t>(m) * K);
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const int i = threadIdx.x + j * blockDim.x;
+            if (i >= K8) break;
+            const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const __half2 h = __floats2half2_rn(ldexpf(bf16_bits_to_f32(w[e] & 0xFFFFu), f),
+                                                    ldexpf(bf16_bits_to_f32(w[e] >> 16), f));
+                o[e] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            out[i] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        __syncthreads();  // wmax / fsh are rewritten for the next row
+    }
+}
+
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -80,83 +157,183 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-constexpr int LR_ROWS = 64;       // rows of x per CTA (16 per warp, 4 warps)
-constexpr int LR_KC = 64;         // K chunk
-constexpr int LR_PITCH = LR_KC + 8;  // smem row pitch in bf16 elements (144 bytes)
+constexpr int LR_ROWS = 64;          // rows of x per CTA (16 per warp, 4 warps)
+constexpr int LR_KC = 64;            // K chunk per pipeline stage
+constexpr int LR_STAGES = 3;         // cp.async pipeline depth
+constexpr int LR_XP = LR_KC + 8;     // x tile row pitch in bf16 elements (144 bytes: ldmatrix conflict-free)
+constexpr int LR_LP = 64 + 8;        // L1 tile row pitch in bf16 elements (r <= 64)
+constexpr int LR_MAX_SPLITS = 8;     // CTAs of a cluster splitting K
+constexpr uint32_t LR_STAGE_BYTES = (LR_ROWS * LR_XP + LR_KC * LR_LP) * 2u;
+__host__ __device__ constexpr size_t lr_t_smem_bytes() {
+    return 128 + static_cast<size_t>(LR_STAGES) * LR_STAGE_BYTES + static_cast<size_t>(LR_ROWS) * 64 * 4;
+}
 
-// T = x L1 -> Thl[m] = [Th(0..r) | Tl(0..r) | 0 ... ] with width W = lr_kb * 64.
-// r in {16, 32, 64}.  128 threads, one CTA per 64 rows.
+__device__ __forceinline__ void lr_cp16(uint32_t dst, const void* src, bool valid) {
+    // 16-byte asynchronous copy; an invalid source reads as zeros (src-size 0)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t (&r)[2], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+                 : "=r"(r[0]), "=r"(r[1])
+                 : "r"(addr));
+}
+
+// T' = (x L1) / xs -> Thl[m] = [T'h(0..r) | T'l(0..r) | T'h(0..r) | 0 ...] with
+// width W = lr_kb * 64, r in {16, 32, 64}; xs == null means 1.  CTA (q, i) of a cluster of S along x takes rows
+// 64 i..64 i + 63 over K split q (whole 64-wide chunks); its 4 warps each own
+// 16 rows and run m16n8k16 bf16 MMAs (fp32 accumulate) on x and L1 chunks
+// staged by a three-deep cp.async pipeline (L1 read K-major as stored and
+// turned by ldmatrix.trans).  The S partials are then added in split order
+// through distributed shared memory, CTA q taking rows 64/S q..+64/S, and
+// written as the bf16 pair hi = bf16(T), lo = bf16(T - hi).
 __global__ void __launch_bounds__(128) prep_lr_t_kernel(const uint16_t* __restrict__ x,
-                                                        const uint16_t* __restrict__ L1, int M, int K,
-                                                        int r, int W, uint16_t* __restrict__ thl) {
-    grid_dependency_sync();
-    __shared__ __align__(16) uint16_t xt[LR_ROWS * LR_PITCH];
-    __shared__ __align__(16) uint16_t lt[64 * LR_PITCH];  // [j][k]
+                                                        const uint16_t* __restrict__ L1, const float* __restrict__ xs,
+                                                        int M, int K, int r, int W, int S, int kc_per,
+                                                        uint16_t* __restrict__ thl) {
+    extern __shared__ uint8_t lr_smem_raw[];
+    uint8_t* base = lr_smem_raw + ((128u - (smem_u32(lr_smem_raw) & 127u)) & 127u);
+    uint16_t* stage0 = reinterpret_cast<uint16_t*>(base);
+    float* part = reinterpret_cast<float*>(base + LR_STAGES * LR_STAGE_BYTES);  // [64 rows][r]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int m0 = blockIdx.x * LR_ROWS;
+    const int q = (S > 1) ? static_cast<int>(cluster_ctarank()) : 0;
+    const int KC = (K + LR_KC - 1) / LR_KC;
+    const int c0 = q * kc_per, c1 = min(KC, c0 + kc_per);
+    const int nchunks = max(0, c1 - c0);
     const int ntile = r / 8;
-    float acc[8][4];
-    for (int t = 0; t < 8; ++t)
-        for (int e = 0; e < 4; ++e) acc[t][e] = 0.0f;
-    for (int k0 = 0; k0 < K; k0 += LR_KC) {
-        // x tile: 64 rows x 64 k, 8 elements per uint4
+    const int lchunks = r / 8;  // 16-byte pieces per L1 row
+    grid_dependency_sync();
+    // every CTA of a cluster shares blockIdx.y, so all take the same row tiles
+    for (int m0 = blockIdx.y * LR_ROWS; m0 < M; m0 += gridDim.y * LR_ROWS) {
+
+    auto issue = [&](int c, int st) {
+        uint16_t* xt = stage0 + st * (LR_STAGE_BYTES / 2);
+        uint16_t* lt = xt + LR_ROWS * LR_XP;
+        const int k0 = (c0 + c) * LR_KC;
         for (int idx = tid; idx < LR_ROWS * (LR_KC / 8); idx += 128) {
-            const int rr = idx / (LR_KC / 8), c8 = idx % (LR_KC / 8);
+            const int rr = idx >> 3, c8 = idx & 7;
             const int m = m0 + rr, k = k0 + c8 * 8;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (m < M && k < K) v = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(m) * K + k));
-            *reinterpret_cast<uint4*>(&xt[rr * LR_PITCH + c8 * 8]) = v;
+            const bool ok = m < M && k < K;
+            lr_cp16(smem_u32(xt + rr * LR_XP + c8 * 8), ok ? x + static_cast<size_t>(m) * K + k : x, ok);
         }
-        // L1 chunk transposed: lt[j][kk] = L1[k0 + kk][j]
-        for (int idx = tid; idx < LR_KC * r; idx += 128) {
-            const int kk = idx / r, j = idx % r;
+        for (int idx = tid; idx < LR_KC * lchunks; idx += 128) {
+            const int kk = idx / lchunks, j8 = idx % lchunks;
             const int k = k0 + kk;
-            lt[j * LR_PITCH + kk] = (k < K) ? L1[static_cast<size_t>(k) * r + j] : static_cast<uint16_t>(0);
+            const bool ok = k < K;
+            lr_cp16(smem_u32(lt + kk * LR_LP + j8 * 8), ok ? L1 + static_cast<size_t>(k) * r + j8 * 8 : L1, ok);
         }
-        __syncthreads();
+    };
+
+    float acc[8][4];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
+#pragma unroll
+    for (int st = 0; st < LR_STAGES - 1; ++st) {
+        if (st < nchunks) issue(st, st);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    for (int c = 0; c < nchunks; ++c) {
+        asm volatile("cp.async.wait_group %0;" ::"n"(LR_STAGES - 2) : "memory");
+        __syncthreads();  // chunk c has landed for every thread; chunk c - 1's stage is free
+        if (c + LR_STAGES - 1 < nchunks) issue(c + LR_STAGES - 1, (c + LR_STAGES - 1) % LR_STAGES);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        const uint16_t* xt = stage0 + (c % LR_STAGES) * (LR_STAGE_BYTES / 2);
+        const uint16_t* lt = xt + LR_ROWS * LR_XP;
+#pragma unroll
         for (int ks = 0; ks < LR_KC / 16; ++ks) {
             uint32_t a[4];
             const int arow = warp * 16 + (lane & 15);
-            ldsm_x4(a, static_cast<uint32_t>(__cvta_generic_to_shared(&xt[arow * LR_PITCH + ks * 16 + (lane >> 4) * 8])));
-            for (int t = 0; t < ntile; ++t) {
-                uint32_t b[2];
-                const int brow = t * 8 + (lane & 7);
-                ldsm_x2(b, static_cast<uint32_t>(__cvta_generic_to_shared(&lt[brow * LR_PITCH + ks * 16 + ((lane >> 3) & 1) * 8])));
-                mma_bf16_16816(acc[t], a, b);
+            ldsm_x4(a, smem_u32(xt + arow * LR_XP + ks * 16 + (lane >> 4) * 8));
+            // B fragment of n-tile t: rows k = 16 ks + {0..7} (lanes 0-7) and
+            // + {8..15} (lanes 8-15) of the K-major L1 tile, columns 8 t..8 t + 7
+            const int krow = ks * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                if (t < ntile) {
+                    uint32_t b[2];
+                    ldsm_x2_trans(b, smem_u32(lt + krow * LR_LP + t * 8));
+                    mma_bf16_16816(acc[t], a, b);
+                }
             }
         }
-        __syncthreads();
     }
-    // scatter: c0,c1 -> (row g, cols 2q, 2q+1); c2,c3 -> (row g+8, same cols)
-    const int g = lane >> 2, q = lane & 3;
-    for (int half = 0; half < 2; ++half) {
-        const int m = m0 + warp * 16 + g + 8 * half;
-        if (m >= M) continue;
-        uint16_t* out = thl + static_cast<size_t>(m) * W;
-        for (int t = 0; t < ntile; ++t)
-            for (int e = 0; e < 2; ++e) {
-                const int j = t * 8 + 2 * q + e;
-                const float T = acc[t][2 * half + e];
-                const __nv_bfloat16 hi = __float2bfloat16_rn(T);
-                const __nv_bfloat16 lo = __float2bfloat16_rn(T - __bfloat162float(hi));
-                out[j] = *reinterpret_cast<const uint16_t*>(&hi);
-                out[r + j] = *reinterpret_cast<const uint16_t*>(&lo);
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    // this CTA's partial: part[row][j]; c0,c1 -> (row g, cols 2q', 2q'+1), c2,c3 -> row g + 8
+    {
+        const int g = lane >> 2, qq = lane & 3;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            if (t < ntile) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int row = warp * 16 + g + 8 * h;
+                    part[row * r + t * 8 + 2 * qq] = acc[t][2 * h];
+                    part[row * r + t * 8 + 2 * qq + 1] = acc[t][2 * h + 1];
+                }
             }
-        for (int j = 2 * r + q; j < W; j += 4) out[j] = 0;
+        }
     }
+    if (S > 1) cluster_sync_all();
+    else __syncthreads();
+    // rows of this CTA's share, summed over the S partials in split order
+    const int rows_per = LR_ROWS / S;
+    for (int idx = tid; idx < rows_per * r; idx += 128) {
+        const int row = q * rows_per + idx / r, j = idx % r;
+        const uint32_t a0 = smem_u32(part + row * r + j);
+        float T = (S > 1) ? ld_dsmem_f32(mapa_shared(a0, 0)) : part[row * r + j];
+        for (int sp = 1; sp < S; ++sp) T += ld_dsmem_f32(mapa_shared(a0, static_cast<uint32_t>(sp)));
+        const int m = m0 + row;
+        if (m < M) {
+            if (xs) T /= xs[m];  // a power of two: exact
+            uint16_t* out = thl + static_cast<size_t>(m) * W;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(T);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(T - __bfloat162float(hi));
+            out[j] = *reinterpret_cast<const uint16_t*>(&hi);
+            out[r + j] = *reinterpret_cast<const uint16_t*>(&lo);
+            out[2 * r + j] = *reinterpret_cast<const uint16_t*>(&hi);
+            for (int jj = 3 * r + j; jj < W; jj += r) out[jj] = 0;
+        }
+    }
+    // no CTA may exit, or overwrite its partial, while another still reads it
+    if (S > 1) cluster_sync_all();
+    else __syncthreads();
+    }  // row tiles
 }
 
-// L2t[n][c] = L2[c mod r][n] for c < 2r, zero beyond 2r or N.
-__global__ void prep_lr_l2t_kernel(const uint16_t* __restrict__ L2, int N, int N_pad, int r, int W,
-                                   uint16_t* __restrict__ l2t) {
+// L2t[n] = [L2'h(0..r) | L2'h(0..r) | L2'l(0..r) | 0 ...] (width W) with
+// L2' = L2[., n] / rowf[n] (L2 itself where rowf[n] == 0), zero for n >= N.
+// One thread per (row n, 8 columns): the reads of L2 are coalesced across
+// consecutive n, each thread writes one 16-byte piece.
+__global__ void prep_lr_l2t_kernel(const uint16_t* __restrict__ L2, const float* __restrict__ rowf, int N,
+                                   int N_pad, int r, int W, uint16_t* __restrict__ l2t) {
     grid_dependency_sync();
-    const int64_t total = static_cast<int64_t>(N_pad) * W;
+    const int64_t total = static_cast<int64_t>(N_pad) * (W / 8);
     for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
          idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int n = static_cast<int>(idx / W), c = static_cast<int>(idx % W);
-        uint16_t v = 0;
-        if (n < N && c < 2 * r) v = L2[static_cast<size_t>(c % r) * N + n];
-        l2t[idx] = v;
+        const int n = static_cast<int>(idx % N_pad), c8 = static_cast<int>(idx / N_pad);
+        const float rf = (n < N) ? rowf[n] : 0.0f;
+
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            uint32_t h[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int c = c8 * 8 + 2 * e + u;
+                uint16_t v = 0;
+                if (n < N && c < 3 * r) {
+                    const float l2 = bf16_bits_to_f32(L2[static_cast<size_t>(c % r) * N + n]);
+                    const float l = (rf != 0.0f) ? l2 / rf : l2;
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(l);
+                    const __nv_bfloat16 lo = __float2bfloat16_rn(l - __bfloat162float(hi));
+                    const __nv_bfloat16 out = (c < 2 * r) ? hi : lo;
+                    v = *reinterpret_cast<const uint16_t*>(&out);
+                }
+                h[u] = v;
+            }
+            w[e] = h[0] | (h[1] << 16);
+        }
+        reinterpret_cast<uint4*>(l2t + static_cast<size_t>(n) * W)[c8] = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 

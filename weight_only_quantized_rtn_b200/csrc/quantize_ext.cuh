@@ -6,8 +6,8 @@
 //
 // quantize_ex_kernel: for each group (g inputs of a row), a = max|W| exactly,
 // the stored scale s = the value of the scale format nearest to a / qmax
-// (fp32: IEEE division; fp16 / bf16: the fp64 quotient rounded once to the
-// 16-bit format, which equals the correctly rounded one), and
+// (fp32: IEEE division; fp16 / bf16: the exactly rounded quotient, found in
+// fp32 arithmetic by stored_scale), and
 // q = clamp(RTN(W / s), +-qmax) computed exactly with that stored s (a 16-bit
 // s may lie below a / qmax, so the clamp can act).  A group holding a NaN or
 // an infinity, or whose 16-bit scale overflows, gets s = 0 and codes 0 and
@@ -48,6 +48,78 @@ __device__ __forceinline__ uint32_t absbits_max4(float4 v) {
                max(__float_as_uint(v.z) & 0x7FFFFFFFu, __float_as_uint(v.w) & 0x7FFFFFFFu));
 }
 
+// The stored scale: the value of the scale format nearest to a / qmax
+// (ties to even).  fp32: the IEEE division.  fp16 / bf16, from fp32
+// arithmetic: q = RN32(a / qmax) rounds to the same 16-bit value as the exact
+// quotient unless q itself is the midpoint of two 16-bit neighbours (fp32
+// rounding cannot step over such a midpoint, which fp32 represents); there
+// the sign of the exact residual a - q qmax picks the neighbour (a midpoint
+// of two 16-bit values has at most 12 significant bits and qmax at most 7,
+// so q qmax is exact, and so is the fma's result, a small difference of
+// nearby values).  An exact
+// quotient on the midpoint keeps the even neighbour.
+template <int SF>
+__device__ __forceinline__ float stored_scale(float a, int qmax) {
+    const float qf = static_cast<float>(qmax);
+    const float q = __fdiv_rn(a, qf);
+    if constexpr (SF == SCALE_F32) {
+        return q;
+    } else {
+        float lo, hi, rn;
+        if constexpr (SF == SCALE_F16) {
+            lo = __half2float(__float2half_rd(q));
+            hi = __half2float(__float2half_ru(q));
+            rn = __half2float(__float2half_rn(q));
+        } else {
+            lo = __bfloat162float(__float2bfloat16_rd(q));
+            hi = __bfloat162float(__float2bfloat16_ru(q));
+            rn = __bfloat162float(__float2bfloat16_rn(q));
+        }
+        if (lo != hi && __fsub_rn(q, lo) == __fsub_rn(hi, q)) {
+            const float r = __fmaf_rn(-q, qf, a);
+            if (r > 0.0f) return hi;
+            if (r < 0.0f) return lo;
+        }
+        return rn;
+    }
+}
+
+// rtn4_f32 with the codes clamped to [-qmax, qmax] before they are packed:
+// a 16-bit scale may lie below a / qmax, so |W / s| may pass qmax + 1/2 (by at
+// most a 2^-8 fraction: still below 128, where rtn4_f32's estimate holds, but
+// the rounded code can be qmax + 1).
+__device__ __forceinline__ uint32_t rtn4_f32_clamped(float4 v, float s, float inv, float h, float qmax) {
+    const float kMagic = 12582912.0f;  // 1.5 * 2^23
+    const float w[4] = {v.x, v.y, v.z, v.w};
+    float km[4];
+    bool near_half = false;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float t = __fmul_rn(w[i], inv);
+        km[i] = __fadd_rn(t, kMagic);
+        const float d = __fsub_rn(t, __fsub_rn(km[i], kMagic));
+        near_half |= fabsf(d) > 0.499755859375f;  // 1/2 - 2^-12
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float k = __fsub_rn(km[i], kMagic);
+        if (near_half) {
+            const float e = __fmaf_rn(-k, s, w[i]);
+            k = (e > h) ? k + 1.0f : k;
+            k = (e < -h) ? k - 1.0f : k;
+            if (fabsf(e) == h) {  // exact tie between k and k + sign(e): keep the even one
+                if (__float_as_uint(__fadd_rn(k, kMagic)) & 1u) k += (e > 0.0f) ? 1.0f : -1.0f;
+            }
+        }
+        km[i] = __fadd_rn(fminf(fmaxf(k, -qmax), qmax), kMagic);
+    }
+    uint32_t lo, hi, out;
+    asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(lo) : "r"(__float_as_uint(km[0])), "r"(__float_as_uint(km[1])));
+    asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(hi) : "r"(__float_as_uint(km[2])), "r"(__float_as_uint(km[3])));
+    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(out) : "r"(lo), "r"(hi));
+    return out;
+}
+
 template <bool IN_BF16, int SF>
 __global__ void __launch_bounds__(256) quantize_ex_kernel(const void* __restrict__ W, int64_t groups, int g4,
                                                           int qmax, int8_t* __restrict__ codes,
@@ -64,16 +136,7 @@ __global__ void __launch_bounds__(256) quantize_ex_kernel(const void* __restrict
         for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
         bool gbad = m >= 0x7F800000u;  // NaN or infinity in the group
         const float a = gbad ? 0.0f : __uint_as_float(m);
-        float s;
-        if constexpr (SF == SCALE_F32) {
-            s = __fdiv_rn(a, static_cast<float>(qmax));
-        } else if constexpr (SF == SCALE_F16) {
-            const __half h = __double2half(static_cast<double>(a) / static_cast<double>(qmax));
-            s = __half2float(h);
-        } else {
-            const __nv_bfloat16 h = __double2bfloat16(static_cast<double>(a) / static_cast<double>(qmax));
-            s = __bfloat162float(h);
-        }
+        float s = stored_scale<SF>(a, qmax);
         if (isinf(s)) {  // the 16-bit scale overflowed
             gbad = true;
             s = 0.0f;
@@ -132,46 +195,85 @@ __global__ void __launch_bounds__(256) quantize_ex_short_kernel(const void* __re
             const int64_t i4 = (r0 + u) * 32 + lane;  // float4 index: group (r0+u)*GPW + lane / L
             v[u] = i4 < total4 ? load4<IN_BF16>(W, i4) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        uint32_t m[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            m[u] = absbits_max4(v[u]);
+#pragma unroll
+            for (int off = L >> 1; off > 0; off >>= 1) m[u] = max(m[u], __shfl_xor_sync(0xffffffffu, m[u], off));
+        }
+        // The warp holds NGW = U * GPW groups.  When they fit one per lane, lane
+        // j works out the scale of group (j / GPW, j % GPW) -- the division, the
+        // 16-bit rounding and the reciprocal once per group, not once per lane
+        // of it -- and the results go back to each group's lanes by shuffle.
+        constexpr int NGW = U * GPW;
+        float su[U], iu[U];
+        if constexpr (NGW <= 32) {
+            const int ju = lane / GPW, jg = lane % GPW;
+            uint32_t mj = 0;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const uint32_t mu = __shfl_sync(0xffffffffu, m[u], jg * L);
+                if (ju == u) mj = mu;
+            }
+            bool gbad = mj >= 0x7F800000u;  // NaN or infinity in the group
+            float sj = stored_scale<SF>(gbad ? 0.0f : __uint_as_float(mj), qmax);
+            if (isinf(sj)) {  // the 16-bit scale overflowed
+                gbad = true;
+                sj = 0.0f;
+            }
+            const float ij = (sj >= 1.17549435e-38f) ? __frcp_rn(sj) : 0.0f;
+            const int64_t gj = (r0 + ju) * GPW + jg;
+            if (lane < NGW && gj < groups) {
+                bad |= gbad;
+                if constexpr (SF == SCALE_F32) static_cast<float*>(scales)[gj] = sj;
+                else if constexpr (SF == SCALE_F16) static_cast<__half*>(scales)[gj] = __float2half_rn(sj);
+                else static_cast<__nv_bfloat16*>(scales)[gj] = __float2bfloat16_rn(sj);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                su[u] = __shfl_sync(0xffffffffu, sj, u * GPW + lane / L);
+                iu[u] = __shfl_sync(0xffffffffu, ij, u * GPW + lane / L);
+            }
+        } else {
+            // short groups (4 or 8 inputs): at most two lanes share a group
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t i4 = (r0 + u) * 32 + lane;
+                bool gbad = m[u] >= 0x7F800000u;
+                float sg = stored_scale<SF>(gbad ? 0.0f : __uint_as_float(m[u]), qmax);
+                if (isinf(sg)) {
+                    gbad = true;
+                    sg = 0.0f;
+                }
+                su[u] = sg;
+                iu[u] = (sg >= 1.17549435e-38f) ? __frcp_rn(sg) : 0.0f;
+                if (i4 < total4) {
+                    bad |= gbad;
+                    if ((lane & (L - 1)) == 0) {
+                        const int64_t gi = i4 / L;
+                        if constexpr (SF == SCALE_F32) static_cast<float*>(scales)[gi] = sg;
+                        else if constexpr (SF == SCALE_F16) static_cast<__half*>(scales)[gi] = __float2half_rn(sg);
+                        else static_cast<__nv_bfloat16*>(scales)[gi] = __float2bfloat16_rn(sg);
+                    }
+                }
+            }
+        }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int64_t i4 = (r0 + u) * 32 + lane;
-            uint32_t m = absbits_max4(v[u]);
-#pragma unroll
-            for (int off = L >> 1; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
             if (i4 >= total4) continue;
-            bool gbad = m >= 0x7F800000u;
-            const float a = gbad ? 0.0f : __uint_as_float(m);
-            float s;
-            if constexpr (SF == SCALE_F32) {
-                s = __fdiv_rn(a, static_cast<float>(qmax));
-            } else if constexpr (SF == SCALE_F16) {
-                s = __half2float(__double2half(static_cast<double>(a) / static_cast<double>(qmax)));
-            } else {
-                s = __bfloat162float(__double2bfloat16(static_cast<double>(a) / static_cast<double>(qmax)));
-            }
-            if (isinf(s)) {
-                gbad = true;
-                s = 0.0f;
-            }
-            bad |= gbad;
-            if ((lane & (L - 1)) == 0) {
-                const int64_t gi = i4 / L;
-                if constexpr (SF == SCALE_F32) static_cast<float*>(scales)[gi] = s;
-                else if constexpr (SF == SCALE_F16) static_cast<__half*>(scales)[gi] = __float2half_rn(s);
-                else static_cast<__nv_bfloat16*>(scales)[gi] = __float2bfloat16_rn(s);
-            }
+            const float sg = su[u];
             uint32_t c = 0;
-            if (s >= 1.17549435e-38f) {
-                const float inv = __frcp_rn(s);
-                const float w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) c |= rtn_byte_f32(w[e], s, inv, static_cast<float>(qmax)) << (8 * e);
-            } else if (s > 0.0f) {
+            if (sg >= 1.17549435e-38f) {
+                if constexpr (SF == SCALE_F32) c = rtn4_f32(v[u], sg, iu[u], 0.5f * sg);  // |W/s| < qmax + 1/2
+                else c = rtn4_f32_clamped(v[u], sg, iu[u], 0.5f * sg, static_cast<float>(qmax));
+            } else if (sg > 0.0f) {
                 GroupScale gs;
-                gs.s = s;
+                gs.s = sg;
                 gs.normal = false;
                 gs.inv = 0.0f;
-                gs.inv64 = 1.0 / static_cast<double>(s);
+                gs.inv64 = 1.0 / static_cast<double>(sg);
                 bool unused = false;
                 c = pack_codes4(v[u], gs, qmax, unused);
             }

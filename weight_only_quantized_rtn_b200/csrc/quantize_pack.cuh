@@ -91,8 +91,7 @@ __global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
             // group absmax (per group of L lanes; 0 for a group holding a NaN
             // or infinity) and the row's largest group scale over the CTA
             // (scales are non-negative floats: their bit patterns order them)
-            float ga[V];
-            uint32_t smax = 0;
+            uint32_t gm[V];
 #pragma unroll
             for (int i = 0; i < V; ++i) {
                 uint32_t m = max(max(__float_as_uint(v[i].x) & 0x7FFFFFFFu, __float_as_uint(v[i].y) & 0x7FFFFFFFu),
@@ -100,8 +99,30 @@ __global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
                 for (int off = L >> 1; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
                 const bool gbad = m >= 0x7F800000u;
                 bad |= gbad;
-                ga[i] = gbad ? 0.0f : __uint_as_float(m);
-                smax = max(smax, __float_as_uint(__fdiv_rn(ga[i], static_cast<float>(qmax))));
+                gm[i] = gbad ? 0u : m;
+            }
+            // The warp holds V * GPW groups (GPW = 32 / L per float4 slot).
+            // Lane j takes groups j and j + 32: the IEEE division and the
+            // reciprocal once per group rather than once per lane of it; the
+            // results go back to each group's lanes by shuffle.
+            constexpr int GPW = 32 / L;
+            constexpr int NGW = V * GPW;
+            constexpr int PER_LANE = (NGW + 31) / 32;
+            float sj[PER_LANE], ij[PER_LANE];
+            uint32_t smax = 0;
+#pragma unroll
+            for (int t = 0; t < PER_LANE; ++t) {
+                const int j = lane + 32 * t, ji = j / GPW, jg = j % GPW;
+                uint32_t mj = 0;
+#pragma unroll
+                for (int i = 0; i < V; ++i) {
+                    const uint32_t mi = __shfl_sync(0xffffffffu, gm[i], jg * L);
+                    if (ji == i) mj = mi;
+                }
+                const GroupScale gs = group_scale(__uint_as_float(mj), qmax);
+                sj[t] = gs.s;
+                ij[t] = gs.inv;
+                if (j < NGW) smax = max(smax, __float_as_uint(gs.s));
             }
             for (int off = 16; off > 0; off >>= 1) smax = max(smax, __shfl_xor_sync(0xffffffffu, smax, off));
             if (lane == 0) part[warp] = smax;
@@ -122,7 +143,16 @@ __global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
                 const int idx = threadIdx.x + i * blockDim.x;
                 const int k = 4 * idx;
                 bool unused = false;
-                const GroupScale gs = group_scale(ga[i], qmax);
+                // this slot's group scale, from the lane that worked it out
+                // (group i * GPW + lane / L: the same lane slot t = i * GPW / 32 for
+                // every lane, since GPW divides 32)
+                const int src_t = (i * GPW) / 32;
+                const int src = (i * GPW) % 32 + lane / L;
+                GroupScale gs;
+                gs.s = __shfl_sync(0xffffffffu, sj[src_t], src);
+                gs.inv = __shfl_sync(0xffffffffu, ij[src_t], src);
+                gs.normal = gs.s >= 1.17549435e-38f;
+                gs.inv64 = (!gs.normal && gs.s > 0.0f) ? 1.0 / static_cast<double>(gs.s) : 0.0;
                 const uint32_t c4 = gs.normal ? rtn4_f32(v[i], gs.s, gs.inv, 0.5f * gs.s) : pack_codes4(v[i], gs, qmax, unused);
                 // four nibbles (q + 8) at their places among the eight of the word
                 uint32_t w = 0;

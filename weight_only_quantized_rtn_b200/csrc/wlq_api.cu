@@ -20,6 +20,7 @@
 #include "quantize_ext.cuh"
 #include "pack.cuh"
 #include "prep.cuh"
+#include "lowrank.cuh"
 #include "ptx.cuh"
 #include "quantize.cuh"
 
@@ -54,7 +55,7 @@ int fmt_of(int bits, int group) {
 struct DeviceInfo {
     int checked = 0;  // 0 unknown, 1 supported, -1 not
     int sms = 0;
-    bool smem_set[32] = {};
+    bool smem_set[64] = {};
     // resident clusters per (format, cluster size, dynamic smem), queried once
     std::unordered_map<uint64_t, int> max_clusters;
 };
@@ -147,7 +148,7 @@ int token_tile(int64_t M, int r) {
     if (M <= 16) return 16;
     if (M <= 32) return 32;
     if (M <= 64) return 64;
-    if (M <= 128 || r) return 128;
+    if (M <= 128) return 128;
     return 256;
 }
 
@@ -172,7 +173,7 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     p.r = r;
     p.NT = static_cast<int>(cdiv(N, 128));
     p.KT = static_cast<int>(cdiv(K, 64));
-    p.lr_kb = r ? static_cast<int>(cdiv(2 * r, 64)) : 0;
+    p.lr_kb = r ? static_cast<int>(cdiv(3 * r, 64)) : 0;  // [T'h|T'l|T'h] x [L2'h|L2'h|L2'l]
     p.BN = token_tile(M, r);
     p.MT = static_cast<int>(cdiv(M, p.BN));
     // Few 256-token tiles: CTA pairs, with the K range split over up to four
@@ -181,7 +182,7 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     const int cap = (g_grid_limit > 0) ? std::min(g_grid_limit, sms) : sms;
     int S = 1;
     bool pair_split = false;
-    if (variant == 0 && r == 0 && p.BN == 256 && p.NT % 2 == 0) {
+    if (variant == 0 && p.BN == 256 && p.NT % 2 == 0) {
         const int64_t tp = static_cast<int64_t>(p.NT / 2) * p.MT;  // pair tiles
         if (tp * 2 * 2 <= cap) {
             while (S * 2 <= 4 && tp * 2 * (S * 2) <= cap && p.KT >= S * 2 * 4) S *= 2;
@@ -192,7 +193,7 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     // split tiles keep their fp32 partial beside the ring; 256-token ones
     // (variants 0-1, no low-rank term) keep it in the ring's memory.
     if (!pair_split && p.NT * p.MT * 2 <= sms) {
-        if (p.BN > 128 && (variant == 2 || r != 0)) {
+        if (p.BN > 128 && variant == 2) {
             p.BN = 128;
             p.MT = static_cast<int>(cdiv(M, p.BN));
         }
@@ -210,14 +211,14 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     if (S > 1 && p.BN % S != 0) return false;  // every CTA of a split cluster sums whole tokens
     // CTA pairs for large token tiles: two 128-channel tiles share each MMA
     if (pair_split && S == 1) pair_split = false;  // the K range was too short to split
-    p.pair = (r == 0 && p.BN == 256 && p.NT % 2 == 0) && (S == 1 || pair_split);
+    p.pair = (p.BN == 256 && p.NT % 2 == 0) && (S == 1 || pair_split);
     p.red_alias = S > 1 && p.BN == 256;  // split 256-token tiles: pairs or single CTAs
     p.tiles_nm = p.pair ? (p.NT / 2) * p.MT : p.NT * p.MT;
     // TMEM: accumulator(s) first, from column 0, so each starts at a multiple
     // of its own width (main accumulators at ab*BN, low-rank ones after them);
     // then a ks * 32-column A stage per ring slot.  The accumulators are
     // double-buffered when that still leaves room for four 32-column blocks.
-    const uint32_t acc_cols = static_cast<uint32_t>(p.BN) * (r ? 2u : 1u);
+    const uint32_t acc_cols = static_cast<uint32_t>(p.BN);  // the low-rank term shares the accumulator
     if (acc_cols + 2 * wlq::A_STAGE_COLS > 512) return false;
     p.acc_bufs = (2 * acc_cols + 4 * wlq::A_STAGE_COLS <= 512) ? 2 : 1;
     const uint32_t acc_total = p.acc_bufs * acc_cols;
@@ -227,7 +228,7 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     p.xsub = static_cast<uint32_t>(p.pair ? p.BN / 2 : p.BN) * 128u;  // a pair's CTA stages half the tokens
     // token-major fp32 partial (256-token split tiles: in the ring's memory)
     p.red = (S > 1 && !p.red_alias) ? static_cast<uint32_t>(p.BN) * 128u * 4u : 0u;
-    const size_t lr_bytes = r ? (wlq::LR_TILE_A_BYTES + p.xsub) : 0;
+    const size_t lr_bytes = r ? static_cast<size_t>(p.lr_kb) * (wlq::LR_TILE_A_BYTES + p.xsub) : 0;
     p.stage = (S == 1) ? wlq::NUM_EPI_WARPS * wlq::EPI_STAGE_BYTES : 0u;  // epilogue transpose buffers
     const size_t fixed = 1024 /* alignment */ + 1024 /* barriers */ + lr_bytes + p.red + p.stage;
     // Resident x (one token tile, small K range): the CTA's x rows stay in
@@ -352,7 +353,7 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     if (p.red_alias && p.stages * static_cast<size_t>(p.xstage + p.wstage) < static_cast<size_t>(p.BN) * 128u * 4u)
         return variant < 2 ? make_plan(p, M, N, K, fmt, r, sms, variant + 1) : false;
     p.acc_col0 = 0;
-    p.lr_col0 = p.acc_bufs * static_cast<uint32_t>(p.BN);
+    p.lr_col0 = 0;
     p.a_col0 = a_col0;
     const uint32_t need = a_col0 + static_cast<uint32_t>((p.xres ? p.astages : p.stages) * p.ks) * wlq::A_STAGE_COLS;
     p.tmem_cols = 32;
@@ -622,6 +623,78 @@ int grid_for(int64_t work, int per_block, int sms) {
     return static_cast<int>(std::min<int64_t>(b, int64_t(sms) * 32));
 }
 
+// x -> x16 (int4 operands): one CTA per row with the row in registers when
+// it fits (K <= 32768), else one warp per row.
+wlq_status launch_prep_x16(const uint16_t* x, int M, int K, __half* x16, float* xs, DeviceInfo* d, cudaStream_t s) {
+    const int K8 = K / 8;
+    if (M <= 16 && K8 <= 8 * 256) {
+        // few rows: one 256-thread CTA per row
+        const int per = (K8 <= 256) ? 1 : (K8 <= 512) ? 2 : (K8 <= 1024) ? 4 : 8;
+        const int threads = static_cast<int>(std::max<int64_t>(32, (cdiv(K8, per) + 31) / 32 * 32));
+        if (per == 1) launch_k(wlq::prep_x16_rows_kernel<1, 256, 4>, M, threads, 0, s, x, M, K, x16, xs);
+        else if (per == 2) launch_k(wlq::prep_x16_rows_kernel<2, 256, 4>, M, threads, 0, s, x, M, K, x16, xs);
+        else if (per == 4) launch_k(wlq::prep_x16_rows_kernel<4, 256, 4>, M, threads, 0, s, x, M, K, x16, xs);
+        else launch_k(wlq::prep_x16_rows_kernel<8, 256, 4>, M, threads, 0, s, x, M, K, x16, xs);
+    } else if (K8 <= 16 * 128) {
+        // many rows: 128-thread CTAs, up to 16 chunks of the row per thread, so
+        // that the 16 CTAs an SM holds keep about 128 KB of x in flight
+        const int per = (K8 <= 128) ? 1 : (K8 <= 256) ? 2 : (K8 <= 512) ? 4 : (K8 <= 1024) ? 8 : 16;
+        const int threads = static_cast<int>(std::max<int64_t>(32, (cdiv(K8, per) + 31) / 32 * 32));
+        const int grid = static_cast<int>(std::min<int64_t>(M, static_cast<int64_t>(d->sms) * 16));
+        if (per == 1) launch_k(wlq::prep_x16_rows_kernel<1, 128, 1>, grid, threads, 0, s, x, M, K, x16, xs);
+        else if (per == 2) launch_k(wlq::prep_x16_rows_kernel<2, 128, 1>, grid, threads, 0, s, x, M, K, x16, xs);
+        else if (per == 4) launch_k(wlq::prep_x16_rows_kernel<4, 128, 1>, grid, threads, 0, s, x, M, K, x16, xs);
+        else if (per == 8) launch_k(wlq::prep_x16_rows_kernel<8, 128, 1>, grid, threads, 0, s, x, M, K, x16, xs);
+        else launch_k(wlq::prep_x16_rows_kernel<16, 128, 1>, grid, threads, 0, s, x, M, K, x16, xs);
+    } else {
+        launch_k(wlq::prep_x16_kernel, grid_for(static_cast<int64_t>(M) * 32, 256, d->sms), 256, 0, s, x, M, K, x16, xs);
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? WLQ_OK : cuda_fail(e, "prep_x16 launch");
+}
+
+// T = x L1 as [Th | Tl]: 64-row tiles, K split over a cluster of S CTAs
+// (S doubles while the CTAs fit twice on the SMs and every split keeps two
+// 64-wide chunks).
+wlq_status launch_prep_lr_t(const uint16_t* x, const uint16_t* L1, const float* xs, int M, int K, int r, int W,
+                            uint16_t* thl, DeviceInfo* d, cudaStream_t s) {
+    auto kern = wlq::prep_lr_t_kernel;
+    const size_t smem = wlq::lr_t_smem_bytes();
+    if (!d->smem_set[27]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        d->smem_set[27] = true;
+    }
+    const int64_t tiles = cdiv(M, wlq::LR_ROWS);
+    const int KC = static_cast<int>(cdiv(K, wlq::LR_KC));
+    int S = 1;
+    while (S * 2 <= wlq::LR_MAX_SPLITS && tiles * S * 2 <= 2 * d->sms && KC >= S * 2 * 2) S *= 2;
+    int kc_per = static_cast<int>(cdiv(KC, S));
+    while (S > 1 && (S - 1) * kc_per >= KC) {  // every split owns at least one chunk
+        S /= 2;
+        kc_per = static_cast<int>(cdiv(KC, S));
+    }
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3(static_cast<unsigned>(S), static_cast<unsigned>(std::min<int64_t>(tiles, 65535)), 1);
+    cfg.blockDim = dim3(128, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    if (S > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    cudaLaunchAttribute all_attrs[2];
+    add_pdl(cfg, all_attrs);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, x, L1, xs, M, K, r, W, S, kc_per, thl);
+    return e == cudaSuccess ? WLQ_OK : cuda_fail(e, "prep_lr_t launch");
+}
+
 wlq_status launch_linear(Plan& p, int fmt, int64_t M, int64_t N, int64_t K, int r, const void* xin, float* xs,
                          uint16_t* thl, uint16_t* l2t, int W, const void* packed, const void* bias, void* y,
                          int y_dtype, DeviceInfo* d, cudaStream_t s) {
@@ -634,7 +707,7 @@ wlq_status launch_linear(Plan& p, int fmt, int64_t M, int64_t N, int64_t K, int 
     std::memset(&tx, 0, sizeof tx);
     if (!p.gemv && (st = make_map_2d(&tx, xin, M, K, p.pair ? p.BN / 2 : p.BN)) != WLQ_OK) return st;
     if (r) {
-        if ((st = make_map_2d(&tt, thl, M, W, p.BN)) != WLQ_OK) return st;
+        if ((st = make_map_2d(&tt, thl, M, W, p.pair ? p.BN / 2 : p.BN)) != WLQ_OK) return st;
         if ((st = make_map_2d(&tl, l2t, NT * 128, W, 128)) != WLQ_OK) return st;
     }
     wlq::GemmArgs a;
@@ -919,11 +992,18 @@ size_t wlq_linear_workspace(int64_t M, int64_t N, int64_t K, int bits, int group
     return p.ws;
 }
 
-wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, int64_t K, int bits, int group,
-                      const void* bias, const void* L1, const void* L2, int r, void* y, int y_dtype,
-                      void* workspace, size_t ws_bytes, void* stream) {
-    const int fmt = fmt_of(bits, group);
-    if (fmt < 0) return fail(WLQ_ERR_UNSUPPORTED, "linear supports (8,0), (4,64) and (4,16)");
+}  // extern "C"
+
+namespace {
+
+// Argument checks of the Linear entry points, all made before any device
+// access or planning.  *noop is set when the call has nothing to do (M == 0
+// or N == 0 after valid arguments).
+wlq_status check_linear_args(const void* x, int64_t M, const void* packed, int64_t N, int64_t K, int bits,
+                             int group, const void* bias, const void* L1, const void* L2, int r, const void* y,
+                             int y_dtype, bool* noop) {
+    *noop = false;
+    if (fmt_of(bits, group) < 0) return fail(WLQ_ERR_UNSUPPORTED, "linear supports (8,0), (4,64) and (4,16)");
     wlq_status st = check_shape(N, K, bits, group);
     if (st != WLQ_OK) return st;
     if (M < 0) return fail(WLQ_ERR_INVALID_ARG, "M < 0");
@@ -931,12 +1011,29 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
     if (!(r == 0 || r == 16 || r == 32 || r == 64)) return fail(WLQ_ERR_SHAPE, "r must be 0, 16, 32 or 64");
     if (r && (!L1 || !L2)) return fail(WLQ_ERR_INVALID_ARG, "r > 0 needs L1 and L2");
     if (y_dtype != WLQ_OUT_BF16 && y_dtype != WLQ_OUT_F32) return fail(WLQ_ERR_INVALID_ARG, "bad y_dtype");
-    if (M == 0 || N == 0) return WLQ_OK;
+    if (M == 0 || N == 0) {
+        *noop = true;
+        return WLQ_OK;
+    }
     if (!x || !packed || !y) return fail(WLQ_ERR_INVALID_ARG, "null pointer");
     if (!aligned16(x) || !aligned16(packed)) return fail(WLQ_ERR_ALIGN, "x and packed must be 16-byte aligned");
-    if ((bias && (reinterpret_cast<uintptr_t>(bias) & 1u)) || (L1 && (reinterpret_cast<uintptr_t>(L1) & 1u)) ||
+    if ((bias && (reinterpret_cast<uintptr_t>(bias) & 1u)) || (L1 && !aligned16(L1)) ||
         (L2 && (reinterpret_cast<uintptr_t>(L2) & 1u)) || (reinterpret_cast<uintptr_t>(y) & 3u))
-        return fail(WLQ_ERR_ALIGN, "bias/L1/L2 must be 2-byte aligned, y 4-byte aligned");
+        return fail(WLQ_ERR_ALIGN, "L1 must be 16-byte aligned, bias/L2 2-byte aligned, y 4-byte aligned");
+    return WLQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, int64_t K, int bits, int group,
+                      const void* bias, const void* L1, const void* L2, int r, void* y, int y_dtype,
+                      void* workspace, size_t ws_bytes, void* stream) {
+    bool noop = false;
+    wlq_status st = check_linear_args(x, M, packed, N, K, bits, group, bias, L1, L2, r, y, y_dtype, &noop);
+    if (st != WLQ_OK || noop) return st;
+    const int fmt = fmt_of(bits, group);
     int dev;
     DeviceInfo* d;
     if ((st = current_device(&dev, &d)) != WLQ_OK) return st;
@@ -955,8 +1052,7 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
     if (fmt != wlq::FMT_W8) {
         __half* x16 = reinterpret_cast<__half*>(ws + p.off_x16);
         xs = reinterpret_cast<float*>(ws + p.off_xs);
-        launch_k(wlq::prep_x16_kernel, grid_for(M * 32, 256, d->sms), 256, 0, s, static_cast<const uint16_t*>(x), p.M,
-                                                                          p.K, x16, xs);
+        if ((st = launch_prep_x16(static_cast<const uint16_t*>(x), p.M, p.K, x16, xs, d, s)) != WLQ_OK) return st;
         xin = x16;
     }
     uint16_t* thl = nullptr;
@@ -965,10 +1061,15 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
     if (r) {
         thl = reinterpret_cast<uint16_t*>(ws + p.off_thl);
         l2t = reinterpret_cast<uint16_t*>(ws + p.off_l2t);
-        launch_k(wlq::prep_lr_t_kernel, static_cast<unsigned>(cdiv(M, wlq::LR_ROWS)), 128, 0, s, 
-            static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(L1), p.M, p.K, r, W, thl);
-        launch_k(wlq::prep_lr_l2t_kernel, grid_for(NT * 128 * W, 256, d->sms), 256, 0, s, 
-            static_cast<const uint16_t*>(L2), p.N, static_cast<int>(NT * 128), r, W, l2t);
+        // the branch is folded into the GEMM's accumulator: T' = T / xs (int4) and
+        // L2' = L2 / rowf, rowf read from the packed operand
+        if ((st = launch_prep_lr_t(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(L1), xs, p.M, p.K, r,
+                                   W, thl, d, s)) != WLQ_OK)
+            return st;
+        const float* rowf = reinterpret_cast<const float*>(static_cast<const uint8_t*>(packed) +
+                                                           static_cast<size_t>(NT) * p.KT * wlq::tile_bytes(fmt));
+        launch_k(wlq::prep_lr_l2t_kernel, grid_for(NT * 128 * (W / 8), 256, d->sms), 256, 0, s,
+            static_cast<const uint16_t*>(L2), rowf, p.N, static_cast<int>(NT * 128), r, W, l2t);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "prep launch");
@@ -1001,9 +1102,19 @@ namespace {
 void* g_static_scratch_ptr[kMaxDevices] = {};
 std::mutex g_static_mu;
 
-wlq_status static_scratch(int dev, void** out) {
+wlq_status static_scratch(int dev, cudaStream_t stream, void** out) {
     std::lock_guard<std::mutex> lk(g_static_mu);
     if (!g_static_scratch_ptr[dev]) {
+        // The address lookup is not a stream operation and may load the
+        // module; inside a stream capture it would fail or invalidate the
+        // capture, so the first call on a device must come before any capture.
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        cudaError_t ce = cudaStreamIsCapturing(stream, &cs);
+        if (ce != cudaSuccess) return cuda_fail(ce, "cudaStreamIsCapturing");
+        if (cs != cudaStreamCaptureStatusNone)
+            return fail(WLQ_ERR_INVALID_ARG,
+                        "the first wlq_linear_noalloc call on a device looks up its built-in scratch and must "
+                        "come before any stream capture");
         void* ptr = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_scratch);
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
@@ -1019,15 +1130,15 @@ extern "C" {
 wlq_status wlq_linear_noalloc(const void* x, int64_t M, const void* packed, int64_t N, int64_t K, int bits,
                               int group, const void* bias, const void* L1, const void* L2, int r, void* y,
                               int y_dtype, void* stream) {
-    // Shapes the ordinary entry point rejects, and empty problems, go straight
-    // through it (it reports the error or does nothing); nothing here allocates.
+    // The same argument checks as wlq_linear, before any planning or device
+    // access, so an invalid call gets the same status from both entry points.
+    bool noop = false;
+    wlq_status st = check_linear_args(x, M, packed, N, K, bits, group, bias, L1, L2, r, y, y_dtype, &noop);
+    if (st != WLQ_OK || noop) return st;
     const int fmt = fmt_of(bits, group);
-    if (fmt < 0 || M <= 0 || N <= 0 || check_shape(N, K, bits, group) != WLQ_OK)
-        return wlq_linear(x, M, packed, N, K, bits, group, bias, L1, L2, r, y, y_dtype, nullptr, 0, stream);
     int dev;
     DeviceInfo* d;
-    wlq_status st = current_device(&dev, &d);
-    if (st != WLQ_OK) return st;
+    if ((st = current_device(&dev, &d)) != WLQ_OK) return st;
     Plan p;
     if (!make_plan(p, M, N, K, fmt, r, d->sms)) return fail(WLQ_ERR_UNSUPPORTED, "no launch plan for this shape");
     if (p.ws > kStaticScratchBytes)
@@ -1036,11 +1147,161 @@ wlq_status wlq_linear_noalloc(const void* x, int64_t M, const void* packed, int6
                     "call wlq_linear with a caller-owned workspace instead",
                     p.ws, kStaticScratchBytes);
     void* scratch = nullptr;
-    if ((st = static_scratch(dev, &scratch)) != WLQ_OK) return st;
+    if ((st = static_scratch(dev, static_cast<cudaStream_t>(stream), &scratch)) != WLQ_OK) return st;
     // Nothing in the scratch has to start at zero: every region is fully
     // written by the call's preparation kernels before the GEMM reads it.
     return wlq_linear(x, M, packed, N, K, bits, group, bias, L1, L2, r, y, y_dtype, scratch, kStaticScratchBytes,
                       stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Workspace of the low-rank split: two [K, l] and two [N, l] fp32 panels,
+// the fp64 Gram partials (one per chunk of LR_GRAM_ROWS rows), the small
+// l x l / l x r matrices.
+constexpr int LR_GRAM_ROWS = 64;
+struct LrLayout {
+    size_t y0, y1, z0, z1, parts, rinv, b1, b2, total;
+};
+LrLayout lr_layout(int64_t N, int64_t K, int l, int r) {
+    LrLayout o;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { const size_t at = off; off = align256(off + bytes); return at; };
+    o.y0 = take(static_cast<size_t>(K) * l * 4);
+    o.y1 = take(static_cast<size_t>(K) * l * 4);
+    o.z0 = take(static_cast<size_t>(N) * l * 4);
+    o.z1 = take(static_cast<size_t>(N) * l * 4);
+    const int64_t parts = cdiv(std::max(N, K), LR_GRAM_ROWS);
+    o.parts = take(static_cast<size_t>(parts) * l * l * 8);
+    o.rinv = take(static_cast<size_t>(l) * l * 4);
+    o.b1 = take(static_cast<size_t>(l) * r * 4);
+    o.b2 = take(static_cast<size_t>(l) * r * 4);
+    o.total = off;
+    return o;
+}
+
+bool lr_shape_ok(int64_t N, int64_t K, int r, int l, int q) {
+    return (r == 16 || r == 32 || r == 64) && (l == 32 || l == 64) && l >= r && q >= 0 && q <= 8 && N >= l &&
+           K >= l && N <= (int64_t(1) << 24) && K <= (int64_t(1) << 24);
+}
+
+template <bool TRANS>
+void lr_gemm(const float* A, const float* B, int R, int inner, int c, float* out, uint16_t* out_bf16,
+             uint16_t* out_bf16_t, cudaStream_t s) {
+    launch_k(wlq::lr_skinny_gemm<TRANS>, static_cast<unsigned>(cdiv(R, wlq::LRS_ROWS)), wlq::LRS_THREADS, 0, s, A, B, R,
+             inner, c, out, out_bf16, out_bf16_t);
+}
+
+wlq_status lr_small(const double* parts, int nparts, int l, int r, int mode, float* o1, float* o2, float* sigma,
+                    DeviceInfo* d, cudaStream_t s) {
+    const size_t smem = static_cast<size_t>(2) * l * l * 8;
+    if (!d->smem_set[40]) {
+        cudaError_t e = cudaFuncSetAttribute(wlq::lr_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(2 * wlq::LRS_MAX_L * wlq::LRS_MAX_L * 8));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        d->smem_set[40] = true;
+    }
+    launch_k(wlq::lr_small_kernel, 1, 256, smem, s, parts, nparts, l, r, mode, o1, o2, sigma, static_cast<int*>(nullptr));
+    return WLQ_OK;
+}
+
+// Y <- orth(Y) by CholeskyQR2 (Y [R, l] in `cur`, `tmp` the same size); the
+// orthonormal result ends in `cur`.
+wlq_status lr_orth(float* cur, float* tmp, int R, int l, const LrLayout& L, uint8_t* ws, DeviceInfo* d,
+                   cudaStream_t s) {
+    double* parts = reinterpret_cast<double*>(ws + L.parts);
+    float* rinv = reinterpret_cast<float*>(ws + L.rinv);
+    const int nparts = static_cast<int>(cdiv(R, LR_GRAM_ROWS));
+    wlq_status st;
+    for (int pass = 0; pass < 2; ++pass) {
+        launch_k(wlq::lr_gram_partial, nparts, 256, 0, s, static_cast<const float*>(cur), R, l, LR_GRAM_ROWS, parts);
+        if ((st = lr_small(parts, nparts, l, 0, 0, rinv, nullptr, nullptr, d, s)) != WLQ_OK) return st;
+        lr_gemm<false>(cur, rinv, R, l, l, tmp, nullptr, nullptr, s);
+        std::swap(cur, tmp);
+    }
+    // two swaps: the result is back in the caller's `cur`
+    return WLQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t wlq_lowrank_workspace(int64_t N, int64_t K, int r, int l) {
+    if (!lr_shape_ok(N, K, r, l, 0)) return 0;
+    return lr_layout(N, K, l, r).total;
+}
+
+wlq_status wlq_lowrank_split(const float* W, int64_t N, int64_t K, int r, int l, int power_iters, const float* omega,
+                             void* L1, void* L2, float* sigma, void* workspace, size_t ws_bytes, void* stream) {
+    if (!lr_shape_ok(N, K, r, l, power_iters))
+        return fail(WLQ_ERR_SHAPE, "low-rank split needs r in {16,32,64}, l in {32,64} with l >= r, "
+                                   "0 <= power_iters <= 8 and N, K >= l");
+    if (!W || !omega || !L1 || !L2 || !workspace) return fail(WLQ_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(W) || !aligned16(omega) || !aligned16(L1) || !aligned16(L2) || !aligned16(workspace) ||
+        (sigma && (reinterpret_cast<uintptr_t>(sigma) & 3u)))
+        return fail(WLQ_ERR_ALIGN, "W, omega, L1, L2 and workspace must be 16-byte aligned");
+    const LrLayout L = lr_layout(N, K, l, r);
+    if (ws_bytes < L.total) return fail(WLQ_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", L.total, ws_bytes);
+    int dev;
+    DeviceInfo* d;
+    wlq_status st = current_device(&dev, &d);
+    if (st != WLQ_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* y0 = reinterpret_cast<float*>(ws + L.y0);
+    float* y1 = reinterpret_cast<float*>(ws + L.y1);
+    float* z0 = reinterpret_cast<float*>(ws + L.z0);
+    float* z1 = reinterpret_cast<float*>(ws + L.z1);
+    const int n = static_cast<int>(N), k = static_cast<int>(K);
+    // Y = W^T Omega, orthonormalised
+    lr_gemm<true>(W, omega, k, n, l, y0, nullptr, nullptr, s);
+    if ((st = lr_orth(y0, y1, k, l, L, ws, d, s)) != WLQ_OK) return st;
+    for (int it = 0; it < power_iters; ++it) {
+        lr_gemm<false>(W, y0, n, k, l, z0, nullptr, nullptr, s);   // Z = W Q
+        if ((st = lr_orth(z0, z1, n, l, L, ws, d, s)) != WLQ_OK) return st;
+        lr_gemm<true>(W, z0, k, n, l, y0, nullptr, nullptr, s);    // Y = W^T P
+        if ((st = lr_orth(y0, y1, k, l, L, ws, d, s)) != WLQ_OK) return st;
+    }
+    // C = W Q; H = C^T C = U~ Lambda U~^T
+    lr_gemm<false>(W, y0, n, k, l, z0, nullptr, nullptr, s);
+    double* parts = reinterpret_cast<double*>(ws + L.parts);
+    const int nparts = static_cast<int>(cdiv(N, LR_GRAM_ROWS));
+    launch_k(wlq::lr_gram_partial, nparts, 256, 0, s, static_cast<const float*>(z0), n, l, LR_GRAM_ROWS, parts);
+    float* b1 = reinterpret_cast<float*>(ws + L.b1);
+    float* b2 = reinterpret_cast<float*>(ws + L.b2);
+    if ((st = lr_small(parts, nparts, l, r, 1, b1, b2, sigma, d, s)) != WLQ_OK) return st;
+    // L1 = Q U~_r Lambda_r^(1/4) [K, r]; L2 = (C U~_r Lambda_r^(-1/4))^T [r, N]
+    lr_gemm<false>(y0, b1, k, l, r, nullptr, static_cast<uint16_t*>(L1), nullptr, s);
+    lr_gemm<false>(z0, b2, n, l, r, nullptr, nullptr, static_cast<uint16_t*>(L2), s);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "low-rank split launch");
+    return WLQ_OK;
+}
+
+wlq_status wlq_lowrank_residual(const float* W, const void* L1, const void* L2, int64_t N, int64_t K, int r, float* R,
+                                void* stream) {
+    if (N < 0 || K <= 0 || !(r == 16 || r == 32 || r == 64) || N > (int64_t(1) << 30) || K > (int64_t(1) << 30))
+        return fail(WLQ_ERR_SHAPE, "residual needs r in {16,32,64}, N >= 0, K > 0");
+    if (N == 0) return WLQ_OK;
+    if (!W || !L1 || !L2 || !R) return fail(WLQ_ERR_INVALID_ARG, "null pointer");
+    if ((reinterpret_cast<uintptr_t>(W) & 3u) || (reinterpret_cast<uintptr_t>(R) & 3u) ||
+        (reinterpret_cast<uintptr_t>(L1) & 1u) || (reinterpret_cast<uintptr_t>(L2) & 1u))
+        return fail(WLQ_ERR_ALIGN, "W and R must be 4-byte aligned, L1 and L2 2-byte aligned");
+    int dev;
+    DeviceInfo* d;
+    wlq_status st = current_device(&dev, &d);
+    if (st != WLQ_OK) return st;
+    const dim3 grid(static_cast<unsigned>(cdiv(K, 32)), static_cast<unsigned>(cdiv(N, 32)), 1);
+    if (grid.y > 65535) return fail(WLQ_ERR_SHAPE, "N too large for the residual kernel");
+    launch_k(wlq::lr_residual_kernel, grid, 256, 0, static_cast<cudaStream_t>(stream), W,
+             static_cast<const uint16_t*>(L1), static_cast<const uint16_t*>(L2), static_cast<int>(N),
+             static_cast<int>(K), r, R);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "residual launch");
+    return WLQ_OK;
 }
 
 void wlq_set_grid_limit(int max_ctas) { g_grid_limit = max_ctas > 0 ? max_ctas : 0; }
