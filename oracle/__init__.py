@@ -49,8 +49,13 @@ def bind(path: str):
     lib.oracle_quantize_ex.argtypes = [vp, i32, i64, i64, i32, i32, i32, vp, vp]
     lib.oracle_quantize_fp8.argtypes = [vp, i32, i64, i64, i32, vp, vp]
     lib.oracle_lowrank_residual.argtypes = [vp, vp, vp, i64, i64, i32, vp]
+    lib.oracle_nvfp4_quantize.argtypes = [vp, i32, i64, i64, vp, vp, vp]
+    lib.oracle_nvfp4_dequantize.argtypes = [vp, vp, ctypes.c_float, i64, i64, vp]
+    lib.oracle_nvfp4_linear.argtypes = [vp, vp, ctypes.c_float, vp, i64, i64, vp, vp, ctypes.c_float, i64,
+                                        vp, vp, vp, i32, vp]
     for f in (lib.oracle_quantize, lib.oracle_dequantize, lib.oracle_linear, lib.oracle_quantize_ex,
-              lib.oracle_quantize_fp8, lib.oracle_lowrank_residual):
+              lib.oracle_quantize_fp8, lib.oracle_lowrank_residual, lib.oracle_nvfp4_quantize,
+              lib.oracle_nvfp4_dequantize, lib.oracle_nvfp4_linear):
         f.restype = ctypes.c_int
     return lib
 
@@ -226,3 +231,64 @@ def lowrank_residual(W: np.ndarray, L1_bits: np.ndarray, L2_bits: np.ndarray) ->
     R = np.empty((N, K), np.float32)
     _check(_load().oracle_lowrank_residual(_p(W), _p(L1_bits), _p(L2_bits), N, K, r, _p(R)))
     return R
+
+
+def nvfp4_quantize(X: np.ndarray):
+    """NVFP4 quantization of a [rows, K] tensor (the 4-bit format of the W4A4
+    path on Blackwell: "Nunchaku Lite" article, hardware and precision
+    support): E2M1 codes, one E4M3 scale per 16 inputs of a row, one fp32
+    tensor scale g = fp32(amax / 2688).  X: fp32, or uint16 bf16 bit patterns.
+    Returns (codes uint8 [rows, K] (E2M1 bits, sign in bit 3), scales uint8
+    [rows, K/16] (E4M3 bits), g)."""
+    if X.dtype == np.uint16:
+        X = np.ascontiguousarray(X)
+        x_dtype = 1
+    else:
+        X = np.ascontiguousarray(X, dtype=np.float32)
+        x_dtype = 0
+    rows, K = X.shape
+    codes = np.empty((rows, K), np.uint8)
+    scales = np.empty((rows, K // 16 if K % 16 == 0 else 1), np.uint8)
+    g = ctypes.c_float(0.0)
+    _check(_load().oracle_nvfp4_quantize(_p(X), x_dtype, rows, K, _p(codes), _p(scales), ctypes.byref(g)))
+    return codes, scales, float(g.value)
+
+
+def nvfp4_dequantize(codes: np.ndarray, scales: np.ndarray, g: float) -> np.ndarray:
+    """x^ = q s_b g (exact, fp64 [rows, K])."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, K = codes.shape
+    out = np.empty((rows, K), np.float64)
+    _check(_load().oracle_nvfp4_dequantize(_p(codes), _p(scales), g, rows, K, _p(out)))
+    return out
+
+
+def nvfp4_linear(xq, xs, xg, x_bits, wq, ws, wg, bias_bits=None, L1_bits=None, L2_bits=None) -> np.ndarray:
+    """The W4A4 Linear in fp64: y = deq(xq) deq(wq)^T [+ (x L1) L2] [+ b].
+
+    xq/xs/xg, wq/ws/wg: NVFP4 codes, block scales and tensor scale of the
+    activations [M, K] and the weights [N, K]; x_bits: the 16-bit activations
+    (bf16 bit patterns, used by the low-rank branch only); bias [N], L1 [K, r],
+    L2 [r, N]: bf16 bit patterns."""
+    xq = np.ascontiguousarray(xq, dtype=np.uint8)
+    xs = np.ascontiguousarray(xs, dtype=np.uint8)
+    wq = np.ascontiguousarray(wq, dtype=np.uint8)
+    ws = np.ascontiguousarray(ws, dtype=np.uint8)
+    M, K = xq.shape
+    N = wq.shape[0]
+    assert wq.shape[1] == K
+    r = 0
+    if L1_bits is not None:
+        L1_bits = np.ascontiguousarray(L1_bits, dtype=np.uint16)
+        L2_bits = np.ascontiguousarray(L2_bits, dtype=np.uint16)
+        x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        r = L1_bits.shape[1]
+        assert L1_bits.shape == (K, r) and L2_bits.shape == (r, N) and x_bits.shape == (M, K)
+    if bias_bits is not None:
+        bias_bits = np.ascontiguousarray(bias_bits, dtype=np.uint16)
+        assert bias_bits.shape == (N,)
+    y = np.empty((M, N), np.float64)
+    _check(_load().oracle_nvfp4_linear(_p(xq), _p(xs), xg, _p(x_bits) if r else None, M, K, _p(wq), _p(ws), wg,
+                                       N, _p(bias_bits), _p(L1_bits), _p(L2_bits), r, _p(y)))
+    return y

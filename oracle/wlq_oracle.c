@@ -361,3 +361,124 @@ int oracle_lowrank_residual(const float* W, const uint16_t* L1, const uint16_t* 
     }
     return ORACLE_OK;
 }
+
+/*
+ * NVFP4, the 4-bit format of the W4A4 path's Blackwell kernels [NL, section
+ * "hardware and precision support": the NVFP4 variant of svdq_w4a4 runs on
+ * Blackwell; section "how it works": W4A4 quantizes weights and activations
+ * to 4 bits and keeps a 16-bit low-rank branch].  The pages name the format
+ * without defining it; it is read as NVIDIA's NVFP4: E2M1 elements (sign,
+ * magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), one E4M3 scale per 16 consecutive
+ * inputs of a row, one fp32 scale per tensor:
+ *   g   = fp32(amax(X) / (6 * 448))            (0 for an all-zero tensor)
+ *   s_b = E4M3 nearest to a_b / (6 g)          (a_b = max |x| over the block;
+ *                                                ties to even, saturated at 448)
+ *   q   = E2M1 nearest to x / (s_b g)          (ties to an even significand,
+ *                                                saturated at 6; 0 when s_b = 0)
+ *   x^  = q s_b g
+ * The quotients are taken in fp64 from the exact operands: s_b g has at most
+ * 28 significant bits, so it is exact, and a quotient of fp32 values cannot
+ * come within fp64's rounding error of a midpoint of these short formats
+ * without lying on it (the same argument as for the scales above).
+ * X: fp32 or bf16 [rows, K], K % 16 == 0; codes: E2M1 bits (sign in bit 3)
+ * [rows, K]; scales: E4M3 bits [rows, K / 16]; *gscale: g.
+ */
+static const double E2M1_MAG[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+static double e4m3_value(uint8_t bits) {
+    const int e = (bits >> 3) & 15, m = bits & 7;
+    const double v = (e == 0) ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return (bits & 0x80) ? -v : v;
+}
+
+static uint8_t e2m1_encode(double t) {
+    const int neg = signbit(t) ? 1 : 0;
+    double r = round_to_format(fabs(t), 2, 0, 6.0);
+    if (isinf(r)) r = 6.0; /* saturate */
+    uint8_t code = 0;
+    for (int i = 0; i < 8; ++i)
+        if (E2M1_MAG[i] == r) code = (uint8_t)i;
+    return (uint8_t)(code | (neg << 3));
+}
+
+static double e2m1_value(uint8_t code) {
+    const double v = E2M1_MAG[code & 7];
+    return (code & 8) ? -v : v;
+}
+
+int oracle_nvfp4_quantize(const void* X, int x_dtype, int64_t rows, int64_t K, uint8_t* codes,
+                          uint8_t* scales, float* gscale) {
+    if (rows < 0 || K <= 0 || K % 16 != 0 || (x_dtype != 0 && x_dtype != 1)) return ORACLE_ERR_ARG;
+    double amax = 0.0;
+    for (int64_t i = 0; i < rows * K; ++i) {
+        const double v = in_value(X, x_dtype, i);
+        if (!isfinite(v)) return ORACLE_ERR_NONFINITE;
+        if (fabs(v) > amax) amax = fabs(v);
+    }
+    const float g = (float)(amax / (6.0 * 448.0));
+    *gscale = g;
+    for (int64_t row = 0; row < rows; ++row) {
+        for (int64_t b = 0; b < K / 16; ++b) {
+            const int64_t base = row * K + b * 16;
+            double ab = 0.0;
+            for (int j = 0; j < 16; ++j) {
+                const double v = fabs(in_value(X, x_dtype, base + j));
+                if (v > ab) ab = v;
+            }
+            uint8_t sb = 0;
+            if (g > 0.0f) sb = e4m3_encode(ab / (6.0 * (double)g));
+            scales[row * (K / 16) + b] = sb;
+            const double d = e4m3_value(sb) * (double)g; /* exact: <= 28 significant bits */
+            for (int j = 0; j < 16; ++j)
+                codes[base + j] = (d > 0.0) ? e2m1_encode(in_value(X, x_dtype, base + j) / d) : 0;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* x^ = q s_b g for every element: fp64 [rows, K] (exact). */
+int oracle_nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, float g, int64_t rows, int64_t K,
+                            double* out) {
+    if (rows < 0 || K <= 0 || K % 16 != 0) return ORACLE_ERR_ARG;
+    for (int64_t row = 0; row < rows; ++row)
+        for (int64_t k = 0; k < K; ++k)
+            out[row * K + k] = e2m1_value(codes[row * K + k]) * e4m3_value(scales[row * (K / 16) + k / 16]) *
+                               (double)g;
+    return ORACLE_OK;
+}
+
+/*
+ * The W4A4 Linear [NL, "how it works": 4-bit weights and activations with a
+ * 16-bit low-rank correction]:
+ *   y[m,n] = sum_k x^[m,k] w^[n,k] + sum_j (sum_k x[m,k] L1[k,j]) L2[j,n] + b[n]
+ * x^, w^: NVFP4 dequantized activations [M, K] and weights [N, K]; the
+ * low-rank branch takes the 16-bit x (bf16 bits) as it is.  fp64, naive loops.
+ */
+int oracle_nvfp4_linear(const uint8_t* xq, const uint8_t* xs, float xg, const uint16_t* x, int64_t M, int64_t K,
+                        const uint8_t* wq, const uint8_t* ws, float wg, int64_t N, const uint16_t* bias,
+                        const uint16_t* L1, const uint16_t* L2, int r, double* y) {
+    if (M < 0 || N < 0 || K <= 0 || K % 16 != 0 || r < 0 || r > 256) return ORACLE_ERR_ARG;
+    if (r > 0 && (L1 == 0 || L2 == 0 || x == 0)) return ORACLE_ERR_ARG;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; ++m) {
+        double T[256];
+        for (int j = 0; j < r; ++j) {
+            double t = 0.0;
+            for (int64_t k = 0; k < K; ++k) t += bf16_value(x[m * K + k]) * bf16_value(L1[k * r + j]);
+            T[j] = t;
+        }
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                const double a = e2m1_value(xq[m * K + k]) * e4m3_value(xs[m * (K / 16) + k / 16]) * (double)xg;
+                const double w = e2m1_value(wq[n * K + k]) * e4m3_value(ws[n * (K / 16) + k / 16]) * (double)wg;
+                acc += a * w;
+            }
+            double lr = 0.0;
+            for (int j = 0; j < r; ++j) lr += T[j] * bf16_value(L2[(int64_t)j * N + n]);
+            const double b = bias ? bf16_value(bias[n]) : 0.0;
+            y[m * N + n] = acc + lr + b;
+        }
+    }
+    return ORACLE_OK;
+}

@@ -146,6 +146,8 @@ def test_parity_low_rank_zero_weight_rows(bits, group, r, M):
     (512, 1024, 512, 32, 0),   # low rank on split pairs: the term on K split 0 only
     (256, 1920, 1024, 64, 0),  # low rank, 256-token tiles on single CTAs with the partial in the ring
     (1024, 2048, 1024, 16, 20),# low rank on pairs, several tiles per pair
+    (256, 4096, 1024, 0, 0),   # pairs over 128-token tiles, K split over the two pairs of a 4-CTA cluster
+    (200, 4096, 512, 32, 0),   # the same with low rank and a ragged token tile
 
     (40, 1100, 320, 0, 4),     # 9 tiles on 4 CTAs: both accumulator buffers in use
     (16, 33000, 128, 0, 16),   # 258 tiles of 16 tokens on 16 CTAs

@@ -13,6 +13,7 @@ import pytest
 import oracle
 import tests.test_oracle_ext_pins as ext
 import tests.test_oracle_lowrank_pins as lr
+import tests.test_oracle_nvfp4_pins as nv
 import tests.test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "wlq_oracle.c")
@@ -37,6 +38,14 @@ MUTATIONS = {
     "residual_last_rank_dropped": ("for (int j = 0; j < r; ++j) {\n                const double prod",
                                    "for (int j = 0; j < r - 1; ++j) {\n                const double prod"),
     "residual_sign": ("const double d = (double)W[n * K + k] - p;", "const double d = (double)W[n * K + k] + p;"),
+    "nvfp4_tensor_scale_off": ("(float)(amax / (6.0 * 448.0))", "(float)(amax / (6.0 * 480.0))"),
+    "nvfp4_block_max_signed": ("const double v = fabs(in_value(X, x_dtype, base + j));",
+                               "const double v = in_value(X, x_dtype, base + j);"),
+    "e2m1_no_subnormals": ("round_to_format(fabs(t), 2, 0, 6.0)", "round_to_format(fabs(t), 2, 1, 6.0)"),
+    "e2m1_sign_dropped": ("return (uint8_t)(code | (neg << 3));", "(void)neg; return code;"),
+    "nvfp4_weight_block_index": ("e4m3_value(ws[n * (K / 16) + k / 16])", "e4m3_value(ws[n * (K / 16) + k % (K / 16)])"),
+    "nvfp4_low_rank_dropped": ("y[m * N + n] = acc + lr + b;", "y[m * N + n] = acc + b;"),
+    "nvfp4_e4m3_decode_bias": ("ldexp(1.0 + (double)m / 8.0, e - 7)", "ldexp(1.0 + (double)m / 8.0, e - 8)"),
 }
 
 PIN_TESTS = [
@@ -54,6 +63,12 @@ PIN_TESTS = [
     lambda: ext.test_fp8_codes_are_the_nearest_e4m3_ties_to_even_saturated(),
     lambda: ext.test_fp8_codes_match_torch_e4m3fn_conversion(),
     lambda: lr.test_residual_equals_fp64_matmul_when_every_sum_is_exact(),
+    lambda: nv.test_every_e2m1_code_and_midpoint_with_unit_scales(),
+    lambda: nv.test_block_scales_are_the_nearest_e4m3_with_ties_to_even(),
+    lambda: nv.test_codes_are_the_brute_force_nearest_for_random_tensors(),
+    lambda: nv.test_dequantize_decodes_the_fields(),
+    lambda: nv.test_w4a4_linear_matches_numpy_matmul(16, True),
+    lambda: nv.test_w4a4_linear_exact_small_case(),
 ]
 
 

@@ -30,98 +30,135 @@
 namespace wlq {
 
 constexpr int LRS_MAX_L = 64;      // columns of the sketch (l)
-constexpr int LRS_ROWS = 32;       // output rows per CTA of the skinny GEMM
+constexpr int LRS_ROWS = 64;       // output rows per CTA of the skinny GEMM
 constexpr int LRS_KC = 32;         // inner chunk
 constexpr int LRS_THREADS = 256;
 
-// out[R, c] (+ fp32, row-major, ld c) = op(A)[R, inner] * B[inner, c]
-// op(A): TRANS == false: A is [R, inner] row-major (lda = inner);
-//        TRANS == true : A is [inner, R] row-major, read transposed (lda = R).
-// B is [inner, c] row-major fp32.  c <= LRS_MAX_L, a multiple of 16.
-// bf16_t_out: write the result as bf16 transposed, out_t[c][R] (row-major).
+// part[split][R, c] = op(A)[R, inner-range of split] * B[inner-range, c], fp32.
+// op(A): TRANS == false: A is [R, inner] row-major;
+//        TRANS == true : A is [inner, R] row-major, read transposed.
+// B is [inner, c] row-major, c in {16, 32, 64}.  A CTA takes 64 rows and one
+// inner range (blockIdx.y); thread (tr, tc) accumulates rows 4 tr..+3 and
+// columns 4 tc..+3; the next chunk is loaded into registers while the
+// current one is used.
 template <bool TRANS>
 __global__ void __launch_bounds__(LRS_THREADS) lr_skinny_gemm(const float* __restrict__ A, const float* __restrict__ B,
-                                                              int R, int inner, int c, float* __restrict__ out,
-                                                              uint16_t* __restrict__ out_bf16,
-                                                              uint16_t* __restrict__ out_bf16_t) {
+                                                              int R, int inner, int c, int kper,
+                                                              float* __restrict__ part) {
     grid_dependency_sync();
-    __shared__ float As[LRS_KC][LRS_ROWS + 1];      // [k][row]
-    __shared__ float Bs[LRS_KC][LRS_MAX_L];         // [k][col]
+    __shared__ __align__(16) float As[2][LRS_KC][LRS_ROWS + 4];  // [k][row]
+    __shared__ __align__(16) float Bs[2][LRS_KC][LRS_MAX_L];     // [k][col]
     const int r0 = blockIdx.x * LRS_ROWS;
+    const int kb = blockIdx.y * kper, ke = min(inner, kb + kper);
     const int tid = threadIdx.x;
-    // thread -> 4 rows (tid / (c/4) ...) x up to 4 columns: 32 rows x c columns
-    // over 256 threads: each thread holds (32 * c / 256) = c / 8 outputs
-    const int cg = c / 4;                 // column groups of 4
-    const int per_row_threads = cg;       // threads covering one row's columns
-    const int rows_per_pass = LRS_THREADS / per_row_threads;  // rows a pass covers
-    float acc[LRS_MAX_L / 8][4];
-    const int nouts = (LRS_ROWS + rows_per_pass - 1) / rows_per_pass;  // <= c / 8 (c >= 32) or more
+    const int cg = c / 4;
+    const bool active = tid < 16 * cg;
+    const int tr = tid / cg, tc = tid % cg;
+    constexpr int AV = LRS_KC * LRS_ROWS / LRS_THREADS;  // A values per thread per chunk (8)
+    float ra[AV], rb[AV];
+    auto load = [&](int k0) {
 #pragma unroll
-    for (int i = 0; i < LRS_MAX_L / 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
-    const int myc = (tid % per_row_threads) * 4;
-    const int myr = tid / per_row_threads;
-    for (int k0 = 0; k0 < inner; k0 += LRS_KC) {
-        // A chunk -> As[k][row]
-        for (int idx = tid; idx < LRS_KC * LRS_ROWS; idx += LRS_THREADS) {
+        for (int u = 0; u < AV; ++u) {
+            const int idx = tid + u * LRS_THREADS;
             int kk, rr;
-            if (TRANS) { rr = idx % LRS_ROWS; kk = idx / LRS_ROWS; }   // coalesced along rows of A^T (R)
-            else { kk = idx % LRS_KC; rr = idx / LRS_KC; }             // coalesced along inner
+            if (TRANS) { rr = idx % LRS_ROWS; kk = idx / LRS_ROWS; }
+            else { kk = idx % LRS_KC; rr = idx / LRS_KC; }
             const int row = r0 + rr, k = k0 + kk;
-            float v = 0.0f;
-            if (row < R && k < inner) v = TRANS ? A[static_cast<size_t>(k) * R + row] : A[static_cast<size_t>(row) * inner + k];
-            As[kk][rr] = v;
+            ra[u] = (row < R && k < ke) ? (TRANS ? A[static_cast<size_t>(k) * R + row] : A[static_cast<size_t>(row) * inner + k]) : 0.0f;
         }
-        for (int idx = tid; idx < LRS_KC * c; idx += LRS_THREADS) {
+#pragma unroll
+        for (int u = 0; u < AV; ++u) {
+            const int idx = tid + u * LRS_THREADS;
             const int kk = idx / c, j = idx % c;
             const int k = k0 + kk;
-            Bs[kk][j] = (k < inner) ? B[static_cast<size_t>(k) * c + j] : 0.0f;
+            rb[u] = (idx < LRS_KC * c && k < ke) ? B[static_cast<size_t>(k) * c + j] : 0.0f;
         }
-        __syncthreads();
-#pragma unroll 4
-        for (int kk = 0; kk < LRS_KC; ++kk) {
-            const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][myc]);
+    };
+    auto store = [&](int buf) {
 #pragma unroll
-            for (int i = 0; i < LRS_MAX_L / 8; ++i) {
-                if (i < nouts) {
-                    const int rr = myr + i * rows_per_pass;
-                    const float a = (rr < LRS_ROWS) ? As[kk][rr] : 0.0f;
-                    acc[i][0] = fmaf(a, b.x, acc[i][0]);
-                    acc[i][1] = fmaf(a, b.y, acc[i][1]);
-                    acc[i][2] = fmaf(a, b.z, acc[i][2]);
-                    acc[i][3] = fmaf(a, b.w, acc[i][3]);
-                }
+        for (int u = 0; u < AV; ++u) {
+            const int idx = tid + u * LRS_THREADS;
+            int kk, rr;
+            if (TRANS) { rr = idx % LRS_ROWS; kk = idx / LRS_ROWS; }
+            else { kk = idx % LRS_KC; rr = idx / LRS_KC; }
+            As[buf][kk][rr] = ra[u];
+        }
+#pragma unroll
+        for (int u = 0; u < AV; ++u) {
+            const int idx = tid + u * LRS_THREADS;
+            if (idx < LRS_KC * c) Bs[buf][idx / c][idx % c] = rb[u];
+        }
+    };
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
+    int buf = 0;
+    if (kb < ke) {
+        load(kb);
+        store(0);
+    }
+    __syncthreads();
+    for (int k0 = kb; k0 < ke; k0 += LRS_KC) {
+        const bool more = k0 + LRS_KC < ke;
+        if (more) load(k0 + LRS_KC);
+        if (active) {
+#pragma unroll 8
+            for (int kk = 0; kk < LRS_KC; ++kk) {
+                const float4 a = *reinterpret_cast<const float4*>(&As[buf][kk][4 * tr]);
+                const float4 b = *reinterpret_cast<const float4*>(&Bs[buf][kk][4 * tc]);
+                const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
             }
         }
+        if (more) store(buf ^ 1);
         __syncthreads();
+        buf ^= 1;
     }
+    if (!active) return;
+    float* out = part + static_cast<size_t>(blockIdx.y) * R * c;
 #pragma unroll
-    for (int i = 0; i < LRS_MAX_L / 8; ++i) {
-        if (i >= nouts) continue;
-        const int rr = myr + i * rows_per_pass;
-        const int row = r0 + rr;
-        if (rr >= LRS_ROWS || row >= R) continue;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int j = myc + e;
-            if (out) out[static_cast<size_t>(row) * c + j] = acc[i][e];
-            const __nv_bfloat16 h = __float2bfloat16_rn(acc[i][e]);
-            if (out_bf16) out_bf16[static_cast<size_t>(row) * c + j] = *reinterpret_cast<const uint16_t*>(&h);
-            if (out_bf16_t) out_bf16_t[static_cast<size_t>(j) * R + row] = *reinterpret_cast<const uint16_t*>(&h);
-        }
+    for (int i = 0; i < 4; ++i) {
+        const int row = r0 + 4 * tr + i;
+        if (row < R)
+            *reinterpret_cast<float4*>(out + static_cast<size_t>(row) * c + 4 * tc) =
+                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    }
+}
+
+// out = sum over the S splits of part (in split order), as fp32 [R, c],
+// bf16 [R, c] and / or bf16 transposed [c, R] (each optional).
+__global__ void lr_sum_splits(const float* __restrict__ part, int S, int R, int c, float* __restrict__ out,
+                              uint16_t* __restrict__ out_bf16, uint16_t* __restrict__ out_bf16_t) {
+    grid_dependency_sync();
+    const int64_t total = static_cast<int64_t>(R) * c;
+    for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        float v = part[e];
+        for (int sp = 1; sp < S; ++sp) v += part[static_cast<size_t>(sp) * total + e];
+        const int row = static_cast<int>(e / c), j = static_cast<int>(e % c);
+        if (out) out[e] = v;
+        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+        if (out_bf16) out_bf16[e] = *reinterpret_cast<const uint16_t*>(&h);
+        if (out_bf16_t) out_bf16_t[static_cast<size_t>(j) * R + row] = *reinterpret_cast<const uint16_t*>(&h);
     }
 }
 
 // Gram partials: part[b][i][j] = sum over rows of chunk b of Y[row][i] Y[row][j]
 // (fp64, rows in order inside the chunk).  One CTA per chunk of rows_per rows;
 // thread t owns the entries t, t + 256, ... of the l x l matrix.
-__global__ void __launch_bounds__(256) lr_gram_partial(const float* __restrict__ Y, int R, int l, int rows_per,
+template <int L>
+__global__ void __launch_bounds__(256) lr_gram_partial(const float* __restrict__ Y, int R, int rows_per,
                                                        double* __restrict__ part) {
     grid_dependency_sync();
-    __shared__ float rows[32][LRS_MAX_L];
+    constexpr int l = L;
+    __shared__ float rows[32][L];
     const int b = blockIdx.x;
     const int rs = b * rows_per, re = min(R, rs + rows_per);
-    const int ll = l * l;
-    constexpr int OWN = LRS_MAX_L * LRS_MAX_L / 256;
+    constexpr int ll = L * L;
+    constexpr int OWN = (ll + 255) / 256;
     double acc[OWN];
 #pragma unroll
     for (int i = 0; i < OWN; ++i) acc[i] = 0.0;
@@ -154,7 +191,8 @@ __global__ void __launch_bounds__(256) lr_gram_partial(const float* __restrict__
 //         and sets *status = 1.
 // mode 1: H = sum of partials; Jacobi eigen-decomposition H = V diag(w) V^T
 //         (parallel round-robin order, sweeps until the off-diagonal mass
-//         is below 1e-28 of the total or 40 sweeps); then for the r largest
+//         is below 1e-20 of the total -- a norm ratio of 1e-10, far below the
+//         fp32 the results are stored in -- or 40 sweeps); then for the r largest
 //         eigenvalues w_k (descending): out1 [l][r] = V_k w_k^(1/4),
 //         out2 [l][r] = V_k w_k^(-1/4) (fp32), sigma[k] = sqrt(w_k).
 __global__ void __launch_bounds__(256) lr_small_kernel(const double* __restrict__ part, int nparts, int l, int r,
@@ -171,8 +209,17 @@ __global__ void __launch_bounds__(256) lr_small_kernel(const double* __restrict_
     const int tid = threadIdx.x;
     const int ll = l * l;
     for (int e = tid; e < ll; e += 256) {
+        // chunk order, eight partials loaded at a time
         double s = 0.0;
-        for (int b = 0; b < nparts; ++b) s += part[static_cast<size_t>(b) * ll + e];  // chunk order
+        int b = 0;
+        for (; b + 8 <= nparts; b += 8) {
+            double p[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) p[u] = part[static_cast<size_t>(b + u) * ll + e];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) s += p[u];
+        }
+        for (; b < nparts; ++b) s += part[static_cast<size_t>(b) * ll + e];
         Am[e] = s;
     }
     __syncthreads();
@@ -239,7 +286,7 @@ __global__ void __launch_bounds__(256) lr_small_kernel(const double* __restrict_
             atomicAdd(&wsum[1], tot);
         }
         __syncthreads();
-        if (wsum[0] <= 1e-28 * wsum[1]) break;
+        if (wsum[0] <= 1e-20 * wsum[1]) break;  // off-diagonal norm <= 1e-10 of the whole: far below fp32
         for (int step = 0; step < l - 1; ++step) {
             // pairs of this step: (order[i], order[l-1-i]), i < l/2
             if (tid < l / 2) {

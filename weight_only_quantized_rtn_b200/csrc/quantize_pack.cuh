@@ -152,8 +152,13 @@ __global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
                 gs.s = __shfl_sync(0xffffffffu, sj[src_t], src);
                 gs.inv = __shfl_sync(0xffffffffu, ij[src_t], src);
                 gs.normal = gs.s >= 1.17549435e-38f;
-                gs.inv64 = (!gs.normal && gs.s > 0.0f) ? 1.0 / static_cast<double>(gs.s) : 0.0;
-                const uint32_t c4 = gs.normal ? rtn4_f32(v[i], gs.s, gs.inv, 0.5f * gs.s) : pack_codes4(v[i], gs, qmax, unused);
+                uint32_t c4;
+                if (gs.normal) {
+                    c4 = rtn4_f32(v[i], gs.s, gs.inv, 0.5f * gs.s);
+                } else {  // rare: a subnormal (or zero) scale takes the fp64 path
+                    gs.inv64 = (gs.s > 0.0f) ? 1.0 / static_cast<double>(gs.s) : 0.0;
+                    c4 = pack_codes4(v[i], gs, qmax, unused);
+                }
                 // four nibbles (q + 8) at their places among the eight of the word
                 uint32_t w = 0;
 #pragma unroll

@@ -139,7 +139,8 @@ struct Plan {
     int astages = 0;    // resident x: TMEM A-stage ring depth
     uint32_t tmem_cols = 0, acc_col0 = 0, lr_col0 = 0, a_col0 = 0, wtile = 0, wstage = 0, xsub = 0, xstage = 0, red = 0, stage = 0;
     size_t smem = 0;
-    size_t off_x16 = 0, off_xs = 0, off_thl = 0, off_l2t = 0, ws = 0;
+    size_t off_x16 = 0, off_xs = 0, off_thl = 0, off_l2t = 0, off_l1t = 0, ws = 0;
+    bool fused_lr_prep = false;  // int4 + low rank, K <= 4096: x16, xs and T' in one pass (L1 transposed first)
 };
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -163,8 +164,8 @@ constexpr wlq_status kRetryPlan = static_cast<wlq_status>(-100);
 // variant 0: CTA pairs may split K (over up to four pairs of a cluster);
 // variant 1: no split pairs, but 256-token tiles may split K (partial in the
 // ring); variant 2: splits use 128-token tiles (partial beside the ring).
-// Variants 0 and 1 need one tile per cluster; the launcher reports
-// kRetryPlan when the device cannot hold that many clusters.
+// Variant 0 needs one tile per cluster; the launcher reports kRetryPlan when
+// the device cannot hold that many clusters.
 bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms, int variant = 0) {
     p.fmt = fmt;
     p.M = static_cast<int>(M);
@@ -367,6 +368,8 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     if (r) {
         p.off_thl = off; off = align256(off + static_cast<size_t>(M) * p.lr_kb * 64 * 2);
         p.off_l2t = off; off = align256(off + static_cast<size_t>(p.NT) * 128 * p.lr_kb * 64 * 2);
+        p.fused_lr_prep = fmt != wlq::FMT_W8 && K <= 4096;
+        if (p.fused_lr_prep) { p.off_l1t = off; off = align256(off + static_cast<size_t>(r) * K * 2); }
     }
     p.ws = off;
     return true;
@@ -651,6 +654,25 @@ wlq_status launch_prep_x16(const uint16_t* x, int M, int K, __half* x16, float* 
     }
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? WLQ_OK : cuda_fail(e, "prep_x16 launch");
+}
+
+// x16, xs and T' in one pass (int4 + low rank, K <= 4096): 16 rows per CTA.
+wlq_status launch_prep_x16_lr(const uint16_t* x, const uint16_t* l1t, int M, int K, int r, int W, __half* x16,
+                              float* xs, uint16_t* thl, DeviceInfo* d, cudaStream_t s) {
+    const size_t smem = wlq::xlr_smem_bytes(K, r);
+    const int kid = 41 + (r == 16 ? 0 : r == 32 ? 1 : 2);  // 41..43
+    auto kern = (r == 16) ? wlq::prep_x16_lr_kernel<16> : (r == 32) ? wlq::prep_x16_lr_kernel<32>
+                                                                    : wlq::prep_x16_lr_kernel<64>;
+    if (!d->smem_set[kid]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(wlq::xlr_smem_bytes(4096, r)));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        d->smem_set[kid] = true;
+    }
+    const int grid = static_cast<int>(std::min<int64_t>(cdiv(M, wlq::XLR_ROWS), static_cast<int64_t>(d->sms) * 8));
+    launch_k(kern, grid, wlq::XLR_WARPS * 32, smem, s, x, l1t, M, K, W, x16, xs, thl);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? WLQ_OK : cuda_fail(e, "prep_x16_lr launch");
 }
 
 // T = x L1 as [Th | Tl]: 64-row tiles, K split over a cluster of S CTAs
@@ -1052,7 +1074,9 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
     if (fmt != wlq::FMT_W8) {
         __half* x16 = reinterpret_cast<__half*>(ws + p.off_x16);
         xs = reinterpret_cast<float*>(ws + p.off_xs);
-        if ((st = launch_prep_x16(static_cast<const uint16_t*>(x), p.M, p.K, x16, xs, d, s)) != WLQ_OK) return st;
+        if (!p.fused_lr_prep &&
+            (st = launch_prep_x16(static_cast<const uint16_t*>(x), p.M, p.K, x16, xs, d, s)) != WLQ_OK)
+            return st;
         xin = x16;
     }
     uint16_t* thl = nullptr;
@@ -1063,9 +1087,17 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
         l2t = reinterpret_cast<uint16_t*>(ws + p.off_l2t);
         // the branch is folded into the GEMM's accumulator: T' = T / xs (int4) and
         // L2' = L2 / rowf, rowf read from the packed operand
-        if ((st = launch_prep_lr_t(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(L1), xs, p.M, p.K, r,
-                                   W, thl, d, s)) != WLQ_OK)
+        if (p.fused_lr_prep) {
+            uint16_t* l1t = reinterpret_cast<uint16_t*>(ws + p.off_l1t);
+            launch_k(wlq::prep_l1t_kernel, grid_for(K * r, 256, d->sms), 256, 0, s, static_cast<const uint16_t*>(L1),
+                     p.K, r, l1t);
+            if ((st = launch_prep_x16_lr(static_cast<const uint16_t*>(x), l1t, p.M, p.K, r, W,
+                                         reinterpret_cast<__half*>(ws + p.off_x16), xs, thl, d, s)) != WLQ_OK)
+                return st;
+        } else if ((st = launch_prep_lr_t(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(L1), xs, p.M,
+                                          p.K, r, W, thl, d, s)) != WLQ_OK) {
             return st;
+        }
         const float* rowf = reinterpret_cast<const float*>(static_cast<const uint8_t*>(packed) +
                                                            static_cast<size_t>(NT) * p.KT * wlq::tile_bytes(fmt));
         launch_k(wlq::prep_lr_l2t_kernel, grid_for(NT * 128 * (W / 8), 256, d->sms), 256, 0, s,
@@ -1163,8 +1195,9 @@ namespace {
 // l x l / l x r matrices.
 constexpr int LR_GRAM_ROWS = 64;
 struct LrLayout {
-    size_t y0, y1, z0, z1, parts, rinv, b1, b2, total;
+    size_t y0, y1, z0, z1, parts, rinv, b1, b2, gpart, total;
 };
+constexpr int LR_MAX_GSPLIT = 8;  // inner-dimension splits of the skinny GEMM
 LrLayout lr_layout(int64_t N, int64_t K, int l, int r) {
     LrLayout o;
     size_t off = 0;
@@ -1178,6 +1211,7 @@ LrLayout lr_layout(int64_t N, int64_t K, int l, int r) {
     o.rinv = take(static_cast<size_t>(l) * l * 4);
     o.b1 = take(static_cast<size_t>(l) * r * 4);
     o.b2 = take(static_cast<size_t>(l) * r * 4);
+    o.gpart = take(static_cast<size_t>(LR_MAX_GSPLIT) * std::max(N, K) * l * 4);
     o.total = off;
     return o;
 }
@@ -1187,11 +1221,20 @@ bool lr_shape_ok(int64_t N, int64_t K, int r, int l, int q) {
            K >= l && N <= (int64_t(1) << 24) && K <= (int64_t(1) << 24);
 }
 
+// out = op(A) B through the skinny GEMM: the inner range split S ways (S <= 8,
+// each at least 256 long) until the CTAs cover the SMs twice, the splits'
+// partials (in `gpart`) added in order by a second pass.
 template <bool TRANS>
 void lr_gemm(const float* A, const float* B, int R, int inner, int c, float* out, uint16_t* out_bf16,
-             uint16_t* out_bf16_t, cudaStream_t s) {
-    launch_k(wlq::lr_skinny_gemm<TRANS>, static_cast<unsigned>(cdiv(R, wlq::LRS_ROWS)), wlq::LRS_THREADS, 0, s, A, B, R,
-             inner, c, out, out_bf16, out_bf16_t);
+             uint16_t* out_bf16_t, float* gpart, int sms, cudaStream_t s) {
+    const int tiles = static_cast<int>(cdiv(R, wlq::LRS_ROWS));
+    int S = 1;
+    while (S * 2 <= LR_MAX_GSPLIT && tiles * S < 2 * sms && inner / (S * 2) >= 256) S *= 2;
+    const int kper = static_cast<int>(cdiv(cdiv(inner, S), wlq::LRS_KC) * wlq::LRS_KC);
+    launch_k(wlq::lr_skinny_gemm<TRANS>, dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(S), 1),
+             wlq::LRS_THREADS, 0, s, A, B, R, inner, c, kper, gpart);
+    launch_k(wlq::lr_sum_splits, grid_for(static_cast<int64_t>(R) * c, 256, sms), 256, 0, s,
+             static_cast<const float*>(gpart), S, R, c, out, out_bf16, out_bf16_t);
 }
 
 wlq_status lr_small(const double* parts, int nparts, int l, int r, int mode, float* o1, float* o2, float* sigma,
@@ -1207,6 +1250,12 @@ wlq_status lr_small(const double* parts, int nparts, int l, int r, int mode, flo
     return WLQ_OK;
 }
 
+void lr_gram(const float* Y, int R, int l, double* parts, cudaStream_t s) {
+    const int nparts = static_cast<int>(cdiv(R, LR_GRAM_ROWS));
+    if (l == 32) launch_k(wlq::lr_gram_partial<32>, nparts, 256, 0, s, Y, R, LR_GRAM_ROWS, parts);
+    else launch_k(wlq::lr_gram_partial<64>, nparts, 256, 0, s, Y, R, LR_GRAM_ROWS, parts);
+}
+
 // Y <- orth(Y) by CholeskyQR2 (Y [R, l] in `cur`, `tmp` the same size); the
 // orthonormal result ends in `cur`.
 wlq_status lr_orth(float* cur, float* tmp, int R, int l, const LrLayout& L, uint8_t* ws, DeviceInfo* d,
@@ -1216,9 +1265,9 @@ wlq_status lr_orth(float* cur, float* tmp, int R, int l, const LrLayout& L, uint
     const int nparts = static_cast<int>(cdiv(R, LR_GRAM_ROWS));
     wlq_status st;
     for (int pass = 0; pass < 2; ++pass) {
-        launch_k(wlq::lr_gram_partial, nparts, 256, 0, s, static_cast<const float*>(cur), R, l, LR_GRAM_ROWS, parts);
+        lr_gram(cur, R, l, parts, s);
         if ((st = lr_small(parts, nparts, l, 0, 0, rinv, nullptr, nullptr, d, s)) != WLQ_OK) return st;
-        lr_gemm<false>(cur, rinv, R, l, l, tmp, nullptr, nullptr, s);
+        lr_gemm<false>(cur, rinv, R, l, l, tmp, nullptr, nullptr, reinterpret_cast<float*>(ws + L.gpart), d->sms, s);
         std::swap(cur, tmp);
     }
     // two swaps: the result is back in the caller's `cur`
@@ -1255,27 +1304,28 @@ wlq_status wlq_lowrank_split(const float* W, int64_t N, int64_t K, int r, int l,
     float* y1 = reinterpret_cast<float*>(ws + L.y1);
     float* z0 = reinterpret_cast<float*>(ws + L.z0);
     float* z1 = reinterpret_cast<float*>(ws + L.z1);
+    float* gpart = reinterpret_cast<float*>(ws + L.gpart);
     const int n = static_cast<int>(N), k = static_cast<int>(K);
     // Y = W^T Omega, orthonormalised
-    lr_gemm<true>(W, omega, k, n, l, y0, nullptr, nullptr, s);
+    lr_gemm<true>(W, omega, k, n, l, y0, nullptr, nullptr, gpart, d->sms, s);
     if ((st = lr_orth(y0, y1, k, l, L, ws, d, s)) != WLQ_OK) return st;
     for (int it = 0; it < power_iters; ++it) {
-        lr_gemm<false>(W, y0, n, k, l, z0, nullptr, nullptr, s);   // Z = W Q
+        lr_gemm<false>(W, y0, n, k, l, z0, nullptr, nullptr, gpart, d->sms, s);   // Z = W Q
         if ((st = lr_orth(z0, z1, n, l, L, ws, d, s)) != WLQ_OK) return st;
-        lr_gemm<true>(W, z0, k, n, l, y0, nullptr, nullptr, s);    // Y = W^T P
+        lr_gemm<true>(W, z0, k, n, l, y0, nullptr, nullptr, gpart, d->sms, s);    // Y = W^T P
         if ((st = lr_orth(y0, y1, k, l, L, ws, d, s)) != WLQ_OK) return st;
     }
     // C = W Q; H = C^T C = U~ Lambda U~^T
-    lr_gemm<false>(W, y0, n, k, l, z0, nullptr, nullptr, s);
+    lr_gemm<false>(W, y0, n, k, l, z0, nullptr, nullptr, gpart, d->sms, s);
     double* parts = reinterpret_cast<double*>(ws + L.parts);
     const int nparts = static_cast<int>(cdiv(N, LR_GRAM_ROWS));
-    launch_k(wlq::lr_gram_partial, nparts, 256, 0, s, static_cast<const float*>(z0), n, l, LR_GRAM_ROWS, parts);
+    lr_gram(z0, n, l, parts, s);
     float* b1 = reinterpret_cast<float*>(ws + L.b1);
     float* b2 = reinterpret_cast<float*>(ws + L.b2);
     if ((st = lr_small(parts, nparts, l, r, 1, b1, b2, sigma, d, s)) != WLQ_OK) return st;
     // L1 = Q U~_r Lambda_r^(1/4) [K, r]; L2 = (C U~_r Lambda_r^(-1/4))^T [r, N]
-    lr_gemm<false>(y0, b1, k, l, r, nullptr, static_cast<uint16_t*>(L1), nullptr, s);
-    lr_gemm<false>(z0, b2, n, l, r, nullptr, nullptr, static_cast<uint16_t*>(L2), s);
+    lr_gemm<false>(y0, b1, k, l, r, nullptr, static_cast<uint16_t*>(L1), nullptr, gpart, d->sms, s);
+    lr_gemm<false>(z0, b2, n, l, r, nullptr, nullptr, static_cast<uint16_t*>(L2), gpart, d->sms, s);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "low-rank split launch");
     return WLQ_OK;
