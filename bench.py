@@ -322,6 +322,69 @@ def time_lowrank_producer(wlq, torch, dev, evict_l2, reps=3):
             "timing": "each call alone, L2 flushed before, CUDA events, median of %d" % reps}
 
 
+def time_w4a4(wlq, torch, dev, evict_l2, tc_peak, reps=3):
+    """The NVFP4 W4A4 forward on the SVDQuant projection ([4096, 4096], r = 32):
+    x quantized to NVFP4, the low-rank pre-pass, the block-scaled GEMM with the
+    low-rank accumulator; graphs of back-to-back forwards over weight copies
+    (> 3x L2), L2 flushed before each replay.  FP4 peak: the measured bf16
+    figure x 4 (the nominal dense fp4 / bf16 ratio, 9 / 2.25)."""
+    N = K = wi.HIDDEN
+    r = wi.RANK
+    W = torch.from_numpy(wi.svdq_w4_lr(1)["W"]).to(dev)
+    wq, ws, wg = wlq.nvfp4_quantize(W)
+    del W
+    wbytes = wq.numel() + ws.numel()
+    copies = int(min(16, max(1, -(-3 * L2_BYTES // wbytes))))
+    units = max(8, copies)
+    ops = [(wq, ws, wg)] + [(wq.clone(), ws.clone(), wg.clone()) for _ in range(copies - 1)]
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+    L1 = bf(wi.normal_bf16(wi.rng(5, 3), (K, r), 0.05))
+    L2 = bf(wi.normal_bf16(wi.rng(5, 4), (r, N), 0.05))
+    b = bf(wi.bias(5, 2, N))
+    out = {}
+    fp4_peak = 4.0 * tc_peak
+    for M in (256, 4096):
+        x = bf(wi.activations(5, 1, M, K))
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        wsp = wlq.w4a4_workspace(M, N, K, r, device=dev)
+
+        def unit(i):
+            q, s_, g_ = ops[i % copies]
+            wlq.w4a4_linear_into(y, x, q, s_, g_, N, K, b, L1, L2, workspace=wsp)
+
+        for i in range(3):
+            unit(i)
+        torch.cuda.synchronize()
+        wlq.check_status()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(units):
+                unit(i)
+        g.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            evict_l2()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e-3 / units)
+        wlq.check_status()
+        t = statistics.median(ts)
+        flops = 2.0 * M * N * K + 2.0 * M * r * (K + N)
+        out["m%d" % M] = {"M": M, "us": round(t * 1e6, 2), "tflops": round(flops / t / 1e12, 1),
+                          "fp4_tensor_frac": round(flops / t / 1e12 / fp4_peak, 4),
+                          "bf16_tensor_frac": round(flops / t / 1e12 / tc_peak, 4)}
+        del g
+    out["workload"] = ("W4A4 NVFP4 forward, [4096, 4096] weight (SVDQuant recipe's residual), r = 32, bf16 x "
+                       "quantized per call; weight copies %d, units per replay %d" % (copies, units))
+    out["fp4_peak_tflops"] = round(fp4_peak, 1)
+    out["fp4_peak_source"] = "measured bf16 burst x 4 (nominal dense fp4 / bf16 ratio)"
+    return out
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
@@ -625,6 +688,7 @@ def run_gpu(args):
     if not args.no_configs:
         line["configs"] = time_workloads(wlq, torch, dev, evict_l2, hbm_peak, tc_peak)
         line["lowrank_producer"] = time_lowrank_producer(wlq, torch, dev, evict_l2)
+        line["w4a4_nvfp4"] = time_w4a4(wlq, torch, dev, evict_l2, tc_peak)
         line["configs_timing"] = ("per unit = one CUDA-graph replay of back-to-back units / units; units rotate over "
                                   "weight copies totalling >= 3x L2 and L2 is flushed before each replay; "
                                   "median of 3 replays; bf16 outputs")

@@ -154,6 +154,36 @@ wlq_status wlq_quantize_fp8(const void* W, int w_dtype, int64_t N, int64_t K, in
                             uint8_t* codes, float* scales, void* stream);
 
 /*
+ * NVFP4 quantization: the 4-bit format of the W4A4 SVDQuant kernels on
+ * Blackwell ("Nunchaku Lite: loading and running 4-bit SVDQuant", section
+ * "hardware and precision support": the NVFP4 variant of svdq_w4a4 runs on
+ * Blackwell GPUs, B200 included; section "why it matters": weights AND
+ * activations in 4 bits).  The pages name the format without defining it;
+ * it is read as NVIDIA's NVFP4:
+ *   g   = fp32(amax(X) / 2688)                 (one scale per tensor)
+ *   s_b = E4M3 nearest a_b / (6 g)             (a_b = max |x| of 16 inputs of
+ *                                               a row; ties to even, <= 448)
+ *   q   = E2M1 nearest x / (s_b g)             (values 0, .5, 1, 1.5, 2, 3, 4, 6
+ *                                               with sign; ties to even; <= 6)
+ * with every rounding decision exact (see nvfp4.cuh).  An all-zero block
+ * (or one whose scale rounds to 0) gets codes 0.
+ * X      : [rows, K] fp32 or bf16 (x_dtype), 16-byte aligned; K % 64 == 0
+ * codes  : uint8 [rows, K / 2]: input k in byte k / 2, low nibble for even k;
+ *          a code is sign << 3 | magnitude index; 16-byte aligned
+ * scales : wlq_nvfp4_scales_bytes(rows, K) bytes, E4M3 bits in the tensor
+ *          cores' 512-byte atom layout: atom (t, a) = 128 rows from 128 t,
+ *          inputs 64 a .. 64 a + 63, at ((t * KA) + a) * 512 with
+ *          KA = ceil(K / 256) * 4; the scale of row 128 t + 32 i + j, block
+ *          4 a + c (16 inputs each) at byte 16 j + 4 i + c of its atom; padding
+ *          rows and blocks hold 0; 16-byte aligned
+ * gscale : fp32 [2], 8-byte aligned: [0] = g, [1] = amax(X)
+ * Non-finite inputs set the device error word (WLQ_ERR_NONFINITE).
+ */
+size_t wlq_nvfp4_scales_bytes(int64_t rows, int64_t K);
+wlq_status wlq_nvfp4_quantize(const void* X, int x_dtype, int64_t rows, int64_t K, void* codes,
+                              void* scales, float* gscale, void* stream);
+
+/*
  * Inverse of the code part of wlq_pack: packed -> codes int8 [N, K].  No
  * passage of the pages defines it: a layout helper that lets a caller (and
  * the tests) read the packed codes back.
@@ -296,6 +326,43 @@ const char* wlq_last_error(void);
 
 /* Library version, e.g. "0.1.0". */
 const char* wlq_version(void);
+
+/*
+ * The W4A4 Linear of the NVFP4 SVDQuant path ("Nunchaku Lite", section "how
+ * it works": svdq_w4a4 = 4-bit weights and activations plus the SVDQuant
+ * low-rank correction, used for the attention and MLP projections):
+ *   y[m, n] = g_x g_w sum_k qx[m,k] sx[m,k/16] qw[n,k] sw[n,k/16]
+ *             + sum_j (sum_k x[m,k] L1[k,j]) L2[j,n] + b[n]
+ * on the block-scaled tensor cores (E2M1 x E2M1 products scaled by UE4M3
+ * block scales, fp32 accumulation); the low-rank term from the 16-bit x
+ * through a bf16 hi/lo split (relative error ~2^-16) into a second fp32
+ * accumulator.
+ * xq, xs, xg : the activations [M, K] as wlq_nvfp4_quantize writes them
+ *              (xg: its gscale, read on the device)
+ * x          : bf16 [M, K] (only read when r > 0; may be NULL otherwise)
+ * wq, ws, wg : the weights [N, K] from wlq_nvfp4_quantize
+ * bias [N], L1 [K, r], L2 [r, N]: bf16 (bias may be NULL; r in {0,16,32,64})
+ * y          : [M, N] in y_dtype
+ * workspace  : wlq_nvfp4_linear_workspace(M, N, K, r) bytes (0 when r == 0),
+ *              16-byte aligned
+ * K % 64 == 0; codes, scales, x, L1 and the workspace 16-byte aligned.
+ */
+size_t wlq_nvfp4_linear_workspace(int64_t M, int64_t N, int64_t K, int r);
+wlq_status wlq_nvfp4_linear(const void* xq, const void* xs, const float* xg, const void* x, int64_t M,
+                            const void* wq, const void* ws, const float* wg, int64_t N, int64_t K,
+                            const void* bias, const void* L1, const void* L2, int r, void* y,
+                            int y_dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * The W4A4 forward from bf16 activations: x [M, K] is quantized to NVFP4 in
+ * the workspace (wlq_nvfp4_quantize), then wlq_nvfp4_linear runs.  Same
+ * arguments as wlq_nvfp4_linear otherwise; workspace: wlq_w4a4_workspace()
+ * bytes (never 0 for M, N > 0), 16-byte aligned.
+ */
+size_t wlq_w4a4_workspace(int64_t M, int64_t N, int64_t K, int r);
+wlq_status wlq_w4a4_linear(const void* x, int64_t M, const void* wq, const void* ws, const float* wg,
+                           int64_t N, int64_t K, const void* bias, const void* L1, const void* L2, int r,
+                           void* y, int y_dtype, void* workspace, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -15,7 +15,11 @@ HEADER = os.path.join(ROOT, "include", "wlq.h")
 
 @pytest.fixture(scope="module")
 def lib():
-    from weight_only_quantized_rtn_b200 import _build
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_wlq_build", os.path.join(ROOT, "weight_only_quantized_rtn_b200", "_build.py"))
+    _build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(_build)
     path = _build.build()
     L = ctypes.CDLL(path)
     L.wlq_packed_bytes.restype = ctypes.c_size_t
@@ -30,7 +34,7 @@ def lib():
 def declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(wlq_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(wlq_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -169,3 +173,51 @@ def test_noalloc_argument_errors_match_the_workspace_entry_point(lib):
     for args, want in cases:
         assert lib.wlq_linear(*args, None, 0, None) == want, args
         assert lib.wlq_linear_noalloc(*args, None) == want, args
+
+
+def test_nvfp4_sizes_and_argument_errors(lib):
+    """NVFP4 scale storage: one 512-byte atom per 128 rows and 64 inputs, K
+    padded to 256 and rows to 128; argument checks of the NVFP4 calls come
+    before any device access."""
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    lib.wlq_nvfp4_scales_bytes.restype = sz
+    lib.wlq_nvfp4_scales_bytes.argtypes = [i64, i64]
+    assert lib.wlq_nvfp4_scales_bytes(4096, 4096) == 32 * 64 * 512     # = 4096 * 4096 / 16 bytes
+    assert lib.wlq_nvfp4_scales_bytes(130, 320) == 2 * 8 * 512          # rows -> 256, K -> 512
+    assert lib.wlq_nvfp4_scales_bytes(4, 96) == 0                       # K % 64
+    lib.wlq_nvfp4_quantize.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp]
+    assert lib.wlq_nvfp4_quantize(vp(16), 2, 4, 64, vp(16), vp(16), vp(16), None) == 4    # input dtype
+    assert lib.wlq_nvfp4_quantize(vp(16), 0, 4, 96, vp(16), vp(16), vp(16), None) == 2    # K % 64
+    assert lib.wlq_nvfp4_quantize(None, 0, 4, 64, vp(16), vp(16), vp(16), None) == 1      # null
+    assert lib.wlq_nvfp4_quantize(vp(16), 0, 4, 64, vp(24), vp(16), vp(16), None) == 3    # codes misaligned
+    assert lib.wlq_nvfp4_quantize(vp(16), 0, 4, 64, vp(16), vp(16), vp(12), None) == 3    # gscale misaligned
+    lib.wlq_nvfp4_linear_workspace.restype = sz
+    lib.wlq_nvfp4_linear_workspace.argtypes = [i64, i64, i64, i32]
+    assert lib.wlq_nvfp4_linear_workspace(256, 4096, 4096, 0) == 0
+    # r = 32: T [M, 128] and L2 [N_pad, 128] in bf16, each 256-byte aligned
+    assert lib.wlq_nvfp4_linear_workspace(200, 300, 512, 32) == 200 * 128 * 2 + 384 * 128 * 2
+    assert lib.wlq_nvfp4_linear_workspace(200, 300, 512, 8) == 0        # bad rank
+    lib.wlq_w4a4_workspace.restype = sz
+    lib.wlq_w4a4_workspace.argtypes = [i64, i64, i64, i32]
+    # codes M * K / 2, scale atoms, 256 bytes for the tensor scale, then the Linear's own
+    assert lib.wlq_w4a4_workspace(256, 4096, 4096, 0) == 256 * 2048 + 2 * 64 * 512 + 256
+    lib.wlq_nvfp4_linear.argtypes = [vp, vp, vp, vp, i64, vp, vp, vp, i64, i64, vp, vp, vp, i32, vp, i32, vp, sz, vp]
+    ok = dict(xq=vp(16), xs=vp(16), xg=vp(16), x=vp(16), M=4, wq=vp(16), ws=vp(16), wg=vp(16), N=64, K=64,
+              bias=None, L1=None, L2=None, r=0, y=vp(16), yd=0)
+    cases = [
+        (dict(K=96), 2), (dict(r=8), 2), (dict(r=16), 1), (dict(yd=3), 1), (dict(M=-1), 1),
+        (dict(xq=None), 1), (dict(wg=None), 1), (dict(xs=vp(24)), 3), (dict(y=vp(18)), 3),
+        (dict(M=0, xq=None), 0),
+    ]
+    for change, want in cases:
+        a = dict(ok, **change)
+        got = lib.wlq_nvfp4_linear(a["xq"], a["xs"], a["xg"], a["x"], a["M"], a["wq"], a["ws"], a["wg"], a["N"],
+                                   a["K"], a["bias"], a["L1"], a["L2"], a["r"], a["y"], a["yd"], None, 0, None)
+        assert got == want, (change, got)
+    lib.wlq_w4a4_linear.argtypes = [vp, i64, vp, vp, vp, i64, i64, vp, vp, vp, i32, vp, i32, vp, sz, vp]
+    assert lib.wlq_w4a4_linear(vp(16), 4, vp(16), vp(16), vp(16), 64, 64, None, None, None, 0, vp(16), 0,
+                               None, 0, None) == 6                      # no workspace
+    assert lib.wlq_w4a4_linear(None, 4, vp(16), vp(16), vp(16), 64, 64, None, None, None, 0, vp(16), 0,
+                               vp(256), 1 << 20, None) == 1            # null x
+    assert lib.wlq_w4a4_linear(vp(16), 4, vp(16), vp(16), vp(16), 64, 96, None, None, None, 0, vp(16), 0,
+                               vp(256), 1 << 20, None) == 2            # K % 64

@@ -26,11 +26,13 @@ STATUS_NAMES = {
 }
 EXPORTS = ("wlq_quantize", "wlq_quantize_pack", "wlq_quantize_ex", "wlq_quantize_fp8", "wlq_packed_bytes",
            "wlq_pack", "wlq_unpack", "wlq_linear_workspace", "wlq_linear", "wlq_linear_noalloc",
-           "wlq_lowrank_workspace", "wlq_lowrank_split", "wlq_lowrank_residual", "wlq_get_status",
+           "wlq_lowrank_workspace", "wlq_lowrank_split", "wlq_lowrank_residual", "wlq_nvfp4_scales_bytes",
+           "wlq_nvfp4_quantize", "wlq_nvfp4_linear_workspace", "wlq_nvfp4_linear", "wlq_w4a4_workspace",
+           "wlq_w4a4_linear", "wlq_get_status",
            "wlq_probe_wait_timeout", "wlq_set_grid_limit", "wlq_last_error", "wlq_version")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError("libwlq.so is not built; run `python -m weight_only_quantized_rtn_b200._build`")
+    raise ImportError("libwlq.so is not built; run `python weight_only_quantized_rtn_b200/_build.py`")
 
 lib = ctypes.CDLL(LIB_PATH)
 _i64, _i32, _vp, _sz, _u64 = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint64
@@ -50,6 +52,16 @@ lib.wlq_lowrank_workspace.argtypes = [_i64, _i64, _i32, _i32]
 lib.wlq_lowrank_workspace.restype = _sz
 lib.wlq_lowrank_split.argtypes = [_vp, _i64, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 lib.wlq_lowrank_residual.argtypes = [_vp, _vp, _vp, _i64, _i64, _i32, _vp, _vp]
+lib.wlq_nvfp4_scales_bytes.argtypes = [_i64, _i64]
+lib.wlq_nvfp4_scales_bytes.restype = _sz
+lib.wlq_nvfp4_quantize.argtypes = [_vp, _i32, _i64, _i64, _vp, _vp, _vp, _vp]
+lib.wlq_nvfp4_linear_workspace.argtypes = [_i64, _i64, _i64, _i32]
+lib.wlq_nvfp4_linear_workspace.restype = _sz
+lib.wlq_nvfp4_linear.argtypes = [_vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _i32, _vp, _i32,
+                                 _vp, _sz, _vp]
+lib.wlq_w4a4_workspace.argtypes = [_i64, _i64, _i64, _i32]
+lib.wlq_w4a4_workspace.restype = _sz
+lib.wlq_w4a4_linear.argtypes = [_vp, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _sz, _vp]
 lib.wlq_get_status.argtypes = [_vp]
 lib.wlq_probe_wait_timeout.argtypes = [_u64, _vp]
 lib.wlq_set_grid_limit.argtypes = [_i32]
@@ -57,7 +69,8 @@ lib.wlq_set_grid_limit.restype = None
 lib.wlq_last_error.restype = ctypes.c_char_p
 lib.wlq_version.restype = ctypes.c_char_p
 for _f in ("wlq_quantize", "wlq_quantize_pack", "wlq_quantize_ex", "wlq_quantize_fp8", "wlq_pack", "wlq_unpack", "wlq_linear",
-           "wlq_linear_noalloc", "wlq_lowrank_split", "wlq_lowrank_residual", "wlq_get_status", "wlq_probe_wait_timeout"):
+           "wlq_linear_noalloc", "wlq_lowrank_split", "wlq_lowrank_residual", "wlq_nvfp4_quantize", "wlq_nvfp4_linear",
+           "wlq_w4a4_linear", "wlq_get_status", "wlq_probe_wait_timeout"):
     getattr(lib, _f).restype = ctypes.c_int
 
 
@@ -229,6 +242,59 @@ def lowrank_residual(W: torch.Tensor, L1: torch.Tensor, L2: torch.Tensor, stream
     R = torch.empty_like(W)
     _check(lib.wlq_lowrank_residual(_ptr(W), _ptr(L1), _ptr(L2), N, K, r, _ptr(R), _stream(stream)))
     return R
+
+
+def nvfp4_scales_bytes(rows: int, K: int) -> int:
+    return int(lib.wlq_nvfp4_scales_bytes(rows, K))
+
+
+def nvfp4_quantize(X: torch.Tensor, stream=None):
+    """NVFP4 quantization of fp32 or bf16 X [rows, K] -> (codes uint8 [rows, K/2]
+    (two E2M1 codes a byte, low nibble first), scales uint8 (E4M3, the MMA's
+    512-byte atom layout), gscale fp32 [2] = (tensor scale, amax))."""
+    assert X.is_cuda and X.is_contiguous()
+    rows, K = X.shape
+    codes = torch.empty((rows, K // 2), dtype=torch.uint8, device=X.device)
+    scales = torch.empty(max(nvfp4_scales_bytes(rows, K), 16), dtype=torch.uint8, device=X.device)
+    gscale = torch.empty(2, dtype=torch.float32, device=X.device)
+    _check(lib.wlq_nvfp4_quantize(_ptr(X), _in_dtype(X), rows, K, _ptr(codes), _ptr(scales), _ptr(gscale),
+                                  _stream(stream)))
+    return codes, scales, gscale
+
+
+def nvfp4_linear_into(y, xq, xs, xg, wq, ws, wg, N, K, x=None, bias=None, L1=None, L2=None, workspace=None,
+                      stream=None):
+    """y = deq(xq) deq(wq)^T [+ (x L1) L2] [+ b] (NVFP4 operands from nvfp4_quantize)."""
+    M = xq.shape[0]
+    r = 0 if L1 is None else L1.shape[1]
+    out = OUT_F32 if y.dtype == torch.float32 else OUT_BF16
+    if workspace is None:
+        n = int(lib.wlq_nvfp4_linear_workspace(M, N, K, r))
+        workspace = torch.empty(n, dtype=torch.uint8, device=y.device) if n else None
+    ws_n = 0 if workspace is None else workspace.numel()
+    _check(lib.wlq_nvfp4_linear(_ptr(xq), _ptr(xs), _ptr(xg), _ptr(x), M, _ptr(wq), _ptr(ws), _ptr(wg), N, K,
+                                _ptr(bias), _ptr(L1), _ptr(L2), r, _ptr(y), out, _ptr(workspace), ws_n,
+                                _stream(stream)))
+    return y
+
+
+def w4a4_workspace(M: int, N: int, K: int, r: int = 0, device="cuda"):
+    n = int(lib.wlq_w4a4_workspace(M, N, K, r))
+    return torch.empty(n, dtype=torch.uint8, device=device) if n else None
+
+
+def w4a4_linear_into(y, x, wq, ws, wg, N, K, bias=None, L1=None, L2=None, workspace=None, stream=None):
+    """The W4A4 forward from bf16 x [M, K]: x quantized to NVFP4 in the
+    workspace, then y = deq(xq) deq(wq)^T [+ (x L1) L2] [+ b]."""
+    M = x.shape[0]
+    r = 0 if L1 is None else L1.shape[1]
+    out = OUT_F32 if y.dtype == torch.float32 else OUT_BF16
+    if workspace is None:
+        workspace = w4a4_workspace(M, N, K, r, device=x.device)
+    ws_n = 0 if workspace is None else workspace.numel()
+    _check(lib.wlq_w4a4_linear(_ptr(x), M, _ptr(wq), _ptr(ws), _ptr(wg), N, K, _ptr(bias), _ptr(L1), _ptr(L2), r,
+                               _ptr(y), out, _ptr(workspace), ws_n, _stream(stream)))
+    return y
 
 
 def get_status(stream=None) -> int:

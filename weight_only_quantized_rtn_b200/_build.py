@@ -1,6 +1,6 @@
 """Build libwlq.so (sm_100a) in-tree with nvcc.
 
-    python -m weight_only_quantized_rtn_b200._build [--verbose]
+    python weight_only_quantized_rtn_b200/_build.py [--verbose]
 """
 from __future__ import annotations
 

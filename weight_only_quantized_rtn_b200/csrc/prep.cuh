@@ -300,203 +300,47 @@ __global__ void __launch_bounds__(128) prep_lr_t_kernel(const uint16_t* __restri
     }  // row tiles
 }
 
-// L1t[j][k] = L1[k][j] (bf16, [r, K]): the fused pass below reads four
-// consecutive inputs of one rank component as one 8-byte load.
-__global__ void prep_l1t_kernel(const uint16_t* __restrict__ L1, int K, int r, uint16_t* __restrict__ l1t) {
-    grid_dependency_sync();
-    const int64_t total = static_cast<int64_t>(K) * r;
-    for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
-         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int j = static_cast<int>(e / K), k = static_cast<int>(e % K);  // coalesced writes along k
-        l1t[e] = L1[static_cast<size_t>(k) * r + j];
-    }
-}
-
-// x -> x16, xs and T' = (x L1) / xs = (x L1) 2^f in one pass over x (int4
-// weights with a low-rank term, K <= 4096).  A CTA holds 16 rows of x in
-// shared memory (the whole K), so each row's maximum -- which x16's scale
-// needs before any element is converted -- is known without a second read.
-// T is formed from the bf16 rows on the tensor cores (m16n8k16, fp32
-// accumulate; the 8 warps split K, their partials added in warp order; each
-// warp fetches the L1 fragments of four steps before using any), with
-// the inputs of an MMA renumbered so that lane (g, t) takes inputs 4t..4t+3
-// of its 16: A from one 8-byte shared-memory load per row, B from one 8-byte
-// load of L1t.  Same x16 / xs arithmetic as prep_x16_kernel; T' written as
-// [T'h | T'l | T'h | 0 ...] like prep_lr_t_kernel.
-constexpr int XLR_ROWS = 16;
-constexpr int XLR_WARPS = 8;
-__host__ __device__ constexpr size_t xlr_smem_bytes(int K, int r) {
-    return 128 + static_cast<size_t>(XLR_ROWS) * (K + 8) * 2 + static_cast<size_t>(XLR_WARPS) * XLR_ROWS * r * 4 + 256;
-}
-template <int R>
-__global__ void __launch_bounds__(XLR_WARPS * 32) prep_x16_lr_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ l1t,
-                                                          int M, int K, int W, __half* __restrict__ x16,
-                                                          float* __restrict__ xs, uint16_t* __restrict__ thl) {
-    extern __shared__ uint8_t xlr_smem_raw[];
-    uint8_t* base = xlr_smem_raw + ((128u - (smem_u32(xlr_smem_raw) & 127u)) & 127u);
-    const int KP = K + 8;  // row pitch (bf16 elements)
-    uint16_t* slab = reinterpret_cast<uint16_t*>(base);
-    float* tpart = reinterpret_cast<float*>(base + static_cast<size_t>(XLR_ROWS) * KP * 2);  // [8][16][R]
-    uint32_t* rmax = reinterpret_cast<uint32_t*>(tpart + XLR_WARPS * XLR_ROWS * R);      // [16]
-    int* rf = reinterpret_cast<int*>(rmax + XLR_ROWS);                                    // [16]
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int K8 = K / 8;
-    grid_dependency_sync();
-    constexpr int NT_ = XLR_WARPS * 32;
-    for (int m0 = blockIdx.x * XLR_ROWS; m0 < M; m0 += gridDim.x * XLR_ROWS) {
-        // the slab: rows m0..m0+15 (zeros past M), 16-byte asynchronous copies
-        for (int i = tid; i < XLR_ROWS * K8; i += NT_) {
-            const int rr = i / K8, c8 = i % K8;
-            const int m = m0 + rr;
-            const bool ok = m < M;
-            lr_cp16(smem_u32(slab + rr * KP + c8 * 8), ok ? x + static_cast<size_t>(m) * K + c8 * 8 : x, ok);
-        }
-        asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
-        __syncthreads();
-        // row maxima over bf16 magnitude bit patterns (NaN ignored, as fmaxf
-        // does): 16 threads per row (half a warp), then a shuffle reduction
-        {
-            const int rr = tid >> 4, q = tid & 15;
-            uint32_t a = 0;
-            for (int c8 = q; c8 < K8; c8 += 16) {
-                const uint4 v = *reinterpret_cast<const uint4*>(slab + rr * KP + c8 * 8);
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const uint32_t lo = w[e] & 0x7FFFu, hi = (w[e] >> 16) & 0x7FFFu;
-                    a = max(a, lo > 0x7F80u ? 0u : lo);
-                    a = max(a, hi > 0x7F80u ? 0u : hi);
-                }
-            }
-            for (int off = 8; off > 0; off >>= 1) a = max(a, __shfl_xor_sync(0xffffffffu, a, off));
-            if (q == 0) rmax[rr] = a;
-        }
-        // T over this warp's quarter of K (16-input steps)
-        float acc[R / 8][4];
-#pragma unroll
-        for (int jt = 0; jt < R / 8; ++jt) acc[jt][0] = acc[jt][1] = acc[jt][2] = acc[jt][3] = 0.0f;
-        const int ksteps = K / 16;
-        constexpr int B4 = 4;  // steps whose L1 fragments are fetched together
-        for (int st0 = warp; st0 < ksteps; st0 += XLR_WARPS * B4) {
-            uint2 bf[B4][R / 8];
-#pragma unroll
-            for (int u = 0; u < B4; ++u) {
-                const int st = st0 + u * XLR_WARPS;
-                const int k0 = st * 16 + 4 * t;
-#pragma unroll
-                for (int jt = 0; jt < R / 8; ++jt)
-                    bf[u][jt] = (st < ksteps) ? __ldg(reinterpret_cast<const uint2*>(l1t + static_cast<size_t>(jt * 8 + g) * K + k0))
-                                              : make_uint2(0u, 0u);
-            }
-#pragma unroll
-            for (int u = 0; u < B4; ++u) {
-                const int st = st0 + u * XLR_WARPS;
-                if (st >= ksteps) break;
-                const int k0 = st * 16 + 4 * t;
-                const uint2 alo = *reinterpret_cast<const uint2*>(slab + g * KP + k0);
-                const uint2 ahi = *reinterpret_cast<const uint2*>(slab + (g + 8) * KP + k0);
-                const uint32_t a[4] = {alo.x, ahi.x, alo.y, ahi.y};
-#pragma unroll
-                for (int jt = 0; jt < R / 8; ++jt) {
-                    const uint32_t bb[2] = {bf[u][jt].x, bf[u][jt].y};
-                    mma_bf16_16816(acc[jt], a, bb);
-                }
-            }
-        }
-        // this warp's partial: rows g, g + 8; columns 8 jt + 2t, + 1
-#pragma unroll
-        for (int jt = 0; jt < R / 8; ++jt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                tpart[(warp * XLR_ROWS + g + 8 * h) * R + jt * 8 + 2 * t] = acc[jt][2 * h];
-                tpart[(warp * XLR_ROWS + g + 8 * h) * R + jt * 8 + 2 * t + 1] = acc[jt][2 * h + 1];
-            }
-        __syncthreads();
-        if (tid < XLR_ROWS) {
-            const float fa = bf16_bits_to_f32(rmax[tid]);
-            int f = 0;
-            if (fa > 0.0f && isfinite(fa)) {
-                int ex;
-                frexpf(fa, &ex);  // fa in [2^(ex-1), 2^ex)
-                f = 9 - ex;
-            }
-            rf[tid] = f;
-            if (m0 + tid < M) xs[m0 + tid] = ldexpf(1.0f, -f);
-        }
-        __syncthreads();
-        // T' = T 2^f (the warps' partials in warp order), as the bf16 pair
-        for (int i = tid; i < XLR_ROWS * R; i += NT_) {
-            const int rr = i / R, j = i % R;
-            const int m = m0 + rr;
-            if (m >= M) continue;
-            float T = tpart[rr * R + j];
-#pragma unroll
-            for (int w = 1; w < XLR_WARPS; ++w) T += tpart[(w * XLR_ROWS + rr) * R + j];
-            T = ldexpf(T, rf[rr]);  // a power of two: exact
-            uint16_t* out = thl + static_cast<size_t>(m) * W;
-            const __nv_bfloat16 hi = __float2bfloat16_rn(T);
-            const __nv_bfloat16 lo = __float2bfloat16_rn(T - __bfloat162float(hi));
-            out[j] = *reinterpret_cast<const uint16_t*>(&hi);
-            out[R + j] = *reinterpret_cast<const uint16_t*>(&lo);
-            out[2 * R + j] = *reinterpret_cast<const uint16_t*>(&hi);
-            for (int jj = 3 * R + j; jj < W; jj += R) out[jj] = 0;
-        }
-        // x16 = fp16(x 2^f), row by row
-        for (int i = tid; i < XLR_ROWS * K8; i += NT_) {
-            const int rr = i / K8, c8 = i % K8;
-            const int m = m0 + rr;
-            if (m >= M) continue;
-            const uint4 v = *reinterpret_cast<const uint4*>(slab + rr * KP + c8 * 8);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            const int f = rf[rr];
-            uint32_t o[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const __half2 h = __floats2half2_rn(ldexpf(bf16_bits_to_f32(w[e] & 0xFFFFu), f),
-                                                    ldexpf(bf16_bits_to_f32(w[e] >> 16), f));
-                o[e] = *reinterpret_cast<const uint32_t*>(&h);
-            }
-            reinterpret_cast<uint4*>(x16 + static_cast<size_t>(m) * K)[c8] = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-        __syncthreads();  // the slab and partials are rewritten for the next rows
-    }
-}
-
 // L2t[n] = [L2'h(0..r) | L2'h(0..r) | L2'l(0..r) | 0 ...] (width W) with
-// L2' = L2[., n] / rowf[n] (L2 itself where rowf[n] == 0), zero for n >= N.
-// One thread per (row n, 8 columns): the reads of L2 are coalesced across
-// consecutive n, each thread writes one 16-byte piece.
-__global__ void prep_lr_l2t_kernel(const uint16_t* __restrict__ L2, const float* __restrict__ rowf, int N,
-                                   int N_pad, int r, int W, uint16_t* __restrict__ l2t) {
+// L2' = L2[., n] / rowf[n] (L2 itself where rowf[n] == 0 or rowf is null),
+// zero for n >= N.
+// A CTA builds 32 rows of L2t in shared memory: its reads of L2 are 64-byte
+// row pieces (consecutive n), its writes one contiguous 32 * W * 2-byte block.
+constexpr int L2T_ROWS = 32;
+constexpr int L2T_MAX_W = 192;  // lr_kb <= 3
+__global__ void __launch_bounds__(256) prep_lr_l2t_kernel(const uint16_t* __restrict__ L2, const float* __restrict__ rowf,
+                                                          int N, int N_pad, int r, int W, uint16_t* __restrict__ l2t) {
     grid_dependency_sync();
-    const int64_t total = static_cast<int64_t>(N_pad) * (W / 8);
-    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
-         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int n = static_cast<int>(idx % N_pad), c8 = static_cast<int>(idx / N_pad);
-        const float rf = (n < N) ? rowf[n] : 0.0f;
-
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            uint32_t h[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int c = c8 * 8 + 2 * e + u;
-                uint16_t v = 0;
-                if (n < N && c < 3 * r) {
-                    const float l2 = bf16_bits_to_f32(L2[static_cast<size_t>(c % r) * N + n]);
-                    const float l = (rf != 0.0f) ? l2 / rf : l2;
-                    const __nv_bfloat16 hi = __float2bfloat16_rn(l);
-                    const __nv_bfloat16 lo = __float2bfloat16_rn(l - __bfloat162float(hi));
-                    const __nv_bfloat16 out = (c < 2 * r) ? hi : lo;
-                    v = *reinterpret_cast<const uint16_t*>(&out);
-                }
-                h[u] = v;
+    __shared__ __align__(16) uint16_t tile[L2T_ROWS][L2T_MAX_W + 8];
+    const int tid = threadIdx.x;
+    for (int n0 = blockIdx.x * L2T_ROWS; n0 < N_pad; n0 += gridDim.x * L2T_ROWS) {
+        for (int e = tid; e < L2T_ROWS * r; e += 256) {
+            const int j = e / L2T_ROWS, nn = e % L2T_ROWS, n = n0 + nn;
+            uint16_t hb = 0, lb = 0;
+            if (n < N) {
+                const float rf = rowf ? rowf[n] : 0.0f;
+                const float l2 = bf16_bits_to_f32(L2[static_cast<size_t>(j) * N + n]);
+                const float l = (rf != 0.0f) ? l2 / rf : l2;
+                const __nv_bfloat16 hi = __float2bfloat16_rn(l);
+                const __nv_bfloat16 lo = __float2bfloat16_rn(l - __bfloat162float(hi));
+                hb = *reinterpret_cast<const uint16_t*>(&hi);
+                lb = *reinterpret_cast<const uint16_t*>(&lo);
             }
-            w[e] = h[0] | (h[1] << 16);
+            tile[nn][j] = hb;
+            tile[nn][r + j] = hb;
+            tile[nn][2 * r + j] = lb;
         }
-        reinterpret_cast<uint4*>(l2t + static_cast<size_t>(n) * W)[c8] = make_uint4(w[0], w[1], w[2], w[3]);
+        for (int e = tid; e < L2T_ROWS * (W - 3 * r); e += 256) {
+            const int nn = e / (W - 3 * r), c = 3 * r + e % (W - 3 * r);
+            tile[nn][c] = 0;
+        }
+        __syncthreads();
+        const int w8 = W / 8;  // 16-byte pieces per row
+        uint4* dst = reinterpret_cast<uint4*>(l2t + static_cast<size_t>(n0) * W);
+        for (int e = tid; e < L2T_ROWS * w8; e += 256) {
+            const int nn = e / w8, c8 = e % w8;
+            dst[e] = *reinterpret_cast<const uint4*>(&tile[nn][c8 * 8]);
+        }
+        __syncthreads();
     }
 }
 

@@ -23,6 +23,7 @@
 #include "lowrank.cuh"
 #include "ptx.cuh"
 #include "quantize.cuh"
+#include "nvfp4.cuh"
 
 namespace {
 
@@ -139,8 +140,7 @@ struct Plan {
     int astages = 0;    // resident x: TMEM A-stage ring depth
     uint32_t tmem_cols = 0, acc_col0 = 0, lr_col0 = 0, a_col0 = 0, wtile = 0, wstage = 0, xsub = 0, xstage = 0, red = 0, stage = 0;
     size_t smem = 0;
-    size_t off_x16 = 0, off_xs = 0, off_thl = 0, off_l2t = 0, off_l1t = 0, ws = 0;
-    bool fused_lr_prep = false;  // int4 + low rank, K <= 4096: x16, xs and T' in one pass (L1 transposed first)
+    size_t off_x16 = 0, off_xs = 0, off_thl = 0, off_l2t = 0, ws = 0;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -368,8 +368,6 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
     if (r) {
         p.off_thl = off; off = align256(off + static_cast<size_t>(M) * p.lr_kb * 64 * 2);
         p.off_l2t = off; off = align256(off + static_cast<size_t>(p.NT) * 128 * p.lr_kb * 64 * 2);
-        p.fused_lr_prep = fmt != wlq::FMT_W8 && K <= 4096;
-        if (p.fused_lr_prep) { p.off_l1t = off; off = align256(off + static_cast<size_t>(r) * K * 2); }
     }
     p.ws = off;
     return true;
@@ -657,24 +655,6 @@ wlq_status launch_prep_x16(const uint16_t* x, int M, int K, __half* x16, float* 
 }
 
 // x16, xs and T' in one pass (int4 + low rank, K <= 4096): 16 rows per CTA.
-wlq_status launch_prep_x16_lr(const uint16_t* x, const uint16_t* l1t, int M, int K, int r, int W, __half* x16,
-                              float* xs, uint16_t* thl, DeviceInfo* d, cudaStream_t s) {
-    const size_t smem = wlq::xlr_smem_bytes(K, r);
-    const int kid = 41 + (r == 16 ? 0 : r == 32 ? 1 : 2);  // 41..43
-    auto kern = (r == 16) ? wlq::prep_x16_lr_kernel<16> : (r == 32) ? wlq::prep_x16_lr_kernel<32>
-                                                                    : wlq::prep_x16_lr_kernel<64>;
-    if (!d->smem_set[kid]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(wlq::xlr_smem_bytes(4096, r)));
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-        d->smem_set[kid] = true;
-    }
-    const int grid = static_cast<int>(std::min<int64_t>(cdiv(M, wlq::XLR_ROWS), static_cast<int64_t>(d->sms) * 8));
-    launch_k(kern, grid, wlq::XLR_WARPS * 32, smem, s, x, l1t, M, K, W, x16, xs, thl);
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? WLQ_OK : cuda_fail(e, "prep_x16_lr launch");
-}
-
 // T = x L1 as [Th | Tl]: 64-row tiles, K split over a cluster of S CTAs
 // (S doubles while the CTAs fit twice on the SMs and every split keeps two
 // 64-wide chunks).
@@ -943,6 +923,42 @@ wlq_status wlq_quantize_fp8(const void* W, int w_dtype, int64_t N, int64_t K, in
     return WLQ_OK;
 }
 
+size_t wlq_nvfp4_scales_bytes(int64_t rows, int64_t K) {
+    if (rows < 0 || K <= 0 || K % 64) return 0;
+    return wlq::nv_scale_bytes(rows, K);
+}
+
+wlq_status wlq_nvfp4_quantize(const void* X, int x_dtype, int64_t rows, int64_t K, void* codes, void* scales,
+                              float* gscale, void* stream) {
+    if (x_dtype != WLQ_IN_F32 && x_dtype != WLQ_IN_BF16) return fail(WLQ_ERR_UNSUPPORTED, "input must be fp32 or bf16");
+    if (rows < 0 || K <= 0 || K % 64) return fail(WLQ_ERR_SHAPE, "NVFP4 needs rows >= 0 and K a positive multiple of 64");
+    if (!X || !codes || !scales || !gscale) return fail(WLQ_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(X) || !aligned16(codes) || !aligned16(scales) || (reinterpret_cast<uintptr_t>(gscale) & 7u))
+        return fail(WLQ_ERR_ALIGN, "X, codes and scales must be 16-byte aligned, gscale 8-byte aligned");
+    int dev;
+    DeviceInfo* d;
+    wlq_status st;
+    if ((st = current_device(&dev, &d)) != WLQ_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(gscale, 0, 2 * sizeof(float), s);
+    if (e == cudaSuccess && (rows % 128 || K % 256)) e = cudaMemsetAsync(scales, 0, wlq::nv_scale_bytes(rows, K), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    const int64_t nblocks = rows * (K / 16);
+    const int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(cdiv(nblocks, 256), 1), int64_t(d->sms) * 8));
+    if (x_dtype == WLQ_IN_BF16) {
+        launch_k(wlq::nvfp4_amax_kernel<1>, grid, 256, 0, s, X, nblocks, gscale);
+        launch_k(wlq::nvfp4_quantize_kernel<1>, grid, 256, 0, s, X, rows, K, gscale, static_cast<uint8_t*>(codes),
+                 static_cast<uint8_t*>(scales));
+    } else {
+        launch_k(wlq::nvfp4_amax_kernel<0>, grid, 256, 0, s, X, nblocks, gscale);
+        launch_k(wlq::nvfp4_quantize_kernel<0>, grid, 256, 0, s, X, rows, K, gscale, static_cast<uint8_t*>(codes),
+                 static_cast<uint8_t*>(scales));
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "nvfp4 quantize launch");
+    return WLQ_OK;
+}
+
 size_t wlq_packed_bytes(int64_t N, int64_t K, int bits, int group) {
     const int fmt = fmt_of(bits, group);
     if (fmt < 0 || N < 0 || K <= 0 || K % 8 || (group && K % group)) return 0;
@@ -1074,9 +1090,7 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
     if (fmt != wlq::FMT_W8) {
         __half* x16 = reinterpret_cast<__half*>(ws + p.off_x16);
         xs = reinterpret_cast<float*>(ws + p.off_xs);
-        if (!p.fused_lr_prep &&
-            (st = launch_prep_x16(static_cast<const uint16_t*>(x), p.M, p.K, x16, xs, d, s)) != WLQ_OK)
-            return st;
+        if ((st = launch_prep_x16(static_cast<const uint16_t*>(x), p.M, p.K, x16, xs, d, s)) != WLQ_OK) return st;
         xin = x16;
     }
     uint16_t* thl = nullptr;
@@ -1087,21 +1101,13 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
         l2t = reinterpret_cast<uint16_t*>(ws + p.off_l2t);
         // the branch is folded into the GEMM's accumulator: T' = T / xs (int4) and
         // L2' = L2 / rowf, rowf read from the packed operand
-        if (p.fused_lr_prep) {
-            uint16_t* l1t = reinterpret_cast<uint16_t*>(ws + p.off_l1t);
-            launch_k(wlq::prep_l1t_kernel, grid_for(K * r, 256, d->sms), 256, 0, s, static_cast<const uint16_t*>(L1),
-                     p.K, r, l1t);
-            if ((st = launch_prep_x16_lr(static_cast<const uint16_t*>(x), l1t, p.M, p.K, r, W,
-                                         reinterpret_cast<__half*>(ws + p.off_x16), xs, thl, d, s)) != WLQ_OK)
-                return st;
-        } else if ((st = launch_prep_lr_t(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(L1), xs, p.M,
-                                          p.K, r, W, thl, d, s)) != WLQ_OK) {
+        if ((st = launch_prep_lr_t(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(L1), xs, p.M, p.K, r,
+                                   W, thl, d, s)) != WLQ_OK)
             return st;
-        }
         const float* rowf = reinterpret_cast<const float*>(static_cast<const uint8_t*>(packed) +
                                                            static_cast<size_t>(NT) * p.KT * wlq::tile_bytes(fmt));
-        launch_k(wlq::prep_lr_l2t_kernel, grid_for(NT * 128 * (W / 8), 256, d->sms), 256, 0, s,
-            static_cast<const uint16_t*>(L2), rowf, p.N, static_cast<int>(NT * 128), r, W, l2t);
+        launch_k(wlq::prep_lr_l2t_kernel, static_cast<int>(NT * 128 / wlq::L2T_ROWS), 256, 0, s,
+                 static_cast<const uint16_t*>(L2), rowf, p.N, static_cast<int>(NT * 128), r, W, l2t);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "prep launch");
@@ -1383,6 +1389,236 @@ wlq_status wlq_probe_wait_timeout(uint64_t timeout_ns, void* stream) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "probe launch");
     return WLQ_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// NVFP4 W4A4 Linear (block-scaled tensor-core GEMM plus the low-rank branch)
+namespace {
+
+// 2-D tensor of bytes [rows, cols] (cols contiguous), 128 x 128-byte boxes
+// with a 128-byte swizzle; out-of-range bytes read as zero.
+wlq_status make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(WLQ_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {128, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(WLQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return WLQ_OK;
+}
+
+struct NvPlan {
+    int NT = 0, MT = 0, KS = 0, KA = 0, tiles = 0, stages = 0, lr_kb = 0, W = 0, acc_bufs = 2;
+    size_t smem = 0, off_thl = 0, off_l2t = 0, ws = 0;
+};
+
+constexpr size_t kMaxDynSmem = 232448;  // 227 KB per CTA
+
+bool nv_plan(NvPlan& p, int64_t M, int64_t N, int64_t K, int r) {
+    p.NT = static_cast<int>(cdiv(N, 128));
+    p.MT = static_cast<int>(cdiv(M, 128));
+    p.KS = static_cast<int>(cdiv(K, 256));
+    p.KA = p.KS * 4;
+    p.tiles = p.NT * p.MT;
+    p.lr_kb = r ? static_cast<int>(cdiv(3 * r, 64)) : 0;
+    p.W = 64 * p.lr_kb;
+    p.acc_bufs = r ? 1 : 2;  // a low-rank accumulator takes the second buffer's columns
+    p.stages = 0;
+    for (int st = wlq::NV_MAX_STAGES; st >= 2; --st)
+        if (wlq::nv_smem_bytes(st, p.lr_kb) <= kMaxDynSmem) {
+            p.stages = st;
+            break;
+        }
+    if (!p.stages) return false;
+    p.smem = wlq::nv_smem_bytes(p.stages, p.lr_kb);
+    size_t off = 0;
+    if (r) {
+        p.off_thl = off;
+        off = align256(off + static_cast<size_t>(M) * p.W * 2);
+        p.off_l2t = off;
+        off = align256(off + static_cast<size_t>(p.NT) * 128 * p.W * 2);
+    }
+    p.ws = off;
+    return true;
+}
+
+wlq_status check_nvfp4_linear(const void* xq, const void* xs, const float* xg, const void* x, int64_t M, const void* wq,
+                              const void* ws, const float* wg, int64_t N, int64_t K, const void* bias, const void* L1,
+                              const void* L2, int r, const void* y, int y_dtype, bool* noop) {
+    *noop = false;
+    if (M < 0 || N < 0) return fail(WLQ_ERR_INVALID_ARG, "M and N must be >= 0");
+    if (K <= 0 || K % 64) return fail(WLQ_ERR_SHAPE, "NVFP4 needs K a positive multiple of 64");
+    if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30)) return fail(WLQ_ERR_SHAPE, "M or N too large");
+    if (!(r == 0 || r == 16 || r == 32 || r == 64)) return fail(WLQ_ERR_SHAPE, "r must be 0, 16, 32 or 64");
+    if (r && (!L1 || !L2 || !x)) return fail(WLQ_ERR_INVALID_ARG, "r > 0 needs x, L1 and L2");
+    if (y_dtype != WLQ_OUT_BF16 && y_dtype != WLQ_OUT_F32) return fail(WLQ_ERR_INVALID_ARG, "bad y_dtype");
+    if (M == 0 || N == 0) {
+        *noop = true;
+        return WLQ_OK;
+    }
+    if (!xq || !xs || !xg || !wq || !ws || !wg || !y) return fail(WLQ_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(xq) || !aligned16(xs) || !aligned16(wq) || !aligned16(ws) || (x && !aligned16(x)) ||
+        (L1 && !aligned16(L1)) || (L2 && (reinterpret_cast<uintptr_t>(L2) & 1u)) ||
+        (bias && (reinterpret_cast<uintptr_t>(bias) & 1u)) || (reinterpret_cast<uintptr_t>(y) & 3u) ||
+        (reinterpret_cast<uintptr_t>(xg) & 3u) || (reinterpret_cast<uintptr_t>(wg) & 3u))
+        return fail(WLQ_ERR_ALIGN, "codes, scales, x and L1 must be 16-byte aligned, bias/L2 2-byte, y/xg/wg 4-byte");
+    return WLQ_OK;
+}
+
+template <bool LR>
+wlq_status launch_nvfp4_gemm(const NvPlan& p, const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& tl,
+                             const CUtensorMap& tt, const wlq::NvArgs& a, DeviceInfo* d, cudaStream_t s) {
+    auto kern = wlq::nvfp4_gemm_kernel<LR>;
+    const int kid = LR ? 51 : 50;
+    if (!d->smem_set[kid]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kMaxDynSmem));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        d->smem_set[kid] = true;
+    }
+    const int grid = std::min(p.tiles, d->sms);
+    cudaError_t e = launch_k(kern, grid, wlq::NV_THREADS, p.smem, s, tw, tx, tl, tt, a);
+    return e == cudaSuccess ? WLQ_OK : cuda_fail(e, "nvfp4 gemm launch");
+}
+
+wlq_status nvfp4_linear_impl(const void* xq, const void* xs, const float* xg, const void* x, int64_t M, const void* wq,
+                             const void* wsf, const float* wg, int64_t N, int64_t K, const void* bias, const void* L1,
+                             const void* L2, int r, void* y, int y_dtype, uint8_t* ws, size_t ws_bytes, DeviceInfo* d,
+                             cudaStream_t s) {
+    NvPlan p;
+    if (!nv_plan(p, M, N, K, r)) return fail(WLQ_ERR_UNSUPPORTED, "no NVFP4 launch plan for this shape");
+    if (p.ws > 0 && (!ws || ws_bytes < p.ws)) return fail(WLQ_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", p.ws, ws_bytes);
+    if (ws && !aligned16(ws)) return fail(WLQ_ERR_ALIGN, "workspace must be 16-byte aligned");
+    wlq_status st;
+    uint16_t* thl = nullptr;
+    uint16_t* l2t = nullptr;
+    if (r) {
+        thl = reinterpret_cast<uint16_t*>(ws + p.off_thl);
+        l2t = reinterpret_cast<uint16_t*>(ws + p.off_l2t);
+        // T = x L1 split into bf16 [T_h | T_l | T_h], L2 into [L2_h | L2_h | L2_l] (no scaling)
+        if ((st = launch_prep_lr_t(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(L1), nullptr,
+                                   static_cast<int>(M), static_cast<int>(K), r, p.W, thl, d, s)) != WLQ_OK)
+            return st;
+        launch_k(wlq::prep_lr_l2t_kernel, p.NT * 128 / wlq::L2T_ROWS, 256, 0, s, static_cast<const uint16_t*>(L2),
+                 static_cast<const float*>(nullptr), static_cast<int>(N), p.NT * 128, r, p.W, l2t);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "low-rank prep launch");
+    }
+    CUtensorMap tw, tx, tl, tt;
+    std::memset(&tl, 0, sizeof tl);
+    std::memset(&tt, 0, sizeof tt);
+    if ((st = make_map_u8(&tw, wq, N, K / 2)) != WLQ_OK) return st;
+    if ((st = make_map_u8(&tx, xq, M, K / 2)) != WLQ_OK) return st;
+    if (r) {
+        if ((st = make_map_2d(&tl, l2t, static_cast<uint64_t>(p.NT) * 128, p.W, 128)) != WLQ_OK) return st;
+        if ((st = make_map_2d(&tt, thl, M, p.W, 128)) != WLQ_OK) return st;
+    }
+    wlq::NvArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.wsf = static_cast<const uint8_t*>(wsf);
+    a.xsf = static_cast<const uint8_t*>(xs);
+    a.wg = wg;
+    a.xg = xg;
+    a.bias = static_cast<const uint16_t*>(bias);
+    a.y = y;
+    a.M = static_cast<int>(M);
+    a.N = static_cast<int>(N);
+    a.K = static_cast<int>(K);
+    a.NT = p.NT;
+    a.MT = p.MT;
+    a.KS = p.KS;
+    a.KA = p.KA;
+    a.tiles = p.tiles;
+    a.stages = p.stages;
+    a.lr_kb = p.lr_kb;
+    a.y_f32 = (y_dtype == WLQ_OUT_F32) ? 1 : 0;
+    a.acc_bufs = p.acc_bufs;
+    a.timeout_ns = kDefaultTimeoutNs;
+    return r ? launch_nvfp4_gemm<true>(p, tw, tx, tl, tt, a, d, s) : launch_nvfp4_gemm<false>(p, tw, tx, tl, tt, a, d, s);
+}
+
+struct W4a4Layout {
+    size_t off_xq = 0, off_xs = 0, off_xg = 0, off_lin = 0, total = 0;
+};
+W4a4Layout w4a4_layout(int64_t M, int64_t K, size_t lin) {
+    W4a4Layout L;
+    size_t off = 0;
+    L.off_xq = off;
+    off = align256(off + static_cast<size_t>(M) * (K / 2));
+    L.off_xs = off;
+    off = align256(off + wlq::nv_scale_bytes(M, K));
+    L.off_xg = off;
+    off = align256(off + 16);
+    L.off_lin = off;
+    L.total = off + lin;
+    return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t wlq_nvfp4_linear_workspace(int64_t M, int64_t N, int64_t K, int r) {
+    if (M <= 0 || N <= 0 || K <= 0 || K % 64 || !(r == 0 || r == 16 || r == 32 || r == 64)) return 0;
+    NvPlan p;
+    if (!nv_plan(p, M, N, K, r)) return 0;
+    return p.ws;
+}
+
+wlq_status wlq_nvfp4_linear(const void* xq, const void* xs, const float* xg, const void* x, int64_t M, const void* wq,
+                            const void* ws, const float* wg, int64_t N, int64_t K, const void* bias, const void* L1,
+                            const void* L2, int r, void* y, int y_dtype, void* workspace, size_t ws_bytes,
+                            void* stream) {
+    bool noop = false;
+    wlq_status st = check_nvfp4_linear(xq, xs, xg, x, M, wq, ws, wg, N, K, bias, L1, L2, r, y, y_dtype, &noop);
+    if (st != WLQ_OK || noop) return st;
+    int dev;
+    DeviceInfo* d;
+    if ((st = current_device(&dev, &d)) != WLQ_OK) return st;
+    return nvfp4_linear_impl(xq, xs, xg, x, M, wq, ws, wg, N, K, bias, L1, L2, r, y, y_dtype,
+                             static_cast<uint8_t*>(workspace), ws_bytes, d, static_cast<cudaStream_t>(stream));
+}
+
+size_t wlq_w4a4_workspace(int64_t M, int64_t N, int64_t K, int r) {
+    if (M <= 0 || N <= 0 || K <= 0 || K % 64 || !(r == 0 || r == 16 || r == 32 || r == 64)) return 0;
+    NvPlan p;
+    if (!nv_plan(p, M, N, K, r)) return 0;
+    return w4a4_layout(M, K, p.ws).total;
+}
+
+wlq_status wlq_w4a4_linear(const void* x, int64_t M, const void* wq, const void* ws, const float* wg, int64_t N,
+                           int64_t K, const void* bias, const void* L1, const void* L2, int r, void* y, int y_dtype,
+                           void* workspace, size_t ws_bytes, void* stream) {
+    if (M > 0 && N > 0 && !x) return fail(WLQ_ERR_INVALID_ARG, "null pointer");
+    if (M > 0 && N > 0 && !workspace) return fail(WLQ_ERR_WORKSPACE, "the W4A4 Linear needs a workspace");
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    bool noop = false;
+    // the activations' codes and scales are checked as if they were already in the workspace
+    const W4a4Layout L = w4a4_layout(std::max<int64_t>(M, 0), K > 0 ? K : 64, 0);
+    const void* xq = w ? w + L.off_xq : nullptr;
+    const void* xs = w ? w + L.off_xs : nullptr;
+    const float* xg = w ? reinterpret_cast<const float*>(w + L.off_xg) : nullptr;
+    wlq_status st = check_nvfp4_linear(xq, xs, xg, x, M, wq, ws, wg, N, K, bias, L1, L2, r, y, y_dtype, &noop);
+    if (st != WLQ_OK || noop) return st;
+    if (!aligned16(x) || !aligned16(workspace)) return fail(WLQ_ERR_ALIGN, "x and workspace must be 16-byte aligned");
+    int dev;
+    DeviceInfo* d;
+    if ((st = current_device(&dev, &d)) != WLQ_OK) return st;
+    NvPlan p;
+    if (!nv_plan(p, M, N, K, r)) return fail(WLQ_ERR_UNSUPPORTED, "no NVFP4 launch plan for this shape");
+    const W4a4Layout LL = w4a4_layout(M, K, p.ws);
+    if (ws_bytes < LL.total) return fail(WLQ_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", LL.total, ws_bytes);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = wlq_nvfp4_quantize(x, WLQ_IN_BF16, M, K, w + LL.off_xq, w + LL.off_xs,
+                                 reinterpret_cast<float*>(w + LL.off_xg), stream)) != WLQ_OK)
+        return st;
+    return nvfp4_linear_impl(w + LL.off_xq, w + LL.off_xs, reinterpret_cast<const float*>(w + LL.off_xg), x, M, wq, ws,
+                             wg, N, K, bias, L1, L2, r, y, y_dtype, w + LL.off_lin, ws_bytes - LL.off_lin, d, s);
 }
 
 }  // extern "C"
