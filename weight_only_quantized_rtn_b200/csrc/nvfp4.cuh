@@ -16,8 +16,11 @@
 // operands: a quotient of a 24-bit by a 26-bit number is either an E4M3
 // midpoint exactly or at least 2^-31 away from one (relative), far above
 // fp64's rounding error.  The element decision compares |x| with the seven
-// midpoints t (0.25, 0.75, ..., 5) times d = s_b g, each product exact in
-// fp64 (at most 3 + 4 + 24 significant bits), so no division is rounded.
+// midpoints t (0.25, 0.75, ..., 5) times d = s_b g: in fp32 each threshold
+// is carried as a rounded product plus its exact fma error, and |x| minus the
+// rounded product is exact wherever the comparison can go either way (in
+// fp64 for tensors with amax below ~1e-26, where the error could underflow);
+// no division is rounded.
 //
 // Layouts (what the block-scaled tensor-core MMA reads):
 //   codes  : [rows, K / 2] bytes, input k in byte k / 2, low nibble for even k;
@@ -25,7 +28,8 @@
 //   scales : 512-byte atoms, one per (128-row tile, 64 inputs of K); atom
 //            (t, a) at ((t * KA) + a) * 512 with KA = ceil(K / 256) * 4, and in
 //            it the scale of row 128 t + 32 i + j, block 4 a + c at byte
-//            16 j + 4 i + c (rows and blocks past the tensor hold 0)
+//            16 j + 4 i + c; rows are padded to a multiple of 256 and K to one
+//            of 256, and rows and blocks past the tensor hold 0
 //   gscale : [0] g, [1] amax(X) (the first pass's accumulator)
 #pragma once
 #include <cuda_bf16.h>
@@ -39,8 +43,9 @@ namespace wlq {
 constexpr int NV_ATOM_BYTES = 512;
 
 __host__ __device__ constexpr int64_t nv_atoms_per_row_tile(int64_t K) { return ((K + 255) / 256) * 4; }
+// rows padded to 256 (two 128-row tiles): a 256-token GEMM tile always has both halves
 __host__ __device__ constexpr size_t nv_scale_bytes(int64_t rows, int64_t K) {
-    return static_cast<size_t>((rows + 127) / 128) * static_cast<size_t>(nv_atoms_per_row_tile(K)) * NV_ATOM_BYTES;
+    return static_cast<size_t>((rows + 255) / 256) * 2 * static_cast<size_t>(nv_atoms_per_row_tile(K)) * NV_ATOM_BYTES;
 }
 __device__ __forceinline__ size_t nv_scale_offset(int64_t row, int64_t blk, int64_t KA) {
     const int64_t atom = (row >> 7) * KA + (blk >> 2);
@@ -49,25 +54,30 @@ __device__ __forceinline__ size_t nv_scale_offset(int64_t row, int64_t blk, int6
 
 // E4M3 (no infinities; 0x7f is NaN) nearest to q >= 0, ties to an even
 // mantissa, saturated at 448 (0x7e).  Spacing 2^(E-3) in [2^E, 2^(E+1)),
-// 2^-9 below 2^-6; q / spacing is exact, rint rounds half to even.
+// 2^-9 below 2^-6: q / spacing is an exact scaling, rounded half to even by
+// the conversion to an integer.  q is an fp64 normal here (a quotient of
+// fp32 values), so its exponent field is E + 1023.
 __device__ __forceinline__ uint32_t e4m3_from_f64(double q) {
     if (!(q > 0.0)) return 0u;
     if (q >= 448.0) return 0x7eu;
-    int e;
-    (void)frexp(q, &e);  // q in [2^(e-1), 2^e)
-    int E = e - 1;
+    int E = static_cast<int>((static_cast<unsigned long long>(__double_as_longlong(q)) >> 52) & 0x7ff) - 1023;
     if (E < -6) E = -6;
-    double n = rint(ldexp(q, 3 - E));  // q / 2^(E-3): in [0, 16]
-    if (n >= 16.0) {
-        n = 8.0;
+    const double sc = __longlong_as_double(static_cast<long long>(1023 + 3 - E) << 52);  // 2^(3-E)
+    long long n = __double2ll_rn(q * sc);                                                   // in [0, 16]
+    if (n >= 16) {
+        n = 8;
         E += 1;
     }
-    if (n < 8.0) return static_cast<uint32_t>(n);  // below 2^-6 (E = -6): subnormal, or zero
-    return (static_cast<uint32_t>(E + 7) << 3) | static_cast<uint32_t>(n - 8.0);
+    if (n < 8) return static_cast<uint32_t>(n);  // below 2^-6 (E = -6): subnormal, or zero
+    return (static_cast<uint32_t>(E + 7) << 3) | static_cast<uint32_t>(n - 8);
 }
 __device__ __forceinline__ double e4m3_to_f64(uint32_t b) {
     const int e = (b >> 3) & 15, m = b & 7;
     return e == 0 ? ldexp(static_cast<double>(m), -9) : ldexp(static_cast<double>(8 + m), e - 10);
+}
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+    const int e = (b >> 3) & 15, m = b & 7;
+    return e == 0 ? static_cast<float>(m) * 0x1p-9f : static_cast<float>(8 + m) * __int_as_float((e - 10 + 127) << 23);
 }
 
 // |x| of 16 inputs (fp32 or bf16) into v[], with the sign bits in *sign.
@@ -164,20 +174,48 @@ __global__ void __launch_bounds__(256) nvfp4_quantize_kernel(const void* __restr
 #pragma unroll
         for (int i = 0; i < 16; ++i) ab = fmaxf(ab, v[i]);
         const uint32_t sb = (g > 0.0f) ? e4m3_from_f64(static_cast<double>(ab) / (6.0 * static_cast<double>(g))) : 0u;
-        const double d = e4m3_to_f64(sb) * static_cast<double>(g);  // exact
-        const double T0 = 0.25 * d, T1 = 0.75 * d, T2 = 1.25 * d, T3 = 1.75 * d, T4 = 2.5 * d, T5 = 3.5 * d,
-                     T6 = 5.0 * d;
         uint32_t lo = 0, hi = 0;
+        if (sb != 0 && g >= 1e-30f) {
+            // fp32: T_i = t_i s_b g as p_i + e_i exactly (u_i = t_i s_b has at most 7 bits; the fma
+            // error is exact because u_i g stays far above the subnormals), and |x| - p_i is exact
+            // whenever |x| is within a factor 2 of p_i, which is the only case it can tie or flip
+            const float sf = e4m3_to_f32(sb);
+            float P[7], E[7];
+            const float tau[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f};
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const double a = static_cast<double>(v[i]);
-            const bool p4 = a >= T3;               // past T_3 (odd index: ties round up)
-            const bool p2 = a >= (p4 ? T5 : T1);   // past T_5 / T_1 (odd)
-            const bool p1 = a > (p4 ? (p2 ? T6 : T4) : (p2 ? T2 : T0));  // even index: ties stay
-            uint32_t c = (p4 ? 4u : 0u) + (p2 ? 2u : 0u) + (p1 ? 1u : 0u);
-            c = (d > 0.0) ? (c | (((sg >> i) & 1u) << 3)) : 0u;
-            if (i < 8) lo |= c << (4 * i);
-            else hi |= c << (4 * (i - 8));
+            for (int t = 0; t < 7; ++t) {
+                const float u = tau[t] * sf;
+                P[t] = __fmul_rn(u, g);
+                E[t] = __fmaf_rn(u, g, -P[t]);
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float a = v[i];
+                const bool p4 = __fsub_rn(a, P[3]) >= E[3];                      // past T_3 (odd: ties up)
+                const float p1v = p4 ? P[5] : P[1], e1v = p4 ? E[5] : E[1];
+                const bool p2 = __fsub_rn(a, p1v) >= e1v;                        // past T_5 / T_1 (odd)
+                const float p0v = p4 ? (p2 ? P[6] : P[4]) : (p2 ? P[2] : P[0]);
+                const float e0v = p4 ? (p2 ? E[6] : E[4]) : (p2 ? E[2] : E[0]);
+                const bool p1 = __fsub_rn(a, p0v) > e0v;                         // even: ties stay
+                const uint32_t c = (p4 ? 4u : 0u) + (p2 ? 2u : 0u) + (p1 ? 1u : 0u) + (((sg >> i) & 1u) << 3);
+                if (i < 8) lo |= c << (4 * i);
+                else hi |= c << (4 * (i - 8));
+            }
+        } else if (sb != 0) {
+            // tensors whose amax is below ~1e-26: the same decisions in fp64
+            const double d = e4m3_to_f64(sb) * static_cast<double>(g);  // exact
+            const double T0 = 0.25 * d, T1 = 0.75 * d, T2 = 1.25 * d, T3 = 1.75 * d, T4 = 2.5 * d, T5 = 3.5 * d,
+                         T6 = 5.0 * d;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const double a = static_cast<double>(v[i]);
+                const bool p4 = a >= T3;
+                const bool p2 = a >= (p4 ? T5 : T1);
+                const bool p1 = a > (p4 ? (p2 ? T6 : T4) : (p2 ? T2 : T0));
+                const uint32_t c = (p4 ? 4u : 0u) + (p2 ? 2u : 0u) + (p1 ? 1u : 0u) + (((sg >> i) & 1u) << 3);
+                if (i < 8) lo |= c << (4 * i);
+                else hi |= c << (4 * (i - 8));
+            }
         }
         *reinterpret_cast<uint2*>(codes + static_cast<size_t>(row) * (K / 2) + kb * 8) = make_uint2(lo, hi);
         scales[nv_scale_offset(row, kb, KA)] = static_cast<uint8_t>(sb);
@@ -190,31 +228,44 @@ __global__ void __launch_bounds__(256) nvfp4_quantize_kernel(const void* __restr
 // tensor cores (tcgen05.mma kind::mxf4nvf4, E2M1 operands, one UE4M3 scale
 // per 16 inputs, fp32 accumulation in tensor memory).
 //
-// Tile: 128 output channels (the MMA's M: weight rows, operand A) x 128
+// Tile: 128 output channels (the MMA's M: weight rows, operand A) x 256
 // tokens (its N: activation rows, operand B).  A stage holds 256 inputs of K:
-// a 128 x 128-byte code tile of each operand (TMA, 128-byte swizzle) and the
-// four 512-byte scale atoms of each (bulk copies).  The MMA thread moves the
+// the 128 x 128-byte weight code tile and the 256 x 128-byte token code tile
+// (TMA, 128-byte swizzle), the weights' four 512-byte scale atoms and the
+// tokens' eight (two 128-row halves; bulk copies).  The MMA thread moves the
 // atoms into tensor memory (tcgen05.cp 32x128b.warpx4: lane 32 i + j gets
 // atom bytes 16 j .. 16 j + 15 for every i, i.e. rows j, j + 32, j + 64,
-// j + 96 in four columns) and issues four K = 64 MMAs per stage.
+// j + 96 of the atom in four columns; the token atoms of one 64-input block
+// take eight columns, rows 0-127 then 128-255) and issues four K = 64 MMAs.
+// The low-rank term shares the accumulator: its operands are pre-divided by
+// the tensor scales (T / g_x and L2 / g_w, each as a bf16 hi + lo pair, the
+// [T_h | T_l | T_h] x [L2_h | L2_h | L2_l] split the W4A16 path uses) and
+// pass through the same ring as ceil(3r / 64) bf16 stages ahead of each
+// tile's FP4 stages (a 128 x 64 bf16 tile is 16 KB like the weight codes, a
+// 256 x 64 one 32 KB like the token codes), so y = acc g_x g_w + b.  A tensor
+// scale of 0 (an all-zero operand) is taken as 1 on both sides.
 // Persistent CTAs walk the tiles (channel tile fastest); warp 0 loads, warp 1
-// issues MMAs, warps 2-5 drain the accumulator: y = acc g_x g_w + lr + b.
-// The low-rank term comes from a second accumulator: its operands are the
-// same [T_h | T_l | T_h] x [L2_h | L2_h | L2_l] bf16 split the W4A16 path
-// uses (kind::f16 MMAs, 64 inputs per block).
-constexpr int NV_TILE = 128;
-constexpr uint32_t NV_OP_BYTES = 128u * 128u;
-constexpr uint32_t NV_SF_STAGE = 4u * NV_ATOM_BYTES;
-constexpr uint32_t NV_STAGE_BYTES = 2u * NV_OP_BYTES + 2u * NV_SF_STAGE;  // 36 KB
-constexpr int NV_MAX_STAGES = 6;
-constexpr uint32_t NV_LR_TILE = 128u * 64u * 2u;  // 16 KB bf16 tile
-constexpr int NV_MAX_LR_KB = 3;
+// issues MMAs, warps 2-5 drain the accumulator.  One 256-column accumulator
+// and 48 scale columns per stage fill the 512 TMEM columns, so a tile's
+// epilogue and the next tile's MMAs do not overlap.
+constexpr int NV_TM = 128;  // channels per tile
+constexpr int NV_TN = 256;  // tokens per tile
+constexpr uint32_t NV_A_BYTES = 128u * 128u;
+constexpr uint32_t NV_B_BYTES = 256u * 128u;
+constexpr uint32_t NV_SFA_BYTES = 4u * NV_ATOM_BYTES;
+constexpr uint32_t NV_SFB_BYTES = 8u * NV_ATOM_BYTES;
+constexpr uint32_t NV_STAGE_BYTES = NV_A_BYTES + NV_B_BYTES + NV_SFA_BYTES + NV_SFB_BYTES;  // 54 KB
+constexpr uint32_t NV_LR_STAGE_BYTES = NV_A_BYTES + NV_B_BYTES;  // one bf16 low-rank block
+constexpr int NV_MAX_STAGES = 4;
 constexpr int NV_THREADS = 192;
 constexpr uint32_t NV_TMEM_COLS = 512;
-constexpr uint32_t NV_SF_COL0 = 256;  // stage s: A scales at 256 + 32 s, B scales 16 columns after
+constexpr uint32_t NV_SF_COL0 = 256;  // stage s: weight scales at 256 + 48 s, token scales 16 columns after
+constexpr uint32_t NV_SF_COLS = 48;
 
-__host__ __device__ constexpr size_t nv_smem_bytes(int stages, int lr_kb) {
-    return 1024 + static_cast<size_t>(stages) * NV_STAGE_BYTES + static_cast<size_t>(lr_kb) * 2 * NV_LR_TILE + 256;
+constexpr uint32_t NV_EPI_STAGE = 2048;  // per epilogue warp: 16 tokens x 32 channels of y (two bf16 halves or one fp32)
+
+__host__ __device__ constexpr size_t nv_smem_bytes(int stages) {
+    return 1024 + static_cast<size_t>(stages) * NV_STAGE_BYTES + 256 + 4 * NV_EPI_STAGE;
 }
 
 struct NvArgs {
@@ -225,11 +276,26 @@ struct NvArgs {
     const uint16_t* bias;
     void* y;
     int M, N, K;
-    int NT, MT, KS;  // channel tiles, token tiles, 256-input stages
+    int NT, MT, KS;  // channel tiles (128), token tiles (256), 256-input stages
     int KA;          // scale atoms per 128-row tile
-    int tiles, stages, lr_kb, y_f32, acc_bufs;
+    int tiles, stages, lr_kb, y_f32;
+    int tma_store;  // y written by TMA stores from a per-warp staging tile (y 16-byte aligned, rows 16-byte multiples)
     uint64_t timeout_ns;
 };
+
+// y[box] <- shared staging (bulk async group of this thread).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t c0, int32_t c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(src)), "r"(c0), "r"(c1)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
 
 // D[tmem] (+)= A[smem] B[smem]^T with one UE4M3 scale per 16 inputs of each
 // operand row (scales in tensor memory at sfa / sfb).
@@ -281,21 +347,19 @@ template <bool LR>
 __global__ void __launch_bounds__(NV_THREADS, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                       const __grid_constant__ CUtensorMap tm_l2, const __grid_constant__ CUtensorMap tm_t,
-                      const NvArgs a) {
+                      const __grid_constant__ CUtensorMap tm_y, const NvArgs a) {
     extern __shared__ uint8_t nv_smem_raw[];
     uint8_t* base = nv_smem_raw + ((1024u - (smem_u32(nv_smem_raw) & 1023u)) & 1023u);
     uint8_t* stage0 = base;
-    uint8_t* lrbuf = base + static_cast<size_t>(a.stages) * NV_STAGE_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(lrbuf + static_cast<size_t>(a.lr_kb) * 2 * NV_LR_TILE);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base + static_cast<size_t>(a.stages) * NV_STAGE_BYTES);
     uint64_t* full = bars;
     uint64_t* empty = full + NV_MAX_STAGES;
     uint64_t* accfull = empty + NV_MAX_STAGES;
-    uint64_t* accempty = accfull + 2;
-    uint64_t* lrfull = accempty + 2;
-    uint64_t* lrempty = lrfull + 1;
-    uint64_t* drain = lrempty + 1;
+    uint64_t* accempty = accfull + 1;
+    uint64_t* drain = accempty + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    uint8_t* epi_stage = reinterpret_cast<uint8_t*>(bars) + 256;  // 4 x NV_EPI_STAGE, 256-byte aligned
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -303,12 +367,8 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&accfull[i], 1);
-            mbar_init(&accempty[i], 4);
-        }
-        mbar_init(lrfull, 1);
-        mbar_init(lrempty, 1);
+        mbar_init(accfull, 1);
+        mbar_init(accempty, 4);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -317,6 +377,7 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tm_w);
         prefetch_tensormap(&tm_x);
+        if (a.tma_store) prefetch_tensormap(&tm_y);
         if (LR) {
             prefetch_tensormap(&tm_l2);
             prefetch_tensormap(&tm_t);
@@ -328,35 +389,39 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     grid_dependency_sync();
+    const int per_tile = a.KS + (LR ? a.lr_kb : 0);  // ring stages per tile
 
     if (warp == 0) {
         if (lane == 0) {
             // ---------------------------------------------------------- loads
-            uint32_t it = 0, lr_it = 0;
+            uint32_t it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x) {
                 const int nt = tile % a.NT, mt = tile / a.NT;
-                if (LR) {
-                    if (!nv_wait(lrempty, (lr_it & 1) ^ 1, a.timeout_ns, abort_flag)) { ok = false; break; }
-                    mbar_arrive_expect_tx(lrfull, static_cast<uint32_t>(a.lr_kb) * 2 * NV_LR_TILE);
-                    for (int j = 0; j < a.lr_kb; ++j) {
-                        uint8_t* t = lrbuf + static_cast<size_t>(j) * 2 * NV_LR_TILE;
-                        tma_load_2d(t, &tm_l2, lrfull, j * 64, nt * NV_TILE);
-                        tma_load_2d(t + NV_LR_TILE, &tm_t, lrfull, j * 64, mt * NV_TILE);
-                    }
-                    ++lr_it;
-                }
-                for (int ks = 0; ks < a.KS; ++ks, ++it) {
+                for (int s = 0; s < per_tile; ++s, ++it) {
                     const uint32_t st = it % a.stages, ph = (it / a.stages) & 1;
                     if (!nv_wait(&empty[st], ph ^ 1, a.timeout_ns, abort_flag)) { ok = false; break; }
                     uint8_t* sb = stage0 + static_cast<size_t>(st) * NV_STAGE_BYTES;
-                    mbar_arrive_expect_tx(&full[st], NV_STAGE_BYTES);
-                    tma_load_2d(sb, &tm_w, &full[st], ks * 128, nt * NV_TILE);
-                    tma_load_2d(sb + NV_OP_BYTES, &tm_x, &full[st], ks * 128, mt * NV_TILE);
-                    bulk_load(sb + 2 * NV_OP_BYTES, a.wsf + (static_cast<size_t>(nt) * a.KA + ks * 4) * NV_ATOM_BYTES,
-                              NV_SF_STAGE, &full[st]);
-                    bulk_load(sb + 2 * NV_OP_BYTES + NV_SF_STAGE,
-                              a.xsf + (static_cast<size_t>(mt) * a.KA + ks * 4) * NV_ATOM_BYTES, NV_SF_STAGE, &full[st]);
+                    const int ks = s - (LR ? a.lr_kb : 0);
+                    if (ks < 0) {  // low-rank block j: L2'' rows of this channel tile, T'' rows of this token tile
+                        const int j = s;
+                        mbar_arrive_expect_tx(&full[st], NV_LR_STAGE_BYTES);
+                        tma_load_2d(sb, &tm_l2, &full[st], j * 64, nt * NV_TM);
+                        tma_load_2d(sb + NV_A_BYTES, &tm_t, &full[st], j * 64, mt * NV_TN);
+                    } else {
+                        mbar_arrive_expect_tx(&full[st], NV_STAGE_BYTES);
+                        tma_load_2d(sb, &tm_w, &full[st], ks * 128, nt * NV_TM);
+                        tma_load_2d(sb + NV_A_BYTES, &tm_x, &full[st], ks * 128, mt * NV_TN);
+                        uint8_t* sf = sb + NV_A_BYTES + NV_B_BYTES;
+                        bulk_load(sf, a.wsf + (static_cast<size_t>(nt) * a.KA + ks * 4) * NV_ATOM_BYTES, NV_SFA_BYTES,
+                                  &full[st]);
+                        // the two 128-row halves of the token tile (scale rows are padded to 256)
+                        bulk_load(sf + NV_SFA_BYTES, a.xsf + (static_cast<size_t>(2 * mt) * a.KA + ks * 4) * NV_ATOM_BYTES,
+                                  NV_SFA_BYTES, &full[st]);
+                        bulk_load(sf + 2 * NV_SFA_BYTES,
+                                  a.xsf + (static_cast<size_t>(2 * mt + 1) * a.KA + ks * 4) * NV_ATOM_BYTES, NV_SFA_BYTES,
+                                  &full[st]);
+                    }
                 }
             }
             // copies still in flight land before the CTA leaves (bounded)
@@ -366,59 +431,46 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
                 while (!mbar_try_wait(&full[i % a.stages], (i / a.stages) & 1) && globaltimer_ns() - t0 < a.timeout_ns) {
                 }
             }
-            if (LR && lr_it > 0) {
-                const uint64_t t0 = globaltimer_ns();
-                while (!mbar_try_wait(lrfull, (lr_it - 1) & 1) && globaltimer_ns() - t0 < a.timeout_ns) {
-                }
-            }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ----------------------------------------------------------- MMAs
-            const uint32_t idesc = idesc_nvf4(128, NV_TILE);
-            const uint32_t idesc_lr = idesc_f16(1, 128, NV_TILE);
-            uint32_t it = 0, lr_it = 0, tc = 0;
+            const uint32_t idesc = idesc_nvf4(NV_TM, NV_TN);
+            const uint32_t idesc_lr = idesc_f16(1, NV_TM, NV_TN);
+            uint32_t it = 0, tc = 0;
             for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x, ++tc) {
-                const uint32_t b = tc % a.acc_bufs, use = tc / a.acc_bufs;
-                if (!nv_wait(&accempty[b], (use & 1) ^ 1, a.timeout_ns, abort_flag)) break;
+                if (!nv_wait(accempty, (tc & 1) ^ 1, a.timeout_ns, abort_flag)) break;
                 tc_fence_after();
-                const uint32_t acc = tmem + b * NV_TILE;
-                if (LR) {
-                    if (!nv_wait(lrfull, lr_it & 1, a.timeout_ns, abort_flag)) break;
-                    tc_fence_after();
-                    const uint32_t lacc = tmem + NV_TILE;  // one main buffer with a low-rank term
-                    for (int j = 0; j < a.lr_kb; ++j) {
-                        const uint8_t* t = lrbuf + static_cast<size_t>(j) * 2 * NV_LR_TILE;
-                        const uint64_t da = smem_desc_sw128(smem_u32(t)), db = smem_desc_sw128(smem_u32(t + NV_LR_TILE));
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_ss(lacc, da + 2 * kk, db + 2 * kk, idesc_lr, (j > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    mma_commit(lrempty);
-                    ++lr_it;
-                }
                 bool ok = true;
-                for (int ks = 0; ks < a.KS; ++ks, ++it) {
+                for (int s = 0; s < per_tile; ++s, ++it) {
                     const uint32_t st = it % a.stages, ph = (it / a.stages) & 1;
                     if (!nv_wait(&full[st], ph, a.timeout_ns, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint8_t* sb = stage0 + static_cast<size_t>(st) * NV_STAGE_BYTES;
-                    const uint32_t sfa = tmem + NV_SF_COL0 + 32 * st, sfb = sfa + 16;
-                    const uint32_t sa = smem_u32(sb + 2 * NV_OP_BYTES), sbb = sa + NV_SF_STAGE;
+                    const uint64_t da = smem_desc_sw128(smem_u32(sb)), db = smem_desc_sw128(smem_u32(sb + NV_A_BYTES));
+                    if (LR && s < a.lr_kb) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        tmem_cp_32x128b_x4(sfa + 4 * i, smem_desc_rows16(sa + i * NV_ATOM_BYTES));
-                        tmem_cp_32x128b_x4(sfb + 4 * i, smem_desc_rows16(sbb + i * NV_ATOM_BYTES));
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ss(tmem, da + 2 * kk, db + 2 * kk, idesc_lr, (s > 0 || kk > 0) ? 1u : 0u);
+                    } else {
+                        const bool first = s == 0;  // no low-rank block before it
+                        const uint32_t sfa = tmem + NV_SF_COL0 + NV_SF_COLS * st, sfb = sfa + 16;
+                        const uint32_t sa = smem_u32(sb + NV_A_BYTES + NV_B_BYTES);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            tmem_cp_32x128b_x4(sfa + 4 * i, smem_desc_rows16(sa + i * NV_ATOM_BYTES));
+                            tmem_cp_32x128b_x4(sfb + 8 * i, smem_desc_rows16(sa + NV_SFA_BYTES + i * NV_ATOM_BYTES));
+                            tmem_cp_32x128b_x4(sfb + 8 * i + 4, smem_desc_rows16(sa + 2 * NV_SFA_BYTES + i * NV_ATOM_BYTES));
+                        }
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            mma_nvf4(tmem, da + 2 * k, db + 2 * k, idesc, sfa + 4 * k, sfb + 8 * k,
+                                     (first && k == 0) ? 0u : 1u);
                     }
-                    const uint64_t da = smem_desc_sw128(smem_u32(sb)), db = smem_desc_sw128(smem_u32(sb + NV_OP_BYTES));
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        mma_nvf4(acc, da + 2 * k, db + 2 * k, idesc, sfa + 4 * k, sfb + 4 * k,
-                                 (ks > 0 || k > 0) ? 1u : 0u);
                     mma_commit(&empty[st]);
                 }
                 if (!ok) break;
-                mma_commit(&accfull[b]);
+                mma_commit(accfull);
             }
             // every MMA issued has completed before tensor memory is freed
             mma_commit(drain);
@@ -429,16 +481,16 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may read
-        const float e = __ldg(a.xg) * __ldg(a.wg);
-        uint32_t tc = 0;
+        const float gx = __ldg(a.xg), gw = __ldg(a.wg);
+        const float ex = (gx != 0.0f) ? gx : 1.0f, ew = (gw != 0.0f) ? gw : 1.0f;
+        uint32_t tc = 0, chunk = 0;  // chunk: staging halves alternate across tiles too
         for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x, ++tc) {
             const int nt = tile % a.NT, mt = tile / a.NT;
-            const uint32_t b = tc % a.acc_bufs, use = tc / a.acc_bufs;
             // every lane polls (each acquires for itself); lane 0 decides to give up
             bool ready = false;
             uint64_t t0 = 0;
             for (uint32_t spin = 0;; ++spin) {
-                ready = mbar_try_wait(&accfull[b], use & 1);
+                ready = mbar_try_wait(accfull, tc & 1);
                 if (__all_sync(0xffffffffu, ready)) break;
                 int give_up = 0;
                 if (lane == 0 && (spin & 255) == 255) {
@@ -455,31 +507,53 @@ __global__ void __launch_bounds__(NV_THREADS, 1)
             }
             if (!__all_sync(0xffffffffu, ready)) break;
             tc_fence_after();
-            const int n = nt * NV_TILE + q * 32 + lane;
+            const int n = nt * NV_TM + q * 32 + lane;
             const float bv = (a.bias && n < a.N) ? bf16_bits_to_f32(a.bias[n]) : 0.0f;
-            const uint32_t acc = tmem + b * NV_TILE + (static_cast<uint32_t>(q * 32) << 16);
-            const uint32_t lacc = tmem + NV_TILE + (static_cast<uint32_t>(q * 32) << 16);
-            for (int c0 = 0; c0 < NV_TILE; c0 += 16) {
-                uint32_t v[16], w[16];
+            const uint32_t acc = tmem + (static_cast<uint32_t>(q * 32) << 16);
+            const int m_end = min(NV_TN, a.M - mt * NV_TN);
+            uint8_t* stg = epi_stage + static_cast<size_t>(warp - 2) * NV_EPI_STAGE;
+            for (int c0 = 0; c0 < m_end; c0 += 16) {
+                uint32_t v[16];
                 tmem_ld16(acc + c0, v);
-                if (LR) tmem_ld16(lacc + c0, w);
                 tmem_wait_ld();
+                if (a.tma_store) {
+                    // 16 tokens x this warp's 32 channels into the staging tile (token-major, like y),
+                    // then one TMA store; out-of-range rows and channels are clipped by the store
+                    uint8_t* buf = a.y_f32 ? stg : stg + (chunk++ & 1) * 1024;
+                    if (lane == 0) {
+                        if (a.y_f32) bulk_wait_read<0>();
+                        else bulk_wait_read<1>();  // the other half may still be read
+                    }
+                    __syncwarp();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int m = mt * NV_TILE + c0 + j;
-                    float o = __uint_as_float(v[j]) * e + bv;
-                    if (LR) o += __uint_as_float(w[j]);
-                    if (m < a.M && n < a.N) {
-                        const size_t off = static_cast<size_t>(m) * a.N + n;
-                        if (a.y_f32) static_cast<float*>(a.y)[off] = o;
-                        else static_cast<__nv_bfloat16*>(a.y)[off] = __float2bfloat16_rn(o);
+                    for (int j = 0; j < 16; ++j) {
+                        const float o = (__uint_as_float(v[j]) * ex) * ew + bv;
+                        if (a.y_f32) reinterpret_cast<float*>(buf)[j * 32 + lane] = o;
+                        else reinterpret_cast<__nv_bfloat16*>(buf)[j * 32 + lane] = __float2bfloat16_rn(o);
+                    }
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0 && nt * NV_TM + q * 32 < a.N) tma_store_2d(&tm_y, buf, nt * NV_TM + q * 32, mt * NV_TN + c0);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int m = mt * NV_TN + c0 + j;
+                        const float o = (__uint_as_float(v[j]) * ex) * ew + bv;
+                        if (c0 + j < m_end && n < a.N) {
+                            const size_t off = static_cast<size_t>(m) * a.N + n;
+                            if (a.y_f32) static_cast<float*>(a.y)[off] = o;
+                            else static_cast<__nv_bfloat16*>(a.y)[off] = __float2bfloat16_rn(o);
+                        }
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&accempty[b]);
+            if (lane == 0) mbar_arrive(accempty);
         }
+        // the staging tiles stay valid until their stores have read them
+        if (a.tma_store && lane == 0) bulk_wait_read<0>();
+        __syncwarp();
     }
 
     tc_fence_before();

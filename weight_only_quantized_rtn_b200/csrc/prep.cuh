@@ -121,6 +121,12 @@ __global__ void __launch_bounds__(THREADS, MINB) prep_x16_rows_kernel(const uint
         __syncthreads();
         const int f = fsh;
         uint4* out = reinterpret_cast<uint4*>(x16 + static_cast<size_t>(m) * K);
+        // 2^f as a float when it is one (f in [-126, 127], every row but those
+        // spanning extreme ranges): the product is then exact whenever it can
+        // round to a nonzero fp16 (a product below 2^-126 gives fp16 0 either
+        // way), so it converts exactly as ldexpf's result does
+        const bool fast = f >= -126 && f <= 127;
+        const float p2 = __int_as_float((f + 127) << 23);
 #pragma unroll
         for (int j = 0; j < PER; ++j) {
             const int i = threadIdx.x + j * blockDim.x;
@@ -129,8 +135,8 @@ __global__ void __launch_bounds__(THREADS, MINB) prep_x16_rows_kernel(const uint
             uint32_t o[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const __half2 h = __floats2half2_rn(ldexpf(bf16_bits_to_f32(w[e] & 0xFFFFu), f),
-                                                    ldexpf(bf16_bits_to_f32(w[e] >> 16), f));
+                const float a = bf16_bits_to_f32(w[e] & 0xFFFFu), b = bf16_bits_to_f32(w[e] >> 16);
+                const __half2 h = fast ? __floats2half2_rn(a * p2, b * p2) : __floats2half2_rn(ldexpf(a, f), ldexpf(b, f));
                 o[e] = *reinterpret_cast<const uint32_t*>(&h);
             }
             out[i] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -159,7 +165,7 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
 
 constexpr int LR_ROWS = 64;          // rows of x per CTA (16 per warp, 4 warps)
 constexpr int LR_KC = 64;            // K chunk per pipeline stage
-constexpr int LR_STAGES = 3;         // cp.async pipeline depth
+constexpr int LR_STAGES = 4;         // cp.async pipeline depth
 constexpr int LR_XP = LR_KC + 8;     // x tile row pitch in bf16 elements (144 bytes: ldmatrix conflict-free)
 constexpr int LR_LP = 64 + 8;        // L1 tile row pitch in bf16 elements (r <= 64)
 constexpr int LR_MAX_SPLITS = 8;     // CTAs of a cluster splitting K
@@ -190,7 +196,7 @@ __device__ __forceinline__ void ldsm_x2_trans(uint32_t (&r)[2], uint32_t addr) {
 __global__ void __launch_bounds__(128) prep_lr_t_kernel(const uint16_t* __restrict__ x,
                                                         const uint16_t* __restrict__ L1, const float* __restrict__ xs,
                                                         int M, int K, int r, int W, int S, int kc_per,
-                                                        uint16_t* __restrict__ thl) {
+                                                        int xs_scalar, uint16_t* __restrict__ thl) {
     extern __shared__ uint8_t lr_smem_raw[];
     uint8_t* base = lr_smem_raw + ((128u - (smem_u32(lr_smem_raw) & 127u)) & 127u);
     uint16_t* stage0 = reinterpret_cast<uint16_t*>(base);
@@ -284,7 +290,8 @@ __global__ void __launch_bounds__(128) prep_lr_t_kernel(const uint16_t* __restri
         for (int sp = 1; sp < S; ++sp) T += ld_dsmem_f32(mapa_shared(a0, static_cast<uint32_t>(sp)));
         const int m = m0 + row;
         if (m < M) {
-            if (xs) T /= xs[m];  // a power of two: exact
+            if (xs && !xs_scalar) T /= xs[m];  // a power of two: exact
+            if (xs && xs_scalar && xs[0] != 0.0f) T /= xs[0];  // one tensor scale (0: left unscaled)
             uint16_t* out = thl + static_cast<size_t>(m) * W;
             const __nv_bfloat16 hi = __float2bfloat16_rn(T);
             const __nv_bfloat16 lo = __float2bfloat16_rn(T - __bfloat162float(hi));
@@ -301,14 +308,15 @@ __global__ void __launch_bounds__(128) prep_lr_t_kernel(const uint16_t* __restri
 }
 
 // L2t[n] = [L2'h(0..r) | L2'h(0..r) | L2'l(0..r) | 0 ...] (width W) with
-// L2' = L2[., n] / rowf[n] (L2 itself where rowf[n] == 0 or rowf is null),
-// zero for n >= N.
+// L2' = L2[., n] / rowf[n] (rowf[0] for every n when rowf_scalar; L2 itself
+// where that factor is 0 or rowf is null), zero for n >= N.
 // A CTA builds 32 rows of L2t in shared memory: its reads of L2 are 64-byte
 // row pieces (consecutive n), its writes one contiguous 32 * W * 2-byte block.
 constexpr int L2T_ROWS = 32;
 constexpr int L2T_MAX_W = 192;  // lr_kb <= 3
 __global__ void __launch_bounds__(256) prep_lr_l2t_kernel(const uint16_t* __restrict__ L2, const float* __restrict__ rowf,
-                                                          int N, int N_pad, int r, int W, uint16_t* __restrict__ l2t) {
+                                                          int rowf_scalar, int N, int N_pad, int r, int W,
+                                                          uint16_t* __restrict__ l2t) {
     grid_dependency_sync();
     __shared__ __align__(16) uint16_t tile[L2T_ROWS][L2T_MAX_W + 8];
     const int tid = threadIdx.x;
@@ -317,7 +325,7 @@ __global__ void __launch_bounds__(256) prep_lr_l2t_kernel(const uint16_t* __rest
             const int j = e / L2T_ROWS, nn = e % L2T_ROWS, n = n0 + nn;
             uint16_t hb = 0, lb = 0;
             if (n < N) {
-                const float rf = rowf ? rowf[n] : 0.0f;
+                const float rf = rowf ? rowf[rowf_scalar ? 0 : n] : 0.0f;
                 const float l2 = bf16_bits_to_f32(L2[static_cast<size_t>(j) * N + n]);
                 const float l = (rf != 0.0f) ? l2 / rf : l2;
                 const __nv_bfloat16 hi = __float2bfloat16_rn(l);

@@ -658,8 +658,8 @@ wlq_status launch_prep_x16(const uint16_t* x, int M, int K, __half* x16, float* 
 // T = x L1 as [Th | Tl]: 64-row tiles, K split over a cluster of S CTAs
 // (S doubles while the CTAs fit twice on the SMs and every split keeps two
 // 64-wide chunks).
-wlq_status launch_prep_lr_t(const uint16_t* x, const uint16_t* L1, const float* xs, int M, int K, int r, int W,
-                            uint16_t* thl, DeviceInfo* d, cudaStream_t s) {
+wlq_status launch_prep_lr_t(const uint16_t* x, const uint16_t* L1, const float* xs, int xs_scalar, int M, int K, int r,
+                            int W, uint16_t* thl, DeviceInfo* d, cudaStream_t s) {
     auto kern = wlq::prep_lr_t_kernel;
     const size_t smem = wlq::lr_t_smem_bytes();
     if (!d->smem_set[27]) {
@@ -693,7 +693,7 @@ wlq_status launch_prep_lr_t(const uint16_t* x, const uint16_t* L1, const float* 
     }
     cudaLaunchAttribute all_attrs[2];
     add_pdl(cfg, all_attrs);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, x, L1, xs, M, K, r, W, S, kc_per, thl);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, x, L1, xs, M, K, r, W, S, kc_per, xs_scalar, thl);
     return e == cudaSuccess ? WLQ_OK : cuda_fail(e, "prep_lr_t launch");
 }
 
@@ -941,7 +941,7 @@ wlq_status wlq_nvfp4_quantize(const void* X, int x_dtype, int64_t rows, int64_t 
     if ((st = current_device(&dev, &d)) != WLQ_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemsetAsync(gscale, 0, 2 * sizeof(float), s);
-    if (e == cudaSuccess && (rows % 128 || K % 256)) e = cudaMemsetAsync(scales, 0, wlq::nv_scale_bytes(rows, K), s);
+    if (e == cudaSuccess && (rows % 256 || K % 256)) e = cudaMemsetAsync(scales, 0, wlq::nv_scale_bytes(rows, K), s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
     const int64_t nblocks = rows * (K / 16);
     const int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(cdiv(nblocks, 256), 1), int64_t(d->sms) * 8));
@@ -1101,13 +1101,13 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
         l2t = reinterpret_cast<uint16_t*>(ws + p.off_l2t);
         // the branch is folded into the GEMM's accumulator: T' = T / xs (int4) and
         // L2' = L2 / rowf, rowf read from the packed operand
-        if ((st = launch_prep_lr_t(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(L1), xs, p.M, p.K, r,
-                                   W, thl, d, s)) != WLQ_OK)
+        if ((st = launch_prep_lr_t(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(L1), xs, 0, p.M, p.K,
+                                   r, W, thl, d, s)) != WLQ_OK)
             return st;
         const float* rowf = reinterpret_cast<const float*>(static_cast<const uint8_t*>(packed) +
                                                            static_cast<size_t>(NT) * p.KT * wlq::tile_bytes(fmt));
         launch_k(wlq::prep_lr_l2t_kernel, static_cast<int>(NT * 128 / wlq::L2T_ROWS), 256, 0, s,
-                 static_cast<const uint16_t*>(L2), rowf, p.N, static_cast<int>(NT * 128), r, W, l2t);
+                 static_cast<const uint16_t*>(L2), rowf, 0, p.N, static_cast<int>(NT * 128), r, W, l2t);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "prep launch");
@@ -1397,14 +1397,14 @@ wlq_status wlq_probe_wait_timeout(uint64_t timeout_ns, void* stream) {
 // NVFP4 W4A4 Linear (block-scaled tensor-core GEMM plus the low-rank branch)
 namespace {
 
-// 2-D tensor of bytes [rows, cols] (cols contiguous), 128 x 128-byte boxes
-// with a 128-byte swizzle; out-of-range bytes read as zero.
-wlq_status make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+// 2-D tensor of bytes [rows, cols] (cols contiguous), box_rows x 128-byte
+// boxes with a 128-byte swizzle; out-of-range bytes read as zero.
+wlq_status make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(WLQ_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {cols};
-    const cuuint32_t box[2] = {128, 128};
+    const cuuint32_t box[2] = {128, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1414,29 +1414,28 @@ wlq_status make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64
 }
 
 struct NvPlan {
-    int NT = 0, MT = 0, KS = 0, KA = 0, tiles = 0, stages = 0, lr_kb = 0, W = 0, acc_bufs = 2;
+    int NT = 0, MT = 0, KS = 0, KA = 0, tiles = 0, stages = 0, lr_kb = 0, W = 0;
     size_t smem = 0, off_thl = 0, off_l2t = 0, ws = 0;
 };
 
 constexpr size_t kMaxDynSmem = 232448;  // 227 KB per CTA
 
 bool nv_plan(NvPlan& p, int64_t M, int64_t N, int64_t K, int r) {
-    p.NT = static_cast<int>(cdiv(N, 128));
-    p.MT = static_cast<int>(cdiv(M, 128));
+    p.NT = static_cast<int>(cdiv(N, wlq::NV_TM));
+    p.MT = static_cast<int>(cdiv(M, wlq::NV_TN));
     p.KS = static_cast<int>(cdiv(K, 256));
     p.KA = p.KS * 4;
     p.tiles = p.NT * p.MT;
     p.lr_kb = r ? static_cast<int>(cdiv(3 * r, 64)) : 0;
     p.W = 64 * p.lr_kb;
-    p.acc_bufs = r ? 1 : 2;  // a low-rank accumulator takes the second buffer's columns
     p.stages = 0;
     for (int st = wlq::NV_MAX_STAGES; st >= 2; --st)
-        if (wlq::nv_smem_bytes(st, p.lr_kb) <= kMaxDynSmem) {
+        if (wlq::nv_smem_bytes(st) <= kMaxDynSmem) {
             p.stages = st;
             break;
         }
     if (!p.stages) return false;
-    p.smem = wlq::nv_smem_bytes(p.stages, p.lr_kb);
+    p.smem = wlq::nv_smem_bytes(p.stages);
     size_t off = 0;
     if (r) {
         p.off_thl = off;
@@ -1473,7 +1472,8 @@ wlq_status check_nvfp4_linear(const void* xq, const void* xs, const float* xg, c
 
 template <bool LR>
 wlq_status launch_nvfp4_gemm(const NvPlan& p, const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& tl,
-                             const CUtensorMap& tt, const wlq::NvArgs& a, DeviceInfo* d, cudaStream_t s) {
+                             const CUtensorMap& tt, const CUtensorMap& ty, const wlq::NvArgs& a, DeviceInfo* d,
+                             cudaStream_t s) {
     auto kern = wlq::nvfp4_gemm_kernel<LR>;
     const int kid = LR ? 51 : 50;
     if (!d->smem_set[kid]) {
@@ -1482,7 +1482,7 @@ wlq_status launch_nvfp4_gemm(const NvPlan& p, const CUtensorMap& tw, const CUten
         d->smem_set[kid] = true;
     }
     const int grid = std::min(p.tiles, d->sms);
-    cudaError_t e = launch_k(kern, grid, wlq::NV_THREADS, p.smem, s, tw, tx, tl, tt, a);
+    cudaError_t e = launch_k(kern, grid, wlq::NV_THREADS, p.smem, s, tw, tx, tl, tt, ty, a);
     return e == cudaSuccess ? WLQ_OK : cuda_fail(e, "nvfp4 gemm launch");
 }
 
@@ -1500,23 +1500,24 @@ wlq_status nvfp4_linear_impl(const void* xq, const void* xs, const float* xg, co
     if (r) {
         thl = reinterpret_cast<uint16_t*>(ws + p.off_thl);
         l2t = reinterpret_cast<uint16_t*>(ws + p.off_l2t);
-        // T = x L1 split into bf16 [T_h | T_l | T_h], L2 into [L2_h | L2_h | L2_l] (no scaling)
-        if ((st = launch_prep_lr_t(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(L1), nullptr,
+        // T / g_x and L2 / g_w, each split into bf16 [h | l | h] and [h | h | l]: the
+        // branch then adds into the FP4 accumulator, which the epilogue scales by g_x g_w
+        if ((st = launch_prep_lr_t(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(L1), xg, 1,
                                    static_cast<int>(M), static_cast<int>(K), r, p.W, thl, d, s)) != WLQ_OK)
             return st;
-        launch_k(wlq::prep_lr_l2t_kernel, p.NT * 128 / wlq::L2T_ROWS, 256, 0, s, static_cast<const uint16_t*>(L2),
-                 static_cast<const float*>(nullptr), static_cast<int>(N), p.NT * 128, r, p.W, l2t);
+        launch_k(wlq::prep_lr_l2t_kernel, p.NT * 128 / wlq::L2T_ROWS, 256, 0, s, static_cast<const uint16_t*>(L2), wg, 1,
+                 static_cast<int>(N), p.NT * 128, r, p.W, l2t);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "low-rank prep launch");
     }
     CUtensorMap tw, tx, tl, tt;
     std::memset(&tl, 0, sizeof tl);
     std::memset(&tt, 0, sizeof tt);
-    if ((st = make_map_u8(&tw, wq, N, K / 2)) != WLQ_OK) return st;
-    if ((st = make_map_u8(&tx, xq, M, K / 2)) != WLQ_OK) return st;
+    if ((st = make_map_u8(&tw, wq, N, K / 2, wlq::NV_TM)) != WLQ_OK) return st;
+    if ((st = make_map_u8(&tx, xq, M, K / 2, wlq::NV_TN)) != WLQ_OK) return st;
     if (r) {
-        if ((st = make_map_2d(&tl, l2t, static_cast<uint64_t>(p.NT) * 128, p.W, 128)) != WLQ_OK) return st;
-        if ((st = make_map_2d(&tt, thl, M, p.W, 128)) != WLQ_OK) return st;
+        if ((st = make_map_2d(&tl, l2t, static_cast<uint64_t>(p.NT) * 128, p.W, wlq::NV_TM)) != WLQ_OK) return st;
+        if ((st = make_map_2d(&tt, thl, M, p.W, wlq::NV_TN)) != WLQ_OK) return st;
     }
     wlq::NvArgs a;
     std::memset(&a, 0, sizeof a);
@@ -1537,9 +1538,26 @@ wlq_status nvfp4_linear_impl(const void* xq, const void* xs, const float* xg, co
     a.stages = p.stages;
     a.lr_kb = p.lr_kb;
     a.y_f32 = (y_dtype == WLQ_OUT_F32) ? 1 : 0;
-    a.acc_bufs = p.acc_bufs;
+    // y through TMA stores when its rows are whole 16-byte units (else plain stores)
+    CUtensorMap ty;
+    std::memset(&ty, 0, sizeof ty);
+    const size_t esize = a.y_f32 ? 4 : 2;
+    if (aligned16(y) && (static_cast<size_t>(N) * esize) % 16 == 0) {
+        EncodeTiledFn fn = encode_fn();
+        if (!fn) return fail(WLQ_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * esize};
+        const cuuint32_t box[2] = {32, 16};
+        const cuuint32_t estr[2] = {1, 1};
+        CUresult cr = fn(&ty, a.y_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, y, dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (cr != CUDA_SUCCESS) return fail(WLQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(cr));
+        a.tma_store = 1;
+    }
     a.timeout_ns = kDefaultTimeoutNs;
-    return r ? launch_nvfp4_gemm<true>(p, tw, tx, tl, tt, a, d, s) : launch_nvfp4_gemm<false>(p, tw, tx, tl, tt, a, d, s);
+    return r ? launch_nvfp4_gemm<true>(p, tw, tx, tl, tt, ty, a, d, s)
+             : launch_nvfp4_gemm<false>(p, tw, tx, tl, tt, ty, a, d, s);
 }
 
 struct W4a4Layout {
