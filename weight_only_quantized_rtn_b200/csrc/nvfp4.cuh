@@ -16,11 +16,11 @@
 // operands: a quotient of a 24-bit by a 26-bit number is either an E4M3
 // midpoint exactly or at least 2^-31 away from one (relative), far above
 // fp64's rounding error.  The element decision compares |x| with the seven
-// midpoints t (0.25, 0.75, ..., 5) times d = s_b g: in fp32 each threshold
-// is carried as a rounded product plus its exact fma error, and |x| minus the
-// rounded product is exact wherever the comparison can go either way (in
-// fp64 for tensors with amax below ~1e-26, where the error could underflow);
-// no division is rounded.
+// midpoints t (0.25, 0.75, ..., 5) times d = s_b g: each threshold's rounded
+// product and exact fma error give the smallest fp32 value that passes it,
+// so the decision is one exact fp32 comparison per threshold (in fp64 for
+// tensors with amax below ~1e-26, where the error could underflow); no
+// division is rounded.
 //
 // Layouts (what the block-scaled tensor-core MMA reads):
 //   codes  : [rows, K / 2] bytes, input k in byte k / 2, low nibble for even k;
@@ -149,24 +149,26 @@ __global__ void __launch_bounds__(256) nvfp4_amax_kernel(const void* __restrict_
 }
 
 // Pass 2: one thread per block of 16 inputs (consecutive threads take
-// consecutive blocks of a row): block scale, then each code by a three-step
+// consecutive blocks of a row, 2^lg_tpr threads a row): block scale, then each code by a three-step
 // search over the midpoints.  A midpoint between codes i and i + 1 rounds up
 // when i is odd (the even neighbour is i + 1), so "passed" is |x| >= T_i for
 // odd i and |x| > T_i for even i.
 template <int DT>
 __global__ void __launch_bounds__(256) nvfp4_quantize_kernel(const void* __restrict__ X, int64_t rows, int64_t K,
                                                              float* __restrict__ gscale, uint8_t* __restrict__ codes,
-                                                             uint8_t* __restrict__ scales) {
+                                                             uint8_t* __restrict__ scales, int lg_tpr) {
     grid_dependency_sync();
     const float amax = __uint_as_float(*reinterpret_cast<const volatile unsigned int*>(gscale + 1));
     const float g = __fdiv_rn(amax, 2688.0f);
-    const int64_t kb_per_row = K / 16;
-    const int64_t nblocks = rows * kb_per_row;
+    const int kb_per_row = static_cast<int>(K / 16);
     const int64_t KA = nv_atoms_per_row_tile(K);
     if (blockIdx.x == 0 && threadIdx.x == 0) gscale[0] = g;
-    for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nblocks;
-         b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t row = b / kb_per_row, kb = b - row * kb_per_row;
+    // 2^lg_tpr threads per row (the CTA covers 256 >> lg_tpr rows a pass): no index division
+    const int tpr = 1 << lg_tpr, rpc = 256 >> lg_tpr;
+    for (int64_t row = static_cast<int64_t>(blockIdx.x) * rpc + (threadIdx.x >> lg_tpr); row < rows;
+         row += static_cast<int64_t>(gridDim.x) * rpc)
+    for (int kb = threadIdx.x & (tpr - 1); kb < kb_per_row; kb += tpr) {
+        const int64_t b = row * kb_per_row + kb;
         float v[16];
         uint32_t sg;
         nv_load16<DT>(X, static_cast<size_t>(b) * 16, v, &sg);
@@ -176,27 +178,28 @@ __global__ void __launch_bounds__(256) nvfp4_quantize_kernel(const void* __restr
         const uint32_t sb = (g > 0.0f) ? e4m3_from_f64(static_cast<double>(ab) / (6.0 * static_cast<double>(g))) : 0u;
         uint32_t lo = 0, hi = 0;
         if (sb != 0 && g >= 1e-30f) {
-            // fp32: T_i = t_i s_b g as p_i + e_i exactly (u_i = t_i s_b has at most 7 bits; the fma
-            // error is exact because u_i g stays far above the subnormals), and |x| - p_i is exact
-            // whenever |x| is within a factor 2 of p_i, which is the only case it can tie or flip
+            // T_i = t_i s_b g is carried as p_i = fl(u_i g) plus its exact fma error e_i (u_i = t_i s_b
+            // has at most 7 bits; the error is exact while u_i g stays far above the subnormals).  From
+            // them, A_i = the smallest fp32 value that passes T_i: p_i itself when p_i already passes
+            // (p_i >= T_i for odd i, > T_i for even i), else the next float up.  |x| is an fp32 value,
+            // so |x| passes T_i exactly when |x| >= A_i: one comparison per threshold.
             const float sf = e4m3_to_f32(sb);
-            float P[7], E[7];
+            float A[7];
             const float tau[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f};
 #pragma unroll
             for (int t = 0; t < 7; ++t) {
                 const float u = tau[t] * sf;
-                P[t] = __fmul_rn(u, g);
-                E[t] = __fmaf_rn(u, g, -P[t]);
+                const float pt = __fmul_rn(u, g);
+                const float et = __fmaf_rn(u, g, -pt);  // T_t - p_t, exact
+                const bool p_passes = (t & 1) ? (et <= 0.0f) : (et < 0.0f);
+                A[t] = p_passes ? pt : __int_as_float(__float_as_int(pt) + 1);
             }
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const float a = v[i];
-                const bool p4 = __fsub_rn(a, P[3]) >= E[3];                      // past T_3 (odd: ties up)
-                const float p1v = p4 ? P[5] : P[1], e1v = p4 ? E[5] : E[1];
-                const bool p2 = __fsub_rn(a, p1v) >= e1v;                        // past T_5 / T_1 (odd)
-                const float p0v = p4 ? (p2 ? P[6] : P[4]) : (p2 ? P[2] : P[0]);
-                const float e0v = p4 ? (p2 ? E[6] : E[4]) : (p2 ? E[2] : E[0]);
-                const bool p1 = __fsub_rn(a, p0v) > e0v;                         // even: ties stay
+                const bool p4 = a >= A[3];
+                const bool p2 = a >= (p4 ? A[5] : A[1]);
+                const bool p1 = a >= (p4 ? (p2 ? A[6] : A[4]) : (p2 ? A[2] : A[0]));
                 const uint32_t c = (p4 ? 4u : 0u) + (p2 ? 2u : 0u) + (p1 ? 1u : 0u) + (((sg >> i) & 1u) << 3);
                 if (i < 8) lo |= c << (4 * i);
                 else hi |= c << (4 * (i - 8));

@@ -945,14 +945,17 @@ wlq_status wlq_nvfp4_quantize(const void* X, int x_dtype, int64_t rows, int64_t 
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
     const int64_t nblocks = rows * (K / 16);
     const int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(cdiv(nblocks, 256), 1), int64_t(d->sms) * 8));
+    int lg_tpr = 0;  // threads per row of the quantize pass: the 16-input blocks of a row, up to 256
+    while ((1 << lg_tpr) < 256 && (int64_t(1) << lg_tpr) < K / 16) ++lg_tpr;
+    const int qgrid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(cdiv(rows, 256 >> lg_tpr), 1), int64_t(d->sms) * 8));
     if (x_dtype == WLQ_IN_BF16) {
         launch_k(wlq::nvfp4_amax_kernel<1>, grid, 256, 0, s, X, nblocks, gscale);
-        launch_k(wlq::nvfp4_quantize_kernel<1>, grid, 256, 0, s, X, rows, K, gscale, static_cast<uint8_t*>(codes),
-                 static_cast<uint8_t*>(scales));
+        launch_k(wlq::nvfp4_quantize_kernel<1>, qgrid, 256, 0, s, X, rows, K, gscale, static_cast<uint8_t*>(codes),
+                 static_cast<uint8_t*>(scales), lg_tpr);
     } else {
         launch_k(wlq::nvfp4_amax_kernel<0>, grid, 256, 0, s, X, nblocks, gscale);
-        launch_k(wlq::nvfp4_quantize_kernel<0>, grid, 256, 0, s, X, rows, K, gscale, static_cast<uint8_t*>(codes),
-                 static_cast<uint8_t*>(scales));
+        launch_k(wlq::nvfp4_quantize_kernel<0>, qgrid, 256, 0, s, X, rows, K, gscale, static_cast<uint8_t*>(codes),
+                 static_cast<uint8_t*>(scales), lg_tpr);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "nvfp4 quantize launch");
