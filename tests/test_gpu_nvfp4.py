@@ -187,3 +187,84 @@ def test_nvfp4_linear_from_quantized_operands_equals_w4a4():
     m.w4a4_linear_into(y2, x, wq, ws, wg, N, K, L1=L1, L2=L2)
     m.check_status()
     assert torch.equal(y1, y2)
+
+
+@pytest.mark.parametrize("M,N,K,r,out", [
+    (1, 301, 128, 0, torch.float32),     # one token; odd N: rows of y are not 16-byte units (plain stores)
+    (17, 300, 192, 16, torch.bfloat16),  # N * 2 bytes not a multiple of 16 (plain stores), K % 256 != 0
+    (257, 136, 320, 32, torch.float32),  # a second 256-token tile holding one token
+])
+def test_w4a4_linear_ragged_shapes_and_plain_store_epilogue(M, N, K, r, out):
+    assert _linear_case(M, N, K, r, True, out, seed=M + N + K) <= TOL_F32
+
+
+def test_w4a4_linear_misaligned_output_takes_plain_stores():
+    """y 4 bytes past a 16-byte boundary: the epilogue cannot use TMA stores
+    and must write the same values with plain stores."""
+    m = wlq()
+    M, N, K = 64, 256, 256
+    x_bits = wi.activations(41, 1, M, K)
+    W = wi.weight(41, 2, N, K)
+    x = dev_bf16(x_bits)
+    wq, ws, wg = m.nvfp4_quantize(dev_f32(W))
+    y_al = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    buf = torch.empty(M * N + 4, dtype=torch.float32, device="cuda")
+    y_mis = buf[1:1 + M * N].view(M, N)
+    m.w4a4_linear_into(y_al, x, wq, ws, wg, N, K)
+    m.w4a4_linear_into(y_mis, x, wq, ws, wg, N, K)
+    m.check_status()
+    assert torch.equal(y_al, y_mis)
+
+
+def test_w4a4_zero_weights_keep_the_low_rank_term_and_zero_x_gives_bias():
+    """An all-zero weight tensor has tensor scale 0: the low-rank operand is then
+    left unscaled, so y = (x L1) L2 + b.  An all-zero x gives y = b."""
+    m = wlq()
+    M, N, K, r = 48, 128, 256, 32
+    x_bits = wi.activations(43, 1, M, K)
+    b_bits = wi.bias(43, 3, N)
+    L1 = wi.normal_bf16(wi.rng(43, 4), (K, r), 0.05)
+    L2 = wi.normal_bf16(wi.rng(43, 5), (r, N), 0.05)
+    W = np.zeros((N, K), np.float32)
+    wq, ws, wg = m.nvfp4_quantize(dev_f32(W))
+    assert float(wg[0]) == 0.0
+    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    m.w4a4_linear_into(y, dev_bf16(x_bits), wq, ws, wg, N, K, dev_bf16(b_bits), dev_bf16(L1), dev_bf16(L2))
+    m.check_status()
+    xq_o, xs_o, xg_o = oracle.nvfp4_quantize(x_bits)
+    wq_o, ws_o, wg_o = oracle.nvfp4_quantize(W)
+    y_ref = oracle.nvfp4_linear(xq_o, xs_o, xg_o, x_bits, wq_o, ws_o, wg_o, b_bits, L1, L2)
+    assert rel_err(y.cpu().numpy(), y_ref) <= TOL_F32
+    # x = 0: every code and the low-rank term vanish
+    xz = np.zeros((M, K), np.uint16)
+    W2 = wi.weight(43, 2, N, K)
+    wq2, ws2, wg2 = m.nvfp4_quantize(dev_f32(W2))
+    m.w4a4_linear_into(y, dev_bf16(xz), wq2, ws2, wg2, N, K, dev_bf16(b_bits), dev_bf16(L1), dev_bf16(L2))
+    m.check_status()
+    np.testing.assert_array_equal(y.cpu().numpy(), np.broadcast_to(oracle._bf16_value(b_bits), (M, N)))
+
+
+def test_nvfp4_nonfinite_input_is_reported():
+    m = wlq()
+    X = np.ones((4, 64), np.float32)
+    X[2, 5] = np.inf
+    m.nvfp4_quantize(dev_f32(X))
+    with pytest.raises(m.WlqError):
+        m.check_status()
+    m.check_status()  # the status word was cleared by the report
+
+
+def test_w4a4_forward_is_bitwise_reproducible():
+    m = wlq()
+    M, N, K, r = 300, 384, 512, 32
+    x = dev_bf16(wi.activations(47, 1, M, K))
+    wq, ws, wg = m.nvfp4_quantize(dev_f32(wi.weight(47, 2, N, K)))
+    L1 = dev_bf16(wi.normal_bf16(wi.rng(47, 4), (K, r), 0.05))
+    L2 = dev_bf16(wi.normal_bf16(wi.rng(47, 5), (r, N), 0.05))
+    ys = []
+    for _ in range(3):
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        m.w4a4_linear_into(y, x, wq, ws, wg, N, K, L1=L1, L2=L2)
+        ys.append(y)
+    m.check_status()
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[0], ys[2])
