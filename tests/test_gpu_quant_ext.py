@@ -170,3 +170,43 @@ def test_quantize_ex_scale_midpoints_and_subnormal_scales(bits, scale_dtype):
     m.check_status()
     np.testing.assert_array_equal(sg.float().cpu().numpy(), so)
     np.testing.assert_array_equal(cg.cpu().numpy(), co)
+
+
+@pytest.mark.parametrize("group", [8, 32, 64, 256])
+@pytest.mark.parametrize("bits,scale_dtype", [(8, 1), (4, 0), (5, 2)])
+def test_quantize_ex_bf16_power_of_two_groups_bit_exact(group, bits, scale_dtype):
+    """bf16 input with groups of 8..256 (8 inputs a lane, groups across 1..32
+    lanes) against the oracle."""
+    m = wlq()
+    W = _edge_weights(group + bits + scale_dtype, 29, 1024)
+    if scale_dtype == 1:
+        W[2] = 0.001
+    co, so = oracle.quantize_ex(_host_in(W, True), bits, group, scale_dtype)
+    cg, sg = m.quantize_ex(_dev(W, True), bits, group, scale_dtype)
+    torch.cuda.synchronize()
+    m.check_status()
+    np.testing.assert_array_equal(cg.cpu().numpy(), co)
+    np.testing.assert_array_equal(sg.float().cpu().numpy(), so)
+
+
+def test_quantize_ex_bf16_nonfinite_group_and_unaligned_codes():
+    """A NaN zeroes its group and raises the flag; codes that are only 4-byte
+    aligned take the general path and give the same bytes."""
+    m = wlq()
+    m.check_status()
+    W = (np.random.default_rng(5).standard_normal((16, 256)) * 0.3).astype(np.float32)
+    W[3, 70] = np.nan
+    x = _dev(W, True)
+    c, s = m.quantize_ex(x, 8, 64, 1)
+    assert m.get_status() == m.ERR_NONFINITE
+    assert float(s[3, 1]) == 0.0 and not c[3, 64:128].any()
+    W[3, 70] = 0.25
+    x = _dev(W, True)
+    c, s = m.quantize_ex(x, 8, 64, 1)
+    m.check_status()
+    buf = torch.empty(16 * 256 + 4, dtype=torch.int8, device="cuda")
+    c_mis = buf[4:4 + 16 * 256].view(16, 256)
+    s2 = torch.empty_like(s)
+    m.lib.wlq_quantize_ex(m._ptr(x), 1, 16, 256, 8, 64, 1, m._ptr(c_mis), m._ptr(s2), m._stream())
+    m.check_status()
+    assert torch.equal(c, c_mis) and torch.equal(s, s2)

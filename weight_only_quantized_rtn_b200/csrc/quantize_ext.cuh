@@ -283,6 +283,129 @@ __global__ void __launch_bounds__(256) quantize_ex_short_kernel(const void* __re
     if (bad) raise_error(ERRBIT_NONFINITE);
 }
 
+// bf16 input, groups of G = 8 * LG inputs (LG a power of two, at most 32):
+// a lane takes 8 adjacent inputs (one 16-byte load) a round, so a warp covers
+// 256 inputs (256 / G groups) a round, four rounds in flight; when the warp's
+// groups fit one per lane, each scale is worked out once, by one lane.  The group's
+// absmax is the maximum of the bf16 magnitude bits (two at a time, 16-bit
+// lanes), reduced over its LG lanes; the stored scale and the exactly rounded
+// codes are those of quantize_ex_short_kernel (same stored_scale, same
+// rtn4_f32 / rtn4_f32_clamped), so the results are bit-identical.  Codes go
+// out as one 8-byte store per lane (codes 8-byte aligned).
+template <int SF, int LG>
+__global__ void __launch_bounds__(256) quantize_ex_bf16_kernel(const uint16_t* __restrict__ W, int64_t total8,
+                                                               int qmax, int8_t* __restrict__ codes,
+                                                               void* __restrict__ scales) {
+    grid_dependency_sync();
+    constexpr int U = 4;            // rounds in flight
+    constexpr int GPR = 32 / LG;    // groups per warp-round
+    constexpr int NGW = U * GPR;    // groups the warp holds
+    const int lane = threadIdx.x & 31;
+    const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    const uint4* W8 = reinterpret_cast<const uint4*>(W);
+    uint2* out = reinterpret_cast<uint2*>(codes);
+    bool bad = false;
+    for (int64_t r0 = w0 * U; r0 * 32 < total8; r0 += nw * U) {
+        uint4 raw[U];
+        uint32_t m[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i8 = (r0 + u) * 32 + lane;
+            raw[u] = i8 < total8 ? __ldcs(W8 + i8) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint4 r = raw[u];
+            const uint32_t m2 = __vmaxu2(__vmaxu2(r.x & 0x7FFF7FFFu, r.y & 0x7FFF7FFFu),
+                                         __vmaxu2(r.z & 0x7FFF7FFFu, r.w & 0x7FFF7FFFu));
+            m[u] = max(m2 & 0xFFFFu, m2 >> 16);
+#pragma unroll
+            for (int off = LG >> 1; off > 0; off >>= 1) m[u] = max(m[u], __shfl_xor_sync(0xffffffffu, m[u], off));
+        }
+        float su[U], iu[U];
+        bool bu[U];
+        if constexpr (NGW <= 32) {
+            // lane j works out the scale of group (j / GPR, j % GPR) once -- the 16-bit rounding and
+            // the reciprocal per group, not per lane of it -- and the results go back by shuffle
+            const int ju = lane / GPR, jg = lane % GPR;
+            uint32_t mj = 0;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const uint32_t mu = __shfl_sync(0xffffffffu, m[u], jg * LG);
+                if (ju == u) mj = mu;
+            }
+            bool gbad = mj >= 0x7F80u;  // NaN or infinity in the group
+            float sj = stored_scale<SF>(gbad ? 0.0f : __uint_as_float(mj << 16), qmax);
+            if (isinf(sj)) {  // the 16-bit scale overflowed
+                gbad = true;
+                sj = 0.0f;
+            }
+            const float ij = (sj >= 1.17549435e-38f) ? __frcp_rn(sj) : 0.0f;
+            const int gb = gbad ? 1 : 0;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                su[u] = __shfl_sync(0xffffffffu, sj, u * GPR + lane / LG);
+                iu[u] = __shfl_sync(0xffffffffu, ij, u * GPR + lane / LG);
+                bu[u] = __shfl_sync(0xffffffffu, gb, u * GPR + lane / LG) != 0;
+            }
+        } else {
+            // one group per lane or two lanes a group: each lane its own
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                bool gbad = m[u] >= 0x7F80u;
+                float sg = stored_scale<SF>(gbad ? 0.0f : __uint_as_float(m[u] << 16), qmax);
+                if (isinf(sg)) {
+                    gbad = true;
+                    sg = 0.0f;
+                }
+                su[u] = sg;
+                iu[u] = (sg >= 1.17549435e-38f) ? __frcp_rn(sg) : 0.0f;
+                bu[u] = gbad;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i8 = (r0 + u) * 32 + lane;
+            if (i8 >= total8) continue;
+            const uint4 r = raw[u];
+            const float sg = su[u];
+            bad |= bu[u];
+            if ((lane & (LG - 1)) == 0) {
+                const int64_t gi = i8 / LG;
+                if constexpr (SF == SCALE_F32) static_cast<float*>(scales)[gi] = sg;
+                else if constexpr (SF == SCALE_F16) static_cast<__half*>(scales)[gi] = __float2half_rn(sg);
+                else static_cast<__nv_bfloat16*>(scales)[gi] = __float2bfloat16_rn(sg);
+            }
+            const float4 lo = make_float4(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xFFFF0000u),
+                                          __uint_as_float(r.y << 16), __uint_as_float(r.y & 0xFFFF0000u));
+            const float4 hi = make_float4(__uint_as_float(r.z << 16), __uint_as_float(r.z & 0xFFFF0000u),
+                                          __uint_as_float(r.w << 16), __uint_as_float(r.w & 0xFFFF0000u));
+            uint32_t c0 = 0, c1 = 0;
+            if (sg >= 1.17549435e-38f) {
+                if constexpr (SF == SCALE_F32) {
+                    c0 = rtn4_f32(lo, sg, iu[u], 0.5f * sg);
+                    c1 = rtn4_f32(hi, sg, iu[u], 0.5f * sg);
+                } else {
+                    c0 = rtn4_f32_clamped(lo, sg, iu[u], 0.5f * sg, static_cast<float>(qmax));
+                    c1 = rtn4_f32_clamped(hi, sg, iu[u], 0.5f * sg, static_cast<float>(qmax));
+                }
+            } else if (sg > 0.0f) {
+                GroupScale gs;
+                gs.s = sg;
+                gs.normal = false;
+                gs.inv = 0.0f;
+                gs.inv64 = 1.0 / static_cast<double>(sg);
+                bool unused = false;
+                c0 = pack_codes4(lo, gs, qmax, unused);
+                c1 = pack_codes4(hi, gs, qmax, unused);
+            }
+            out[i8] = make_uint2(c0, c1);
+        }
+    }
+    if (bad) raise_error(ERRBIT_NONFINITE);
+}
+
 __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));

@@ -865,7 +865,29 @@ wlq_status wlq_quantize_ex(const void* W, int w_dtype, int64_t N, int64_t K, int
     const int g4 = static_cast<int>(g / 4);
     const int qmax = (1 << (bits - 1)) - 1;
     const bool bf = (w_dtype == WLQ_IN_BF16);
-    if (g4 <= 32 && 32 % g4 == 0) {
+    const int LG = static_cast<int>(g / 8);  // bf16: lanes per group at 8 inputs a lane
+    if (bf && g % 8 == 0 && g <= 256 && (LG & (LG - 1)) == 0 && (reinterpret_cast<uintptr_t>(codes) & 7u) == 0) {
+        // bf16 with power-of-two groups of 8..256: 8 inputs a lane, four rounds in flight, persistent
+        const int64_t total8 = N * K / 8;
+        const int64_t rounds = cdiv(total8, 32);
+        const int grid = static_cast<int>(std::min<int64_t>(cdiv(cdiv(rounds, 4), 8), static_cast<int64_t>(d->sms) * 8));
+        const uint16_t* Wb = static_cast<const uint16_t*>(W);
+#define WLQ_QB(F, L) launch_k(wlq::quantize_ex_bf16_kernel<F, L>, grid, 256, 0, s, Wb, total8, qmax, codes, scales)
+#define WLQ_QBL(F)                 \
+    switch (LG) {                  \
+        case 1: WLQ_QB(F, 1); break;   \
+        case 2: WLQ_QB(F, 2); break;   \
+        case 4: WLQ_QB(F, 4); break;   \
+        case 8: WLQ_QB(F, 8); break;   \
+        case 16: WLQ_QB(F, 16); break; \
+        default: WLQ_QB(F, 32); break; \
+    }
+        if (scale_dtype == WLQ_SCALE_F32) { WLQ_QBL(wlq::SCALE_F32) }
+        else if (scale_dtype == WLQ_SCALE_F16) { WLQ_QBL(wlq::SCALE_F16) }
+        else { WLQ_QBL(wlq::SCALE_BF16) }
+#undef WLQ_QBL
+#undef WLQ_QB
+    } else if (g4 <= 32 && 32 % g4 == 0) {
         // short groups: one pass from registers, 32 / g4 groups per warp, four rounds in flight
         // persistent: the CTAs that fit at once (8 per SM) loop over the rounds
         const int64_t rounds = cdiv(groups * g4, 32);
