@@ -159,13 +159,12 @@ __global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
                     gs.inv64 = (gs.s > 0.0f) ? 1.0 / static_cast<double>(gs.s) : 0.0;
                     c4 = pack_codes4(v[i], gs, qmax, unused);
                 }
-                // four nibbles (q + 8) at their places among the eight of the word
-                uint32_t w = 0;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t u = ((c4 >> (8 * j)) + 8u) & 0xFu;
-                    w |= u << (4 * int4_nibble_pos(4 * (idx & 1) + j));
-                }
+                // four nibbles (q + 8) at their places among the eight of the word: the low nibble of
+                // each code byte with its top bit flipped is q + 8 (|q| <= 7, no carry between bytes);
+                // codes t = 0..3 of an even lane go to nibbles 0, 4, 1, 5, an odd lane's to 2, 6, 3, 7
+                const uint32_t x = c4 ^ 0x08080808u;
+                uint32_t w = (x & 0xFu) | ((x >> 12) & 0xF0u) | ((x << 8) & 0xF0000u) | ((x >> 4) & 0xF00000u);
+                w <<= 8 * (idx & 1);
                 w |= __shfl_xor_sync(0xffffffffu, w, 1);
                 if (idx >= KP4) continue;
                 uint8_t* blk = tiles + (k >> 6) * TB;
