@@ -19,15 +19,16 @@ namespace wlq {
 
 // One CTA per padded output row (grid-stride over ceil(N/128)*128 rows).  The
 // row's ceil(K/64)*64 inputs (zeros past K and for rows >= N) are held in
-// registers: thread j takes float4 j + i*blockDim (i < V), so the lanes of a
-// warp hold consecutive inputs and a group of g inputs is g/4 adjacent lanes.
+// registers: thread j takes the float4 pairs j + i*blockDim (i < V/2), so the
+// lanes of a warp hold consecutive 8-input runs and a group of g inputs is g/8
+// adjacent lanes.
 //  - int8: the row's absmax is reduced over the CTA (magnitude bit patterns,
 //    as in quantize_rows_cta_kernel); each float4 becomes one 32-bit word of
 //    four offset-binary bytes at its place in the row's 16-byte run.
-//  - int4: each group's absmax is reduced over its lanes; the row's largest
-//    group scale (over the CTA) fixes the fp16 normalisation 2^e_n and the
-//    row factor 2^-e_n; two adjacent lanes merge their four nibbles each into
-//    one 32-bit word of eight.
+//  - int4: a lane holds pairs of adjacent float4 (8 inputs, one 32-byte run
+//    per slot); each group's absmax is reduced over its lanes; the row's
+//    largest group scale (over the CTA) fixes the fp16 normalisation 2^e_n
+//    and the row factor 2^-e_n; a lane's eight codes make one 32-bit word.
 template <int FMT, int V>
 __global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
     const float* __restrict__ W, int64_t N, int64_t K, int KT, int64_t rows, int qmax,
@@ -51,7 +52,9 @@ __global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
         float4 v[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            const int idx = threadIdx.x + i * blockDim.x;
+            // pairs of float4 (8 inputs, one 32-byte run) at pair p = threadIdx.x + (i / 2) * blockDim:
+            // a lane's eight int4 codes fill one word, its eight int8 codes one 8-byte store
+            const int idx = 2 * (threadIdx.x + (i >> 1) * blockDim.x) + (i & 1);
             v[i] = (row_ok && idx < K4) ? __ldcs(row + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
         if constexpr (FMT == FMT_W8) {
@@ -77,36 +80,43 @@ __global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
             }
             const float h = 0.5f * g.s;
 #pragma unroll
-            for (int i = 0; i < V; ++i) {
-                const int idx = threadIdx.x + i * blockDim.x;
-                if (idx >= KP4) continue;
+            for (int i = 0; i < V / 2; ++i) {
+                const int p8 = threadIdx.x + i * blockDim.x;
+                if (p8 >= KP4 / 2) continue;
                 bool unused = false;
-                const uint32_t c4 = g.normal ? rtn4_f32(v[i], g.s, g.inv, h) : pack_codes4(v[i], g, qmax, unused);
-                const int k = 4 * idx;  // inputs k..k+3 of block k/64, run (k%64)/16
-                *reinterpret_cast<uint32_t*>(tiles + (k >> 6) * TB + ((k >> 4) & 3) * 2048 + 16 * i_row + (k & 15)) =
-                    c4 ^ 0x80808080u;  // offset binary q + 128
+                const uint32_t ca = g.normal ? rtn4_f32(v[2 * i], g.s, g.inv, h) : pack_codes4(v[2 * i], g, qmax, unused);
+                const uint32_t cb = g.normal ? rtn4_f32(v[2 * i + 1], g.s, g.inv, h)
+                                             : pack_codes4(v[2 * i + 1], g, qmax, unused);
+                const int k = 8 * p8;  // inputs k..k+7 of block k/64, run (k%64)/16, bytes k%16 (0 or 8)
+                *reinterpret_cast<uint2*>(tiles + (k >> 6) * TB + ((k >> 4) & 3) * 2048 + 16 * i_row + (k & 15)) =
+                    make_uint2(ca ^ 0x80808080u, cb ^ 0x80808080u);  // offset binary q + 128
             }
             __syncthreads();  // part[] is rewritten for the next row
         } else {
-            // group absmax (per group of L lanes; 0 for a group holding a NaN
-            // or infinity) and the row's largest group scale over the CTA
-            // (scales are non-negative floats: their bit patterns order them)
-            uint32_t gm[V];
+            // each lane holds V / 2 slots of 8 adjacent inputs; a group is L8 = GS / 8 adjacent lanes.
+            // Group absmax (0 for a group holding a NaN or infinity) reduced over its lanes, and the
+            // row's largest group scale over the CTA (scales are non-negative floats: their bit
+            // patterns order them)
+            constexpr int V2 = V / 2;
+            constexpr int L8 = GS / 8;
+            uint32_t gm[V2];
 #pragma unroll
-            for (int i = 0; i < V; ++i) {
-                uint32_t m = max(max(__float_as_uint(v[i].x) & 0x7FFFFFFFu, __float_as_uint(v[i].y) & 0x7FFFFFFFu),
-                                 max(__float_as_uint(v[i].z) & 0x7FFFFFFFu, __float_as_uint(v[i].w) & 0x7FFFFFFFu));
-                for (int off = L >> 1; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+            for (int i = 0; i < V2; ++i) {
+                const float4 a = v[2 * i], b = v[2 * i + 1];
+                uint32_t m = max(max(max(__float_as_uint(a.x) & 0x7FFFFFFFu, __float_as_uint(a.y) & 0x7FFFFFFFu),
+                                     max(__float_as_uint(a.z) & 0x7FFFFFFFu, __float_as_uint(a.w) & 0x7FFFFFFFu)),
+                                 max(max(__float_as_uint(b.x) & 0x7FFFFFFFu, __float_as_uint(b.y) & 0x7FFFFFFFu),
+                                     max(__float_as_uint(b.z) & 0x7FFFFFFFu, __float_as_uint(b.w) & 0x7FFFFFFFu)));
+                for (int off = L8 >> 1; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
                 const bool gbad = m >= 0x7F800000u;
                 bad |= gbad;
                 gm[i] = gbad ? 0u : m;
             }
-            // The warp holds V * GPW groups (GPW = 32 / L per float4 slot).
-            // Lane j takes groups j and j + 32: the IEEE division and the
-            // reciprocal once per group rather than once per lane of it; the
-            // results go back to each group's lanes by shuffle.
-            constexpr int GPW = 32 / L;
-            constexpr int NGW = V * GPW;
+            // The warp holds V2 * GPW groups (GPW = 32 / L8 per slot).  Lane j takes groups j and
+            // j + 32: the IEEE division and the reciprocal once per group rather than once per lane
+            // of it; the results go back to each group's lanes by shuffle.
+            constexpr int GPW = 32 / L8;
+            constexpr int NGW = V2 * GPW;
             constexpr int PER_LANE = (NGW + 31) / 32;
             float sj[PER_LANE], ij[PER_LANE];
             uint32_t smax = 0;
@@ -115,8 +125,8 @@ __global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
                 const int j = lane + 32 * t, ji = j / GPW, jg = j % GPW;
                 uint32_t mj = 0;
 #pragma unroll
-                for (int i = 0; i < V; ++i) {
-                    const uint32_t mi = __shfl_sync(0xffffffffu, gm[i], jg * L);
+                for (int i = 0; i < V2; ++i) {
+                    const uint32_t mi = __shfl_sync(0xffffffffu, gm[i], jg * L8);
                     if (ji == i) mj = mi;
                 }
                 const GroupScale gs = group_scale(__uint_as_float(mj), qmax);
@@ -138,39 +148,40 @@ __global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
             }
             if (threadIdx.x == 0) rowf[n] = rf;
             const int sh = (rf > 0.0f) ? -ilogbf(rf) : 0;  // s * 2^sh = s / rf exactly
+            const int KP8 = KP4 / 2;
 #pragma unroll
-            for (int i = 0; i < V; ++i) {
-                const int idx = threadIdx.x + i * blockDim.x;
-                const int k = 4 * idx;
-                bool unused = false;
-                // this slot's group scale, from the lane that worked it out
-                // (group i * GPW + lane / L: the same lane slot t = i * GPW / 32 for
-                // every lane, since GPW divides 32)
+            for (int i = 0; i < V2; ++i) {
+                const int p8 = threadIdx.x + i * blockDim.x;  // this lane's 8 inputs: k = 8 p8 ..
+                const int k = 8 * p8;
+                // this slot's group scale, from the lane that worked it out (group i * GPW + lane / L8:
+                // the same lane slot t = i * GPW / 32 for every lane, since GPW divides 32)
                 const int src_t = (i * GPW) / 32;
-                const int src = (i * GPW) % 32 + lane / L;
+                const int src = (i * GPW) % 32 + lane / L8;
                 GroupScale gs;
                 gs.s = __shfl_sync(0xffffffffu, sj[src_t], src);
                 gs.inv = __shfl_sync(0xffffffffu, ij[src_t], src);
                 gs.normal = gs.s >= 1.17549435e-38f;
-                uint32_t c4;
+                uint32_t ca, cb;
                 if (gs.normal) {
-                    c4 = rtn4_f32(v[i], gs.s, gs.inv, 0.5f * gs.s);
+                    ca = rtn4_f32(v[2 * i], gs.s, gs.inv, 0.5f * gs.s);
+                    cb = rtn4_f32(v[2 * i + 1], gs.s, gs.inv, 0.5f * gs.s);
                 } else {  // rare: a subnormal (or zero) scale takes the fp64 path
+                    bool unused = false;
                     gs.inv64 = (gs.s > 0.0f) ? 1.0 / static_cast<double>(gs.s) : 0.0;
-                    c4 = pack_codes4(v[i], gs, qmax, unused);
+                    ca = pack_codes4(v[2 * i], gs, qmax, unused);
+                    cb = pack_codes4(v[2 * i + 1], gs, qmax, unused);
                 }
-                // four nibbles (q + 8) at their places among the eight of the word: the low nibble of
-                // each code byte with its top bit flipped is q + 8 (|q| <= 7, no carry between bytes);
-                // codes t = 0..3 of an even lane go to nibbles 0, 4, 1, 5, an odd lane's to 2, 6, 3, 7
-                const uint32_t x = c4 ^ 0x08080808u;
-                uint32_t w = (x & 0xFu) | ((x >> 12) & 0xF0u) | ((x << 8) & 0xF0000u) | ((x >> 4) & 0xF00000u);
-                w <<= 8 * (idx & 1);
-                w |= __shfl_xor_sync(0xffffffffu, w, 1);
-                if (idx >= KP4) continue;
-                uint8_t* blk = tiles + (k >> 6) * TB;
-                if ((idx & 1) == 0)  // word (k%32)/8 of run (k%64)/32
-                    *reinterpret_cast<uint32_t*>(blk + ((k >> 5) & 1) * 2048 + 16 * i_row + 4 * ((k >> 3) & 3)) = w;
-                if ((idx & (L - 1)) == 0) {  // first lane of the group: its scales
+                // eight nibbles (q + 8): the low nibble of each code byte with its top bit flipped is
+                // q + 8 (|q| <= 7, no carry between bytes); codes t = 0..3 go to nibbles 0, 4, 1, 5 and
+                // t = 4..7 to nibbles 2, 6, 3, 7
+                const uint32_t xa = ca ^ 0x08080808u, xb = cb ^ 0x08080808u;
+                const uint32_t wa = (xa & 0xFu) | ((xa >> 12) & 0xF0u) | ((xa << 8) & 0xF0000u) | ((xa >> 4) & 0xF00000u);
+                const uint32_t wb = (xb & 0xFu) | ((xb >> 12) & 0xF0u) | ((xb << 8) & 0xF0000u) | ((xb >> 4) & 0xF00000u);
+                const uint32_t w = wa | (wb << 8);
+                if (p8 >= KP8) continue;
+                uint8_t* blk = tiles + (k >> 6) * TB;  // word (k%32)/8 of run (k%64)/32
+                *reinterpret_cast<uint32_t*>(blk + ((k >> 5) & 1) * 2048 + 16 * i_row + 4 * ((k >> 3) & 3)) = w;
+                if ((p8 & (L8 - 1)) == 0) {  // first lane of the group: its scales
                     const int64_t gi = k / GS;
                     const bool real = row_ok && gi < G;
                     if (real) scales[n * G + gi] = gs.s;
