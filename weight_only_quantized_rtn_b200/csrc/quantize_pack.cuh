@@ -19,16 +19,17 @@ namespace wlq {
 
 // One CTA per padded output row (grid-stride over ceil(N/128)*128 rows).  The
 // row's ceil(K/64)*64 inputs (zeros past K and for rows >= N) are held in
-// registers: thread j takes the float4 pairs j + i*blockDim (i < V/2), so the
-// lanes of a warp hold consecutive 8-input runs and a group of g inputs is g/8
-// adjacent lanes.
+// registers: thread j takes runs of Q adjacent float4 at j + i*blockDim, so
+// the lanes of a warp hold consecutive runs (Q = 2 for int8, 4 for int4: the
+// faster of the two for each).
 //  - int8: the row's absmax is reduced over the CTA (magnitude bit patterns,
-//    as in quantize_rows_cta_kernel); each float4 becomes one 32-bit word of
-//    four offset-binary bytes at its place in the row's 16-byte run.
-//  - int4: a lane holds pairs of adjacent float4 (8 inputs, one 32-byte run
-//    per slot); each group's absmax is reduced over its lanes; the row's
+//    as in quantize_rows_cta_kernel); a lane's eight codes leave as one
+//    8-byte store of offset-binary bytes at its place in the row.
+//  - int4: a lane holds quads of adjacent float4 (16 inputs, one 64-byte run
+//    per slot), so a group of g inputs is g/16 adjacent lanes (one lane for
+//    gs16); each group's absmax is reduced over its lanes; the row's
 //    largest group scale (over the CTA) fixes the fp16 normalisation 2^e_n
-//    and the row factor 2^-e_n; a lane's eight codes make one 32-bit word.
+//    and the row factor 2^-e_n; a lane's sixteen codes make two 32-bit words.
 template <int FMT, int V>
 __global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
     const float* __restrict__ W, int64_t N, int64_t K, int KT, int64_t rows, int qmax,
@@ -37,6 +38,7 @@ __global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
     constexpr uint32_t TB = tile_bytes(FMT);
     constexpr int L = (FMT == FMT_W4G64) ? 16 : 4;  // int4: lanes per group (group / 4)
     constexpr int GS = 4 * L;                        // int4: group size
+    constexpr int Q = (FMT == FMT_W8) ? 2 : 4;       // float4 per run of a lane
     __shared__ uint32_t part[32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nwarps = blockDim.x >> 5;
@@ -52,9 +54,9 @@ __global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
         float4 v[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            // pairs of float4 (8 inputs, one 32-byte run) at pair p = threadIdx.x + (i / 2) * blockDim:
-            // a lane's eight int4 codes fill one word, its eight int8 codes one 8-byte store
-            const int idx = 2 * (threadIdx.x + (i >> 1) * blockDim.x) + (i & 1);
+            // runs of Q float4 at run p = threadIdx.x + (i / Q) * blockDim: int8 pairs (8 inputs, one
+            // 8-byte code store), int4 quads (16 inputs, two whole code words); measured best each
+            const int idx = Q * (threadIdx.x + (i / Q) * blockDim.x) + (i % Q);
             v[i] = (row_ok && idx < K4) ? __ldcs(row + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
         if constexpr (FMT == FMT_W8) {
@@ -93,30 +95,32 @@ __global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
             }
             __syncthreads();  // part[] is rewritten for the next row
         } else {
-            // each lane holds V / 2 slots of 8 adjacent inputs; a group is L8 = GS / 8 adjacent lanes.
-            // Group absmax (0 for a group holding a NaN or infinity) reduced over its lanes, and the
-            // row's largest group scale over the CTA (scales are non-negative floats: their bit
-            // patterns order them)
-            constexpr int V2 = V / 2;
-            constexpr int L8 = GS / 8;
-            uint32_t gm[V2];
+            // each lane holds V / 4 slots of 16 adjacent inputs; a group is L16 = GS / 16 adjacent lanes
+            // (one lane for gs16).  Group absmax (0 for a group holding a NaN or infinity) reduced over
+            // its lanes, and the row's largest group scale over the CTA (scales are non-negative
+            // floats: their bit patterns order them)
+            constexpr int V4 = V / 4;
+            constexpr int L16 = GS / 16;
+            uint32_t gm[V4];
 #pragma unroll
-            for (int i = 0; i < V2; ++i) {
-                const float4 a = v[2 * i], b = v[2 * i + 1];
-                uint32_t m = max(max(max(__float_as_uint(a.x) & 0x7FFFFFFFu, __float_as_uint(a.y) & 0x7FFFFFFFu),
-                                     max(__float_as_uint(a.z) & 0x7FFFFFFFu, __float_as_uint(a.w) & 0x7FFFFFFFu)),
-                                 max(max(__float_as_uint(b.x) & 0x7FFFFFFFu, __float_as_uint(b.y) & 0x7FFFFFFFu),
-                                     max(__float_as_uint(b.z) & 0x7FFFFFFFu, __float_as_uint(b.w) & 0x7FFFFFFFu)));
-                for (int off = L8 >> 1; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+            for (int i = 0; i < V4; ++i) {
+                uint32_t m = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float4 a = v[4 * i + j];
+                    m = max(m, max(max(__float_as_uint(a.x) & 0x7FFFFFFFu, __float_as_uint(a.y) & 0x7FFFFFFFu),
+                                   max(__float_as_uint(a.z) & 0x7FFFFFFFu, __float_as_uint(a.w) & 0x7FFFFFFFu)));
+                }
+                for (int off = L16 >> 1; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
                 const bool gbad = m >= 0x7F800000u;
                 bad |= gbad;
                 gm[i] = gbad ? 0u : m;
             }
-            // The warp holds V2 * GPW groups (GPW = 32 / L8 per slot).  Lane j takes groups j and
-            // j + 32: the IEEE division and the reciprocal once per group rather than once per lane
-            // of it; the results go back to each group's lanes by shuffle.
-            constexpr int GPW = 32 / L8;
-            constexpr int NGW = V2 * GPW;
+            // The warp holds V4 * GPW groups (GPW = 32 / L16 per slot).  Lane j takes groups j, j + 32,
+            // ...: the IEEE division and the reciprocal once per group rather than once per lane of
+            // it; the results go back to each group's lanes by shuffle.
+            constexpr int GPW = 32 / L16;
+            constexpr int NGW = V4 * GPW;
             constexpr int PER_LANE = (NGW + 31) / 32;
             float sj[PER_LANE], ij[PER_LANE];
             uint32_t smax = 0;
@@ -125,8 +129,8 @@ __global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
                 const int j = lane + 32 * t, ji = j / GPW, jg = j % GPW;
                 uint32_t mj = 0;
 #pragma unroll
-                for (int i = 0; i < V2; ++i) {
-                    const uint32_t mi = __shfl_sync(0xffffffffu, gm[i], jg * L8);
+                for (int i = 0; i < V4; ++i) {
+                    const uint32_t mi = __shfl_sync(0xffffffffu, gm[i], jg * L16);
                     if (ji == i) mj = mi;
                 }
                 const GroupScale gs = group_scale(__uint_as_float(mj), qmax);
@@ -148,40 +152,43 @@ __global__ void __launch_bounds__(1024) quantize_pack_rows_kernel(
             }
             if (threadIdx.x == 0) rowf[n] = rf;
             const int sh = (rf > 0.0f) ? -ilogbf(rf) : 0;  // s * 2^sh = s / rf exactly
-            const int KP8 = KP4 / 2;
+            const int KP16 = KP4 / 4;
 #pragma unroll
-            for (int i = 0; i < V2; ++i) {
-                const int p8 = threadIdx.x + i * blockDim.x;  // this lane's 8 inputs: k = 8 p8 ..
-                const int k = 8 * p8;
-                // this slot's group scale, from the lane that worked it out (group i * GPW + lane / L8:
+            for (int i = 0; i < V4; ++i) {
+                const int p16 = threadIdx.x + i * blockDim.x;  // this lane's 16 inputs: k = 16 p16 ..
+                const int k = 16 * p16;
+                // this slot's group scale, from the lane that worked it out (group i * GPW + lane / L16:
                 // the same lane slot t = i * GPW / 32 for every lane, since GPW divides 32)
                 const int src_t = (i * GPW) / 32;
-                const int src = (i * GPW) % 32 + lane / L8;
+                const int src = (i * GPW) % 32 + lane / L16;
                 GroupScale gs;
                 gs.s = __shfl_sync(0xffffffffu, sj[src_t], src);
                 gs.inv = __shfl_sync(0xffffffffu, ij[src_t], src);
                 gs.normal = gs.s >= 1.17549435e-38f;
-                uint32_t ca, cb;
+                uint32_t c[4];
                 if (gs.normal) {
-                    ca = rtn4_f32(v[2 * i], gs.s, gs.inv, 0.5f * gs.s);
-                    cb = rtn4_f32(v[2 * i + 1], gs.s, gs.inv, 0.5f * gs.s);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) c[j] = rtn4_f32(v[4 * i + j], gs.s, gs.inv, 0.5f * gs.s);
                 } else {  // rare: a subnormal (or zero) scale takes the fp64 path
                     bool unused = false;
                     gs.inv64 = (gs.s > 0.0f) ? 1.0 / static_cast<double>(gs.s) : 0.0;
-                    ca = pack_codes4(v[2 * i], gs, qmax, unused);
-                    cb = pack_codes4(v[2 * i + 1], gs, qmax, unused);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) c[j] = pack_codes4(v[4 * i + j], gs, qmax, unused);
                 }
-                // eight nibbles (q + 8): the low nibble of each code byte with its top bit flipped is
-                // q + 8 (|q| <= 7, no carry between bytes); codes t = 0..3 go to nibbles 0, 4, 1, 5 and
-                // t = 4..7 to nibbles 2, 6, 3, 7
-                const uint32_t xa = ca ^ 0x08080808u, xb = cb ^ 0x08080808u;
-                const uint32_t wa = (xa & 0xFu) | ((xa >> 12) & 0xF0u) | ((xa << 8) & 0xF0000u) | ((xa >> 4) & 0xF00000u);
-                const uint32_t wb = (xb & 0xFu) | ((xb >> 12) & 0xF0u) | ((xb << 8) & 0xF0000u) | ((xb >> 4) & 0xF00000u);
-                const uint32_t w = wa | (wb << 8);
-                if (p8 >= KP8) continue;
-                uint8_t* blk = tiles + (k >> 6) * TB;  // word (k%32)/8 of run (k%64)/32
-                *reinterpret_cast<uint32_t*>(blk + ((k >> 5) & 1) * 2048 + 16 * i_row + 4 * ((k >> 3) & 3)) = w;
-                if ((p8 & (L8 - 1)) == 0) {  // first lane of the group: its scales
+                // sixteen nibbles (q + 8): the low nibble of each code byte with its top bit flipped is
+                // q + 8 (|q| <= 7, no carry between bytes); in each word of eight, codes t = 0..3 go to
+                // nibbles 0, 4, 1, 5 and t = 4..7 to nibbles 2, 6, 3, 7
+                uint32_t wn[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t x = c[j] ^ 0x08080808u;
+                    wn[j] = (x & 0xFu) | ((x >> 12) & 0xF0u) | ((x << 8) & 0xF0000u) | ((x >> 4) & 0xF00000u);
+                }
+                if (p16 >= KP16) continue;
+                uint8_t* blk = tiles + (k >> 6) * TB;  // words (k%32)/8 and +1 of run (k%64)/32
+                *reinterpret_cast<uint2*>(blk + ((k >> 5) & 1) * 2048 + 16 * i_row + 4 * ((k >> 3) & 3)) =
+                    make_uint2(wn[0] | (wn[1] << 8), wn[2] | (wn[3] << 8));
+                if ((p16 & (L16 - 1)) == 0) {  // first lane of the group: its scales
                     const int64_t gi = k / GS;
                     const bool real = row_ok && gi < G;
                     if (real) scales[n * G + gi] = gs.s;
