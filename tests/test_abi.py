@@ -98,6 +98,10 @@ def test_workspace_sizes(lib):
     assert lib.wlq_linear_workspace(4096, 4096, 4096, 8, 0, 0) == 0
     # small M splits K across a cluster; partial sums stay in shared memory
     assert lib.wlq_linear_workspace(16, 4096, 4096, 8, 0, 0) == 0
+    # int4 at most 16 tokens: the few-token kernel reads the bf16 x itself
+    assert lib.wlq_linear_workspace(16, 4096, 4096, 4, 64, 0) == 0
+    assert lib.wlq_linear_workspace(16, 4096, 4096, 4, 16, 0) == 0
+    assert lib.wlq_linear_workspace(17, 4096, 4096, 4, 64, 0) >= 17 * 4096 * 2
     # int4 stages an fp16 copy of x (+ row scales)
     assert lib.wlq_linear_workspace(4096, 4096, 4096, 4, 64, 0) >= 4096 * 4096 * 2 + 4096 * 4
     # low rank adds T (hi/lo) and the transposed L2

@@ -69,6 +69,36 @@ def test_parity_few_tokens(bits, group, M, N, K):
     assert err <= TOL, err
 
 
+@pytest.mark.parametrize("bits,group", RECIPES)
+def test_few_tokens_per_token_magnitudes(bits, group):
+    """Direct-load kernel: each CTA rescales each token's x by its own power
+    of two before the fp16 MMAs.  Tokens of size 1e-30 and 1e30, an all-zero
+    token, tokens with one large entry among small ones, and ordinary tokens:
+    each row within 1e-2 of its own rms (the zero row exactly 0).  At most 16
+    tokens no workspace is needed."""
+    m = wlq()
+    M, N, K = 12, 384, 1536
+    assert m.workspace_bytes(M, N, K, bits, group) == 0
+    g = np.random.default_rng(31 + bits + group)
+    x = g.standard_normal((M, K)).astype(np.float32)
+    x[0] *= 1e-30
+    x[1] *= 1e30
+    x[2] = 0.0
+    x[3] *= 1e-4
+    x[3, 100] = 3e4
+    x[4] = 1e-3
+    x[4, 1500] = -2e5   # in the last K split of a cluster
+    x[5, ::2] *= 1e-20  # every other input tiny
+    W = wi.weight(5, 2, N, K)
+    _, yg, y_ref = linear_case(wi.bf16_bits(x), W, bits, group)
+    for i in range(M):
+        rms = float(np.sqrt(np.mean(y_ref[i] ** 2)))
+        if rms == 0.0:
+            assert np.all(yg[i] == 0.0), i
+        else:
+            assert np.max(np.abs(yg[i] - y_ref[i])) <= TOL * rms, (i, np.max(np.abs(yg[i] - y_ref[i])) / rms)
+
+
 @pytest.mark.parametrize("bits,group,M,N,K", [
     (8, 0, 3, 200, 200),      # one K split, three whole K blocks and 8 inputs
     (8, 0, 12, 700, 4040),    # 8-CTA clusters, the last split ends in a ragged block
@@ -238,9 +268,15 @@ def test_empty_and_errors():
         with pytest.raises(m.WlqError) as e:
             m.linear_into(y, x, packed, 64, 128, 8, 0, workspace=small)
         assert e.value.status == m.ERR_WORKSPACE
+    # int4 beyond 16 tokens prepares x in a workspace: none given is an error
+    c4, s4 = m.quantize(dev_f32(W), 4, 64)
+    p4 = m.pack(c4, s4, 4, 64)
+    x32 = dev_bf16(wi.activations(8, 4, 32, 128))
+    y32 = torch.empty((32, 64), dtype=torch.float32, device="cuda")
+    assert m.workspace_bytes(32, 64, 128, 4, 64) > 0
     with pytest.raises(m.WlqError) as e:
-        m.linear_into(y, x, packed, 64, 128, 4, 64)
-    assert e.value.status in (m.ERR_WORKSPACE, m.ERR_UNSUPPORTED, m.ERR_SHAPE)
+        m.linear_into(y32, x32, p4, 64, 128, 4, 64)
+    assert e.value.status == m.ERR_WORKSPACE
     m.check_status()
 
 

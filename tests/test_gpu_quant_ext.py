@@ -172,13 +172,14 @@ def test_quantize_ex_scale_midpoints_and_subnormal_scales(bits, scale_dtype):
     np.testing.assert_array_equal(cg.cpu().numpy(), co)
 
 
-@pytest.mark.parametrize("group", [8, 32, 64, 256])
+@pytest.mark.parametrize("group,N,K", [(8, 29, 1024), (16, 29, 1024), (32, 29, 1024), (64, 29, 1024),
+                                       (256, 29, 1024), (512, 29, 1024), (16, 7, 80), (128, 5, 384)])
 @pytest.mark.parametrize("bits,scale_dtype", [(8, 1), (4, 0), (5, 2)])
-def test_quantize_ex_bf16_power_of_two_groups_bit_exact(group, bits, scale_dtype):
-    """bf16 input with groups of 8..256 (8 inputs a lane, groups across 1..32
-    lanes) against the oracle."""
+def test_quantize_ex_bf16_power_of_two_groups_bit_exact(group, N, K, bits, scale_dtype):
+    """bf16 input with groups of 8..512 (8 or 16 inputs a lane, groups across
+    1..32 lanes, a last warp-round only partly filled) against the oracle."""
     m = wlq()
-    W = _edge_weights(group + bits + scale_dtype, 29, 1024)
+    W = _edge_weights(group + bits + scale_dtype, N, K)
     if scale_dtype == 1:
         W[2] = 0.001
     co, so = oracle.quantize_ex(_host_in(W, True), bits, group, scale_dtype)
@@ -190,8 +191,9 @@ def test_quantize_ex_bf16_power_of_two_groups_bit_exact(group, bits, scale_dtype
 
 
 def test_quantize_ex_bf16_nonfinite_group_and_unaligned_codes():
-    """A NaN zeroes its group and raises the flag; codes that are only 4-byte
-    aligned take the general path and give the same bytes."""
+    """A NaN zeroes its group and raises the flag; codes that are only 8-byte
+    aligned (8 inputs a lane) or 4-byte aligned (the general path) give the
+    same bytes."""
     m = wlq()
     m.check_status()
     W = (np.random.default_rng(5).standard_normal((16, 256)) * 0.3).astype(np.float32)
@@ -204,9 +206,10 @@ def test_quantize_ex_bf16_nonfinite_group_and_unaligned_codes():
     x = _dev(W, True)
     c, s = m.quantize_ex(x, 8, 64, 1)
     m.check_status()
-    buf = torch.empty(16 * 256 + 4, dtype=torch.int8, device="cuda")
-    c_mis = buf[4:4 + 16 * 256].view(16, 256)
-    s2 = torch.empty_like(s)
-    m.lib.wlq_quantize_ex(m._ptr(x), 1, 16, 256, 8, 64, 1, m._ptr(c_mis), m._ptr(s2), m._stream())
-    m.check_status()
-    assert torch.equal(c, c_mis) and torch.equal(s, s2)
+    buf = torch.empty(16 * 256 + 16, dtype=torch.int8, device="cuda")
+    for off in (4, 8):
+        c_mis = buf[off:off + 16 * 256].view(16, 256)
+        s2 = torch.empty_like(s)
+        m.lib.wlq_quantize_ex(m._ptr(x), 1, 16, 256, 8, 64, 1, m._ptr(c_mis), m._ptr(s2), m._stream())
+        m.check_status()
+        assert torch.equal(c, c_mis) and torch.equal(s, s2)

@@ -2,11 +2,12 @@
 // ("Joy-face_change_optimized" model card, files table: weight-only Linear;
 // "Nunchaku Lite", how it works: 4-bit weights, 16-bit activations).
 //
-//   y[m,n] = rowf[n] * xs[m] * sum_k xin[m,k] * w16[n,k]  +  b[n]
+//   y[m,n] = rowf[n] * sum_k x[m,k] * w16[n,k]  +  b[n]
 //
-// Same packed operand, row factors and x (bf16, or the fp16 x16 of the int4
-// formats) as the other engines.  Here streaming the packed weights from HBM
-// is the whole cost, so the kernel is built around that stream:
+// Same packed operand and row factors as the other engines; x is the bf16
+// input itself for every format (no preparation pass).  Here streaming the
+// packed weights from HBM is the whole cost, so the kernel is built around
+// that stream:
 //
 //  - a cluster of S CTAs takes one 128-channel tile of the packed operand, CTA
 //    (cluster rank) q its K split q of kbps 64-wide blocks; clusters are
@@ -21,9 +22,16 @@
 //    ldmatrix (8 rows x 16 bytes per matrix: conflict-free), are dequantised
 //    in registers and feed m16n8k16 warp MMAs (fp32 accumulate) against x
 //    fragments read from shared memory once per block;
-//  - the CTA's x rows ([M][its K range]) are copied to shared memory once, by
-//    16-byte asynchronous copies from the compute threads; token rows >= M
-//    are never read back into an output;
+//  - the CTA's x rows ([M][its K range]) are copied to shared memory once,
+//    warp m row m, by 16-byte asynchronous copies; token rows >= M are never
+//    read back into an output.  The warp then rewrites its row in place as
+//    fp16 of x times 2^e_m, e_m chosen from the largest |x| of the token over
+//    the CTA's K range so that it lands in [2^14, 2^15): bf16 values keep all
+//    8 significand bits (only those below 2^-32 of the largest can round),
+//    and the partials are multiplied back by 2^-e_m (exact) before they are
+//    summed.  The MMAs are fp16: int8 codes become fp16 in two instructions a
+//    pair (0x64 above the offset-binary byte is 1024 + c + 128, less 1152),
+//    int4 codes times their group scale as in the other engines;
 //  - the warps' partial sums are staged in shared memory and added in K-part
 //    order; each thread then sends four adjacent rows of one token of the sum
 //    to the CTA that owns them (rows [q' 128/S, (q'+1) 128/S) belong to CTA
@@ -92,6 +100,41 @@ __device__ __forceinline__ void ldmatrix_x2(uint32_t addr, uint32_t (&d)[2]) {
                  : "=r"(d[0]), "=r"(d[1]) : "r"(addr) : "memory");
 }
 
+// two int8 codes (offset-binary bytes b0, b1 of w picked by sel) -> fp16x2
+// of the signed codes: 0x64 above each byte is the fp16 1024 + byte, less 1152
+__device__ __forceinline__ uint32_t bytes_to_f16x2(uint32_t w, uint32_t sel) {
+    uint32_t v;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(v) : "r"(w), "r"(0x64646464u), "r"(sel));
+    return h2u(__hsub2(u2h(v), u2h(0x64806480u)));
+}
+
+// one landed 64-input int8 block, this warp's rows and K step: ldmatrix of
+// the codes, fp16 x fragments of NB token groups (xrow: this lane's place in
+// x row g), 2 RB x NB warp MMAs
+template <int NB>
+__device__ __forceinline__ void gv_w8_block(const uint8_t* blk, uint32_t lm_off, const uint8_t* xrow, int g,
+                                            uint32_t pitch, float (&acc)[2][NB][4], uint32_t& held) {
+    uint32_t d[4];
+    ldmatrix_x4(smem_u32(blk) + lm_off, d);
+    held ^= d[0] ^ d[1] ^ d[2] ^ d[3];
+    uint32_t b[NB][2];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+        const uint2 u = *reinterpret_cast<const uint2*>(xrow + (nb * 8 + g) * pitch);
+        b[nb][0] = u.x;
+        b[nb][1] = u.y;
+    }
+#pragma unroll
+    for (int bk = 0; bk < 2; ++bk) {
+        const uint32_t lo0 = bytes_to_f16x2(d[2 * bk], 0x4140u);
+        const uint32_t hi0 = bytes_to_f16x2(d[2 * bk], 0x4342u);
+        const uint32_t lo1 = bytes_to_f16x2(d[2 * bk + 1], 0x4140u);
+        const uint32_t hi1 = bytes_to_f16x2(d[2 * bk + 1], 0x4342u);
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) mma16816_f16(acc[bk][nb], lo0, lo1, hi0, hi1, b[nb][0], b[nb][1]);
+    }
+}
+
 template <int FMT, int NB>
 __global__ void __launch_bounds__(GV_THREADS, 1) gemv_kernel(const GemmArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -99,7 +142,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1) gemv_kernel(const GemmArgs a) {
     uint8_t* base = smem_raw + (((raw + 127u) & ~127u) - raw);
     uint64_t* full = reinterpret_cast<uint64_t*>(base);            // [GV_MAX_STAGES]
     uint64_t* empty = full + GV_MAX_STAGES;                          // [GV_MAX_STAGES]
-    float* xs_sm = reinterpret_cast<float*>(base + 256);            // [16]
+    float* xinv_sm = reinterpret_cast<float*>(base + 192);          // [16] 2^-e_m
     uint8_t* xsm = base + 256 + 64;                                  // [NB*8][pitch]
     const uint32_t pitch = gv_x_pitch(a.kbps, FMT);
     constexpr int P = gv_parts(FMT);
@@ -136,17 +179,47 @@ __global__ void __launch_bounds__(GV_THREADS, 1) gemv_kernel(const GemmArgs a) {
         const uint32_t chunks = static_cast<uint32_t>(nkb) * 8u;  // 16-byte chunks per row
         const int kin = min(a.K, kb1 * 64) - kb0 * 64;            // real inputs of the range
         const uint8_t* xg = static_cast<const uint8_t*>(a.xg);
-        for (uint32_t i = threadIdx.x; i < static_cast<uint32_t>(Mv) * chunks; i += GV_WARPS * 32) {
-            const uint32_t m = i / chunks, c = i % chunks;
-            uint8_t* dst = xsm + m * pitch + c * 16u;
-            if (static_cast<int>(c) * 8 < kin)
-                cp_async_16(smem_u32(dst), xg + (static_cast<size_t>(m) * a.K + kb0 * 64) * 2 + c * 16u);
-            else
-                *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+        // warp m takes token row m: copies it, finds its largest |x|
+        // (bf16 magnitudes order as integers) and rewrites it in place as
+        // fp16 of x * 2^e_m, e_m = 141 - E for the bf16 exponent field E
+        // of that largest |x| (at most 126, so 2^-e_m is a normal float
+        // too; a non-finite x keeps e_m = 0 and carries through)
+        const int m = warp;
+        if (m < Mv) {
+            uint8_t* row = xsm + m * pitch;
+            const uint8_t* src = xg + (static_cast<size_t>(m) * a.K + kb0 * 64) * 2;
+            for (uint32_t c = lane; c < chunks; c += 32) {
+                if (static_cast<int>(c) * 8 < kin) cp_async_16(smem_u32(row + c * 16u), src + c * 16u);
+                else *reinterpret_cast<uint4*>(row + c * 16u) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            cp_async_wait_all();
+            __syncwarp();
+            uint32_t mx = 0;
+            for (uint32_t c = lane; c < chunks; c += 32) {
+                const uint4 v = *reinterpret_cast<const uint4*>(row + c * 16u);
+                mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                                           __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu)));
+            }
+            mx = max(mx & 0xFFFFu, mx >> 16);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            const int E = static_cast<int>(mx >> 7);
+            const int e = (E >= 255) ? 0 : min(126, 141 - E);
+            const float sc = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+            for (uint32_t c = lane; c < chunks; c += 32) {
+                uint4* p = reinterpret_cast<uint4*>(row + c * 16u);
+                const uint4 v = *p;
+                uint4 h;
+                h.x = h2u(__floats2half2_rn(__uint_as_float(v.x << 16) * sc, __uint_as_float(v.x & 0xFFFF0000u) * sc));
+                h.y = h2u(__floats2half2_rn(__uint_as_float(v.y << 16) * sc, __uint_as_float(v.y & 0xFFFF0000u) * sc));
+                h.z = h2u(__floats2half2_rn(__uint_as_float(v.z << 16) * sc, __uint_as_float(v.z & 0xFFFF0000u) * sc));
+                h.w = h2u(__floats2half2_rn(__uint_as_float(v.w << 16) * sc, __uint_as_float(v.w & 0xFFFF0000u) * sc));
+                *p = h;
+            }
+            if (lane == 0) xinv_sm[m] = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+        } else if (m < NB * 8 && lane == 0) {
+            xinv_sm[m] = 1.0f;
         }
-        if (threadIdx.x < NB * 8)
-            xs_sm[threadIdx.x] = (FMT != FMT_W8 && static_cast<int>(threadIdx.x) < a.M) ? a.xs[threadIdx.x] : 1.0f;
-        cp_async_wait_all();
         named_sync(1, GV_WARPS * 32);  // x in shared memory for every compute warp
     }
 
@@ -200,31 +273,23 @@ __global__ void __launch_bounds__(GV_THREADS, 1) gemv_kernel(const GemmArgs a) {
                 const uint8_t* slot = ring + st * SLOT;
                 const int nk = min(GV_SLOT_KB, nkb - i * GV_SLOT_KB);
                 uint32_t held = 0;
-                for (int j = 0; j < nk; ++j) {
-                    const uint8_t* blk = slot + j * TB;
-                    const int kx = (i * GV_SLOT_KB + j) * 128;  // byte offset of the block in an x row
-                    if constexpr (FMT == FMT_W8) {
-                        uint32_t d[4];
-                        ldmatrix_x4(smem_u32(blk) + lm_off, d);
-                        held ^= d[0] ^ d[1] ^ d[2] ^ d[3];
-                        uint32_t b[NB][2];
+                if constexpr (FMT == FMT_W8) {
+                    // a full slot: its four blocks unrolled, so the four
+                    // ldmatrix and x reads are in flight together
+                    if (nk == GV_SLOT_KB) {
 #pragma unroll
-                        for (int nb = 0; nb < NB; ++nb) {
-                            const uint2 u = *reinterpret_cast<const uint2*>(xsm + (nb * 8 + g) * pitch + kx + 32 * ks + 8 * t);
-                            b[nb][0] = u.x;
-                            b[nb][1] = u.y;
-                        }
-#pragma unroll
-                        for (int bk = 0; bk < RB; ++bk) {
-                            const uint32_t lo0 = bytes_to_bf16x2(d[2 * bk], 0x7440u, 0x7441u);
-                            const uint32_t hi0 = bytes_to_bf16x2(d[2 * bk], 0x7442u, 0x7443u);
-                            const uint32_t lo1 = bytes_to_bf16x2(d[2 * bk + 1], 0x7440u, 0x7441u);
-                            const uint32_t hi1 = bytes_to_bf16x2(d[2 * bk + 1], 0x7442u, 0x7443u);
-#pragma unroll
-                            for (int nb = 0; nb < NB; ++nb)
-                                mma16816_bf16(acc[bk][nb], lo0, lo1, hi0, hi1, b[nb][0], b[nb][1]);
-                        }
+                        for (int j = 0; j < GV_SLOT_KB; ++j)
+                            gv_w8_block<NB>(slot + j * TB, lm_off, xsm + (i * GV_SLOT_KB + j) * 128 + 32 * ks + 8 * t, g,
+                                            pitch, acc, held);
                     } else {
+                        for (int j = 0; j < nk; ++j)
+                            gv_w8_block<NB>(slot + j * TB, lm_off, xsm + (i * GV_SLOT_KB + j) * 128 + 32 * ks + 8 * t, g,
+                                            pitch, acc, held);
+                    }
+                } else {
+                    for (int j = 0; j < nk; ++j) {
+                        const uint8_t* blk = slot + j * TB;
+                        const int kx = (i * GV_SLOT_KB + j) * 128;  // byte offset of the block in an x row
                         uint32_t d[2];
                         ldmatrix_x2(smem_u32(blk) + lm_off, d);
                         uint16_t h0, h1;
@@ -253,7 +318,12 @@ __global__ void __launch_bounds__(GV_THREADS, 1) gemv_kernel(const GemmArgs a) {
                 if (lane == 0) mbar_arrive(&empty[st]);
             }
 
-            // stage this warp's partial: stage[ks][m][row]
+            // stage this warp's partial: stage[ks][m][row], times 2^-e_m
+            float xi[NB][2];
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) xi[nb][e] = xinv_sm[nb * 8 + 2 * t + e];
 #pragma unroll
             for (int bk = 0; bk < RB; ++bk)
 #pragma unroll
@@ -263,7 +333,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1) gemv_kernel(const GemmArgs a) {
 #pragma unroll
                         for (int e = 0; e < 2; ++e)
                             stage[(ks * NB * 8 + nb * 8 + 2 * t + e) * 128 + row_g + 16 * bk + 8 * h] =
-                                acc[bk][nb][2 * h + e];
+                                acc[bk][nb][2 * h + e] * xi[nb][e];
             named_sync(2, GV_WARPS * 32);
             // sum the P parts of four adjacent rows of one token, in part order,
             // and send them to the owner of the rows: slot q of its buffer
@@ -294,7 +364,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1) gemv_kernel(const GemmArgs a) {
             for (int m = static_cast<int>(threadIdx.x) / rows_per; m < Mv; m += GV_WARPS * 32 / rows_per) {
                 float v = red[m * rows_per + rl];
                 for (int sp = 1; sp < S; ++sp) v += red[(sp * NB * 8 + m) * rows_per + rl];
-                if (n_out < a.N) store_y(a, m, n_out, v * rf * xs_sm[m] + bias);
+                if (n_out < a.N) store_y(a, m, n_out, v * rf + bias);
             }
         }
         // the buffers are rewritten by the next tile: every CTA of the cluster

@@ -283,42 +283,49 @@ __global__ void __launch_bounds__(256) quantize_ex_short_kernel(const void* __re
     if (bad) raise_error(ERRBIT_NONFINITE);
 }
 
-// bf16 input, groups of G = 8 * LG inputs (LG a power of two, at most 32):
-// a lane takes 8 adjacent inputs (one 16-byte load) a round, so a warp covers
-// 256 inputs (256 / G groups) a round, four rounds in flight; when the warp's
-// groups fit one per lane, each scale is worked out once, by one lane.  The group's
+// bf16 input, groups of G = E * LG inputs (LG a power of two, at most 32):
+// a lane takes E = 8 or 16 adjacent inputs (one or two 16-byte loads) a
+// round, so a warp covers 32 E inputs a round, with four loads a lane in
+// flight; when the warp's groups fit one per lane, each scale is worked out
+// once, by one lane.  The group's
 // absmax is the maximum of the bf16 magnitude bits (two at a time, 16-bit
 // lanes), reduced over its LG lanes; the stored scale and the exactly rounded
 // codes are those of quantize_ex_short_kernel (same stored_scale, same
 // rtn4_f32 / rtn4_f32_clamped), so the results are bit-identical.  Codes go
-// out as one 8-byte store per lane (codes 8-byte aligned).
-template <int SF, int LG>
-__global__ void __launch_bounds__(256) quantize_ex_bf16_kernel(const uint16_t* __restrict__ W, int64_t total8,
+// out as one E-byte store per lane (codes E-byte aligned).
+template <int SF, int LG, int E>
+__global__ void __launch_bounds__(256) quantize_ex_bf16_kernel(const uint16_t* __restrict__ W, int64_t totalE,
                                                                int qmax, int8_t* __restrict__ codes,
                                                                void* __restrict__ scales) {
     grid_dependency_sync();
-    constexpr int U = 4;            // rounds in flight
-    constexpr int GPR = 32 / LG;    // groups per warp-round
-    constexpr int NGW = U * GPR;    // groups the warp holds
+    constexpr int NQ = E / 8;          // 16-byte loads a lane per round
+    constexpr int U = 4 / NQ;          // rounds in flight (four 16-byte loads a lane)
+    constexpr int GPR = 32 / LG;       // groups per warp-round
+    constexpr int NGW = U * GPR;       // groups the warp holds
     const int lane = threadIdx.x & 31;
     const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     const uint4* W8 = reinterpret_cast<const uint4*>(W);
-    uint2* out = reinterpret_cast<uint2*>(codes);
     bool bad = false;
-    for (int64_t r0 = w0 * U; r0 * 32 < total8; r0 += nw * U) {
-        uint4 raw[U];
+    for (int64_t r0 = w0 * U; r0 * 32 < totalE; r0 += nw * U) {
+        uint4 raw[U][NQ];
         uint32_t m[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t i8 = (r0 + u) * 32 + lane;
-            raw[u] = i8 < total8 ? __ldcs(W8 + i8) : make_uint4(0u, 0u, 0u, 0u);
+            const int64_t ie = (r0 + u) * 32 + lane;
+#pragma unroll
+            for (int q = 0; q < NQ; ++q)
+                raw[u][q] = ie < totalE ? __ldcs(W8 + ie * NQ + q) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const uint4 r = raw[u];
-            const uint32_t m2 = __vmaxu2(__vmaxu2(r.x & 0x7FFF7FFFu, r.y & 0x7FFF7FFFu),
-                                         __vmaxu2(r.z & 0x7FFF7FFFu, r.w & 0x7FFF7FFFu));
+            uint32_t m2 = 0;
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+                const uint4 r = raw[u][q];
+                m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(r.x & 0x7FFF7FFFu, r.y & 0x7FFF7FFFu),
+                                           __vmaxu2(r.z & 0x7FFF7FFFu, r.w & 0x7FFF7FFFu)));
+            }
             m[u] = max(m2 & 0xFFFFu, m2 >> 16);
 #pragma unroll
             for (int off = LG >> 1; off > 0; off >>= 1) m[u] = max(m[u], __shfl_xor_sync(0xffffffffu, m[u], off));
@@ -366,41 +373,46 @@ __global__ void __launch_bounds__(256) quantize_ex_bf16_kernel(const uint16_t* _
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t i8 = (r0 + u) * 32 + lane;
-            if (i8 >= total8) continue;
-            const uint4 r = raw[u];
+            const int64_t ie = (r0 + u) * 32 + lane;
+            if (ie >= totalE) continue;
             const float sg = su[u];
             bad |= bu[u];
             if ((lane & (LG - 1)) == 0) {
-                const int64_t gi = i8 / LG;
+                const int64_t gi = ie / LG;
                 if constexpr (SF == SCALE_F32) static_cast<float*>(scales)[gi] = sg;
                 else if constexpr (SF == SCALE_F16) static_cast<__half*>(scales)[gi] = __float2half_rn(sg);
                 else static_cast<__nv_bfloat16*>(scales)[gi] = __float2bfloat16_rn(sg);
             }
-            const float4 lo = make_float4(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xFFFF0000u),
-                                          __uint_as_float(r.y << 16), __uint_as_float(r.y & 0xFFFF0000u));
-            const float4 hi = make_float4(__uint_as_float(r.z << 16), __uint_as_float(r.z & 0xFFFF0000u),
-                                          __uint_as_float(r.w << 16), __uint_as_float(r.w & 0xFFFF0000u));
-            uint32_t c0 = 0, c1 = 0;
-            if (sg >= 1.17549435e-38f) {
-                if constexpr (SF == SCALE_F32) {
-                    c0 = rtn4_f32(lo, sg, iu[u], 0.5f * sg);
-                    c1 = rtn4_f32(hi, sg, iu[u], 0.5f * sg);
-                } else {
-                    c0 = rtn4_f32_clamped(lo, sg, iu[u], 0.5f * sg, static_cast<float>(qmax));
-                    c1 = rtn4_f32_clamped(hi, sg, iu[u], 0.5f * sg, static_cast<float>(qmax));
+            uint32_t c[2 * NQ];
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+                const uint4 r = raw[u][q];
+                const float4 lo = make_float4(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xFFFF0000u),
+                                              __uint_as_float(r.y << 16), __uint_as_float(r.y & 0xFFFF0000u));
+                const float4 hi = make_float4(__uint_as_float(r.z << 16), __uint_as_float(r.z & 0xFFFF0000u),
+                                              __uint_as_float(r.w << 16), __uint_as_float(r.w & 0xFFFF0000u));
+                c[2 * q] = c[2 * q + 1] = 0;
+                if (sg >= 1.17549435e-38f) {
+                    if constexpr (SF == SCALE_F32) {
+                        c[2 * q] = rtn4_f32(lo, sg, iu[u], 0.5f * sg);
+                        c[2 * q + 1] = rtn4_f32(hi, sg, iu[u], 0.5f * sg);
+                    } else {
+                        c[2 * q] = rtn4_f32_clamped(lo, sg, iu[u], 0.5f * sg, static_cast<float>(qmax));
+                        c[2 * q + 1] = rtn4_f32_clamped(hi, sg, iu[u], 0.5f * sg, static_cast<float>(qmax));
+                    }
+                } else if (sg > 0.0f) {
+                    GroupScale gs;
+                    gs.s = sg;
+                    gs.normal = false;
+                    gs.inv = 0.0f;
+                    gs.inv64 = 1.0 / static_cast<double>(sg);
+                    bool unused = false;
+                    c[2 * q] = pack_codes4(lo, gs, qmax, unused);
+                    c[2 * q + 1] = pack_codes4(hi, gs, qmax, unused);
                 }
-            } else if (sg > 0.0f) {
-                GroupScale gs;
-                gs.s = sg;
-                gs.normal = false;
-                gs.inv = 0.0f;
-                gs.inv64 = 1.0 / static_cast<double>(sg);
-                bool unused = false;
-                c0 = pack_codes4(lo, gs, qmax, unused);
-                c1 = pack_codes4(hi, gs, qmax, unused);
             }
-            out[i8] = make_uint2(c0, c1);
+            if constexpr (NQ == 1) reinterpret_cast<uint2*>(codes)[ie] = make_uint2(c[0], c[1]);
+            else reinterpret_cast<uint4*>(codes)[ie] = make_uint4(c[0], c[1], c[2], c[3]);
         }
     }
     if (bad) raise_error(ERRBIT_NONFINITE);

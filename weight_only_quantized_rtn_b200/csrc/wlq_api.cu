@@ -266,12 +266,7 @@ bool make_plan(Plan& p, int64_t M, int64_t N, int64_t K, int fmt, int r, int sms
             p.smem = wlq::gv_smem_bytes(fmt, nb, p.kbps, st);
             p.tiles_nm = p.NT;
             p.grid = static_cast<int>(std::min<int64_t>(p.NT, std::max(1, cap / gs))) * gs;  // persistent over tiles
-            size_t off = 0;
-            if (fmt != wlq::FMT_W8) {
-                p.off_x16 = off; off = align256(off + static_cast<size_t>(M) * K * 2);
-                p.off_xs = off;  off = align256(off + static_cast<size_t>(M) * 4);
-            }
-            p.ws = off;
+            p.ws = 0;  // the kernel reads the bf16 x itself, every format
             return true;
         }
     }
@@ -865,26 +860,38 @@ wlq_status wlq_quantize_ex(const void* W, int w_dtype, int64_t N, int64_t K, int
     const int g4 = static_cast<int>(g / 4);
     const int qmax = (1 << (bits - 1)) - 1;
     const bool bf = (w_dtype == WLQ_IN_BF16);
-    const int LG = static_cast<int>(g / 8);  // bf16: lanes per group at 8 inputs a lane
-    if (bf && g % 8 == 0 && g <= 256 && (LG & (LG - 1)) == 0 && (reinterpret_cast<uintptr_t>(codes) & 7u) == 0) {
-        // bf16 with power-of-two groups of 8..256: 8 inputs a lane, four rounds in flight, persistent
-        const int64_t total8 = N * K / 8;
-        const int64_t rounds = cdiv(total8, 32);
-        const int grid = static_cast<int>(std::min<int64_t>(cdiv(cdiv(rounds, 4), 8), static_cast<int64_t>(d->sms) * 8));
+    // bf16 with power-of-two groups of 8..512: E = 16 inputs a lane (codes 16-byte aligned, groups of
+    // at least 16), else 8; four 16-byte loads a lane in flight, persistent
+    const bool pow2 = g >= 8 && (g & (g - 1)) == 0;
+    const int E = (pow2 && g >= 16 && g <= 512 && (reinterpret_cast<uintptr_t>(codes) & 15u) == 0) ? 16
+                  : (pow2 && g <= 256 && (reinterpret_cast<uintptr_t>(codes) & 7u) == 0)          ? 8
+                                                                                                  : 0;
+    if (bf && E) {
+        const int LG = static_cast<int>(g / E);
+        const int64_t totalE = N * K / E;
+        const int64_t rounds = cdiv(totalE, 32);
+        const int U = 4 / (E / 8);
+        const int grid = static_cast<int>(std::min<int64_t>(cdiv(cdiv(rounds, U), 8), static_cast<int64_t>(d->sms) * 8));
         const uint16_t* Wb = static_cast<const uint16_t*>(W);
-#define WLQ_QB(F, L) launch_k(wlq::quantize_ex_bf16_kernel<F, L>, grid, 256, 0, s, Wb, total8, qmax, codes, scales)
-#define WLQ_QBL(F)                 \
-    switch (LG) {                  \
-        case 1: WLQ_QB(F, 1); break;   \
-        case 2: WLQ_QB(F, 2); break;   \
-        case 4: WLQ_QB(F, 4); break;   \
-        case 8: WLQ_QB(F, 8); break;   \
-        case 16: WLQ_QB(F, 16); break; \
-        default: WLQ_QB(F, 32); break; \
+#define WLQ_QB(F, L, EE) launch_k(wlq::quantize_ex_bf16_kernel<F, L, EE>, grid, 256, 0, s, Wb, totalE, qmax, codes, scales)
+#define WLQ_QBL(F, EE)                 \
+    switch (LG) {                      \
+        case 1: WLQ_QB(F, 1, EE); break;   \
+        case 2: WLQ_QB(F, 2, EE); break;   \
+        case 4: WLQ_QB(F, 4, EE); break;   \
+        case 8: WLQ_QB(F, 8, EE); break;   \
+        case 16: WLQ_QB(F, 16, EE); break; \
+        default: WLQ_QB(F, 32, EE); break; \
     }
-        if (scale_dtype == WLQ_SCALE_F32) { WLQ_QBL(wlq::SCALE_F32) }
-        else if (scale_dtype == WLQ_SCALE_F16) { WLQ_QBL(wlq::SCALE_F16) }
-        else { WLQ_QBL(wlq::SCALE_BF16) }
+        if (E == 16) {
+            if (scale_dtype == WLQ_SCALE_F32) { WLQ_QBL(wlq::SCALE_F32, 16) }
+            else if (scale_dtype == WLQ_SCALE_F16) { WLQ_QBL(wlq::SCALE_F16, 16) }
+            else { WLQ_QBL(wlq::SCALE_BF16, 16) }
+        } else {
+            if (scale_dtype == WLQ_SCALE_F32) { WLQ_QBL(wlq::SCALE_F32, 8) }
+            else if (scale_dtype == WLQ_SCALE_F16) { WLQ_QBL(wlq::SCALE_F16, 8) }
+            else { WLQ_QBL(wlq::SCALE_BF16, 8) }
+        }
 #undef WLQ_QBL
 #undef WLQ_QB
     } else if (g4 <= 32 && 32 % g4 == 0) {
@@ -1112,7 +1119,7 @@ wlq_status wlq_linear(const void* x, int64_t M, const void* packed, int64_t N, i
     // --- operand preparation
     const void* xin = x;
     float* xs = nullptr;
-    if (fmt != wlq::FMT_W8) {
+    if (fmt != wlq::FMT_W8 && !p.gemv) {
         __half* x16 = reinterpret_cast<__half*>(ws + p.off_x16);
         xs = reinterpret_cast<float*>(ws + p.off_xs);
         if ((st = launch_prep_x16(static_cast<const uint16_t*>(x), p.M, p.K, x16, xs, d, s)) != WLQ_OK) return st;
