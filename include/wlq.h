@@ -193,7 +193,8 @@ wlq_status wlq_unpack(const void* packed, int64_t N, int64_t K, int bits, int gr
 
 /*
  * Workspace bytes wlq_linear needs for this shape (host-only; 0 when it
- * needs none: int8 weights without the low-rank branch).  No passage of the
+ * needs none: without the low-rank branch, int8 weights at any M and int4
+ * weights at M <= 16, where the few-token kernel reads x itself).  No passage of the
  * pages defines it: a sizing helper for the caller-owned scratch.  The contents need
  * no initialisation.  A workspace must not be shared by calls that may run
  * concurrently.

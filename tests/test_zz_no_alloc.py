@@ -24,7 +24,7 @@ pytestmark = pytest.mark.gpu
 
 CASES = [
     # bits, group, M, N, K, r     (what the scratch holds)
-    (4, 64, 16, 1024, 2048, 0),   # few-token kernel: fp16 copy of x + row scales
+    (4, 64, 24, 1024, 2048, 0),   # 17-32 tokens, warp-MMA kernel: fp16 copy of x + row scales
     (4, 64, 300, 640, 1024, 0),   # tensor-core kernel: fp16 copy of x + row scales
     (4, 16, 40, 384, 512, 32),    # fp16 x, low-rank T (hi/lo) and L2^T, K split over a cluster
     (8, 0, 200, 256, 320, 16),    # low rank with int8 weights: T and L2^T only
