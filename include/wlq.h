@@ -193,8 +193,10 @@ wlq_status wlq_unpack(const void* packed, int64_t N, int64_t K, int bits, int gr
 
 /*
  * Workspace bytes wlq_linear needs for this shape (host-only; 0 when it
- * needs none: without the low-rank branch, int8 weights at any M and int4
- * weights at M <= 16, where the few-token kernel reads x itself).  No passage of the
+ * needs none: without the low-rank branch, int8 weights at any M, and int4
+ * weights at M <= 16 where the few-token kernel, which reads x itself, holds
+ * its x rows in shared memory -- K up to about 40,000 at 9..16 tokens and
+ * 88,000 at 1..8).  No passage of the
  * pages defines it: a sizing helper for the caller-owned scratch.  The contents need
  * no initialisation.  A workspace must not be shared by calls that may run
  * concurrently.

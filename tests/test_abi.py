@@ -102,6 +102,13 @@ def test_workspace_sizes(lib):
     assert lib.wlq_linear_workspace(16, 4096, 4096, 4, 64, 0) == 0
     assert lib.wlq_linear_workspace(16, 4096, 4096, 4, 16, 0) == 0
     assert lib.wlq_linear_workspace(17, 4096, 4096, 4, 64, 0) >= 17 * 4096 * 2
+    # ... while its x rows fit in shared memory; beyond that the warp-MMA
+    # kernel takes the shape and needs the fp16 copy of x again
+    assert lib.wlq_linear_workspace(16, 4096, 40960, 4, 16, 0) == 0
+    assert lib.wlq_linear_workspace(16, 4096, 65536, 4, 64, 0) >= 16 * 65536 * 2
+    # int8 without low rank: none at any M and K
+    for M, K in ((1, 131072), (16, 65536), (300, 4096)):
+        assert lib.wlq_linear_workspace(M, 4096, K, 8, 0, 0) == 0
     # int4 stages an fp16 copy of x (+ row scales)
     assert lib.wlq_linear_workspace(4096, 4096, 4096, 4, 64, 0) >= 4096 * 4096 * 2 + 4096 * 4
     # low rank adds T (hi/lo) and the transposed L2
