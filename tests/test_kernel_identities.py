@@ -10,6 +10,13 @@ parity tests check the kernels that use them against the oracle.
 - int8 codes to fp16 (few-token kernel): the byte permute that puts 0x64
   above an offset-binary byte q + 128 reads as the fp16 1024 + q + 128, and
   one fp16 subtraction of 1152 leaves q exactly.
+- int8 codes to bf16 (tensor-core GEMM): a byte under 0x4B (as fp32, 2^23 +
+  the byte), one packed fp32 subtraction of 2^23 + 128 and a permute of the
+  two upper halves give bf16 q exactly.
+- int4 codes to fp16 (every int4 engine): a nibble OR-ed into 0x6400 reads
+  as 1024 + n (low nibble of a half) or 1024 + 16 n (high nibble); less 1032,
+  or times 1/16 less 72, leaves n - 8 exactly; with the packed nibble order
+  the four results of a word are the consecutive code pairs (0,1) .. (6,7).
 - x to fp16 (few-token kernel): a bf16 row whose largest magnitude has
   exponent field E is scaled by 2^e, e = min(126, 141 - E) (e = 0 for a
   non-finite maximum): nothing overflows fp16, the largest lands in
@@ -137,3 +144,56 @@ def test_x_rescale_to_fp16_exhaustive_over_bf16():
     for e in es:
         inv = np.float32(2.0 ** -e)
         assert np.isfinite(inv) and inv >= np.finfo(np.float32).tiny and float(inv) * 2.0 ** e == 1.0
+
+
+def _f32(u):
+    return np.array([u], dtype=np.uint32).view(np.float32)[0]
+
+
+def test_int8_codes_to_bf16_by_magic_float():
+    magic = np.float32(2.0 ** 23 + 128)
+    assert _f32(0x4B000080) == magic
+    g = np.random.default_rng(3)
+    words = [int(v) for v in g.integers(0, 2 ** 32, 3000, dtype=np.uint64)]
+    words += [int(np.array([b, b ^ 0xFF, (b + 1) & 0xFF, (b * 7) & 0xFF], dtype=np.uint8).view(np.uint32)[0])
+              for b in range(256)]
+    for w in words:
+        q = [((w >> (8 * k)) & 0xFF) - 128 for k in range(4)]       # offset-binary bytes
+        for sel_lo, sel_hi, pair in ((0x7440, 0x7441, q[0:2]), (0x7442, 0x7443, q[2:4])):
+            a = _f32(_prmt(w, 0x4B000000, sel_lo)) - magic           # fp32 arithmetic
+            b = _f32(_prmt(w, 0x4B000000, sel_hi)) - magic
+            lo = int(np.array([a], dtype=np.float32).view(np.uint32)[0])
+            hi = int(np.array([b], dtype=np.float32).view(np.uint32)[0])
+            out = _prmt(lo, hi, 0x7632)                              # the two upper halves
+            bf = (np.array([out & 0xFFFF, out >> 16], dtype=np.uint32) << np.uint32(16)).view(np.float32)
+            np.testing.assert_array_equal(bf.astype(np.float64), np.array(pair, dtype=np.float64))
+
+
+def _f16x2(u32):
+    return np.array([u32 & 0xFFFF, u32 >> 16], dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def _nibbles_to_pairs(w):
+    """The int4 dequantise of one packed word, unit group scale: four fp16
+    pairs, each rounded once as the fp16 subtract / fused multiply-add does."""
+    def f16(x):
+        return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
+    w8 = w >> 8
+    p0 = f16(_f16x2((w & 0x000F000F) | 0x64006400) - 1032.0)
+    p1 = f16(_f16x2((w & 0x00F000F0) | 0x64006400) * (1.0 / 16.0) - 72.0)
+    p2 = f16(_f16x2((w8 & 0x000F000F) | 0x64006400) - 1032.0)
+    p3 = f16(_f16x2((w8 & 0x00F000F0) | 0x64006400) * (1.0 / 16.0) - 72.0)
+    return np.concatenate([p0, p1, p2, p3])
+
+
+def test_int4_packed_word_dequantises_to_consecutive_code_pairs():
+    g = np.random.default_rng(4)
+    cases = [g.integers(-8, 8, 8) for _ in range(3000)]
+    for t in range(8):                                   # every value at every position
+        for q in range(-8, 8):
+            c = g.integers(-8, 8, 8)
+            c[t] = q
+            cases.append(c)
+    for codes in cases:
+        w = _place_per_nibble(codes)
+        np.testing.assert_array_equal(_nibbles_to_pairs(w), codes.astype(np.float64))
