@@ -97,6 +97,27 @@ def test_sixteen_bit_scale_may_round_down_and_codes_clamp():
     assert codes[0, 3] == qmax
 
 
+@pytest.mark.parametrize("group", [16, 32, 128, 256, 512])
+@pytest.mark.parametrize("bits,fmt", [(8, oracle.SCALE_F16), (4, oracle.SCALE_F32), (5, oracle.SCALE_BF16)])
+def test_groups_are_independent_row_problems(group, bits, fmt):
+    """Grouping is only a partition of each row: the codes and scales of
+    group g equal those of its g-wide slice quantized as rows of their own
+    (group 0), for bf16 input too; a group's scale follows its own maximum."""
+    g = np.random.default_rng(group + 10 * bits + fmt)
+    K = 1024
+    W = (g.standard_normal((5, K)) * np.exp(g.uniform(-3, 3, (5, K // group))).repeat(group, 1)).astype(np.float32)
+    W[2, group:2 * group] = 0.0  # one all-zero group
+    for x in (W, _bf16_bits(W)):
+        codes, scales = oracle.quantize_ex(x, bits, group, fmt)
+        assert codes.shape == (5, K) and scales.shape == (5, K // group)
+        for gi in range(K // group):
+            sl = np.ascontiguousarray(x[:, gi * group:(gi + 1) * group])
+            c1, s1 = oracle.quantize_ex(sl, bits, 0, fmt)
+            np.testing.assert_array_equal(codes[:, gi * group:(gi + 1) * group], c1)
+            np.testing.assert_array_equal(scales[:, gi], s1[:, 0])
+    assert not codes[2, group:2 * group].any() and scales[2, 1] == 0.0
+
+
 @pytest.mark.parametrize("bits,group", [(8, 0), (8, 64), (4, 64), (4, 16)])
 def test_fp32_scales_reduce_to_the_int8_int4_quantizer(bits, group):
     g = np.random.default_rng(11 + bits + group)
